@@ -1,0 +1,183 @@
+/*
+ * vdn.h -- C ABI of libvdn, the B200 (sm_100a) Video DeltaNet hybrid
+ * attention layer.
+ *
+ * The layer replaces video-to-video Softmax attention inside a video DiT by
+ * two branches ("Video DeltaNet", article on 10100.com, section 方法概述):
+ *   1. window-and-anchor Softmax (方法概述 item 1): each query chunk of 5
+ *      latent frames attends to itself and one chunk on each side; the first
+ *      and last latent frames are anchors that every frame sees and that see
+ *      every frame;                                   -> vdn_window_attn
+ *   2. Video Delta Attention (方法概述 item 2): a frame-level delta rule whose
+ *      state is S_t = (S_bar_t + B_t)(I + A_t)^-1 with S_bar_t = alpha_t S_{t-1},
+ *      A_t = sum_i beta_i k_i k_i^T, B_t = sum_i beta_i v_i k_i^T over the
+ *      tokens of frame t, run forward and backward over the frames (figure
+ *      caption under 效率阶梯, 前向加反向扫描);         -> vdn_vda_scan
+ *   3. branch calibration (方法概述 item 3): content-dependent sigmoid gate on
+ *      the Softmax branch, RMSNorm then a sigmoid output gate on the linear
+ *      branch, a separate output projection per branch, summed.
+ *                                                     -> vdn_hybrid_fuse
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tokens are frame-major: token row r = t*N + i (frame t, spatial token i).
+ *    Activations are row-major [L, ld] bf16 with L = T*N; head h occupies
+ *    columns [h*d, (h+1)*d).  bf16 arrays are passed as `const void*`
+ *    (IEEE bfloat16, 2 bytes per element).
+ *  - Every pointer is DEVICE memory owned by the caller.  The library never
+ *    allocates, frees or synchronises; every call only enqueues kernels on
+ *    `stream` (a cudaStream_t; NULL = the legacy default stream) and returns.
+ *  - Inputs are read-only; outputs are overwritten in full.
+ *  - Pointers must be 16-byte aligned; leading dimensions (elements) must be
+ *    multiples of 8 and >= H*d.
+ *  - Workspaces are caller-allocated device memory of at least the size the
+ *    matching *_workspace() query returns, 256-byte aligned.  The first 256
+ *    bytes of every workspace hold the device status word (see
+ *    vdn_get_device_status); call vdn_reset_device_status once after
+ *    allocating a workspace.
+ *  - Host-side argument errors return VDN_ERR_INVALID_ARG or
+ *    VDN_ERR_UNSUPPORTED before anything is enqueued.  A failed launch
+ *    returns VDN_ERR_CUDA.  Errors detected on the device (a non-positive
+ *    Cholesky pivot or NaN, a wait that ran out of time) are OR-ed into the
+ *    workspace status word; no kernel traps.
+ *  - Supported head dims: d in {64, 128}.  N >= 1, T >= 1, H >= 1.
+ */
+#ifndef VDN_H_
+#define VDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VDN_API __attribute__((visibility("default")))
+#else
+#define VDN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VDN_OK = 0,
+  VDN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or stride     */
+  VDN_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head dim 96)    */
+  VDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required      */
+  VDN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed               */
+  VDN_ERR_NUMERIC = 5,     /* device: non-positive pivot or NaN in a solve    */
+  VDN_ERR_TIMEOUT = 6      /* device: a bounded wait ran out                   */
+} vdn_status;
+
+/* Problem shape: T latent frames, N tokens per frame, H heads, head dim d
+ * (dk == dv == d). */
+typedef struct {
+  int T, N, H, d;
+} vdn_shape;
+
+/* ------------------------------------------------------------------------
+ * Video Delta Attention (10100.com article, 方法概述 item 2; the scan
+ * direction from the figure caption under 效率阶梯).
+ *
+ *   A_t,h = sum_{i in frame t} beta[i,h] k_i k_i^T
+ *   B_t,h = sum_{i in frame t} beta[i,h] v_i k_i^T            ([v_dim, k_dim])
+ *   P_t,h = (I + A_t,h)^-1   (Cholesky of the SPD matrix I + A)
+ *   S_fwd_t = (alpha_t S_fwd_{t-1} + B_t) P_t,   S_fwd_{-1} = 0
+ *   S_bwd_t = (alpha_t S_bwd_{t+1} + B_t) P_t,   S_bwd_T   = 0
+ *   o_vda[t*N+i, h*d:(h+1)*d] = (S_fwd_t,h + S_bwd_t,h) q_i     (no q scale)
+ *
+ * q, k, v   : [L, ld] bf16 (keys are taken as given; normalise beforehand)
+ * beta      : [L, H] fp32, row-major          (per-token write strength)
+ * alpha     : [T, H] fp32, row-major          (per-frame decay)
+ * o_vda     : [L, ld_o] bf16, output
+ * states_opt: NULL, or fp32 [2, T, H, d, d] output: [0] = S_fwd, [1] = S_bwd,
+ *             each state row-major [v_dim][k_dim]
+ * ws        : >= vdn_vda_scan_workspace(shape) bytes.  After the call it
+ *             also holds A, B, P and C = B P (see vdn_vda_debug_buffers).
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_vda_scan_workspace(const vdn_shape* shape);
+
+VDN_API vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                        int64_t ld, const float* beta, const float* alpha, void* o_vda,
+                        int64_t ld_o, float* states_opt, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* Pointers into a VDA workspace to the per-(frame, head) fp32 matrices the
+ * last vdn_vda_scan on that workspace produced, each [T, H, d, d]:
+ * A, B (prep), P = (I + A)^-1 and C = B P (solve).  Any out pointer may be
+ * NULL.  Pure pointer arithmetic: enqueues nothing. */
+VDN_API vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
+                                 float** P, float** C);
+
+/* ------------------------------------------------------------------------
+ * Window-and-anchor Softmax (10100.com article, 方法概述 item 1).
+ *
+ * Chunk c(t) = floor(t / chunk_frames).  Query frame tq sees key frame tk iff
+ * |c(tq) - c(tk)| <= window_chunks, or (anchors & 1) and 0 in {tq, tk}, or
+ * (anchors & 2) and T-1 in {tq, tk}.  All tokens of a frame share its mask.
+ *   o[r, h] = softmax_{visible keys}(q_r k^T * scale) v,  per head
+ *
+ * q, k, v  : [L, ld] bf16;  o: [L, ld_o] bf16 output
+ * scale    : <= 0 selects 1/sqrt(d)
+ * lse_opt  : NULL, or fp32 [H, L] output: natural-log sum of exp(scaled
+ *            scores) over the visible keys of each query row
+ * ws       : >= vdn_window_attn_workspace(shape) bytes
+ * chunk_frames >= 1, window_chunks >= 0, anchors in 0..3.
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_window_attn_workspace(const vdn_shape* shape);
+
+VDN_API vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                           int64_t ld, int chunk_frames, int window_chunks, unsigned anchors,
+                           float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Branch calibration and output projections (10100.com article, 方法概述
+ * item 3; hotpaper.ai summary, 기술적 접근법).
+ *
+ *   g_s = sigmoid(x W_gs^T),  g_l = sigmoid(x W_gl^T)              (elementwise)
+ *   n   = per-token, per-head RMSNorm of o_vda over d channels:
+ *         n = o / sqrt(mean_d(o^2) + eps) * gamma
+ *   y   = (g_s * o_s) W_os^T + (g_l * n) W_ol^T
+ *
+ * x, o_s, o_vda, y : [L, D] bf16, contiguous (ld = D), D = H*d
+ * W_gs, W_gl, W_os, W_ol : [D, D] bf16 row-major, W[out][in] (y = z W^T)
+ * gamma    : [D] fp32
+ * ws       : >= vdn_hybrid_fuse_workspace(L, D) bytes (holds the gated
+ *            branch outputs [L, 2D] bf16 between the two GEMMs)
+ * D must be a multiple of 128; L >= 1.
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_hybrid_fuse_workspace(int L, int D);
+
+VDN_API vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
+                           const void* o_vda, const void* W_gs, const void* W_gl,
+                           const float* gamma, float eps, const void* W_os, const void* W_ol,
+                           void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Status and diagnostics.
+ * ------------------------------------------------------------------------ */
+
+/* Static, human-readable message for a status code. */
+VDN_API const char* vdn_status_string(vdn_status s);
+
+/* Synchronise `stream`, then read the device status word of a workspace
+ * (VDN_OK if no kernel recorded an error since the last reset). */
+VDN_API vdn_status vdn_get_device_status(const void* ws, void* stream);
+
+/* Enqueue a clear of the workspace's device status word on `stream`. */
+VDN_API vdn_status vdn_reset_device_status(void* ws, void* stream);
+
+/* Wall-clock budget (ns) of every bounded wait inside the kernels launched
+ * after this call (default 2e9).  0 makes any wait that is not already
+ * satisfied fail at once with VDN_ERR_TIMEOUT: a test hook for the timeout
+ * path.  Process-wide; not thread-safe against concurrent launches. */
+VDN_API void vdn_set_wait_budget_ns(uint64_t ns);
+
+/* Library version string. */
+VDN_API const char* vdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDN_H_ */

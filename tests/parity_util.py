@@ -1,0 +1,29 @@
+"""Shared helpers for the parity tests (tolerance metrics, build hook)."""
+
+import numpy as np
+import torch
+
+# Tolerances: 2e-2 on bf16 outputs, 1e-3 on fp32 states, both as
+# max|gpu - ref| / max|ref| per tensor and per head slice.
+TOL_BF16 = 2e-2
+TOL_STATE = 1e-3
+
+
+def max_rel(gpu, ref):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    scale = np.abs(ref).max()
+    return float(np.abs(gpu - ref).max() / (scale if scale > 0 else 1.0))
+
+
+def per_head_max_rel(gpu, ref, H, d):
+    return max(max_rel(gpu[:, h * d:(h + 1) * d], ref[:, h * d:(h + 1) * d]) for h in range(H))
+
+
+def host(t):
+    return t.detach().to("cpu", torch.float32).numpy()
+
+
+def ensure_built():
+    from video_diffusion_hybrid_vda_b200 import build
+    build.build()

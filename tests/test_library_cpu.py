@@ -1,0 +1,87 @@
+"""libvdn on the CPU side: it builds for sm_100a, loads, exports every symbol
+include/vdn.h declares, and rejects bad arguments on the host before any
+CUDA call (so these run without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.parity_util import ensure_built
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    ensure_built()
+    from video_diffusion_hybrid_vda_b200 import vdn
+    return vdn
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "vdn.h")).read()
+    return sorted(set(re.findall(r"^VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert len(names) >= 12
+    lib = L.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(L.EXPORTS) == names
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert L.status_string(code)
+    assert "unknown" in L.status_string(99)
+    assert "sm_100a" in L.version()
+
+
+def test_workspace_queries(L):
+    lib = L.lib()
+    s = L.Shape(102, 4032, 24, 128)
+    mat = 102 * 24 * 128 * 128 * 4
+    assert lib.vdn_vda_scan_workspace(ctypes.byref(s)) == 256 + 6 * mat
+    assert lib.vdn_vda_scan_workspace(None) == 0
+    assert lib.vdn_vda_scan_workspace(ctypes.byref(L.Shape(0, 1, 1, 64))) == 0
+    assert lib.vdn_hybrid_fuse_workspace(411264, 3072) >= 411264 * 2 * 3072 * 2
+
+
+def _scan(L, shape, q=16, k=16, v=16, ld=128, beta=16, alpha=16, o=16, ld_o=128, states=None,
+          ws=256, ws_bytes=1 << 40):
+    lib = L.lib()
+    P = ctypes.c_void_p
+    return lib.vdn_vda_scan(ctypes.byref(shape) if shape is not None else None,
+                            P(q), P(k), P(v), ld, P(beta), P(alpha), P(o), ld_o,
+                            P(states) if states else None, P(ws), ws_bytes, None)
+
+
+def test_vda_scan_rejects_bad_arguments_on_host(L):
+    ok = L.Shape(4, 8, 1, 128)
+    assert _scan(L, None) == 1
+    assert _scan(L, L.Shape(0, 8, 1, 128)) == 1
+    assert _scan(L, L.Shape(4, 8, 1, 96)) == 2                 # unsupported head dim
+    assert _scan(L, ok, q=0) == 1                              # null pointer
+    assert _scan(L, ok, k=24) == 1                             # misaligned
+    assert _scan(L, ok, ld=100) == 1                           # ld % 8
+    assert _scan(L, ok, ld=64) == 1                            # ld < D
+    assert _scan(L, ok, ld_o=120) == 1
+    assert _scan(L, ok, ws=0) == 3                             # no workspace
+    assert _scan(L, ok, ws=128) == 3                           # misaligned workspace
+    assert _scan(L, ok, ws_bytes=1024) == 3                    # too small
+
+
+def test_window_and_fuse_reject_bad_arguments_on_host(L):
+    lib = L.lib()
+    P = ctypes.c_void_p
+    s = L.Shape(10, 16, 1, 128)
+    r = lib.vdn_window_attn(ctypes.byref(s), None, P(16), P(16), 128, 5, 1, 3, 0.0, P(16), 128,
+                            None, P(256), 1 << 30, None)
+    assert r in (1, 2)
+    r = lib.vdn_hybrid_fuse(16, 128, 1, None, P(16), P(16), P(16), P(16), P(16), 1e-6, P(16),
+                            P(16), P(16), P(256), 1 << 30, None)
+    assert r in (1, 2)

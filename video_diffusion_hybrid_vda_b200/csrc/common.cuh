@@ -1,0 +1,57 @@
+// Internal declarations shared by the libvdn translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/vdn.h"
+
+namespace vdn {
+
+// Bits of the device status word (first 4 bytes of every workspace).
+constexpr uint32_t kStatusNumeric = 1u << 0;
+constexpr uint32_t kStatusTimeout = 1u << 1;
+
+// Workspace bytes reserved in front of every workspace for the status word.
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void record_status(uint32_t* status, uint32_t bits) {
+  if (status != nullptr) atomicOr(status, bits);
+}
+
+// Launch context handed to every launcher.
+struct Launch {
+  cudaStream_t stream;
+  uint32_t* status;     // device status word
+  uint64_t budget_ns;   // bounded-wait budget
+};
+
+// ---- tensor maps (built on the host with the driver's encoder) ----------
+
+// 3-D bf16 view of a frame-major [T*N, ld] activation: dims {cols, N, T}.
+// Rows past the end of a frame fall outside dim 1, so TMA loads read zeros
+// there and TMA stores drop them.  Box {64, box_rows, 1}, 128-byte swizzle.
+bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int N, int T,
+                    int box_rows);
+
+// 2-D bf16 map over a row-major [rows, ld] matrix with box {64, box_rows},
+// 128-byte swizzle.
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int64_t rows,
+                   int box_rows);
+
+// ---- kernel launchers (return cudaSuccess or the launch error) ----------
+
+cudaError_t launch_vda_prep(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
+                            const CUtensorMap& vmap, const float* beta, float* A, float* B);
+
+cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A,
+                             const float* B, float* P, float* C);
+
+cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* P,
+                            const float* C, const float* alpha, float* states);
+
+cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                               const CUtensorMap& omap, const float* states);
+
+}  // namespace vdn

@@ -1,0 +1,279 @@
+// VDA-prep: per (frame t, head h) form
+//     A_t,h = sum_i beta_i k_i k_i^T      B_t,h = sum_i beta_i v_i k_i^T
+// over the N spatial tokens of frame t ("Video DeltaNet", 10100.com article,
+// 方法概述 item 2: A_t gathers key correlations, B_t value-key writes).
+//
+// Design (sm_100a):
+//  * one CTA per (t, h); the token dimension is the GEMM reduction;
+//  * TMA streams [BK tokens x d] tiles of k and v into 128B-swizzled shared
+//    memory through a 3-D frame view, so rows past the frame read as zero;
+//  * four "scaler" warps write beta_i * k_i as a bf16 pair hi + lo (hi the
+//    rounded product, lo the rounded remainder; their sum carries ~16
+//    mantissa bits) into two more tiles;
+//  * one thread issues tcgen05.mma with both operands MN-major (token rows,
+//    feature columns): D_A += K^T hi + K^T lo, D_B += V^T hi + V^T lo, fp32
+//    accumulation in TMEM;
+//    for d = 64 the A operand is the stacked [K | V] feature block (M = 128)
+//    so one instruction produces both A (rows 0..63) and B (rows 64..127);
+//  * the scaler warps then drain TMEM rows to global fp32 A and B.
+// The stage is HBM-bound (k and v are read once); the split doubles the
+// tensor-core work, which stays below the HBM time.
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace vdn {
+namespace {
+
+template <int DH>
+struct PrepCfg {
+  static constexpr int BK = DH == 128 ? 32 : 64;  // tokens per pipeline stage
+  static constexpr int SLABS = DH / 64;           // 64-column slabs per tile
+  static constexpr int SLAB_BYTES = BK * 128;
+  static constexpr int TILE_BYTES = SLABS * SLAB_BYTES;
+  static constexpr int STAGE_BYTES = 4 * TILE_BYTES;  // K, V, (beta*K)_hi, (beta*K)_lo
+  static constexpr int STAGES = 3;
+  static constexpr int TMEM_COLS = DH == 128 ? 256 : 64;
+  static constexpr int THREADS = 192;  // warp0 TMA, warp1 MMA, warps2-5 scale+epilogue
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int CHUNKS_PER_THREAD = TILE_BYTES / 16 / 128;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
+    vda_prep_kernel(const __grid_constant__ CUtensorMap kmap,
+                    const __grid_constant__ CUtensorMap vmap, const float* __restrict__ beta,
+                    float* __restrict__ A, float* __restrict__ B, int T, int N, int H,
+                    uint32_t* status, uint64_t budget_ns) {
+  using C = PrepCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* scaled = full + C::STAGES;
+  uint64_t* empty = scaled + C::STAGES;
+  uint64_t* accum_full = empty + C::STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
+
+  const int th = blockIdx.x;  // = t * H + h
+  const int t = th / H;
+  const int h = th % H;
+  const int nk = (N + C::BK - 1) / C::BK;
+  const uint32_t warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&scaled[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accum_full, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto stage_k = [&](int s) { return smem + s * C::STAGE_BYTES; };
+  auto stage_v = [&](int s) { return smem + s * C::STAGE_BYTES + C::TILE_BYTES; };
+  auto stage_hi = [&](int s) { return smem + s * C::STAGE_BYTES + 2 * C::TILE_BYTES; };
+  auto stage_lo = [&](int s) { return smem + s * C::STAGE_BYTES + 3 * C::TILE_BYTES; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int issued = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nk && ok; ++kb) {
+        const int s = kb % C::STAGES;
+        if (kb >= C::STAGES) {
+          if (!mbar_wait(&empty[s], ((kb / C::STAGES) & 1) ^ 1, budget_ns)) {
+            record_status(status, kStatusTimeout);
+            ok = false;
+            break;
+          }
+        }
+        mbar_arrive_expect_tx(&full[s], 2 * C::TILE_BYTES);
+        for (int j = 0; j < C::SLABS; ++j) {
+          tma_load_3d(stage_k(s) + j * C::SLAB_BYTES, &kmap, &full[s], h * DH + 64 * j,
+                      kb * C::BK, t);
+          tma_load_3d(stage_v(s) + j * C::SLAB_BYTES, &vmap, &full[s], h * DH + 64 * j,
+                      kb * C::BK, t);
+        }
+        ++issued;
+      }
+      // Drain: the last loads of every stage must have landed before exit.
+      for (int kb = (issued > C::STAGES ? issued - C::STAGES : 0); kb < issued; ++kb) {
+        const int s = kb % C::STAGES;
+        if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, 200000000ull)) {
+          record_status(status, kStatusTimeout);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16(128, DH, true, true);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % C::STAGES;
+        if (!mbar_wait(&scaled[s], (kb / C::STAGES) & 1, budget_ns)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kbase = smem_u32(stage_k(s));
+        const uint32_t vbase = smem_u32(stage_v(s));
+        const uint32_t hbase = smem_u32(stage_hi(s));
+        const uint32_t lbase = smem_u32(stage_lo(s));
+#pragma unroll
+        for (int kk = 0; kk < C::BK / 16; ++kk) {
+          const uint32_t acc = (kb | kk) != 0;
+          const uint64_t hdesc = sdesc_sw128(hbase + kk * 2048, C::SLAB_BYTES, 1024);
+          const uint64_t ldesc = sdesc_sw128(lbase + kk * 2048, C::SLAB_BYTES, 1024);
+          const uint64_t kdesc = sdesc_sw128(kbase + kk * 2048, C::SLAB_BYTES, 1024);
+          if constexpr (DH == 128) {
+            const uint64_t vdesc = sdesc_sw128(vbase + kk * 2048, C::SLAB_BYTES, 1024);
+            umma_ss(tmem, kdesc, hdesc, idesc, acc);
+            umma_ss(tmem, kdesc, ldesc, idesc, 1);
+            umma_ss(tmem + 128, vdesc, hdesc, idesc, acc);
+            umma_ss(tmem + 128, vdesc, ldesc, idesc, 1);
+          } else {
+            // [K | V] stacked along M: the V slab sits one slab after K.
+            umma_ss(tmem, kdesc, hdesc, idesc, acc);
+            umma_ss(tmem, kdesc, ldesc, idesc, 1);
+          }
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accum_full);
+    }
+  } else {
+    // ------------------------------------------------------------ scalers
+    const int tid = threadIdx.x - 64;  // 0..127
+    bool ok = true;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % C::STAGES;
+      // beta for the rows this thread touches in this stage
+      float bv[C::CHUNKS_PER_THREAD];
+#pragma unroll
+      for (int j = 0; j < C::CHUNKS_PER_THREAD; ++j) {
+        const int off = (tid + 128 * j) * 16;
+        const int row = (off % C::SLAB_BYTES) / 128;
+        const int i = kb * C::BK + row;
+        bv[j] = i < N ? __ldg(beta + (static_cast<int64_t>(t) * N + i) * H + h) : 0.f;
+      }
+      if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, budget_ns)) {
+        record_status(status, kStatusTimeout);
+        ok = false;
+        break;
+      }
+      const uint8_t* ks = stage_k(s);
+      uint8_t* his = stage_hi(s);
+      uint8_t* los = stage_lo(s);
+#pragma unroll
+      for (int j = 0; j < C::CHUNKS_PER_THREAD; ++j) {
+        const int off = (tid + 128 * j) * 16;
+        uint4 u = *reinterpret_cast<const uint4*>(ks + off);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w[e]);
+          const float px = f.x * bv[j], py = f.y * bv[j];
+          hi[e] = pack_bf16x2(px, py);
+          const float2 fh = unpack_bf16x2(hi[e]);
+          lo[e] = pack_bf16x2(px - fh.x, py - fh.y);
+        }
+        *reinterpret_cast<uint4*>(his + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(los + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&scaled[s]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && mbar_wait(accum_full, 0, budget_ns)) {
+      tc_fence_after();
+      const uint32_t quarter = warp & 3;  // TMEM lane quarter this warp may access
+      const int m = quarter * 32 + lane_id();
+      const uint32_t lane_base = tmem + ((quarter * 32) << 16);
+      const int64_t mat = (static_cast<int64_t>(t) * H + h) * DH * DH;
+      if constexpr (DH == 128) {
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float* dst = (half == 0 ? A : B) + mat + static_cast<int64_t>(m) * DH;
+#pragma unroll 1
+          for (int c = 0; c < DH; c += 32) {
+            uint32_t r[32];
+            tmem_ld32(lane_base + half * 128 + c, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dst + c + e) =
+                  make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                              __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+          }
+        }
+      } else {
+        float* dst = (m < 64 ? A + mat + static_cast<int64_t>(m) * DH
+                             : B + mat + static_cast<int64_t>(m - 64) * DH);
+#pragma unroll 1
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(lane_base + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + c + e) =
+                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+        }
+      }
+    } else if (ok) {
+      record_status(status, kStatusTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    // All MMAs were committed to accum_full; make sure they finished before
+    // the columns are released (no-op on the normal path).
+    mbar_wait(accum_full, 0, 200000000ull);
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int DH>
+cudaError_t launch_prep_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
+                           const CUtensorMap& vmap, const float* beta, float* A, float* B) {
+  using C = PrepCfg<DH>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(vda_prep_kernel<DH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = s.T * s.H;
+  vda_prep_kernel<DH><<<grid, C::THREADS, C::SMEM, ctx.stream>>>(
+      kmap, vmap, beta, A, B, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_vda_prep(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
+                            const CUtensorMap& vmap, const float* beta, float* A, float* B) {
+  if (s.d == 128) return launch_prep_dh<128>(ctx, s, kmap, vmap, beta, A, B);
+  if (s.d == 64) return launch_prep_dh<64>(ctx, s, kmap, vmap, beta, A, B);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace vdn

@@ -1,0 +1,222 @@
+// C ABI of libvdn: host-side validation, workspace layout, TMA descriptor
+// construction and kernel sequencing.  Every entry point validates all of
+// its arguments before it enqueues anything, then launches asynchronously on
+// the caller's stream.  Nothing here allocates, frees or synchronises (except
+// vdn_get_device_status, whose job is to read the status word back).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace vdn {
+
+namespace {
+
+std::atomic<uint64_t> g_budget_ns{2000000000ull};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool shape_ok(const vdn_shape* s) {
+  return s != nullptr && s->T >= 1 && s->N >= 1 && s->H >= 1 && s->d >= 1 &&
+         static_cast<int64_t>(s->T) * s->N < (int64_t(1) << 31) &&
+         static_cast<int64_t>(s->H) * s->d < (int64_t(1) << 24);
+}
+
+bool head_dim_supported(int d) { return d == 64 || d == 128; }
+
+bool ld_ok(int64_t ld, int64_t D) { return ld >= D && ld % 8 == 0; }
+
+// VDA workspace: [status 256 B][A][B][P][C][states (2x)], each region
+// 256-byte aligned, every matrix fp32 [T, H, d, d].
+struct VdaLayout {
+  size_t mat_bytes, A, B, P, C, states, total;
+};
+
+VdaLayout vda_layout(const vdn_shape& s) {
+  VdaLayout l;
+  l.mat_bytes = round_up(static_cast<size_t>(s.T) * s.H * s.d * s.d * sizeof(float), 256);
+  l.A = kStatusBytes;
+  l.B = l.A + l.mat_bytes;
+  l.P = l.B + l.mat_bytes;
+  l.C = l.P + l.mat_bytes;
+  l.states = l.C + l.mat_bytes;
+  l.total = l.states + 2 * l.mat_bytes;
+  return l;
+}
+
+}  // namespace
+
+bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int N, int T,
+                    int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(T)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2,
+                                 static_cast<cuuint64_t>(ld) * 2 * static_cast<cuuint64_t>(N)};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int64_t rows,
+                   int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+const char* vdn_version(void) { return "vdn-b200 0.1 (sm_100a)"; }
+
+const char* vdn_status_string(vdn_status s) {
+  switch (s) {
+    case VDN_OK: return "ok";
+    case VDN_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer, bad size or stride)";
+    case VDN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case VDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case VDN_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case VDN_ERR_NUMERIC: return "numeric failure on the device (non-positive pivot or NaN)";
+    case VDN_ERR_TIMEOUT: return "a bounded wait on the device ran out of time";
+  }
+  return "unknown status";
+}
+
+void vdn_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns); }
+
+vdn_status vdn_reset_device_status(void* ws, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return VDN_ERR_WORKSPACE;
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+vdn_status vdn_get_device_status(const void* ws, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return VDN_ERR_WORKSPACE;
+  uint32_t word = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VDN_ERR_CUDA;
+  if (word & kStatusTimeout) return VDN_ERR_TIMEOUT;
+  if (word & kStatusNumeric) return VDN_ERR_NUMERIC;
+  return VDN_OK;
+}
+
+// ----------------------------------------------------------------- VDA
+
+size_t vdn_vda_scan_workspace(const vdn_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return vda_layout(*shape).total;
+}
+
+vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
+                                 float** P, float** C) {
+  if (!shape_ok(shape) || ws == nullptr) return VDN_ERR_INVALID_ARG;
+  const VdaLayout l = vda_layout(*shape);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (A) *A = reinterpret_cast<float*>(base + l.A);
+  if (B) *B = reinterpret_cast<float*>(base + l.B);
+  if (P) *P = reinterpret_cast<float*>(base + l.P);
+  if (C) *C = reinterpret_cast<float*>(base + l.C);
+  return VDN_OK;
+}
+
+vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                        int64_t ld, const float* beta, const float* alpha, void* o_vda,
+                        int64_t ld_o, float* states_opt, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (!shape_ok(shape)) return VDN_ERR_INVALID_ARG;
+  const vdn_shape s = *shape;
+  if (!head_dim_supported(s.d)) return VDN_ERR_UNSUPPORTED;
+  const int64_t D = static_cast<int64_t>(s.H) * s.d;
+  if (q == nullptr || k == nullptr || v == nullptr || beta == nullptr || alpha == nullptr ||
+      o_vda == nullptr)
+    return VDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_vda, 16) ||
+      !aligned(beta, 4) || !aligned(alpha, 4) || (states_opt && !aligned(states_opt, 16)))
+    return VDN_ERR_INVALID_ARG;
+  if (!ld_ok(ld, D) || !ld_ok(ld_o, D)) return VDN_ERR_INVALID_ARG;
+  const VdaLayout l = vda_layout(s);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < l.total) return VDN_ERR_WORKSPACE;
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* A = reinterpret_cast<float*>(base + l.A);
+  float* B = reinterpret_cast<float*>(base + l.B);
+  float* P = reinterpret_cast<float*>(base + l.P);
+  float* C = reinterpret_cast<float*>(base + l.C);
+  float* states = states_opt ? states_opt : reinterpret_cast<float*>(base + l.states);
+
+  const int prep_rows = s.d == 128 ? 32 : 64;
+  CUtensorMap kmap, vmap, qmap, omap;
+  if (!make_frame_map(&kmap, k, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&vmap, v, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&qmap, q, D, ld, s.N, s.T, 128) ||
+      !make_frame_map(&omap, o_vda, D, ld_o, s.N, s.T, 128))
+    return VDN_ERR_CUDA;
+
+  Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
+             g_budget_ns.load()};
+  if (launch_vda_prep(ctx, s, kmap, vmap, beta, A, B) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+}  // extern "C"
+// ----------------------------------------------------------------- pending
+extern "C" {
+size_t vdn_window_attn_workspace(const vdn_shape* shape) { return shape_ok(shape) ? 256 : 0; }
+vdn_status vdn_window_attn(const vdn_shape*, const void*, const void*, const void*, int64_t, int,
+                           int, unsigned, float, void*, int64_t, float*, void*, size_t, void*) {
+  return VDN_ERR_UNSUPPORTED;
+}
+size_t vdn_hybrid_fuse_workspace(int L, int D) {
+  return kStatusBytes + static_cast<size_t>(L) * 2 * D * 2;
+}
+vdn_status vdn_hybrid_fuse(int, int, int, const void*, const void*, const void*, const void*,
+                           const void*, const float*, float, const void*, const void*, void*,
+                           void*, size_t, void*) {
+  return VDN_ERR_UNSUPPORTED;
+}
+}

@@ -1,0 +1,223 @@
+"""ctypes binding over libvdn.so (declared in include/vdn.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Tensors must live on the current CUDA device; PyTorch provides
+device memory and the stream.  If the library is missing, every call raises
+(there is no CPU fallback).
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvdn.so")
+
+VDN_OK = 0
+STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
+                3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_NUMERIC",
+                6: "VDN_ERR_TIMEOUT"}
+
+# every symbol include/vdn.h declares
+EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
+           "vdn_window_attn_workspace", "vdn_window_attn", "vdn_hybrid_fuse_workspace",
+           "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
+           "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version"]
+
+
+class VdnError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({status_string(code)})")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("N", ctypes.c_int), ("H", ctypes.c_int),
+                ("d", ctypes.c_int)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_FP = ctypes.POINTER(ctypes.c_float)
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+
+
+def lib():
+    """Load libvdn.so once; raise if it is not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libvdn.so not found at {LIB_PATH}; build it with "
+                           "`python -m video_diffusion_hybrid_vda_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    S = ctypes.POINTER(Shape)
+    L.vdn_vda_scan_workspace.argtypes = [S]
+    L.vdn_vda_scan_workspace.restype = _SZ
+    L.vdn_vda_scan.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]
+    L.vdn_vda_scan.restype = ctypes.c_int
+    L.vdn_vda_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 4
+    L.vdn_vda_debug_buffers.restype = ctypes.c_int
+    L.vdn_window_attn_workspace.argtypes = [S]
+    L.vdn_window_attn_workspace.restype = _SZ
+    L.vdn_window_attn.argtypes = [S, _P, _P, _P, _I64, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_uint, ctypes.c_float, _P, _I64, _P, _P, _SZ, _P]
+    L.vdn_window_attn.restype = ctypes.c_int
+    L.vdn_hybrid_fuse_workspace.argtypes = [ctypes.c_int, ctypes.c_int]
+    L.vdn_hybrid_fuse_workspace.restype = _SZ
+    L.vdn_hybrid_fuse.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
+                                  _P, ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
+    L.vdn_hybrid_fuse.restype = ctypes.c_int
+    L.vdn_status_string.argtypes = [ctypes.c_int]
+    L.vdn_status_string.restype = ctypes.c_char_p
+    L.vdn_get_device_status.argtypes = [_P, _P]
+    L.vdn_get_device_status.restype = ctypes.c_int
+    L.vdn_reset_device_status.argtypes = [_P, _P]
+    L.vdn_reset_device_status.restype = ctypes.c_int
+    L.vdn_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
+    L.vdn_set_wait_budget_ns.restype = None
+    L.vdn_version.argtypes = []
+    L.vdn_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(code):
+    return lib().vdn_status_string(int(code)).decode()
+
+
+def version():
+    return lib().vdn_version().decode()
+
+
+def _check(code, where):
+    if code != VDN_OK:
+        raise VdnError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _shape(T, N, H, d):
+    return Shape(int(T), int(N), int(H), int(d))
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libvdn takes CUDA tensors only")
+
+
+def alloc_workspace(nbytes, device=None):
+    """Device workspace with a cleared status word."""
+    ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8,
+                     device=device or torch.device("cuda"))
+    _check(lib().vdn_reset_device_status(_ptr(ws), _stream(None)), "vdn_reset_device_status")
+    return ws
+
+
+def get_device_status(ws, stream=None):
+    """Synchronise the stream and return the workspace status code (0 = ok)."""
+    return lib().vdn_get_device_status(_ptr(ws), _stream(stream))
+
+
+def reset_device_status(ws, stream=None):
+    _check(lib().vdn_reset_device_status(_ptr(ws), _stream(stream)), "vdn_reset_device_status")
+
+
+def set_wait_budget_ns(ns):
+    lib().vdn_set_wait_budget_ns(int(ns))
+
+
+# ---------------------------------------------------------------- VDA
+
+def vda_scan_workspace(T, N, H, d):
+    return int(lib().vdn_vda_scan_workspace(ctypes.byref(_shape(T, N, H, d))))
+
+
+def vda_scan(q, k, v, beta, alpha, T, N, H, d, out=None, states=None, ws=None, stream=None):
+    """Video Delta Attention: o_vda = (S_fwd_t + S_bwd_t) q per token.
+
+    q, k, v: [T*N, ld] bf16; beta [T*N, H] fp32; alpha [T, H] fp32.
+    Returns (o_vda, ws).  ``states`` (fp32 [2, T, H, d, d]) receives both
+    scans' states when given.
+    """
+    _need_cuda(q, k, v, beta, alpha, out, states, ws)
+    shape = _shape(T, N, H, d)
+    if out is None:
+        out = torch.empty((T * N, H * d), dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(vda_scan_workspace(T, N, H, d), q.device)
+    code = lib().vdn_vda_scan(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
+                              _ptr(beta), _ptr(alpha), _ptr(out), out.stride(0), _ptr(states),
+                              _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "vdn_vda_scan")
+    return out, ws
+
+
+def vda_debug_buffers(ws, T, N, H, d):
+    """(A, B, P, C) views into a VDA workspace, each fp32 [T, H, d, d]."""
+    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    _check(lib().vdn_vda_debug_buffers(ctypes.byref(_shape(T, N, H, d)), _ptr(ws),
+                                       *[ctypes.byref(p) for p in ptrs]), "vdn_vda_debug_buffers")
+    base = ws.data_ptr()
+    n = T * H * d * d
+    flat = ws.view(torch.uint8)
+    out = []
+    for p in ptrs:
+        off = p.value - base
+        out.append(flat[off:off + 4 * n].view(torch.float32).view(T, H, d, d))
+    return tuple(out)
+
+
+# ---------------------------------------------------------------- window Softmax
+
+def window_attn_workspace(T, N, H, d):
+    return int(lib().vdn_window_attn_workspace(ctypes.byref(_shape(T, N, H, d))))
+
+
+def window_attn(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3, scale=0.0,
+                out=None, lse=None, ws=None, stream=None):
+    """Window-and-anchor Softmax.  Returns (o, ws); fills ``lse`` [H, T*N] if given."""
+    _need_cuda(q, k, v, out, lse, ws)
+    shape = _shape(T, N, H, d)
+    if out is None:
+        out = torch.empty((T * N, H * d), dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(window_attn_workspace(T, N, H, d), q.device)
+    code = lib().vdn_window_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
+                                 int(chunk_frames), int(window_chunks), int(anchors),
+                                 float(scale), _ptr(out), out.stride(0), _ptr(lse), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    _check(code, "vdn_window_attn")
+    return out, ws
+
+
+# ---------------------------------------------------------------- fuse
+
+def hybrid_fuse_workspace(L, D):
+    return int(lib().vdn_hybrid_fuse_workspace(int(L), int(D)))
+
+
+def hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, H, eps=1e-6, out=None, ws=None,
+                stream=None):
+    """y = (sigmoid(x W_gs^T) o_s) W_os^T + (sigmoid(x W_gl^T) RMSNorm(o_vda)) W_ol^T."""
+    _need_cuda(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, out, ws)
+    L, D = x.shape
+    if out is None:
+        out = torch.empty((L, D), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(hybrid_fuse_workspace(L, D), x.device)
+    code = lib().vdn_hybrid_fuse(int(L), int(D), int(H), _ptr(x), _ptr(o_s), _ptr(o_vda),
+                                 _ptr(W_gs), _ptr(W_gl), _ptr(gamma), float(eps), _ptr(W_os),
+                                 _ptr(W_ol), _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "vdn_hybrid_fuse")
+    return out, ws
