@@ -27,6 +27,9 @@ struct Launch {
   uint64_t budget_ns;   // bounded-wait budget
 };
 
+// Budget (ns) of the bounded device waits, set by vdn_set_wait_budget_ns.
+uint64_t current_wait_budget_ns();
+
 // ---- tensor maps (built on the host with the driver's encoder) ----------
 
 // 3-D bf16 view of a frame-major [T*N, ld] activation: dims {cols, N, T}.

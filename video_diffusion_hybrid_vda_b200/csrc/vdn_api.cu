@@ -72,6 +72,8 @@ VdaLayout vda_layout(const vdn_shape& s) {
 
 }  // namespace
 
+uint64_t current_wait_budget_ns() { return g_budget_ns.load(); }
+
 bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int N, int T,
                     int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -206,11 +208,6 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
 }  // extern "C"
 // ----------------------------------------------------------------- pending
 extern "C" {
-size_t vdn_window_attn_workspace(const vdn_shape* shape) { return shape_ok(shape) ? 256 : 0; }
-vdn_status vdn_window_attn(const vdn_shape*, const void*, const void*, const void*, int64_t, int,
-                           int, unsigned, float, void*, int64_t, float*, void*, size_t, void*) {
-  return VDN_ERR_UNSUPPORTED;
-}
 size_t vdn_hybrid_fuse_workspace(int L, int D) {
   return kStatusBytes + static_cast<size_t>(L) * 2 * D * 2;
 }

@@ -1,0 +1,511 @@
+// Window-and-anchor Softmax attention ("Video DeltaNet", 10100.com article,
+// 方法概述 item 1): latent frames form chunks of `chunk_frames`; a query frame
+// attends to the frames of its own chunk and `window_chunks` chunks on each
+// side, plus the anchor frames 0 and T-1, and the anchor frames attend to
+// every frame.  All spatial tokens of a frame share its mask.
+//
+// Schedule (host): consecutive query frames with the same visible key set
+// form a segment; a segment's keys are at most three contiguous token
+// intervals (the window, frame 0, frame T-1).  Every CTA takes 256 query rows
+// (two 128-row tiles) of one segment and one head and loops over the
+// segment's key tiles (128 keys; the last tile of an interval is masked by
+// column).  CTAs are ordered heaviest segment first so the long anchor rows
+// start early.
+//
+// Kernel (sm_100a, one CTA per SM):
+//   warp 0      TMA: Q0/Q1 once, then K/V tiles through a 2-stage ring
+//   warp 1      tcgen05.mma issue: S_i = Q_i K^T into TMEM, O_i += P_i V with
+//               P_i read from TMEM (the A operand) and V MN-major in smem
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
+//               per query row; online max/sum in the exp2 domain, P written
+//               back over S as packed bf16; O rescaled in TMEM only when the
+//               running max grows by more than 2^8 (lazy rescale)
+// TMEM: S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512) columns.
+// The two softmax groups alternate with the tensor core: while one converts
+// S_i to P_i, the MMA warp runs the other tile's products.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace vdn {
+
+namespace {
+
+constexpr int kMaxSegs = 256;
+
+struct WinSeg {
+  int q0, q1;      // query token rows [q0, q1)
+  int tile_base;   // first CTA tile index of this segment (launch order)
+  int ntiles;      // 256-row CTA tiles
+  int nint;        // key intervals (1..3)
+  int k0[3], k1[3];
+  int nkv;         // 128-key tiles over all intervals
+};
+
+struct WinSched {
+  int nseg;
+  int total_tiles;
+  WinSeg seg[kMaxSegs];
+};
+
+template <int DH>
+struct WinCfg {
+  static constexpr int SLABS = DH / 64;
+  static constexpr int TILE_BYTES = SLABS * 128 * 128;  // 128 rows x DH bf16
+  static constexpr int STAGES = 2;
+  static constexpr int THREADS = 384;
+  static constexpr int SMEM = 1024 + 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 512;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Key tile `j` of a segment: start row and number of valid keys.
+struct KvCursor {
+  int iv, pos;
+  __device__ void init(const WinSeg& s) {
+    iv = 0;
+    pos = s.k0[0];
+  }
+  __device__ void next(const WinSeg& s) {
+    pos += 128;
+    if (pos >= s.k1[iv] && iv + 1 < s.nint) {
+      ++iv;
+      pos = s.k0[iv];
+    }
+  }
+  __device__ int valid(const WinSeg& s) const { return min(128, s.k1[iv] - pos); }
+};
+
+template <int DH>
+__global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
+    window_attn_kernel(const __grid_constant__ CUtensorMap qmap,
+                       const __grid_constant__ CUtensorMap kmap,
+                       const __grid_constant__ CUtensorMap vmap,
+                       const __grid_constant__ WinSched sched, int H, int L, float scale_log2,
+                       __nv_bfloat16* __restrict__ out, int64_t ld_o, float* __restrict__ lse,
+                       uint32_t* status, uint64_t budget_ns) {
+  using Cfg = WinCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* qbuf = smem;                              // Q0, Q1
+  uint8_t* kvbuf = smem + 2 * Cfg::TILE_BYTES;       // stage s: K then V
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kvbuf + Cfg::STAGES * 2 * Cfg::TILE_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;                      // [STAGES]
+  uint64_t* kv_empty = kv_full + Cfg::STAGES;        // [STAGES]
+  uint64_t* s_full = kv_empty + Cfg::STAGES;         // [2]
+  uint64_t* p_ready = s_full + 2;                    // [2]
+  uint64_t* o_done = p_ready + 2;                    // [2]
+  uint64_t* mma_done = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  // ---- which segment / tile / head
+  const int lin = blockIdx.x;
+  const int h = lin % H;
+  const int tile = lin / H;
+  int si = 0;
+  while (si + 1 < sched.nseg && tile >= sched.seg[si + 1].tile_base) ++si;
+  const WinSeg& seg = sched.seg[si];
+  const int q0 = seg.q0 + (tile - seg.tile_base) * 256;
+  const int nkv = seg.nkv;
+  const uint32_t warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_ready[i], 128);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================================================================ TMA
+    if (elect_one()) {
+      mbar_arrive_expect_tx(q_full, 2 * Cfg::TILE_BYTES);
+      for (int i = 0; i < 2; ++i)
+        for (int sl = 0; sl < Cfg::SLABS; ++sl)
+          tma_load_2d(qbuf + i * Cfg::TILE_BYTES + sl * 16384, &qmap, q_full, h * DH + 64 * sl,
+                      q0 + 128 * i);
+      KvCursor cur;
+      cur.init(seg);
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % Cfg::STAGES;
+        if (j >= Cfg::STAGES &&
+            !mbar_wait(&kv_empty[s], ((j / Cfg::STAGES) & 1) ^ 1, budget_ns)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        uint8_t* kb = kvbuf + s * 2 * Cfg::TILE_BYTES;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * Cfg::TILE_BYTES);
+        for (int sl = 0; sl < Cfg::SLABS; ++sl) {
+          tma_load_2d(kb + sl * 16384, &kmap, &kv_full[s], h * DH + 64 * sl, cur.pos);
+          tma_load_2d(kb + Cfg::TILE_BYTES + sl * 16384, &vmap, &kv_full[s], h * DH + 64 * sl,
+                      cur.pos);
+        }
+        ++issued;
+        cur.next(seg);
+      }
+      // drain loads still in flight
+      mbar_wait(q_full, 0, 200000000ull);
+      for (int j = (issued > Cfg::STAGES ? issued - Cfg::STAGES : 0); j < issued; ++j)
+        if (!mbar_wait(&kv_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull))
+          record_status(status, kStatusTimeout);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(128, DH, false, true);
+      const uint32_t qb = smem_u32(qbuf);
+      bool ok = mbar_wait(q_full, 0, budget_ns);
+      auto issue_s = [&](int i, int j) {
+        const uint32_t kb = smem_u32(kvbuf + (j % Cfg::STAGES) * 2 * Cfg::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + 128 * i, sdesc_sw128(qb + i * Cfg::TILE_BYTES + off, 16, 1024),
+                  sdesc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(&s_full[i]);
+      };
+      auto issue_o = [&](int i, int j) {
+        const uint32_t vb =
+            smem_u32(kvbuf + (j % Cfg::STAGES) * 2 * Cfg::TILE_BYTES + Cfg::TILE_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
+          umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8,
+                  sdesc_sw128(vb + kk * 2048, 16384, 1024), idesc_o, (j > 0 || kk > 0));
+        umma_commit(&o_done[i]);
+      };
+      if (ok && (ok = mbar_wait(&kv_full[0], 0, budget_ns))) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % Cfg::STAGES;
+        const bool more = j + 1 < nkv;
+        if (!(ok = mbar_wait(&p_ready[0], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(0, j);
+        if (more) {
+          const int sn = (j + 1) % Cfg::STAGES;
+          if (!(ok = mbar_wait(&kv_full[sn], ((j + 1) / Cfg::STAGES) & 1, budget_ns))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = mbar_wait(&p_ready[1], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(1, j);
+        umma_commit(&kv_empty[s]);
+        if (more) issue_s(1, j + 1);
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+      umma_commit(mma_done);
+    }
+  } else if (warp >= 4) {
+    // ================================================================ softmax
+    const int i = (warp - 4) >> 2;  // query tile of this warpgroup
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane_id();
+    const uint32_t lane_off = (quarter * 32) << 16;
+    const uint32_t s_addr = tmem + 128 * i + lane_off;
+    const uint32_t o_addr = tmem + 256 + 128 * i + lane_off;
+    float m_used = -INFINITY;  // running max, log2 domain (scaled)
+    float l = 0.f;
+    KvCursor cur;
+    cur.init(seg);
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      const int valid = cur.valid(seg);
+      cur.next(seg);
+      if (!mbar_wait(&s_full[i], j & 1, budget_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      {
+        uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+        uint32_t (&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+        tmem_ld32(s_addr, a);
+        tmem_ld32(s_addr + 32, b);
+        tmem_ld32(s_addr + 64, c);
+        tmem_ld32(s_addr + 96, d);
+        tmem_ld_wait();
+      }
+      if (valid < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+      }
+      float mx = __uint_as_float(sr[0]);
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
+      const float mt = mx * scale_log2;
+      if (mt > m_used + 8.f) {
+        // the running max grew by more than 2^8: rescale l and O
+        const float factor = fast_exp2(m_used - mt);  // 0 on the first tile
+        l *= factor;
+        if (j > 0) {
+          if (!mbar_wait(&o_done[i], (j - 1) & 1, budget_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < DH; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(o_addr + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(o_addr + c, o);
+          }
+        }
+        m_used = mt;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[32 * q + 2 * e]), scale_log2, -m_used));
+          const float p1 =
+              fast_exp2(fmaf(__uint_as_float(sr[32 * q + 2 * e + 1]), scale_log2, -m_used));
+          sum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_addr + 16 * q, pk);
+      }
+      l += sum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[i]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns)) {
+      tc_fence_after();
+      const int r = q0 + 128 * i + row;
+      const bool live = r < seg.q1;
+      const float inv = 1.f / l;
+      __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * DH;
+#pragma unroll 1
+      for (int c = 0; c < DH; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(o_addr + c, o);
+        tmem_ld_wait();
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + c + e) = u;
+          }
+        }
+      }
+      if (live && lse != nullptr)
+        lse[static_cast<int64_t>(h) * L + r] = (m_used + log2f(l)) * 0.69314718055994531f;
+    } else {
+      record_status(status, kStatusTimeout);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    mbar_wait(mma_done, 0, 200000000ull);
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- host schedule
+
+bool frame_visible(int tq, int tk, int T, int cf, int wc, unsigned anchors) {
+  if ((anchors & 1u) && (tq == 0 || tk == 0)) return true;
+  if ((anchors & 2u) && (tq == T - 1 || tk == T - 1)) return true;
+  const int cq = tq / cf, ck = tk / cf;
+  return (cq > ck ? cq - ck : ck - cq) <= wc;
+}
+
+// Visible key frames of query frame tq as maximal runs [a, b).
+std::vector<std::pair<int, int>> key_runs(int tq, int T, int cf, int wc, unsigned anchors) {
+  std::vector<std::pair<int, int>> runs;
+  int a = -1;
+  for (int tk = 0; tk <= T; ++tk) {
+    const bool v = tk < T && frame_visible(tq, tk, T, cf, wc, anchors);
+    if (v && a < 0) a = tk;
+    if (!v && a >= 0) {
+      runs.push_back({a, tk});
+      a = -1;
+    }
+  }
+  return runs;
+}
+
+bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSched* out) {
+  struct Raw {
+    int f0, f1;
+    std::vector<std::pair<int, int>> runs;
+    long work;
+  };
+  std::vector<Raw> raw;
+  for (int t = 0; t < s.T; ++t) {
+    auto runs = key_runs(t, s.T, cf, wc, anchors);
+    if (!raw.empty() && raw.back().runs == runs && raw.back().f1 == t) {
+      raw.back().f1 = t + 1;
+    } else {
+      raw.push_back({t, t + 1, runs, 0});
+    }
+  }
+  if (static_cast<int>(raw.size()) > kMaxSegs) return false;
+  for (auto& r : raw) {
+    if (r.runs.size() > 3) return false;
+    long keys = 0;
+    for (auto& p : r.runs) keys += static_cast<long>(p.second - p.first) * s.N;
+    r.work = keys;
+  }
+  std::stable_sort(raw.begin(), raw.end(), [](const Raw& a, const Raw& b) { return a.work > b.work; });
+  memset(out, 0, sizeof(*out));
+  out->nseg = static_cast<int>(raw.size());
+  int base = 0;
+  for (size_t k = 0; k < raw.size(); ++k) {
+    WinSeg& g = out->seg[k];
+    g.q0 = raw[k].f0 * s.N;
+    g.q1 = raw[k].f1 * s.N;
+    g.ntiles = (g.q1 - g.q0 + 255) / 256;
+    g.tile_base = base;
+    base += g.ntiles;
+    g.nint = static_cast<int>(raw[k].runs.size());
+    g.nkv = 0;
+    for (int v = 0; v < g.nint; ++v) {
+      g.k0[v] = raw[k].runs[v].first * s.N;
+      g.k1[v] = raw[k].runs[v].second * s.N;
+      g.nkv += (g.k1[v] - g.k0[v] + 127) / 128;
+    }
+  }
+  out->total_tiles = base;
+  return true;
+}
+
+template <int DH>
+cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                             const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             const WinSched& sched, float scale, void* o, int64_t ld_o,
+                             float* lse) {
+  using Cfg = WinCfg<DH>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(window_attn_kernel<DH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = sched.total_tiles * s.H;
+  window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, kmap, vmap, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
+      static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+size_t vdn_window_attn_workspace(const vdn_shape* shape) {
+  if (shape == nullptr || shape->T < 1 || shape->N < 1 || shape->H < 1 || shape->d < 1) return 0;
+  return kStatusBytes;
+}
+
+vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                           int64_t ld, int chunk_frames, int window_chunks, unsigned anchors,
+                           float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (shape == nullptr || shape->T < 1 || shape->N < 1 || shape->H < 1 || shape->d < 1)
+    return VDN_ERR_INVALID_ARG;
+  const vdn_shape s = *shape;
+  if (static_cast<int64_t>(s.T) * s.N >= (int64_t(1) << 31) - 512) return VDN_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return VDN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse_opt && (reinterpret_cast<uintptr_t>(lse_opt) & 3u)))
+    return VDN_ERR_INVALID_ARG;
+  if (chunk_frames < 1 || window_chunks < 0 || anchors > 3u) return VDN_ERR_INVALID_ARG;
+  if (s.d != 128 && s.d != 64) return VDN_ERR_UNSUPPORTED;
+  const int64_t D = static_cast<int64_t>(s.H) * s.d;
+  if (ld < D || ld % 8 || ld_o < D || ld_o % 8) return VDN_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kStatusBytes)
+    return VDN_ERR_WORKSPACE;
+  thread_local WinSched sched;  // ~12 KB; copied into the launch's parameters
+  if (!build_schedule(s, chunk_frames, window_chunks, anchors, &sched)) return VDN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(sched.total_tiles) * s.H >= (int64_t(1) << 31))
+    return VDN_ERR_UNSUPPORTED;
+  const int64_t L = static_cast<int64_t>(s.T) * s.N;
+  CUtensorMap qmap, kmap, vmap;
+  if (!make_rows_map(&qmap, q, D, ld, L, 128) || !make_rows_map(&kmap, k, D, ld, L, 128) ||
+      !make_rows_map(&vmap, v, D, ld, L, 128))
+    return VDN_ERR_CUDA;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(s.d));
+  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
+             current_wait_budget_ns()};
+  cudaError_t e = s.d == 128 ? launch_window_dh<128>(ctx, s, qmap, kmap, vmap, sched, sc, o, ld_o,
+                                                     lse_opt)
+                             : launch_window_dh<64>(ctx, s, qmap, kmap, vmap, sched, sc, o, ld_o,
+                                                    lse_opt);
+  return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+}  // extern "C"
