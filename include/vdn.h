@@ -144,7 +144,7 @@ VDN_API vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const 
  * gamma    : [D] fp32
  * ws       : >= vdn_hybrid_fuse_workspace(L, D) bytes (holds the gated
  *            branch outputs [L, 2D] bf16 between the two GEMMs)
- * D must be a multiple of 128; L >= 1.
+ * D must be a multiple of 256 and d = D/H a multiple of 32; L >= 1.
  * ------------------------------------------------------------------------ */
 VDN_API size_t vdn_hybrid_fuse_workspace(int L, int D);
 

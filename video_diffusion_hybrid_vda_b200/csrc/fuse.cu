@@ -1,0 +1,349 @@
+// Branch calibration and output projections ("Video DeltaNet", 10100.com
+// article, 方法概述 item 3: the Softmax branch gets a content-dependent
+// sigmoid gate, the linear branch RMSNorm and its own sigmoid output gate,
+// each branch its own output projection, and the two are added):
+//
+//   GEMM 1  G = x [W_gs; W_gl]^T                    (M = L, N = 2D, K = D)
+//           epilogue: Z[:, :D] = sigmoid(G[:, :D]) * o_s
+//                     Z[:, D:] = sigmoid(G[:, D:]) * RMSNorm_head(o_vda) * gamma
+//   GEMM 2  y = Z [W_os | W_ol]^T                   (M = L, N = D, K = 2D)
+//           (the sum of the two projections happens in the accumulator)
+//
+// One persistent tcgen05 GEMM kernel serves both: 128 x 256 output tiles,
+// TMA-fed 4-stage ring of [128 x 64] A and [256 x 64] B tiles (K-major,
+// 128B swizzle), one MMA-issuing thread, two 256-column TMEM accumulators so
+// the four epilogue warps drain tile i while the tensor core runs tile i+1.
+// Tiles are walked m-major (all N blocks of one M block in turn) so the A
+// rows are reused from L2 and the weights stay L2-resident.
+#include <math.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace vdn {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+constexpr int B_BYTES = BN * BK * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int GEMM_THREADS = 192;  // warp0 TMA, warp1 MMA, warps2-5 epilogue
+constexpr int GEMM_SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+
+enum class BSplit { kByN, kByK };
+
+struct GateArgs {
+  const __nv_bfloat16* o_s;
+  const __nv_bfloat16* o_vda;
+  const float* gamma;
+  float eps;
+  int D, d;
+  __nv_bfloat16* Z;  // [M, 2D]
+};
+
+struct StoreArgs {
+  __nv_bfloat16* y;  // [M, N]
+};
+
+__device__ __forceinline__ float sigmoidf_fast(float x) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-x * 1.4426950408889634f));
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
+  return r;
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* p, float (&f)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(q + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v = unpack_bf16x2(w[e]);
+      f[8 * i + 2 * e] = v.x;
+      f[8 * i + 2 * e + 1] = v.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float (&f)[32]) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    q[i] = make_uint4(pack_bf16x2(f[8 * i], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
+                      pack_bf16x2(f[8 * i + 4], f[8 * i + 5]),
+                      pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+}
+
+// Epilogue for GEMM 1 on one 32-column chunk of row r starting at column n.
+__device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
+                                           const uint32_t (&acc)[32], float& rinv) {
+  float z[32];
+  if (n < a.D) {
+    float os[32];
+    load_bf16x32(a.o_s + r * a.D + n, os);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) z[e] = sigmoidf_fast(__uint_as_float(acc[e])) * os[e];
+  } else {
+    const int c = n - a.D;
+    const __nv_bfloat16* orow = a.o_vda + r * a.D;
+    if (c % a.d == 0) {  // first chunk of a head: its RMS over d channels
+      float ss = 0.f;
+      for (int k = 0; k < a.d; k += 32) {
+        float f[32];
+        load_bf16x32(orow + c + k, f);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ss = fmaf(f[e], f[e], ss);
+      }
+      rinv = rsqrtf(ss / static_cast<float>(a.d) + a.eps);
+    }
+    float ov[32];
+    load_bf16x32(orow + c, ov);
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      z[e] = sigmoidf_fast(__uint_as_float(acc[e])) * (ov[e] * rinv * __ldg(a.gamma + c + e));
+  }
+  store_bf16x32(a.Z + r * (2 * static_cast<int64_t>(a.D)) + n, z);
+}
+
+template <BSplit SPLIT, class Args>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap b0map,
+                const __grid_constant__ CUtensorMap b1map, int M, int N, int K, int split_at,
+                Args args, uint32_t* status, uint64_t budget_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int mblocks = (M + BM - 1) / BM;
+  const int nblocks = (N + BN - 1) / BN;
+  const int ntiles = mblocks * nblocks;
+  const int nk = K / BK;
+  const uint32_t warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&b0map);
+    tma_prefetch_desc(&b1map);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int mb = tile / nblocks, nb = tile % nblocks;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(&empty[s], ((it / STAGES) & 1) ^ 1, budget_ns)) {
+            record_status(status, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_2d(sa, &amap, &full[s], kb * BK, mb * BM);
+          int brow = nb * BN, bcol = kb * BK;
+          const CUtensorMap* bm = &b0map;
+          if (SPLIT == BSplit::kByN && brow >= split_at) {
+            bm = &b1map;
+            brow -= split_at;
+          }
+          if (SPLIT == BSplit::kByK && bcol >= split_at) {
+            bm = &b1map;
+            bcol -= split_at;
+          }
+          tma_load_2d(sa + A_BYTES, bm, &full[s], bcol, brow);
+        }
+      }
+      // drain the last loads
+      const uint32_t first = it > STAGES ? it - STAGES : 0;
+      for (uint32_t j = first; j < it; ++j)
+        if (!mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 200000000ull))
+          record_status(status, kStatusTimeout);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_bf16(BM, BN, false, false);
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+        const int b = lt & 1;
+        if (lt >= 2 && !mbar_wait(&tempty[b], ((lt >> 1) & 1) ^ 1, budget_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc_addr = tmem + b * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1, budget_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_ss(acc_addr, sdesc_sw128(sa + kk * 32, 16, 1024),
+                    sdesc_sw128(sa + A_BYTES + kk * 32, 16, 1024), idesc, (kb | kk) != 0);
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[b]);
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+      umma_commit(mma_done);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane_id();
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      if (!mbar_wait(&tfull[b], (lt >> 1) & 1, budget_ns)) {
+        record_status(status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int mb = tile / nblocks, nb = tile % nblocks;
+      const int64_t r = static_cast<int64_t>(mb) * BM + row;
+      const uint32_t taddr = tmem + b * BN + ((quarter * 32) << 16);
+      float rinv = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t acc[32];
+        tmem_ld32(taddr + c, acc);
+        tmem_ld_wait();
+        const int n = nb * BN + c;
+        if (r < M && n < N) {
+          if constexpr (SPLIT == BSplit::kByN) {
+            gate_chunk(args, r, n, acc, rinv);
+          } else {
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(acc[e]);
+            store_bf16x32(args.y + r * N + n, f);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    mbar_wait(mma_done, 0, 200000000ull);
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <BSplit SPLIT, class Args>
+cudaError_t launch_gemm(const Launch& ctx, const CUtensorMap& a, const CUtensorMap& b0,
+                        const CUtensorMap& b1, int M, int N, int K, int split_at, const Args& args,
+                        int sm_count) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<SPLIT, Args>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int ntiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = ntiles < sm_count ? ntiles : sm_count;
+  gemm_kernel<SPLIT, Args><<<grid, GEMM_THREADS, GEMM_SMEM, ctx.stream>>>(
+      a, b0, b1, M, N, K, split_at, args, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sm_count_of_current_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
+}  // namespace
+}  // namespace vdn
+
+using namespace vdn;
+
+extern "C" {
+
+size_t vdn_hybrid_fuse_workspace(int L, int D) {
+  if (L < 1 || D < 1) return 0;
+  return kStatusBytes + static_cast<size_t>(L) * 2 * static_cast<size_t>(D) * 2;
+}
+
+vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
+                           const void* o_vda, const void* W_gs, const void* W_gl,
+                           const float* gamma, float eps, const void* W_os, const void* W_ol,
+                           void* y, void* ws, size_t ws_bytes, void* stream) {
+  if (L < 1 || D < 1 || H < 1 || D % H != 0) return VDN_ERR_INVALID_ARG;
+  if (!x || !o_s || !o_vda || !W_gs || !W_gl || !gamma || !W_os || !W_ol || !y)
+    return VDN_ERR_INVALID_ARG;
+  if (!a16(x) || !a16(o_s) || !a16(o_vda) || !a16(W_gs) || !a16(W_gl) || !a16(W_os) ||
+      !a16(W_ol) || !a16(y) || (reinterpret_cast<uintptr_t>(gamma) & 3u))
+    return VDN_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return VDN_ERR_INVALID_ARG;
+  const int d = D / H;
+  if (D % 256 != 0 || d % 32 != 0) return VDN_ERR_UNSUPPORTED;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      ws_bytes < vdn_hybrid_fuse_workspace(L, D))
+    return VDN_ERR_WORKSPACE;
+  __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+
+  CUtensorMap xmap, wgs, wgl, zmap, wos, wol;
+  if (!make_rows_map(&xmap, x, D, D, L, BM) || !make_rows_map(&wgs, W_gs, D, D, D, BN) ||
+      !make_rows_map(&wgl, W_gl, D, D, D, BN) || !make_rows_map(&zmap, Z, 2 * D, 2 * D, L, BM) ||
+      !make_rows_map(&wos, W_os, D, D, D, BN) || !make_rows_map(&wol, W_ol, D, D, D, BN))
+    return VDN_ERR_CUDA;
+
+  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
+             current_wait_budget_ns()};
+  const int sms = sm_count_of_current_device();
+  GateArgs g{static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_vda),
+             gamma, eps, D, d, Z};
+  if (launch_gemm<BSplit::kByN>(ctx, xmap, wgs, wgl, L, 2 * D, D, D, g, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  StoreArgs st{static_cast<__nv_bfloat16*>(y)};
+  if (launch_gemm<BSplit::kByK>(ctx, zmap, wos, wol, L, D, 2 * D, D, st, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+}  // extern "C"

@@ -206,14 +206,3 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
 }
 
 }  // extern "C"
-// ----------------------------------------------------------------- pending
-extern "C" {
-size_t vdn_hybrid_fuse_workspace(int L, int D) {
-  return kStatusBytes + static_cast<size_t>(L) * 2 * D * 2;
-}
-vdn_status vdn_hybrid_fuse(int, int, int, const void*, const void*, const void*, const void*,
-                           const void*, const float*, float, const void*, const void*, void*,
-                           void*, size_t, void*) {
-  return VDN_ERR_UNSUPPORTED;
-}
-}
