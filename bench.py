@@ -1,0 +1,354 @@
+"""Benchmark of the Video DeltaNet hybrid attention layer on B200.
+
+One step = one pass of the whole layer (window-and-anchor Softmax, Video
+Delta Attention prep/solve/scan/read-out, gated fuse with both output
+projections) over one video's synthetic inputs at 102 latent frames x 4032
+tokens (48x84), 24 heads x 128, bf16, seeded.  Inputs live in HBM when the
+timed region starts; each activation (2.5 GB) is larger than L2, so no L2
+flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload layer102|layer42|small]
+
+With N > 1 (torchrun) every rank runs its own video (independent problems,
+no collective on the data path): weak scaling, time = max over ranks.
+``--impl reference`` times the float64 CPU oracle instead, on a bounded
+sample of the same workload, extrapolated by work.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from video_diffusion_hybrid_vda_b200 import synth  # noqa: E402
+
+WORKLOADS = {
+    "layer102": synth.Shape(102, 4032, 24, 128),
+    "layer42": synth.Shape(42, 4032, 24, 128),
+    "small": synth.Shape(12, 4032, 24, 128),   # for ncu captures: ~2 GB on the device
+}
+METRIC = "VDN hybrid attn layer ms & tokens/s at 102 latent frames; % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "window_attn_traffic.json")
+
+
+def mask_pair_count(T, cf=5, wc=1, anchors=3):
+    """Visible (query frame, key frame) pairs of the window-and-anchor mask."""
+    n = 0
+    for tq in range(T):
+        for tk in range(T):
+            if (anchors & 1 and 0 in (tq, tk)) or (anchors & 2 and T - 1 in (tq, tk)) or \
+                    abs(tq // cf - tk // cf) <= wc:
+                n += 1
+    return n
+
+
+def work_model(s):
+    """Algorithmic work of one layer pass (unmasked pairs only)."""
+    pairs = mask_pair_count(s.T) * s.N * s.N          # token pairs per head
+    softmax_flop = pairs * s.H * 4 * s.d                # QK^T and PV
+    proj_flop = 4 * 2 * s.L * s.D * s.D                 # gate GEMMs + output GEMMs
+    # VDA HBM bytes: prep reads k, v (bf16) and beta; read-out reads q, writes o
+    vda_bytes = 2 * s.L * s.D * 2 + s.L * s.H * 4 + 2 * s.L * s.D * 2
+    # FP32 ALU work of the solve (~3 d^3) and the scan (2 x 2 d^3 per frame)
+    vda_alu_flop = s.T * s.H * (3 * s.d ** 3 + 4 * s.d ** 3) * 2
+    return dict(pairs=pairs, softmax_flop=softmax_flop, proj_flop=proj_flop,
+                vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def clocks_start():
+    fd, path = tempfile.mkstemp(suffix=".csv")
+    os.close(fd)
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    dev = os.environ.get("LOCAL_RANK", "0")
+    try:
+        p = subprocess.Popen(["nvidia-smi", f"--id={dev}", f"--query-gpu={q}",
+                              "--format=csv,noheader,nounits", "-lms", "200"],
+                             stdout=open(path, "w"), stderr=subprocess.DEVNULL)
+    except OSError:
+        p = None
+    return p, path
+
+
+def clocks_stop(handle):
+    p, path = handle
+    if p is None:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    p.terminate()
+    try:
+        p.wait(timeout=5)
+    except subprocess.TimeoutExpired:
+        p.kill()
+    sm, smax, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    with open(path) as f:
+        for line in f:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+    os.unlink(path)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(shape, seed=0, vda_heads=2, frames=None, rows_per_frame=128):
+    """Time the float64 oracle on a bounded sample of the layer and
+    extrapolate to one full layer pass by the work ratio of each step.
+
+    Sample: VDA (prep, solve, both scans, read-out) for `vda_heads` heads over
+    all frames; window Softmax for `rows_per_frame` query rows of each
+    sampled frame (default {0, 1, 4, 5, T/2, T-3, T-2, T-1}) in one head;
+    fuse for 256 rows.  Inputs are drawn on the host with the same laws.
+    """
+    import oracle
+    from threadpoolctl import threadpool_info
+    T, N, H, d = shape.T, shape.N, shape.H, shape.d
+    L, D = shape.L, shape.D
+    sub = synth.Shape(T, N, vda_heads, d)
+    x = {k: v.numpy() for k, v in synth.make_inputs(sub, dtype=torch.float32, seed=seed).items()}
+    t0 = time.perf_counter()
+    oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], T, N, vda_heads, d)
+    t_vda = (time.perf_counter() - t0) * H / vda_heads
+
+    if frames is None:
+        frames = [0, 1, 4, 5, T // 2, T - 3, T - 2, T - 1]
+    frames = sorted(set(frames))
+    rows = np.concatenate([np.arange(f * N, f * N + min(rows_per_frame, N)) for f in frames])
+    c = slice(0, d)
+    t0 = time.perf_counter()
+    oracle.window_attn_rows(x["q"][:, c], x["k"][:, c], x["v"][:, c], T, N, 1, d, rows)
+    t_win_s = time.perf_counter() - t0
+    sampled_pairs = sum(len(oracle.visible_key_frames(int(r) // N, T)) * N for r in rows)
+    t_win = t_win_s * (mask_pair_count(T) * N * N * H) / sampled_pairs
+
+    g = torch.Generator().manual_seed(seed + 7)
+    nr = 256
+    xr = torch.randn((nr, D), generator=g).numpy()
+    o_s = torch.randn((nr, D), generator=g).numpy()
+    o_l = torch.randn((nr, D), generator=g).numpy()
+    W = [(0.02 * torch.randn((D, D), generator=g)).numpy() for _ in range(4)]
+    t0 = time.perf_counter()
+    oracle.hybrid_fuse_rows(xr, o_s, o_l, W[0], W[1], np.ones(D), 1e-6, W[2], W[3], H,
+                            np.arange(nr))
+    t_fuse = (time.perf_counter() - t0) * L / nr
+    total = t_vda + t_win + t_fuse
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {
+        "value": L / total, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+        "sample": ("float64 numpy oracle, extrapolated by work: VDA %d of %d heads x %d frames "
+                   "(%.1f s), window Softmax %d query rows of frames %s x 1 head (%.1f s), "
+                   "fuse %d rows (%.1f s); full layer est. %.0f s"
+                   % (vda_heads, H, T, t_vda * vda_heads / H, len(rows), frames, t_win_s, nr,
+                      t_fuse * nr / L, total)),
+        "seconds_per_layer": total,
+    }
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args, shape, rank, world):
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev, with_fuse=True)
+    layer = vdn.HybridLayer(shape.T, shape.N, shape.H, shape.d, inp["W_gs"], inp["W_gl"],
+                            inp["W_os"], inp["W_ol"], inp["gamma"], device=dev)
+    acts = [inp[k] for k in ("q", "k", "v", "beta", "alpha", "x")]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(timed_win=None):
+        q, k, v, beta, alpha, x = acts
+        cf, wc, an = layer.mask
+        if timed_win is not None:
+            timed_win[0].record(stream)
+        vdn.window_attn(q, k, v, shape.T, shape.N, shape.H, shape.d, cf, wc, an,
+                        out=layer.o_s, ws=layer.ws_win, stream=stream)
+        if timed_win is not None:
+            timed_win[1].record(stream)
+        vdn.vda_scan(q, k, v, beta, alpha, shape.T, shape.N, shape.H, shape.d,
+                     out=layer.o_vda, ws=layer.ws_vda, stream=stream)
+        vdn.hybrid_fuse(x, layer.o_s, layer.o_vda, layer.W_gs, layer.W_gl, layer.gamma,
+                        layer.W_os, layer.W_ol, shape.H, out=layer.y, ws=layer.ws_fuse,
+                        stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if layer.status() != 0:
+        raise RuntimeError("device status after warm-up: %d" % layer.status())
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    win_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = clocks_start()
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        step(win_events[i])
+    end.record(stream)
+    barrier()
+    clocks = clocks_stop(clk)
+    ms = start.elapsed_time(end)
+    win_ms = [a.elapsed_time(b) for a, b in win_events]
+    status = layer.status()
+    if status != 0:
+        raise RuntimeError("device status after timed steps: %d" % status)
+
+    # ---- end to end: pinned host inputs copied in and y copied out every step
+    host_in = [t.to("cpu").pin_memory() for t in acts]
+    host_out = torch.empty((shape.L, shape.D), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+    e2e_steps = max(1, min(args.steps, 3))
+    layer.forward(*host_in, out=host_out, stream=stream)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        layer.forward(*host_in, out=host_out, stream=stream)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if layer.status() != 0:
+        raise RuntimeError("device status after end-to-end steps")
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms, sum(win_ms)], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms, win_total = t.tolist()
+    else:
+        win_total = sum(win_ms)
+    return dict(ms=ms, win_ms=win_total / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                clocks=clocks, launches=layer.KERNELS_PER_FORWARD * args.steps)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="vdn", choices=["vdn", "reference"])
+    ap.add_argument("--workload", default="layer102", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    shape = WORKLOADS[args.workload]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    work = work_model(shape)
+    config = {"workload": f"hybrid_layer_T{shape.T}_N{shape.N}_H{shape.H}_d{shape.d}",
+              "latent_frames": shape.T, "tokens_per_frame": shape.N, "grid": "48x84",
+              "heads": shape.H, "head_dim": shape.d, "hidden": shape.D, "tokens": shape.L,
+              "mask": "chunk 5, +-1 chunk, first/last-frame anchors",
+              "global_batch": world, "parallelism": f"independent videos x{world}",
+              "l2": "inputs larger than L2 (2.5 GB per activation), no flush"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        # each step: a smaller bounded sample (1 VDA head, 4 sampled frames)
+        small = dict(vda_heads=1, frames=[0, 5, shape.T // 2, shape.T - 1])
+        for i in range(args.warmup):
+            oracle_sample(shape, seed=100 + i, **small)
+        runs = [oracle_sample(shape, seed=i, **small) for i in range(args.steps)]
+        secs = statistics.median(r["seconds_per_layer"] for r in runs)
+        cpu = dict(runs[0])
+        cpu["value"] = shape.L / secs
+        cpu["sample"] = ("median of %d steps, each: " % args.steps) + cpu["sample"]
+        line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": secs * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                "e2e": {"value": cpu["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        torch.distributed.init_process_group(
+            "nccl", device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
+            timeout=__import__("datetime").timedelta(seconds=300))
+    r = run_gpu(args, shape, rank, world)
+    peaks, peak_kind = load_peaks()
+    ms_step = r["ms"] / args.steps
+    tokens_per_s = world * shape.L / (ms_step / 1e3)
+    win_tflops = work["softmax_flop"] / (r["win_ms"] / 1e3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = None
+    if os.path.exists(KERNEL_TRAFFIC_FILE):
+        with open(KERNEL_TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        if tr.get("workload") == config["workload"]:
+            traffic = tr.get("bytes_per_launch")
+    # layer roofline: sum over steps of the binding resource at the measured peaks
+    roof_ms = (work["softmax_flop"] / (peak * 1e12) + work["proj_flop"] / (peak * 1e12) +
+               work["vda_bytes"] / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; q,k,v,x ~ N(0,1), k L2-normalised, beta = sigmoid(N), "
+                "alpha ~ U(0.9,1), weights ~ N(0,0.02))",
+        "config": config,
+        "roofline": {"bound": "tensor", "achieved": win_tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": win_tflops / peak, "traffic": traffic,
+                     "kernel": "window_attn_kernel<128> (window-and-anchor Softmax)",
+                     "peak_source": f"{peak_kind} bf16_tflops_sustained",
+                     "flop_per_launch": work["softmax_flop"], "ms_per_launch": r["win_ms"]},
+        "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step,
+                           "terms": "softmax + projections at sustained bf16 peak, VDA bytes "
+                                    "at measured HBM"},
+        "e2e": {"value": world * shape.L / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": r["e2e_ms"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(shape)
+        line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

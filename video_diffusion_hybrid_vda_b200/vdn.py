@@ -221,3 +221,68 @@ def hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, H, eps=1e-6, out=N
                                  _ptr(W_ol), _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
     _check(code, "vdn_hybrid_fuse")
     return out, ws
+
+
+# ---------------------------------------------------------------- full layer
+
+class HybridLayer:
+    """The video-to-video hybrid attention layer on one GPU.
+
+    forward() runs window-and-anchor Softmax, Video Delta Attention and the
+    gated fuse (three C-ABI calls, seven kernels) and returns y [T*N, D].
+    Inputs may be CUDA tensors, or host tensors (pinned for asynchronous
+    copies): host inputs are copied into device buffers owned by the layer
+    and, when ``out`` is a host tensor, y is copied back into it.
+    """
+
+    KERNELS_PER_FORWARD = 7   # prep, solve, scan, read-out, window Softmax, 2 GEMMs
+
+    def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, chunk_frames=5,
+                 window_chunks=1, anchors=3, device=None):
+        self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
+        self.L, self.D = self.T * self.N, self.H * self.d
+        self.device = torch.device(device or "cuda")
+        dev = self.device
+        self.W_gs, self.W_gl, self.W_os, self.W_ol = (
+            w.to(dev, torch.bfloat16).contiguous() for w in (W_gs, W_gl, W_os, W_ol))
+        self.gamma = gamma.to(dev, torch.float32).contiguous()
+        self.eps = float(eps)
+        self.mask = (int(chunk_frames), int(window_chunks), int(anchors))
+        L, D = self.L, self.D
+        self.o_s = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
+        self.o_vda = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
+        self.ws_vda = alloc_workspace(vda_scan_workspace(T, N, H, d), dev)
+        self.ws_win = alloc_workspace(window_attn_workspace(T, N, H, d), dev)
+        self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D), dev)
+        self._staging = None
+
+    def _to_device(self, tensors, stream):
+        if all(t.is_cuda for t in tensors):
+            return tensors
+        if self._staging is None:
+            self._staging = [torch.empty(t.shape, dtype=t.dtype, device=self.device)
+                             for t in tensors]
+        with torch.cuda.stream(stream):
+            for dst, src in zip(self._staging, tensors):
+                dst.copy_(src, non_blocking=True)
+        return self._staging
+
+    def forward(self, q, k, v, beta, alpha, x, out=None, stream=None):
+        stream = stream or torch.cuda.current_stream(self.device)
+        q, k, v, beta, alpha, x = self._to_device([q, k, v, beta, alpha, x], stream)
+        T, N, H, d = self.T, self.N, self.H, self.d
+        cf, wc, an = self.mask
+        window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win, stream=stream)
+        vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda, stream=stream)
+        hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
+                    self.W_ol, H, eps=self.eps, out=self.y, ws=self.ws_fuse, stream=stream)
+        if out is not None and not out.is_cuda:
+            with torch.cuda.stream(stream):
+                out.copy_(self.y, non_blocking=True)
+            return out
+        return self.y
+
+    def status(self):
+        """Worst device status over the layer's workspaces (synchronises)."""
+        return max(get_device_status(w) for w in (self.ws_vda, self.ws_win, self.ws_fuse))
