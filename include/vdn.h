@@ -108,6 +108,34 @@ VDN_API vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const voi
 VDN_API vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
                                  float** P, float** C);
 
+/* vdn_vda_scan without a workspace.  The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory (for
+ * example a plugin inside a host framework that owns every device
+ * allocation, or a loop with a fixed memory budget where cudaMalloc is not
+ * allowed).  It computes exactly what vdn_vda_scan computes, with the same
+ * arguments minus ws/ws_bytes, and allocates nothing: its scratch is a
+ * fixed 64 MiB array of this library's own device memory, present on every
+ * GPU that loads the library until the process exits.
+ *  - Limit: 256 + 6 * T*H*d*d*4 bytes must fit in 64 MiB (e.g. T*H <= 170
+ *    at d = 128, <= 680 at d = 64); larger shapes return VDN_ERR_WORKSPACE
+ *    before anything is enqueued.
+ *  - The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call shares the one array: calls that overlap on the GPU (other
+ *    streams, other host threads) race and corrupt each other's results.
+ *    The array keeps the last call's contents; each call clears the status
+ *    word it uses and overwrites everything else it reads.
+ *  - dev_status_opt: NULL, or device memory that receives, as the call's
+ *    last operation on `stream`, this call's device status bits
+ *    (0 = ok, bit 0 = numeric failure, bit 1 = a wait ran out of time).
+ * No cudaMalloc, cudaFree or allocating library routine is called. */
+VDN_API vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q, const void* k,
+                                       const void* v, int64_t ld, const float* beta,
+                                       const float* alpha, void* o_vda, int64_t ld_o,
+                                       float* states_opt, unsigned* dev_status_opt,
+                                       void* stream);
+
 /* ------------------------------------------------------------------------
  * Window-and-anchor Softmax (10100.com article, 方法概述 item 1).
  *

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
 EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_window_attn_workspace", "vdn_window_attn", "vdn_hybrid_fuse_workspace",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
-           "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version"]
+           "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
+           "vdn_vda_scan_static"]
 
 
 class VdnError(RuntimeError):
