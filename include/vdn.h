@@ -12,7 +12,7 @@
  *      state is S_t = (S_bar_t + B_t)(I + A_t)^-1 with S_bar_t = alpha_t S_{t-1},
  *      A_t = sum_i beta_i k_i k_i^T, B_t = sum_i beta_i v_i k_i^T over the
  *      tokens of frame t, run forward and backward over the frames (figure
- *      caption under 效率阶梯, 前向加反向扫描);         -> vdn_vda_scan
+ *      caption under 效率阶梯: forward and backward scans);         -> vdn_vda_scan
  *   3. branch calibration (方法概述 item 3): content-dependent sigmoid gate on
  *      the Softmax branch, RMSNorm then a sigmoid output gate on the linear
  *      branch, a separate output projection per branch, summed.

@@ -13,8 +13,8 @@ pages' description of the method:
                       form S_t = (S_bar_t + B_t)(I + A_t)^-1, run forward and
                       backward over the latent frames).  Source: "Video
                       DeltaNet" article on 10100.com, section 方法概述 item 2
-                      (帧级delta rule), figure caption under 效率阶梯
-                      (前向加反向扫描).
+                      (frame-level delta rule), figure caption under
+                      效率阶梯 (forward and backward scans).
 * ``window_attn``  -- sliding-window Softmax over 5-frame chunks (+-1 chunk)
                       with first/last-frame anchors.  Source: same article,
                       方法概述 item 1 (Sliding-Window Softmax + Boundary

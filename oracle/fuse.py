@@ -1,6 +1,6 @@
 """Branch calibration and output projections, float64 CPU oracle.  TEST INFRASTRUCTURE ONLY.
 
-Source: "Video DeltaNet" article on 10100.com, 方法概述 item 3 (分支校准):
+Source: "Video DeltaNet" article on 10100.com, 方法概述 item 3 (branch calibration):
 the Softmax branch gets a content-dependent sigmoid gate; the linear branch
 is RMS-normalised and then passes its own sigmoid output gate; each branch
 has its own output projection and the two projections are added.  The

@@ -1,7 +1,7 @@
 """Video Delta Attention (VDA), float64 CPU oracle.  TEST INFRASTRUCTURE ONLY.
 
-Source: "Video DeltaNet" article on 10100.com, 方法概述 item 2 (帧级delta
-rule).  The state of latent frame t is the minimiser of a joint objective:
+Source: "Video DeltaNet" article on 10100.com, 方法概述 item 2 (frame-level
+delta rule).  The state of latent frame t is the minimiser of a joint objective:
 stay close to the decayed previous state S_bar_t, and fit every key-value
 association of frame t at once.  With unit weights on both terms,
 
