@@ -68,6 +68,24 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Blackwell packed fp32x2 arithmetic: two lanes in one 64-bit register
+// (low word = first element).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+
+__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint64_t fadd_f32x2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
@@ -123,9 +141,11 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   // ---- which segment / tile / head
+  // head-major launch order: the CTAs resident at any time mostly share one
+  // head, so the K/V rows they stream stay in L2 across query tiles
   const int lin = blockIdx.x;
-  const int h = lin % H;
-  const int tile = lin / H;
+  const int h = lin / sched.total_tiles;
+  const int tile = lin % sched.total_tiles;
   int si = 0;
   while (si + 1 < sched.nseg && tile >= sched.seg[si + 1].tile_base) ++si;
   const WinSeg& seg = sched.seg[si];
@@ -159,6 +179,12 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // Register split (launched with 168 x 384 = 64512): the TMA/MMA warpgroup
+  // drops to 56, the two softmax warpgroups rise to 200
+  // (128 * 56 + 256 * 200 = 58368 <= 64512).
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+  }
   if (warp == 0) {
     // ================================================================ TMA
     if (elect_one()) {
@@ -247,6 +273,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     }
   } else if (warp >= 4) {
     // ================================================================ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
     const int i = (warp - 4) >> 2;  // query tile of this warpgroup
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane_id();
@@ -283,10 +310,17 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(sr[0]);
+      // row max as 8 independent chains, then a short tree
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(sr[c]));
-      const float mt = mx * scale_log2;
+      for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+#pragma unroll
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) mx8[c] = fmaxf(mx8[c], mx8[c + w]);
+      const float mt = mx8[0] * scale_log2;
       if (mt > m_used + 8.f) {
         // the running max grew by more than 2^8: rescale l and O
         const float factor = fast_exp2(m_used - mt);  // 0 on the first tile
@@ -309,21 +343,29 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         }
         m_used = mt;
       }
-      float sum = 0.f;
+      // p = 2^(s * scale_log2 - m): packed f32x2 FMA for the argument, four
+      // independent packed partial sums
+      const uint64_t cc = pack_f32x2(scale_log2, scale_log2);
+      const uint64_t nm = pack_f32x2(-m_used, -m_used);
+      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[32 * q + 2 * e]), scale_log2, -m_used));
-          const float p1 =
-              fast_exp2(fmaf(__uint_as_float(sr[32 * q + 2 * e + 1]), scale_log2, -m_used));
-          sum += p0 + p1;
+          const uint64_t xs = ffma_f32x2(
+              (static_cast<uint64_t>(sr[32 * q + 2 * e + 1]) << 32) | sr[32 * q + 2 * e], cc, nm);
+          const float p0 = fast_exp2(__uint_as_float(static_cast<uint32_t>(xs)));
+          const float p1 = fast_exp2(__uint_as_float(static_cast<uint32_t>(xs >> 32)));
+          const uint64_t pp = pack_f32x2(p0, p1);
+          acc2[e & 3] = fadd_f32x2(acc2[e & 3], pp);
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(s_addr + 16 * q, pk);
       }
-      l += sum;
+      acc2[0] = fadd_f32x2(fadd_f32x2(acc2[0], acc2[1]), fadd_f32x2(acc2[2], acc2[3]));
+      l += __uint_as_float(static_cast<uint32_t>(acc2[0])) +
+           __uint_as_float(static_cast<uint32_t>(acc2[0] >> 32));
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[i]);
