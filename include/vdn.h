@@ -201,6 +201,14 @@ VDN_API vdn_status vdn_reset_device_status(void* ws, void* stream);
  * path.  Process-wide; not thread-safe against concurrent launches. */
 VDN_API void vdn_set_wait_budget_ns(uint64_t ns);
 
+/* Diagnostic: y_fma[i] = 2^x[i] by the FMA-pipe exponential the Softmax uses
+ * for part of its scores (range reduction x = n + f, cubic for 2^f, 2^n added
+ * to the exponent; inputs below -125 are clamped there), and y_mufu[i] =
+ * 2^x[i] by the hardware ex2.approx.  Device pointers, n >= 0 floats;
+ * enqueued on `stream`. */
+VDN_API vdn_status vdn_selftest_exp2(const float* x, float* y_fma, float* y_mufu, int n,
+                                     void* stream);
+
 /* Library version string. */
 VDN_API const char* vdn_version(void);
 

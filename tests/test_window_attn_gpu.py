@@ -120,3 +120,22 @@ def test_window_attn_full_layer_sampled(vdn, T):
         assert np.abs(lse_s[h] - lse_ref[0]).max() <= TOL_LSE, h
     del inp, o, lse
     torch.cuda.empty_cache()
+
+
+def test_fma_pipe_exp2_error_bound(vdn):
+    """The FMA-pipe exponential stays within 1e-4 relative of exact 2^x and of
+    the MUFU ex2.approx over the range the Softmax feeds it (x <= 8), and
+    clamps far-negative inputs to a tiny non-negative value."""
+    xs = np.concatenate([np.linspace(-124.0, 8.0, 400001), np.arange(-40, 9, 0.5),
+                         [0.0, -0.5, 0.5, -1e-7, 7.999]]).astype(np.float32)
+    x = torch.as_tensor(xs, device="cuda")
+    y_fma, y_mufu = vdn.selftest_exp2(x)
+    torch.cuda.synchronize()
+    ref = np.exp2(xs.astype(np.float64))
+    yf, ym = host(y_fma).astype(np.float64), host(y_mufu).astype(np.float64)
+    assert np.max(np.abs(yf / ref - 1.0)) <= 1e-4
+    assert np.max(np.abs(yf / ym - 1.0)) <= 1e-4
+    far = torch.tensor([-200.0, -1000.0, -float("inf")], device="cuda")
+    yfar, _ = vdn.selftest_exp2(far)
+    v = host(yfar)
+    assert np.all(v >= 0) and np.all(v < 1e-37)

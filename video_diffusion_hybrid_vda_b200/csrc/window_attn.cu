@@ -30,6 +30,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "exp2_fma.cuh"
 #include "ptx.cuh"
 
 namespace vdn {
@@ -62,30 +63,6 @@ struct WinCfg {
   static constexpr int SMEM = 1024 + 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 512;
 };
 
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// Blackwell packed fp32x2 arithmetic: two lanes in one 64-bit register
-// (low word = first element).
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-  return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
-}
-
-__device__ __forceinline__ uint64_t ffma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-
-__device__ __forceinline__ uint64_t fadd_f32x2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
@@ -99,21 +76,51 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-// Key tile `j` of a segment: start row and number of valid keys.
-struct KvCursor {
-  int iv, pos;
-  __device__ void init(const WinSeg& s) {
-    iv = 0;
-    pos = s.k0[0];
+// Compiler-level fence: uses of r cannot be scheduled before this point
+// (placed right after tcgen05.wait::ld, which makes the loaded values valid).
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]));
+}
+
+// The key intervals of one segment, held in registers, and a cursor over
+// its 128-key tiles (start row, number of valid keys).
+struct KvRange {
+  int nint, a0, a1, a2, b0, b1, b2;
+  __device__ void load(const WinSeg& s) {
+    nint = s.nint;
+    a0 = s.k0[0];
+    a1 = s.k0[1];
+    a2 = s.k0[2];
+    b0 = s.k1[0];
+    b1 = s.k1[1];
+    b2 = s.k1[2];
   }
-  __device__ void next(const WinSeg& s) {
+  __device__ int start(int iv) const { return iv == 0 ? a0 : (iv == 1 ? a1 : a2); }
+  __device__ int end(int iv) const { return iv == 0 ? b0 : (iv == 1 ? b1 : b2); }
+};
+
+struct KvCursor {
+  int iv, pos, end;
+  __device__ void init(const KvRange& r) {
+    iv = 0;
+    pos = r.a0;
+    end = r.b0;
+  }
+  __device__ void next(const KvRange& r) {
     pos += 128;
-    if (pos >= s.k1[iv] && iv + 1 < s.nint) {
+    if (pos >= end && iv + 1 < r.nint) {
       ++iv;
-      pos = s.k0[iv];
+      pos = r.start(iv);
+      end = r.end(iv);
     }
   }
-  __device__ int valid(const WinSeg& s) const { return min(128, s.k1[iv] - pos); }
+  __device__ int valid() const { return min(128, end - pos); }
 };
 
 template <int DH>
@@ -135,7 +142,8 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   uint64_t* kv_full = bars + 1;                      // [STAGES]
   uint64_t* kv_empty = kv_full + Cfg::STAGES;        // [STAGES]
   uint64_t* s_full = kv_empty + Cfg::STAGES;         // [2]
-  uint64_t* p_ready = s_full + 2;                    // [2]
+  uint64_t* p_half = s_full + 2;                     // [2] P for keys 0..63 stored
+  uint64_t* p_ready = p_half + 2;                    // [2] all of P stored
   uint64_t* o_done = p_ready + 2;                    // [2]
   uint64_t* mma_done = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -150,7 +158,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   while (si + 1 < sched.nseg && tile >= sched.seg[si + 1].tile_base) ++si;
   const WinSeg& seg = sched.seg[si];
   const int q0 = seg.q0 + (tile - seg.tile_base) * 256;
+  const int q_end = seg.q1;
   const int nkv = seg.nkv;
+  KvRange kr;
+  kr.load(seg);
   const uint32_t warp = warp_id();
 
   if (threadIdx.x == 0) {
@@ -161,6 +172,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_half[i], 128);
       mbar_init(&p_ready[i], 128);
       mbar_init(&o_done[i], 1);
     }
@@ -180,10 +192,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   // Register split (launched with 168 x 384 = 64512): the TMA/MMA warpgroup
-  // drops to 56, the two softmax warpgroups rise to 200
-  // (128 * 56 + 256 * 200 = 58368 <= 64512).
+  // drops to 96, the two softmax warpgroups rise to 200
+  // (128 * 96 + 256 * 200 = 63488 <= 64512).
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;\n" ::: "memory");
   }
   if (warp == 0) {
     // ================================================================ TMA
@@ -194,7 +206,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
           tma_load_2d(qbuf + i * Cfg::TILE_BYTES + sl * 16384, &qmap, q_full, h * DH + 64 * sl,
                       q0 + 128 * i);
       KvCursor cur;
-      cur.init(seg);
+      cur.init(kr);
       int issued = 0;
       for (int j = 0; j < nkv; ++j) {
         const int s = j % Cfg::STAGES;
@@ -211,7 +223,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
                       cur.pos);
         }
         ++issued;
-        cur.next(seg);
+        cur.next(kr);
       }
       // drain loads still in flight
       mbar_wait(q_full, 0, 200000000ull);
@@ -236,14 +248,13 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         }
         umma_commit(&s_full[i]);
       };
-      auto issue_o = [&](int i, int j) {
+      // O_i += P_i V for keys [16 k0, 16 k1) of the tile
+      auto issue_o = [&](int i, int j, int k0, int k1) {
         const uint32_t vb =
             smem_u32(kvbuf + (j % Cfg::STAGES) * 2 * Cfg::TILE_BYTES + Cfg::TILE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 128 keys, 16 per step
+        for (int kk = k0; kk < k1; ++kk)
           umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8,
                   sdesc_sw128(vb + kk * 2048, 16384, 1024), idesc_o, (j > 0 || kk > 0));
-        umma_commit(&o_done[i]);
       };
       if (ok && (ok = mbar_wait(&kv_full[0], 0, budget_ns))) {
         tc_fence_after();
@@ -253,18 +264,26 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % Cfg::STAGES;
         const bool more = j + 1 < nkv;
+        if (!(ok = mbar_wait(&p_half[0], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(0, j, 0, 4);
         if (!(ok = mbar_wait(&p_ready[0], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(0, j);
+        issue_o(0, j, 4, 8);
+        umma_commit(&o_done[0]);
         if (more) {
           const int sn = (j + 1) % Cfg::STAGES;
           if (!(ok = mbar_wait(&kv_full[sn], ((j + 1) / Cfg::STAGES) & 1, budget_ns))) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
+        if (!(ok = mbar_wait(&p_half[1], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(1, j, 0, 4);
         if (!(ok = mbar_wait(&p_ready[1], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(1, j);
+        issue_o(1, j, 4, 8);
+        umma_commit(&o_done[1]);
         umma_commit(&kv_empty[s]);
         if (more) issue_s(1, j + 1);
       }
@@ -283,39 +302,50 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     float m_used = -INFINITY;  // running max, log2 domain (scaled)
     float l = 0.f;
     KvCursor cur;
-    cur.init(seg);
+    cur.init(kr);
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
-      const int valid = cur.valid(seg);
-      cur.next(seg);
+      const int valid = cur.valid();
+      cur.next(kr);
       if (!mbar_wait(&s_full[i], j & 1, budget_ns)) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t sr[128];
-      {
-        uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-        uint32_t (&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-        tmem_ld32(s_addr, a);
-        tmem_ld32(s_addr + 32, b);
-        tmem_ld32(s_addr + 64, c);
-        tmem_ld32(s_addr + 96, d);
-        tmem_ld_wait();
-      }
-      if (valid < 128) {
+      uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+      uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+      uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+      uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+      // first half of the row, then start loading the second half while the
+      // first half's max is taken
+      tmem_ld32(s_addr, s0);
+      tmem_ld32(s_addr + 32, s1);
+      tmem_ld_wait();
+      reg_fence(s0);
+      reg_fence(s1);
+      tmem_ld32(s_addr + 64, s2);
+      tmem_ld32(s_addr + 96, s3);
+      if (valid < 64) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
-      // row max as 8 independent chains, then a short tree
       float mx8[8];
 #pragma unroll
       for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      tmem_ld_wait();
+      reg_fence(s2);
+      reg_fence(s3);
+      if (valid < 128) {
+#pragma unroll
+        for (int c = 64; c < 128; ++c)
+          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+      }
+#pragma unroll
+      for (int c = 64; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
 #pragma unroll
       for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
@@ -323,7 +353,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
       const float mt = mx8[0] * scale_log2;
       if (mt > m_used + 8.f) {
         // the running max grew by more than 2^8: rescale l and O
-        const float factor = fast_exp2(m_used - mt);  // 0 on the first tile
+        const float factor = exp2_mufu(m_used - mt);  // 0 on the first tile
         l *= factor;
         if (j > 0) {
           if (!mbar_wait(&o_done[i], (j - 1) & 1, budget_ns)) {
@@ -336,6 +366,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
             uint32_t o[32];
             tmem_ld32(o_addr + c, o);
             tmem_ld_wait();
+            reg_fence(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
             tmem_st32(o_addr + c, o);
@@ -343,29 +374,38 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         }
         m_used = mt;
       }
-      // p = 2^(s * scale_log2 - m): packed f32x2 FMA for the argument, four
-      // independent packed partial sums
-      const uint64_t cc = pack_f32x2(scale_log2, scale_log2);
-      const uint64_t nm = pack_f32x2(-m_used, -m_used);
+      // p = 2^(s * scale_log2 - m) with the argument by packed f32x2 FMA and
+      // four packed partial sums; one pair in four takes the FMA-pipe
+      // exponential, the rest the MUFU.  P goes back over S as bf16 in two
+      // halves, so the PV product can start on keys 0..63.
+      const uint64_t cc = f32x2_pack(scale_log2, scale_log2);
+      const uint64_t nm = f32x2_pack(-m_used, -m_used);
       uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const uint64_t xs = ffma_f32x2(
+          const uint64_t xs = f32x2_fma(
               (static_cast<uint64_t>(sr[32 * q + 2 * e + 1]) << 32) | sr[32 * q + 2 * e], cc, nm);
-          const float p0 = fast_exp2(__uint_as_float(static_cast<uint32_t>(xs)));
-          const float p1 = fast_exp2(__uint_as_float(static_cast<uint32_t>(xs >> 32)));
-          const uint64_t pp = pack_f32x2(p0, p1);
-          acc2[e & 3] = fadd_f32x2(acc2[e & 3], pp);
-          pk[e] = pack_bf16x2(p0, p1);
+          uint64_t pp;
+          if ((e & 3) == 3) {
+            pp = exp2_fma_x2(xs);
+          } else {
+            pp = f32x2_pack(exp2_mufu(f32x2_lo(xs)), exp2_mufu(f32x2_hi(xs)));
+          }
+          acc2[e & 3] = f32x2_add(acc2[e & 3], pp);
+          pk[e] = pack_bf16x2(f32x2_lo(pp), f32x2_hi(pp));
         }
         tmem_st16(s_addr + 16 * q, pk);
+        if (q == 1) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_half[i]);
+        }
       }
-      acc2[0] = fadd_f32x2(fadd_f32x2(acc2[0], acc2[1]), fadd_f32x2(acc2[2], acc2[3]));
-      l += __uint_as_float(static_cast<uint32_t>(acc2[0])) +
-           __uint_as_float(static_cast<uint32_t>(acc2[0] >> 32));
+      acc2[0] = f32x2_add(f32x2_add(acc2[0], acc2[1]), f32x2_add(acc2[2], acc2[3]));
+      l += f32x2_lo(acc2[0]) + f32x2_hi(acc2[0]);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[i]);
@@ -374,7 +414,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     if (ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns)) {
       tc_fence_after();
       const int r = q0 + 128 * i + row;
-      const bool live = r < seg.q1;
+      const bool live = r < q_end;
       const float inv = 1.f / l;
       __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * DH;
 #pragma unroll 1

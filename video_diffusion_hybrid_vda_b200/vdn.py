@@ -24,7 +24,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_window_attn_workspace", "vdn_window_attn", "vdn_hybrid_fuse_workspace",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
-           "vdn_vda_scan_static"]
+           "vdn_vda_scan_static", "vdn_selftest_exp2"]
 
 
 class VdnError(RuntimeError):
@@ -79,6 +79,8 @@ def lib():
     L.vdn_reset_device_status.restype = ctypes.c_int
     L.vdn_set_wait_budget_ns.argtypes = [ctypes.c_uint64]
     L.vdn_set_wait_budget_ns.restype = None
+    L.vdn_selftest_exp2.argtypes = [_P, _P, _P, ctypes.c_int, _P]
+    L.vdn_selftest_exp2.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -136,6 +138,15 @@ def reset_device_status(ws, stream=None):
 
 def set_wait_budget_ns(ns):
     lib().vdn_set_wait_budget_ns(int(ns))
+
+
+def selftest_exp2(x, stream=None):
+    """(y_fma, y_mufu): the Softmax's two exponential paths on fp32 CUDA x."""
+    _need_cuda(x)
+    y_fma, y_mufu = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().vdn_selftest_exp2(_ptr(x), _ptr(y_fma), _ptr(y_mufu), x.numel(),
+                                   _stream(stream)), "vdn_selftest_exp2")
+    return y_fma, y_mufu
 
 
 # ---------------------------------------------------------------- VDA
