@@ -6,106 +6,171 @@
 //   S_bwd_t = alpha_t S_bwd_{t+1} P_t + C_t      t = T-1 .. 0, S_bwd_T   = 0
 //
 // which is (alpha_t S_prev + B_t)(I + A_t)^-1 with P_t = (I + A_t)^-1 and
-// C_t = B_t P_t precomputed by the solve.  Rows of S evolve independently
-// (row r of S_t only needs row r of S_{t-1}), so the state is split into
-// blocks of R rows: one CTA per (row block, head, direction), all resident
-// at once, each running all T steps with its rows of S in shared memory
-// (transposed) and P_t, C_t streamed from L2.  Arithmetic is fp32 FMA; each
-// thread owns a 4 x 4 tile of the new state.
+// C_t = B_t P_t from the solve.  Rows of S evolve independently (row r of
+// S_t needs only row r of S_{t-1}), so each CTA owns 64 rows of one head's
+// state in one direction and runs all T steps; every CTA of the grid is
+// resident at once.  Per step the CTA stages P_t (d x d fp32) into shared
+// memory with one bulk copy, double-buffered so that P_{t+1} lands while
+// step t computes; the state rows stay in shared memory (transposed) and
+// each thread computes a 4 x 8 tile of the new state with packed f32x2 FMA.
+// The scan is serial over T and FP32-ALU bound.
 #include "common.cuh"
+#include "exp2_fma.cuh"
+#include "ptx.cuh"
 
 namespace vdn {
 namespace {
 
-constexpr int kScanRows = 16;  // rows of S per CTA
-constexpr int kTile = 4;       // 4 x 4 outputs per thread
+constexpr int kRows = 64;   // rows of S per CTA
+constexpr int kTR = 4;      // rows per thread
+constexpr int kTC = 8;      // columns per thread
 
 template <int DH>
-__global__ void __launch_bounds__((kScanRows / kTile) * (DH / kTile))
+struct ScanCfg {
+  static constexpr int THREADS = (kRows / kTR) * (DH / kTC);  // 256 (d=128), 128 (d=64)
+  static constexpr int P_BYTES = DH * DH * 4;
+  static constexpr int SMEM = 2 * P_BYTES + DH * kRows * 4 + 64;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     vda_scan_kernel(const float* __restrict__ P, const float* __restrict__ C,
-                    const float* __restrict__ alpha, float* __restrict__ states, int T, int H) {
-  constexpr int CG = DH / kTile;  // column groups
-  __shared__ __align__(16) float St[DH][kScanRows];  // S^T of this CTA's rows
+                    const float* __restrict__ alpha, float* __restrict__ states, int T, int H,
+                    uint32_t* status, uint64_t budget_ns) {
+  using Cfg = ScanCfg<DH>;
+  constexpr int CG = DH / kTC;  // column groups
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* Pbuf = reinterpret_cast<float*>(smem_raw);                  // 2 x [DH][DH]
+  float* St = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // [DH][kRows]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES + DH * kRows * 4);
 
   const int rb = blockIdx.x;  // row block
   const int h = blockIdx.y;
   const int dir = blockIdx.z;  // 0 forward, 1 backward
   const int cg = threadIdx.x % CG;
   const int rg = threadIdx.x / CG;
-  const int row0 = rb * kScanRows + rg * kTile;  // first row of this thread's tile
-  const int col0 = cg * kTile;
+  const int lrow0 = rg * kTR;                  // first local row of the thread's tile
+  const int row0 = rb * kRows + lrow0;         // first row of S
+  const int col0 = cg * kTC;
+  const int64_t mat = static_cast<int64_t>(DH) * DH;
+  float* out_dir = states + static_cast<int64_t>(dir) * T * H * mat;
+  auto frame = [&](int step) { return dir == 0 ? step : T - 1 - step; };
 
-  for (int i = threadIdx.x; i < DH * kScanRows; i += blockDim.x) (&St[0][0])[i] = 0.f;
+  for (int i = threadIdx.x; i < DH * kRows; i += blockDim.x) St[i] = 0.f;
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&full[0], Cfg::P_BYTES);
+    bulk_load(Pbuf, P + (static_cast<int64_t>(frame(0)) * H + h) * mat, Cfg::P_BYTES, &full[0]);
+  }
   __syncthreads();
 
-  const int64_t mat_stride = static_cast<int64_t>(DH) * DH;
-  float* out_dir = states + static_cast<int64_t>(dir) * T * H * mat_stride;
-
+  int issued = 1;
 #pragma unroll 1
   for (int step = 0; step < T; ++step) {
-    const int t = dir == 0 ? step : T - 1 - step;
+    const int t = frame(step);
+    const int b = step & 1;
+    if (threadIdx.x == 0 && step + 1 < T) {
+      // buffer b^1 was last read in step-1, which every thread has left
+      mbar_arrive_expect_tx(&full[b ^ 1], Cfg::P_BYTES);
+      bulk_load(Pbuf + (b ^ 1) * DH * DH, P + (static_cast<int64_t>(frame(step + 1)) * H + h) * mat,
+                Cfg::P_BYTES, &full[b ^ 1]);
+      ++issued;
+    }
     const float a = __ldg(alpha + t * H + h);
-    const float* Pt = P + (static_cast<int64_t>(t) * H + h) * mat_stride;
-    const float* Ct = C + (static_cast<int64_t>(t) * H + h) * mat_stride;
-
-    float acc[kTile][kTile];
+    const float* Ct = C + (static_cast<int64_t>(t) * H + h) * mat;
+    float4 cv[kTR][2];
 #pragma unroll
-    for (int r = 0; r < kTile; ++r)
+    for (int r = 0; r < kTR; ++r) {
+      cv[r][0] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + col0));
+      cv[r][1] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + col0 + 4));
+    }
+    const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
+    if (!__syncthreads_and(ok)) {
+      if (threadIdx.x == 0) record_status(status, kStatusTimeout);
+      break;
+    }
+    const float* Pt = Pbuf + b * DH * DH;
+    // acc2[r][q] holds columns (col0 + 2q, col0 + 2q + 1) of row r
+    uint64_t acc2[kTR][kTC / 2];
 #pragma unroll
-      for (int e = 0; e < kTile; ++e) acc[r][e] = 0.f;
-
+    for (int r = 0; r < kTR; ++r)
+#pragma unroll
+      for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
     if (step > 0) {
-#pragma unroll 8
+#pragma unroll 4
       for (int k = 0; k < DH; ++k) {
-        const float4 p = __ldg(reinterpret_cast<const float4*>(Pt + k * DH + col0));
-        const float4 s = *reinterpret_cast<const float4*>(&St[k][rg * kTile]);
-        const float sv[4] = {s.x, s.y, s.z, s.w};
+        const float4 s4 = *reinterpret_cast<const float4*>(St + k * kRows + lrow0);
+        const ulonglong2 p01 = *reinterpret_cast<const ulonglong2*>(Pt + k * DH + col0);
+        const ulonglong2 p23 = *reinterpret_cast<const ulonglong2*>(Pt + k * DH + col0 + 4);
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-        for (int r = 0; r < kTile; ++r) {
-          acc[r][0] = fmaf(sv[r], p.x, acc[r][0]);
-          acc[r][1] = fmaf(sv[r], p.y, acc[r][1]);
-          acc[r][2] = fmaf(sv[r], p.z, acc[r][2]);
-          acc[r][3] = fmaf(sv[r], p.w, acc[r][3]);
+        for (int r = 0; r < kTR; ++r) {
+          const uint64_t ss = f32x2_pack(sv[r], sv[r]);
+          acc2[r][0] = f32x2_fma(ss, p01.x, acc2[r][0]);
+          acc2[r][1] = f32x2_fma(ss, p01.y, acc2[r][1]);
+          acc2[r][2] = f32x2_fma(ss, p23.x, acc2[r][2]);
+          acc2[r][3] = f32x2_fma(ss, p23.y, acc2[r][3]);
         }
       }
     }
-    float snew[kTile][kTile];
+    float snew[kTR][kTC];
+    const uint64_t aa = f32x2_pack(a, a);
 #pragma unroll
-    for (int r = 0; r < kTile; ++r) {
-      const float4 c = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + col0));
-      snew[r][0] = fmaf(a, acc[r][0], c.x);
-      snew[r][1] = fmaf(a, acc[r][1], c.y);
-      snew[r][2] = fmaf(a, acc[r][2], c.z);
-      snew[r][3] = fmaf(a, acc[r][3], c.w);
-      float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat_stride +
+    for (int r = 0; r < kTR; ++r) {
+      const float cc[8] = {cv[r][0].x, cv[r][0].y, cv[r][0].z, cv[r][0].w,
+                           cv[r][1].x, cv[r][1].y, cv[r][1].z, cv[r][1].w};
+#pragma unroll
+      for (int q = 0; q < kTC / 2; ++q) {
+        const uint64_t v = f32x2_fma(aa, acc2[r][q], f32x2_pack(cc[2 * q], cc[2 * q + 1]));
+        snew[r][2 * q] = f32x2_lo(v);
+        snew[r][2 * q + 1] = f32x2_hi(v);
+      }
+      float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
                    static_cast<int64_t>(row0 + r) * DH + col0;
       *reinterpret_cast<float4*>(dst) = make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
+      *reinterpret_cast<float4*>(dst + 4) =
+          make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
     }
-    __syncthreads();  // every thread has finished reading St
+    __syncthreads();  // every thread has finished reading St (and Pbuf b)
 #pragma unroll
-    for (int e = 0; e < kTile; ++e)
-      *reinterpret_cast<float4*>(&St[col0 + e][rg * kTile]) =
+    for (int e = 0; e < kTC; ++e)
+      *reinterpret_cast<float4*>(St + (col0 + e) * kRows + lrow0) =
           make_float4(snew[0][e], snew[1][e], snew[2][e], snew[3][e]);
     __syncthreads();
   }
+  // the bulk copies this CTA started must land before it exits
+  if (threadIdx.x == 0) {
+    for (int s = (issued > 2 ? issued - 2 : 0); s < issued; ++s)
+      mbar_wait(&full[s & 1], (s >> 1) & 1, 200000000ull);
+  }
+}
+
+template <int DH>
+cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* C,
+                           const float* alpha, float* states) {
+  using Cfg = ScanCfg<DH>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(vda_scan_kernel<DH>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(DH / kRows, s.H, 2);
+  vda_scan_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      P, C, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* P,
                             const float* C, const float* alpha, float* states) {
-  if (s.d == 128) {
-    dim3 grid(128 / kScanRows, s.H, 2);
-    vda_scan_kernel<128><<<grid, (kScanRows / kTile) * (128 / kTile), 0, ctx.stream>>>(
-        P, C, alpha, states, s.T, s.H);
-  } else if (s.d == 64) {
-    dim3 grid(64 / kScanRows, s.H, 2);
-    vda_scan_kernel<64><<<grid, (kScanRows / kTile) * (64 / kTile), 0, ctx.stream>>>(
-        P, C, alpha, states, s.T, s.H);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (s.d == 128) return launch_scan_dh<128>(ctx, s, P, C, alpha, states);
+  if (s.d == 64) return launch_scan_dh<64>(ctx, s, P, C, alpha, states);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace vdn

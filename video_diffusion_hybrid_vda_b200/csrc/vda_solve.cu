@@ -2,18 +2,19 @@
 // article, 方法概述 item 2: S_t = (S_bar_t + B_t)(I + A_t)^-1).
 //
 // Per (frame t, head h), one CTA of 512 threads:
-//   1. Cholesky  L L^T = I + A   (right-looking, the matrix held in registers
-//      as 4x8 (d=128) tiles per thread; the scaled pivot column is published
-//      through shared memory each step and L is kept in shared memory);
-//   2. forward substitution  L Y = [I | B^T];
-//   3. back substitution     L^T X = Y   ->  X = [P | C^T],
-//      P = (I + A)^-1 and C = B P (because (I + A) C^T = B^T).
-// The solve factors the symmetric part of the prep's A (the tensor-core
-// product rounds beta*k on one side only, so A is symmetric up to that).
+//   1. Cholesky  L L^T = I + A_sym  (right-looking; the matrix lives in
+//      registers as 4x8 (d=128) tiles per thread, the scaled pivot column is
+//      published through shared memory each step, L is kept in shared
+//      memory);
+//   2. W = L^-1 by forward substitution against I (row k of W is published
+//      each step; column blocks that are still zero are skipped);
+//   3. P = (I + A)^-1 = W^T W and 4. C = B P, both as shared-memory GEMMs
+//      without barriers inside their loops.
+// A_sym = (A + A^T) / 2: the tensor-core product in the prep rounds
+// beta*k on one operand only, so A is symmetric up to that rounding.
 // I + A is symmetric positive definite with eigenvalues >= 1 (beta >= 0),
 // so no pivoting is needed; a non-positive or NaN pivot is reported as
-// VDN_ERR_NUMERIC in the status word.
-// This step is FP32-ALU and latency bound (d^3-order work per problem).
+// VDN_ERR_NUMERIC in the status word.  This step is FP32-ALU bound.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -24,11 +25,13 @@ constexpr int kSolveThreads = 512;  // 32 row groups x 16 column groups
 
 template <int DH>
 struct SolveCfg {
-  static constexpr int RA = DH / 32;        // rows per thread
+  static constexpr int RA = DH / 32;        // rows per thread (strided by 32)
   static constexpr int CB = DH / 16;        // matrix columns per thread (phase 1)
-  static constexpr int RG = (2 * DH) / 64;  // 4-wide column groups of the RHS per thread
-  static constexpr int LD = DH + 1;         // padded smem row stride of L
-  static constexpr int SMEM = DH * LD * 4 + 2 * (2 * DH) * 4;
+  static constexpr int RG = DH / 64;        // 4-wide column groups of W per thread
+  static constexpr int LD = DH + 1;         // padded row stride of L (column access)
+  static constexpr int LD2 = DH + 4;        // row stride of W, P, B (float4 rows)
+  static constexpr int MAT = DH * LD2;      // floats per matrix buffer (>= DH * LD)
+  static constexpr int SMEM = 2 * MAT * 4 + 2 * (2 * DH) * 4;
 };
 
 // Scale row group `ka` of the register tile by `dinv`, write it back and
@@ -60,7 +63,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1)
   using Cfg = SolveCfg<DH>;
   extern __shared__ float sm[];
   float* Ls = sm;                    // [DH][LD], lower triangle of L
-  float* buf0 = sm + DH * Cfg::LD;   // two 2*DH broadcast buffers
+  float* buf0 = sm + 2 * Cfg::MAT;   // two 2*DH broadcast buffers
   float* buf1 = buf0 + 2 * DH;
 
   const int tx = threadIdx.x & 15;
@@ -131,25 +134,22 @@ __global__ void __launch_bounds__(kSolveThreads, 1)
   __syncthreads();  // L complete in shared memory
 
   // ---------------------------------------------------------------- phase 2
-  // RHS columns c = 64 g + 4 tx + e; c < DH: identity, c >= DH: B^T.
+  // W = L^-1: forward substitution against I.  Columns c = 64 g + 4 tx + e.
+  // Row k of W is zero beyond column k, so column group g only takes part
+  // once k >= 64 g.
   float r[Cfg::RA][Cfg::RG][4];
 #pragma unroll
   for (int a = 0; a < Cfg::RA; ++a)
 #pragma unroll
     for (int g = 0; g < Cfg::RG; ++g)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = ty + 32 * a, c = 64 * g + 4 * tx + e;
-        r[a][g][e] = c < DH ? (i == c ? 1.f : 0.f) : __ldg(Bm + (c - DH) * DH + i);
-      }
+      for (int e = 0; e < 4; ++e) r[a][g][e] = (ty + 32 * a == 64 * g + 4 * tx + e) ? 1.f : 0.f;
 
 #pragma unroll 1
   for (int k = 0; k < DH; ++k) {
     float* row = (k & 1) ? buf1 : buf0;
     const float dinv = 1.f / Ls[k * Cfg::LD + k];
-    if (ty == (k & 31)) {
-      publish_row<Cfg::RA, Cfg::RG>(r, k >> 5, dinv, row + 4 * tx);
-    }
+    if (ty == (k & 31)) publish_row<Cfg::RA, Cfg::RG>(r, k >> 5, dinv, row + 4 * tx);
     __syncthreads();
 #pragma unroll
     for (int a = 0; a < Cfg::RA; ++a) {
@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kSolveThreads, 1)
       const float lik = i > k ? Ls[i * Cfg::LD + k] : 0.f;
 #pragma unroll
       for (int g = 0; g < Cfg::RG; ++g) {
+        if (64 * g > k) continue;  // W[k][c] = 0 for c > k
         const float4 y = *reinterpret_cast<const float4*>(row + 64 * g + 4 * tx);
         r[a][g][0] = fmaf(-lik, y.x, r[a][g][0]);
         r[a][g][1] = fmaf(-lik, y.y, r[a][g][1]);
@@ -166,51 +167,102 @@ __global__ void __launch_bounds__(kSolveThreads, 1)
       }
     }
   }
+  __syncthreads();  // all reads of L done: its buffer now takes W
+
+  float* Ws = sm;             // [DH][LD2]
+  float* Xs = sm + Cfg::MAT;  // [DH][LD2]: P, then read by phase 4
+#pragma unroll
+  for (int a = 0; a < Cfg::RA; ++a)
+#pragma unroll
+    for (int g = 0; g < Cfg::RG; ++g)
+      *reinterpret_cast<float4*>(Ws + (ty + 32 * a) * Cfg::LD2 + 64 * g + 4 * tx) =
+          make_float4(r[a][g][0], r[a][g][1], r[a][g][2], r[a][g][3]);
   __syncthreads();
 
   // ---------------------------------------------------------------- phase 3
-#pragma unroll 1
-  for (int k = DH - 1; k >= 0; --k) {
-    float* row = (k & 1) ? buf1 : buf0;
-    const float dinv = 1.f / Ls[k * Cfg::LD + k];
-    if (ty == (k & 31)) {
-      publish_row<Cfg::RA, Cfg::RG>(r, k >> 5, dinv, row + 4 * tx);
+  // P = W^T W: each thread a (DH/32) x (DH/16) tile, rows 4 rg.., cols CW cg..
+  constexpr int PR = DH / 32;   // rows per thread
+  constexpr int PC = DH / 16;   // cols per thread
+  const int rg = threadIdx.x >> 4;   // 0..31
+  const int cg = threadIdx.x & 15;   // 0..15
+  const int i0 = rg * PR, c0 = cg * PC;
+  float acc[PR][PC];
+#pragma unroll
+  for (int a = 0; a < PR; ++a)
+#pragma unroll
+    for (int b = 0; b < PC; ++b) acc[a][b] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < DH; ++k) {
+    const float* wk = Ws + k * Cfg::LD2;
+    float wi[PR], wc[PC];
+#pragma unroll
+    for (int a = 0; a < PR; a += 2) {
+      const float2 v = *reinterpret_cast<const float2*>(wk + i0 + a);
+      wi[a] = v.x;
+      wi[a + 1] = v.y;
     }
-    __syncthreads();
 #pragma unroll
-    for (int a = 0; a < Cfg::RA; ++a) {
-      if (32 * a >= k) continue;  // rows i >= k are final
-      const int i = ty + 32 * a;
-      const float lki = i < k ? Ls[k * Cfg::LD + i] : 0.f;
+    for (int b = 0; b < PC; b += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(wk + c0 + b);
+      wc[b] = v.x; wc[b + 1] = v.y; wc[b + 2] = v.z; wc[b + 3] = v.w;
+    }
 #pragma unroll
-      for (int g = 0; g < Cfg::RG; ++g) {
-        const float4 x = *reinterpret_cast<const float4*>(row + 64 * g + 4 * tx);
-        r[a][g][0] = fmaf(-lki, x.x, r[a][g][0]);
-        r[a][g][1] = fmaf(-lki, x.y, r[a][g][1]);
-        r[a][g][2] = fmaf(-lki, x.z, r[a][g][2]);
-        r[a][g][3] = fmaf(-lki, x.w, r[a][g][3]);
+    for (int a = 0; a < PR; ++a)
+#pragma unroll
+      for (int b = 0; b < PC; ++b) acc[a][b] = fmaf(wi[a], wc[b], acc[a][b]);
+  }
+  float* Pm = P + mat;
+#pragma unroll
+  for (int a = 0; a < PR; ++a)
+#pragma unroll
+    for (int b = 0; b < PC; b += 4) {
+      const float4 v = make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+      *reinterpret_cast<float4*>(Xs + (i0 + a) * Cfg::LD2 + c0 + b) = v;
+      *reinterpret_cast<float4*>(Pm + (i0 + a) * DH + c0 + b) = v;
+    }
+  __syncthreads();  // P complete in Xs; W no longer needed: its buffer takes B
+
+  // ---------------------------------------------------------------- phase 4
+  // C = B P (B rows staged through shared memory).
+  for (int idx = threadIdx.x; idx < DH * DH / 4; idx += kSolveThreads) {
+    const int rr = idx / (DH / 4), cc = idx % (DH / 4);
+    *reinterpret_cast<float4*>(Ws + rr * Cfg::LD2 + 4 * cc) =
+        __ldg(reinterpret_cast<const float4*>(Bm) + idx);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int a = 0; a < PR; ++a)
+#pragma unroll
+    for (int b = 0; b < PC; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < DH; k += 4) {
+    float bv[PR][4];
+#pragma unroll
+    for (int a = 0; a < PR; ++a) {
+      const float4 v = *reinterpret_cast<const float4*>(Ws + (i0 + a) * Cfg::LD2 + k);
+      bv[a][0] = v.x; bv[a][1] = v.y; bv[a][2] = v.z; bv[a][3] = v.w;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      float pc[PC];
+#pragma unroll
+      for (int b = 0; b < PC; b += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(Xs + (k + kk) * Cfg::LD2 + c0 + b);
+        pc[b] = v.x; pc[b + 1] = v.y; pc[b + 2] = v.z; pc[b + 3] = v.w;
       }
+#pragma unroll
+      for (int a = 0; a < PR; ++a)
+#pragma unroll
+        for (int b = 0; b < PC; ++b) acc[a][b] = fmaf(bv[a][kk], pc[b], acc[a][b]);
     }
   }
-
-  // ---------------------------------------------------------------- store
-  float* Pm = P + mat;
   float* Cm = Cout + mat;
 #pragma unroll
-  for (int a = 0; a < Cfg::RA; ++a) {
-    const int i = ty + 32 * a;
+  for (int a = 0; a < PR; ++a)
 #pragma unroll
-    for (int g = 0; g < Cfg::RG; ++g) {
-      const int c0 = 64 * g + 4 * tx;
-      if (c0 < DH) {
-        *reinterpret_cast<float4*>(Pm + i * DH + c0) =
-            make_float4(r[a][g][0], r[a][g][1], r[a][g][2], r[a][g][3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Cm[(c0 - DH + e) * DH + i] = r[a][g][e];
-      }
-    }
-  }
+    for (int b = 0; b < PC; b += 4)
+      *reinterpret_cast<float4*>(Cm + (i0 + a) * DH + c0 + b) =
+          make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
   if (bad) record_status(status, kStatusNumeric);
 }
 
