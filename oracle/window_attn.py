@@ -18,6 +18,12 @@ first and last frames are boundary anchors).
 
 ``anchors`` is a bit set: 1 = first frame, 2 = last frame.
 ``origin = 1`` (anchor frames outside the chunk grid) is a study variant.
+
+Context keys: the pages keep every interaction with text or audio tokens as
+full Softmax (ai-feeds.com 方法 section; 10100.com 方法概述 item 1).  Reading
+taken here: when context keys/values ``ctx_k, ctx_v`` ([M, H*d]) are given,
+every video query attends to them in the same softmax as its visible video
+keys (one joint normalisation).
 """
 
 import numpy as np
@@ -54,12 +60,13 @@ def _softmax_rows(s):
 
 
 def window_attn_rows(q, k, v, T, N, H, d, rows, chunk_frames=5, window_chunks=1,
-                     anchors=3, scale=None, origin=0, heads=None):
+                     anchors=3, scale=None, origin=0, heads=None, ctx_k=None, ctx_v=None):
     """Window+anchor Softmax for the given query token rows.
 
     Returns (o [len(rows), H*d], lse [H, len(rows)]) in float64; lse is the
-    natural-log sum of exp(scaled scores) over the visible keys.  ``heads``
-    restricts the computation to a subset of heads (others are left 0).
+    natural-log sum of exp(scaled scores) over the visible keys (video keys
+    and, if given, all context keys).  ``heads`` restricts the computation
+    to a subset of heads (others are left 0).
     """
     scale = 1.0 / np.sqrt(d) if scale is None or scale <= 0 else float(scale)
     rows = np.asarray(rows, dtype=np.int64)
@@ -76,6 +83,9 @@ def window_attn_rows(q, k, v, T, N, H, d, rows, chunk_frames=5, window_chunks=1,
             Q = np.asarray(q[rows[sel], c], dtype=np.float64)
             K = np.asarray(k[key_rows, c], dtype=np.float64)
             V = np.asarray(v[key_rows, c], dtype=np.float64)
+            if ctx_k is not None and len(ctx_k) > 0:
+                K = np.vstack([K, np.asarray(ctx_k[:, c], dtype=np.float64)])
+                V = np.vstack([V, np.asarray(ctx_v[:, c], dtype=np.float64)])
             p, l = _softmax_rows((Q @ K.T) * scale)
             out[sel, c] = p @ V
             lse[h, sel] = l
@@ -83,7 +93,7 @@ def window_attn_rows(q, k, v, T, N, H, d, rows, chunk_frames=5, window_chunks=1,
 
 
 def window_attn(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3,
-                scale=None, origin=0):
+                scale=None, origin=0, ctx_k=None, ctx_v=None):
     """Window+anchor Softmax for every token.  Returns (o [L, H*d], lse [H, L])."""
     return window_attn_rows(q, k, v, T, N, H, d, np.arange(T * N), chunk_frames,
-                            window_chunks, anchors, scale, origin)
+                            window_chunks, anchors, scale, origin, ctx_k=ctx_k, ctx_v=ctx_v)

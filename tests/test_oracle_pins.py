@@ -253,6 +253,31 @@ def test_window_attn_equals_dense_masked(T):
     np.testing.assert_allclose(lse[0], lse_ref, rtol=1e-12)
 
 
+@pytest.mark.parametrize("T,M", [(10, 5), (17, 9)])
+def test_window_attn_with_context_keys_equals_dense_masked(T, M):
+    """Context (text/audio) keys join the same softmax, visible to every query:
+    brute force over [video keys; context keys] with an all-visible block."""
+    s, x = _tiny(T=T, N=8, H=2, d=8, seed=41)
+    rng = np.random.default_rng(T + M)
+    ck = rng.standard_normal((M, s.D))
+    cv = rng.standard_normal((M, s.D))
+    o, lse = oracle.window_attn(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d, ctx_k=ck, ctx_v=cv)
+    _, allowed = _dense_masked_attention(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d)
+    full = np.hstack([allowed, np.ones((s.L, M), dtype=bool)])
+    for h in range(s.H):
+        c = slice(h * s.d, (h + 1) * s.d)
+        K = np.vstack([x["k"][:, c], ck[:, c]])
+        V = np.vstack([x["v"][:, c], cv[:, c]])
+        sc = np.where(full, x["q"][:, c] @ K.T / np.sqrt(s.d), -np.inf)
+        np.testing.assert_allclose(o[:, c], scipy.special.softmax(sc, axis=1) @ V, atol=1e-12)
+        np.testing.assert_allclose(lse[h], scipy.special.logsumexp(sc, axis=1), rtol=1e-12)
+    # no context keys: identical to the plain window attention
+    o0, _ = oracle.window_attn(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d,
+                               ctx_k=ck[:0], ctx_v=cv[:0])
+    o1, _ = oracle.window_attn(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d)
+    np.testing.assert_array_equal(o0, o1)
+
+
 def _closed_form_pair_count(T, cf=5):
     """Visible (query, key) frame pairs for chunk 5, +-1 chunk, both anchors.
 
