@@ -158,6 +158,21 @@ VDN_API vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const 
                            float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* Window-and-anchor Softmax with context keys.  The pages keep every
+ * interaction with text or audio tokens as full Softmax (10100.com 方法概述
+ * item 1; ai-feeds.com 方法).  Here every video query attends, in the same
+ * softmax as its visible video keys, to all m_ctx context keys/values:
+ *   o[r, h] = softmax over {visible video keys} U {context keys}.
+ * ctx_k, ctx_v : [m_ctx, ld_ctx] bf16 (head h at columns [h*d, (h+1)*d)),
+ *                may be NULL when m_ctx == 0.  Everything else as for
+ *                vdn_window_attn, which is this call with m_ctx = 0. */
+VDN_API vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void* k,
+                                       const void* v, int64_t ld, const void* ctx_k,
+                                       const void* ctx_v, int64_t ld_ctx, int m_ctx,
+                                       int chunk_frames, int window_chunks, unsigned anchors,
+                                       float scale, void* o, int64_t ld_o, float* lse_opt,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Branch calibration and output projections (10100.com article, 方法概述
  * item 3; hotpaper.ai summary, 기술적 접근법).

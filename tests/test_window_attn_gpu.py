@@ -139,3 +139,65 @@ def test_fma_pipe_exp2_error_bound(vdn):
     yfar, _ = vdn.selftest_exp2(far)
     v = host(yfar)
     assert np.all(v >= 0) and np.all(v < 1e-37)
+
+
+def _ctx(M, D, seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    ck = torch.randn((M, D), generator=g, device="cuda").to(torch.bfloat16)
+    cv = torch.randn((M, D), generator=g, device="cuda").to(torch.bfloat16)
+    return ck, cv
+
+
+@pytest.mark.parametrize("T,N,H,d,M", [(10, 64, 2, 128, 1), (17, 100, 2, 128, 77),
+                                       (12, 96, 1, 64, 300), (6, 40, 3, 128, 512)])
+def test_window_attn_context_keys_small(vdn, T, N, H, d, M):
+    """Text/audio context keys: every video query also attends to them."""
+    shape = synth.Shape(T, N, H, d)
+    inp = synth.make_inputs(shape, seed=T + M, device="cuda")
+    ck, cv = _ctx(M, shape.D, seed=M)
+    o, lse = _run(vdn, shape, inp, ctx_k=ck, ctx_v=cv)
+    x = {k: host(v) for k, v in inp.items() if k in ("q", "k", "v")}
+    o_ref, lse_ref = oracle.window_attn(x["q"], x["k"], x["v"], T, N, H, d,
+                                        ctx_k=host(ck), ctx_v=host(cv))
+    assert per_head_max_rel(host(o), o_ref, H, d) <= TOL_BF16
+    assert np.abs(host(lse) - lse_ref).max() <= TOL_LSE
+
+
+def test_window_attn_context_keys_full_layer_sampled(vdn):
+    """102 latent frames x 4032 tokens x 24 heads plus 512 text keys."""
+    T, M = 102, 512
+    shape = synth.Shape(T, 4032, 24, 128)
+    inp = synth.make_inputs(shape, seed=3, device="cuda")
+    ck, cv = _ctx(M, shape.D, seed=5)
+    o, lse = _run(vdn, shape, inp, ctx_k=ck, ctx_v=cv)
+    rows = _sample_rows(T, shape.N, np.random.default_rng(7), n_random=12)
+    ridx = torch.as_tensor(rows, device="cuda")
+    o_s, lse_s = host(o[ridx]), host(lse[:, ridx])
+    for h in (2, 17):
+        c = slice(h * 128, (h + 1) * 128)
+        o_ref, lse_ref = oracle.window_attn_rows(
+            host(inp["q"][:, c]), host(inp["k"][:, c]), host(inp["v"][:, c]), T, shape.N, 1, 128,
+            rows, ctx_k=host(ck[:, c]), ctx_v=host(cv[:, c]))
+        assert max_rel(o_s[:, c], o_ref) <= TOL_BF16, h
+        assert np.abs(lse_s[h] - lse_ref[0]).max() <= TOL_LSE, h
+    del inp, o, lse
+    torch.cuda.empty_cache()
+
+
+def test_window_attn_rescale_in_one_row_of_a_warp(vdn):
+    """A context key aligned with one query row makes only that row's running
+    max jump by far more than 2^8 at the last key tiles; the O rescale must
+    stay correct for it and for its warp neighbours."""
+    shape = synth.Shape(6, 64, 1, 128)
+    inp = synth.make_inputs(shape, seed=11, device="cuda")
+    ck, cv = _ctx(130, shape.D, seed=12)
+    ck = (ck.float() * 0.05).to(torch.bfloat16)
+    ck[0] = inp["q"][3]           # row 3 scores |q_3|^2 ~ 128 against this key
+    ck[129] = inp["q"][40] * 2    # another row, in the ragged last context tile
+    o, lse = _run(vdn, shape, inp, ctx_k=ck, ctx_v=cv)
+    x = {k: host(v) for k, v in inp.items() if k in ("q", "k", "v")}
+    o_ref, lse_ref = oracle.window_attn(x["q"], x["k"], x["v"], *shape_args(shape),
+                                        ctx_k=host(ck), ctx_v=host(cv))
+    assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16
+    assert np.abs(host(lse) - lse_ref).max() <= TOL_LSE

@@ -230,7 +230,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int lt = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
       const int b = lt & 1;
-      if (!mbar_wait(&tfull[b], (lt >> 1) & 1, budget_ns)) {
+      // warp-uniform: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[b], (lt >> 1) & 1, budget_ns))) {
         record_status(status, kStatusTimeout);
         break;
       }

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
         const int i = kb * C::BK + row;
         bv[j] = i < N ? __ldg(beta + (static_cast<int64_t>(t) * N + i) * H + h) : 0.f;
       }
-      if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, budget_ns)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kb / C::STAGES) & 1, budget_ns))) {
         record_status(status, kStatusTimeout);
         ok = false;
         break;
@@ -197,7 +197,8 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       mbar_arrive(&scaled[s]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && mbar_wait(accum_full, 0, budget_ns)) {
+    // warp-uniform: the TMEM loads below are warp-collective
+    if (__all_sync(0xffffffffu, ok && mbar_wait(accum_full, 0, budget_ns))) {
       tc_fence_after();
       const uint32_t quarter = warp & 3;  // TMEM lane quarter this warp may access
       const int m = quarter * 32 + lane_id();

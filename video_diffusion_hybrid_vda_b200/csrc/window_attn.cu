@@ -92,7 +92,9 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
 // its 128-key tiles (start row, number of valid keys).
 struct KvRange {
   int nint, a0, a1, a2, b0, b1, b2;
-  __device__ void load(const WinSeg& s) {
+  int mctx;  // context (text/audio) keys, visible to every query, after the video keys
+  __device__ void load(const WinSeg& s, int m_ctx) {
+    mctx = m_ctx;
     nint = s.nint;
     a0 = s.k0[0];
     a1 = s.k0[1];
@@ -107,17 +109,25 @@ struct KvRange {
 
 struct KvCursor {
   int iv, pos, end;
+  bool ctx;  // true once the cursor walks the context keys
   __device__ void init(const KvRange& r) {
     iv = 0;
     pos = r.a0;
     end = r.b0;
+    ctx = false;
   }
   __device__ void next(const KvRange& r) {
     pos += 128;
-    if (pos >= end && iv + 1 < r.nint) {
-      ++iv;
-      pos = r.start(iv);
-      end = r.end(iv);
+    if (pos >= end && !ctx) {
+      if (iv + 1 < r.nint) {
+        ++iv;
+        pos = r.start(iv);
+        end = r.end(iv);
+      } else if (r.mctx > 0) {
+        ctx = true;
+        pos = 0;
+        end = r.mctx;
+      }
     }
   }
   __device__ int valid() const { return min(128, end - pos); }
@@ -128,6 +138,8 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     window_attn_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap kmap,
                        const __grid_constant__ CUtensorMap vmap,
+                       const __grid_constant__ CUtensorMap ckmap,
+                       const __grid_constant__ CUtensorMap cvmap, int m_ctx,
                        const __grid_constant__ WinSched sched, int H, int L, float scale_log2,
                        __nv_bfloat16* __restrict__ out, int64_t ld_o, float* __restrict__ lse,
                        uint32_t* status, uint64_t budget_ns) {
@@ -159,9 +171,9 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   const WinSeg& seg = sched.seg[si];
   const int q0 = seg.q0 + (tile - seg.tile_base) * 256;
   const int q_end = seg.q1;
-  const int nkv = seg.nkv;
+  const int nkv = seg.nkv + (m_ctx + 127) / 128;
   KvRange kr;
-  kr.load(seg);
+  kr.load(seg, m_ctx);
   const uint32_t warp = warp_id();
 
   if (threadIdx.x == 0) {
@@ -181,6 +193,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&kmap);
     tma_prefetch_desc(&vmap);
+    if (m_ctx > 0) {
+      tma_prefetch_desc(&ckmap);
+      tma_prefetch_desc(&cvmap);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -217,9 +233,11 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         }
         uint8_t* kb = kvbuf + s * 2 * Cfg::TILE_BYTES;
         mbar_arrive_expect_tx(&kv_full[s], 2 * Cfg::TILE_BYTES);
+        const CUtensorMap* km = cur.ctx ? &ckmap : &kmap;
+        const CUtensorMap* vm = cur.ctx ? &cvmap : &vmap;
         for (int sl = 0; sl < Cfg::SLABS; ++sl) {
-          tma_load_2d(kb + sl * 16384, &kmap, &kv_full[s], h * DH + 64 * sl, cur.pos);
-          tma_load_2d(kb + Cfg::TILE_BYTES + sl * 16384, &vmap, &kv_full[s], h * DH + 64 * sl,
+          tma_load_2d(kb + sl * 16384, km, &kv_full[s], h * DH + 64 * sl, cur.pos);
+          tma_load_2d(kb + Cfg::TILE_BYTES + sl * 16384, vm, &kv_full[s], h * DH + 64 * sl,
                       cur.pos);
         }
         ++issued;
@@ -307,7 +325,8 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     for (int j = 0; j < nkv; ++j) {
       const int valid = cur.valid();
       cur.next(kr);
-      if (!mbar_wait(&s_full[i], j & 1, budget_ns)) {
+      // warp-uniform decision: tcgen05.ld/st below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[i], j & 1, budget_ns))) {
         ok = false;
         break;
       }
@@ -351,12 +370,16 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < w; ++c) mx8[c] = fmaxf(mx8[c], mx8[c + w]);
       const float mt = mx8[0] * scale_log2;
-      if (mt > m_used + 8.f) {
-        // the running max grew by more than 2^8: rescale l and O
-        const float factor = exp2_mufu(m_used - mt);  // 0 on the first tile
+      // Lazy rescale: only when some row's max grew by more than 2^8.  The
+      // decision is taken per warp (the O accesses are warp-collective); rows
+      // of a rescaling warp move to max(m_used, mt), a factor of 1 for rows
+      // whose max did not grow.
+      if (__any_sync(0xffffffffu, mt > m_used + 8.f)) {
+        const float m_new = fmaxf(m_used, mt);
+        const float factor = exp2_mufu(m_used - m_new);  // 0 on the first tile
         l *= factor;
         if (j > 0) {
-          if (!mbar_wait(&o_done[i], (j - 1) & 1, budget_ns)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&o_done[i], (j - 1) & 1, budget_ns))) {
             ok = false;
             break;
           }
@@ -372,7 +395,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
             tmem_st32(o_addr + c, o);
           }
         }
-        m_used = mt;
+        m_used = m_new;
       }
       // p = 2^(s * scale_log2 - m) with the argument by packed f32x2 FMA and
       // four packed partial sums; one pair in four takes the FMA-pipe
@@ -411,7 +434,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
       mbar_arrive(&p_ready[i]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns)) {
+    if (__all_sync(0xffffffffu, ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns))) {
       tc_fence_after();
       const int r = q0 + 128 * i + row;
       const bool live = r < q_end;
@@ -522,6 +545,7 @@ bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSch
 template <int DH>
 cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                              const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             const CUtensorMap& ckmap, const CUtensorMap& cvmap, int m_ctx,
                              const WinSched& sched, float scale, void* o, int64_t ld_o,
                              float* lse) {
   using Cfg = WinCfg<DH>;
@@ -534,7 +558,7 @@ cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtens
   }
   const int grid = sched.total_tiles * s.H;
   window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, kmap, vmap, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
+      qmap, kmap, vmap, ckmap, cvmap, m_ctx, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
       static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
@@ -553,10 +577,11 @@ size_t vdn_window_attn_workspace(const vdn_shape* shape) {
   return kStatusBytes;
 }
 
-vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k, const void* v,
-                           int64_t ld, int chunk_frames, int window_chunks, unsigned anchors,
-                           float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,
-                           size_t ws_bytes, void* stream) {
+vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void* k,
+                               const void* v, int64_t ld, const void* ctx_k, const void* ctx_v,
+                               int64_t ld_ctx, int m_ctx, int chunk_frames, int window_chunks,
+                               unsigned anchors, float scale, void* o, int64_t ld_o,
+                               float* lse_opt, void* ws, size_t ws_bytes, void* stream) {
   if (shape == nullptr || shape->T < 1 || shape->N < 1 || shape->H < 1 || shape->d < 1)
     return VDN_ERR_INVALID_ARG;
   const vdn_shape s = *shape;
@@ -569,6 +594,10 @@ vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k,
   if (s.d != 128 && s.d != 64) return VDN_ERR_UNSUPPORTED;
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   if (ld < D || ld % 8 || ld_o < D || ld_o % 8) return VDN_ERR_INVALID_ARG;
+  if (m_ctx < 0 || m_ctx >= (1 << 30)) return VDN_ERR_INVALID_ARG;
+  if (m_ctx > 0 && (ctx_k == nullptr || ctx_v == nullptr || !aligned16(ctx_k) ||
+                    !aligned16(ctx_v) || ld_ctx < D || ld_ctx % 8))
+    return VDN_ERR_INVALID_ARG;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kStatusBytes)
     return VDN_ERR_WORKSPACE;
   thread_local WinSched sched;  // ~12 KB; copied into the launch's parameters
@@ -576,18 +605,35 @@ vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k,
   if (static_cast<int64_t>(sched.total_tiles) * s.H >= (int64_t(1) << 31))
     return VDN_ERR_UNSUPPORTED;
   const int64_t L = static_cast<int64_t>(s.T) * s.N;
-  CUtensorMap qmap, kmap, vmap;
+  CUtensorMap qmap, kmap, vmap, ckmap, cvmap;
   if (!make_rows_map(&qmap, q, D, ld, L, 128) || !make_rows_map(&kmap, k, D, ld, L, 128) ||
       !make_rows_map(&vmap, v, D, ld, L, 128))
     return VDN_ERR_CUDA;
+  if (m_ctx > 0) {
+    if (!make_rows_map(&ckmap, ctx_k, D, ld_ctx, m_ctx, 128) ||
+        !make_rows_map(&cvmap, ctx_v, D, ld_ctx, m_ctx, 128))
+      return VDN_ERR_CUDA;
+  } else {
+    ckmap = kmap;  // unused
+    cvmap = vmap;
+  }
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(s.d));
   Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
              current_wait_budget_ns()};
-  cudaError_t e = s.d == 128 ? launch_window_dh<128>(ctx, s, qmap, kmap, vmap, sched, sc, o, ld_o,
-                                                     lse_opt)
-                             : launch_window_dh<64>(ctx, s, qmap, kmap, vmap, sched, sc, o, ld_o,
-                                                    lse_opt);
+  cudaError_t e = s.d == 128 ? launch_window_dh<128>(ctx, s, qmap, kmap, vmap, ckmap, cvmap, m_ctx,
+                                                     sched, sc, o, ld_o, lse_opt)
+                             : launch_window_dh<64>(ctx, s, qmap, kmap, vmap, ckmap, cvmap, m_ctx,
+                                                    sched, sc, o, ld_o, lse_opt);
   return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                           int64_t ld, int chunk_frames, int window_chunks, unsigned anchors,
+                           float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,
+                           size_t ws_bytes, void* stream) {
+  return vdn_window_attn_ctx(shape, q, k, v, ld, nullptr, nullptr, 0, 0, chunk_frames,
+                             window_chunks, anchors, scale, o, ld_o, lse_opt, ws, ws_bytes,
+                             stream);
 }
 
 }  // extern "C"

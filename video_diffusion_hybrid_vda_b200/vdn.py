@@ -24,7 +24,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_window_attn_workspace", "vdn_window_attn", "vdn_hybrid_fuse_workspace",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
-           "vdn_vda_scan_static", "vdn_selftest_exp2"]
+           "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx"]
 
 
 class VdnError(RuntimeError):
@@ -66,6 +66,10 @@ def lib():
     L.vdn_window_attn.argtypes = [S, _P, _P, _P, _I64, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_uint, ctypes.c_float, _P, _I64, _P, _P, _SZ, _P]
     L.vdn_window_attn.restype = ctypes.c_int
+    L.vdn_window_attn_ctx.argtypes = [S, _P, _P, _P, _I64, _P, _P, _I64, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_uint, ctypes.c_float,
+                                      _P, _I64, _P, _P, _SZ, _P]
+    L.vdn_window_attn_ctx.restype = ctypes.c_int
     L.vdn_hybrid_fuse_workspace.argtypes = [ctypes.c_int, ctypes.c_int]
     L.vdn_hybrid_fuse_workspace.restype = _SZ
     L.vdn_hybrid_fuse.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
@@ -197,19 +201,34 @@ def window_attn_workspace(T, N, H, d):
 
 
 def window_attn(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3, scale=0.0,
-                out=None, lse=None, ws=None, stream=None):
-    """Window-and-anchor Softmax.  Returns (o, ws); fills ``lse`` [H, T*N] if given."""
-    _need_cuda(q, k, v, out, lse, ws)
+                out=None, lse=None, ws=None, stream=None, ctx_k=None, ctx_v=None):
+    """Window-and-anchor Softmax.  Returns (o, ws); fills ``lse`` [H, T*N] if given.
+
+    ``ctx_k``/``ctx_v`` ([M, ld] bf16): context (text/audio) keys every video
+    query also attends to, in the same softmax.
+    """
+    _need_cuda(q, k, v, out, lse, ws, ctx_k, ctx_v)
     shape = _shape(T, N, H, d)
     if out is None:
         out = torch.empty((T * N, H * d), dtype=torch.bfloat16, device=q.device)
     if ws is None:
         ws = alloc_workspace(window_attn_workspace(T, N, H, d), q.device)
-    code = lib().vdn_window_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
-                                 int(chunk_frames), int(window_chunks), int(anchors),
-                                 float(scale), _ptr(out), out.stride(0), _ptr(lse), _ptr(ws),
-                                 ws.numel(), _stream(stream))
-    _check(code, "vdn_window_attn")
+    if ctx_k is None:
+        code = lib().vdn_window_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
+                                     int(chunk_frames), int(window_chunks), int(anchors),
+                                     float(scale), _ptr(out), out.stride(0), _ptr(lse), _ptr(ws),
+                                     ws.numel(), _stream(stream))
+        _check(code, "vdn_window_attn")
+    else:
+        if ctx_v is None or ctx_v.shape != ctx_k.shape or ctx_v.stride(0) != ctx_k.stride(0):
+            raise ValueError("ctx_k and ctx_v must have the same shape and row stride")
+        code = lib().vdn_window_attn_ctx(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                         q.stride(0), _ptr(ctx_k), _ptr(ctx_v), ctx_k.stride(0),
+                                         int(ctx_k.shape[0]), int(chunk_frames),
+                                         int(window_chunks), int(anchors), float(scale),
+                                         _ptr(out), out.stride(0), _ptr(lse), _ptr(ws),
+                                         ws.numel(), _stream(stream))
+        _check(code, "vdn_window_attn_ctx")
     return out, ws
 
 
@@ -280,12 +299,15 @@ class HybridLayer:
                 dst.copy_(src, non_blocking=True)
         return self._staging
 
-    def forward(self, q, k, v, beta, alpha, x, out=None, stream=None):
+    def forward(self, q, k, v, beta, alpha, x, out=None, stream=None, ctx_k=None, ctx_v=None):
+        """y for one video; ``ctx_k``/``ctx_v`` (CUDA, [M, D] bf16) are optional
+        text/audio keys the Softmax branch also attends to."""
         stream = stream or torch.cuda.current_stream(self.device)
         q, k, v, beta, alpha, x = self._to_device([q, k, v, beta, alpha, x], stream)
         T, N, H, d = self.T, self.N, self.H, self.d
         cf, wc, an = self.mask
-        window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win, stream=stream)
+        window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win, stream=stream,
+                    ctx_k=ctx_k, ctx_v=ctx_v)
         vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda, stream=stream)
         hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
                     self.W_ol, H, eps=self.eps, out=self.y, ws=self.ws_fuse, stream=stream)
