@@ -40,7 +40,8 @@
  *    returns VDN_ERR_CUDA.  Errors detected on the device (a non-positive
  *    Cholesky pivot or NaN, a wait that ran out of time) are OR-ed into the
  *    workspace status word; no kernel traps.
- *  - Supported head dims: d in {64, 128}.  N >= 1, T >= 1, H >= 1.
+ *  - Head dims: 64 and 128 run directly; 16 and 32 run on zero-padded
+ *    64-wide copies of every head in the workspace (exact).  N, T, H >= 1.
  */
 #ifndef VDN_H_
 #define VDN_H_
@@ -185,11 +186,14 @@ VDN_API vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, co
  * x, o_s, o_vda, y : [L, D] bf16, contiguous (ld = D), D = H*d
  * W_gs, W_gl, W_os, W_ol : [D, D] bf16 row-major, W[out][in] (y = z W^T)
  * gamma    : [D] fp32
- * ws       : >= vdn_hybrid_fuse_workspace(L, D) bytes (holds the gated
+ * ws       : >= vdn_hybrid_fuse_workspace(L, D, H) bytes (holds the gated
  *            branch outputs [L, 2D] bf16 between the two GEMMs)
- * D must be a multiple of 256 and d = D/H a multiple of 32; L >= 1.
+ * D must be a multiple of 8 and of H; L >= 1.  Hidden sizes that are not a
+ * multiple of 256, or head dims not a multiple of 32, run on zero-padded
+ * copies of every head in the workspace (exact; the RMS divides by the true
+ * head dim).
  * ------------------------------------------------------------------------ */
-VDN_API size_t vdn_hybrid_fuse_workspace(int L, int D);
+VDN_API size_t vdn_hybrid_fuse_workspace(int L, int D, int H);
 
 VDN_API vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
                            const void* o_vda, const void* W_gs, const void* W_gl,

@@ -48,7 +48,10 @@ def test_workspace_queries(L):
     assert lib.vdn_vda_scan_workspace(ctypes.byref(s)) == 256 + 6 * mat
     assert lib.vdn_vda_scan_workspace(None) == 0
     assert lib.vdn_vda_scan_workspace(ctypes.byref(L.Shape(0, 1, 1, 64))) == 0
-    assert lib.vdn_hybrid_fuse_workspace(411264, 3072) >= 411264 * 2 * 3072 * 2
+    assert lib.vdn_hybrid_fuse_workspace(411264, 3072, 24) == 256 + 411264 * 2 * 3072 * 2
+    # hidden 16 = 1 head x 16 runs on one head padded to 256 columns
+    assert lib.vdn_hybrid_fuse_workspace(160, 16, 1) > 160 * 2 * 256 * 2
+    assert lib.vdn_hybrid_fuse_workspace(160, 16, 3) == 0
 
 
 def _scan(L, shape, q=16, k=16, v=16, ld=128, beta=16, alpha=16, o=16, ld_o=128, states=None,
@@ -65,6 +68,7 @@ def test_vda_scan_rejects_bad_arguments_on_host(L):
     assert _scan(L, None) == 1
     assert _scan(L, L.Shape(0, 8, 1, 128)) == 1
     assert _scan(L, L.Shape(4, 8, 1, 96)) == 2                 # unsupported head dim
+    assert _scan(L, L.Shape(4, 8, 1, 48)) == 2
     assert _scan(L, ok, q=0) == 1                              # null pointer
     assert _scan(L, ok, k=24) == 1                             # misaligned
     assert _scan(L, ok, ld=100) == 1                           # ld % 8

@@ -19,6 +19,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "repack.cuh"
 
 namespace vdn {
 namespace {
@@ -37,7 +38,8 @@ struct GateArgs {
   const __nv_bfloat16* o_vda;
   const float* gamma;
   float eps;
-  int D, d;
+  int D, d;      // hidden size and head stride (columns per head)
+  float inv_d;   // 1 / (true head dim): the RMS divisor (padded columns are 0)
   __nv_bfloat16* Z;  // [M, 2D]
 };
 
@@ -97,7 +99,7 @@ __device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
 #pragma unroll
         for (int e = 0; e < 32; ++e) ss = fmaf(f[e], f[e], ss);
       }
-      rinv = rsqrtf(ss / static_cast<float>(a.d) + a.eps);
+      rinv = rsqrtf(ss * a.inv_d + a.eps);
     }
     float ov[32];
     load_bf16x32(orow + c, ov);
@@ -305,9 +307,43 @@ using namespace vdn;
 
 extern "C" {
 
-size_t vdn_hybrid_fuse_workspace(int L, int D) {
-  if (L < 1 || D < 1) return 0;
-  return kStatusBytes + static_cast<size_t>(L) * 2 * static_cast<size_t>(D) * 2;
+namespace {
+
+// Fuse layout.  Hidden sizes that 256-wide tiles divide, with head dims that
+// are multiples of 32, run as given: [status][Z].  Others run on heads padded
+// to dp columns (the smallest multiple of 32 >= d with H * dp a multiple of
+// 256): [status][Z][x' o_s' o_vda' y'][W_gs' W_gl' W_os' W_ol'][gamma'].
+struct FusePlan {
+  bool padded;
+  int d, dp, Dp;
+  size_t z, act, w, g, total;
+};
+
+size_t r256(size_t x) { return (x + 255) / 256 * 256; }
+
+FusePlan fuse_plan(int L, int D, int H) {
+  FusePlan p{};
+  p.d = D / H;
+  p.padded = (D % 256 != 0) || (p.d % 32 != 0);
+  p.dp = p.d;
+  if (p.padded) {
+    p.dp = (p.d + 31) / 32 * 32;
+    while ((static_cast<int64_t>(H) * p.dp) % 256 != 0) p.dp += 32;
+  }
+  p.Dp = H * p.dp;
+  p.z = r256(static_cast<size_t>(L) * 2 * p.Dp * 2);
+  p.act = p.padded ? r256(static_cast<size_t>(L) * p.Dp * 2) : 0;
+  p.w = p.padded ? r256(static_cast<size_t>(p.Dp) * p.Dp * 2) : 0;
+  p.g = p.padded ? r256(static_cast<size_t>(p.Dp) * 4) : 0;
+  p.total = kStatusBytes + p.z + 4 * p.act + 4 * p.w + p.g;
+  return p;
+}
+
+}  // namespace
+
+size_t vdn_hybrid_fuse_workspace(int L, int D, int H) {
+  if (L < 1 || D < 1 || H < 1 || D % H != 0) return 0;
+  return fuse_plan(L, D, H).total;
 }
 
 vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
@@ -321,28 +357,65 @@ vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
       !a16(W_ol) || !a16(y) || (reinterpret_cast<uintptr_t>(gamma) & 3u))
     return VDN_ERR_INVALID_ARG;
   if (!(eps >= 0.f)) return VDN_ERR_INVALID_ARG;
-  const int d = D / H;
-  if (D % 256 != 0 || d % 32 != 0) return VDN_ERR_UNSUPPORTED;
-  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
-      ws_bytes < vdn_hybrid_fuse_workspace(L, D))
+  if (D % 8 != 0) return VDN_ERR_UNSUPPORTED;  // rows must stay 16-byte aligned
+  const FusePlan pl = fuse_plan(L, D, H);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < pl.total)
     return VDN_ERR_WORKSPACE;
-  __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  uint8_t* base = static_cast<uint8_t*>(ws) + kStatusBytes;
+  __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int Dp = pl.Dp, d = pl.d, dp = pl.dp;
 
-  CUtensorMap xmap, wgs, wgl, zmap, wos, wol;
-  if (!make_rows_map(&xmap, x, D, D, L, BM) || !make_rows_map(&wgs, W_gs, D, D, D, BN) ||
-      !make_rows_map(&wgl, W_gl, D, D, D, BN) || !make_rows_map(&zmap, Z, 2 * D, 2 * D, L, BM) ||
-      !make_rows_map(&wos, W_os, D, D, D, BN) || !make_rows_map(&wol, W_ol, D, D, D, BN))
+  // operands of the two GEMMs: the caller's, or zero-padded copies per head
+  const void *xg = x, *osg = o_s, *ovg = o_vda, *wgs = W_gs, *wgl = W_gl, *wos = W_os,
+             *wol = W_ol;
+  const float* gg = gamma;
+  void* yg = y;
+  if (pl.padded) {
+    uint8_t* p = base + pl.z;
+    void* xp = p;
+    void* osp = p + pl.act;
+    void* ovp = p + 2 * pl.act;
+    void* yp = p + 3 * pl.act;
+    uint8_t* wp = p + 4 * pl.act;
+    float* gp = reinterpret_cast<float*>(wp + 4 * pl.w);
+    const void* wsrc[4] = {W_gs, W_gl, W_os, W_ol};
+    bool ok = launch_repack_bf16(st, xp, Dp, x, D, 1, L, L, H, dp, d) == cudaSuccess &&
+              launch_repack_bf16(st, osp, Dp, o_s, D, 1, L, L, H, dp, d) == cudaSuccess &&
+              launch_repack_bf16(st, ovp, Dp, o_vda, D, 1, L, L, H, dp, d) == cudaSuccess &&
+              launch_repack_f32(st, gp, Dp, gamma, D, 1, 1, 1, H, dp, d) == cudaSuccess;
+    for (int i = 0; i < 4 && ok; ++i)
+      ok = launch_repack_bf16(st, wp + i * pl.w, Dp, wsrc[i], D, H, dp, d, H, dp, d) ==
+           cudaSuccess;
+    if (!ok) return VDN_ERR_CUDA;
+    xg = xp;
+    osg = osp;
+    ovg = ovp;
+    yg = yp;
+    wgs = wp;
+    wgl = wp + pl.w;
+    wos = wp + 2 * pl.w;
+    wol = wp + 3 * pl.w;
+    gg = gp;
+  }
+
+  CUtensorMap xmap, m_gs, m_gl, zmap, m_os, m_ol;
+  if (!make_rows_map(&xmap, xg, Dp, Dp, L, BM) || !make_rows_map(&m_gs, wgs, Dp, Dp, Dp, BN) ||
+      !make_rows_map(&m_gl, wgl, Dp, Dp, Dp, BN) ||
+      !make_rows_map(&zmap, Z, 2 * Dp, 2 * Dp, L, BM) ||
+      !make_rows_map(&m_os, wos, Dp, Dp, Dp, BN) || !make_rows_map(&m_ol, wol, Dp, Dp, Dp, BN))
     return VDN_ERR_CUDA;
 
-  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
-             current_wait_budget_ns()};
+  Launch ctx{st, static_cast<uint32_t*>(ws), current_wait_budget_ns()};
   const int sms = sm_count_of_current_device();
-  GateArgs g{static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_vda),
-             gamma, eps, D, d, Z};
-  if (launch_gemm<BSplit::kByN>(ctx, xmap, wgs, wgl, L, 2 * D, D, D, g, sms) != cudaSuccess)
+  GateArgs g{static_cast<const __nv_bfloat16*>(osg), static_cast<const __nv_bfloat16*>(ovg),
+             gg, eps, Dp, dp, 1.f / static_cast<float>(d), Z};
+  if (launch_gemm<BSplit::kByN>(ctx, xmap, m_gs, m_gl, L, 2 * Dp, Dp, Dp, g, sms) != cudaSuccess)
     return VDN_ERR_CUDA;
-  StoreArgs st{static_cast<__nv_bfloat16*>(y)};
-  if (launch_gemm<BSplit::kByK>(ctx, zmap, wos, wol, L, D, 2 * D, D, st, sms) != cudaSuccess)
+  StoreArgs so{static_cast<__nv_bfloat16*>(yg)};
+  if (launch_gemm<BSplit::kByK>(ctx, zmap, m_os, m_ol, L, Dp, 2 * Dp, Dp, so, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (pl.padded && launch_repack_bf16(st, y, D, yg, Dp, 1, L, L, H, d, dp) != cudaSuccess)
     return VDN_ERR_CUDA;
   return VDN_OK;
 }

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "repack.cuh"
 
 namespace vdn {
 
@@ -48,7 +49,9 @@ bool shape_ok(const vdn_shape* s) {
          static_cast<int64_t>(s->H) * s->d < (int64_t(1) << 24);
 }
 
-bool head_dim_supported(int d) { return d == 64 || d == 128; }
+bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool head_dim_padded(int d) { return d == 16 || d == 32; }
 
 bool ld_ok(int64_t ld, int64_t D) { return ld >= D && ld % 8 == 0; }
 
@@ -68,6 +71,48 @@ VdaLayout vda_layout(const vdn_shape& s) {
   l.states = l.C + l.mat_bytes;
   l.total = l.states + 2 * l.mat_bytes;
   return l;
+}
+
+// Workspace of a VDA call.  Head dims 16 and 32 run through a 64-wide padded
+// copy: [status][q' k' v' o' bf16 L x H*64][A B P C S_fwd S_bwd for d = 64].
+struct VdaPlan {
+  bool padded;
+  vdn_shape inner;  // shape the kernels run on
+  size_t act;       // bytes of one padded activation
+  size_t inner_off; // where the d = 64 layout (after its status word) starts
+  VdaLayout lay;    // layout of the inner shape
+  size_t total;
+};
+
+VdaPlan vda_plan(const vdn_shape& s) {
+  VdaPlan p;
+  p.padded = head_dim_padded(s.d);
+  p.inner = s;
+  if (p.padded) p.inner.d = 64;
+  p.lay = vda_layout(p.inner);
+  p.act = p.padded ? round_up(static_cast<size_t>(s.T) * s.N * s.H * 64 * 2, 256) : 0;
+  p.inner_off = 4 * p.act;
+  p.total = p.lay.total + p.inner_off;
+  return p;
+}
+
+// The four VDA kernels on head dim 64 or 128.
+vdn_status run_vda(const Launch& ctx, const vdn_shape& s, const void* q, const void* k,
+                   const void* v, int64_t ld, const float* beta, const float* alpha, void* o,
+                   int64_t ld_o, float* A, float* B, float* P, float* C, float* states) {
+  const int64_t D = static_cast<int64_t>(s.H) * s.d;
+  const int prep_rows = s.d == 128 ? 32 : 64;
+  CUtensorMap kmap, vmap, qmap, omap;
+  if (!make_frame_map(&kmap, k, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&vmap, v, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&qmap, q, D, ld, s.N, s.T, 128) ||
+      !make_frame_map(&omap, o, D, ld_o, s.N, s.T, 128))
+    return VDN_ERR_CUDA;
+  if (launch_vda_prep(ctx, s, kmap, vmap, beta, A, B) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
+  return VDN_OK;
 }
 
 }  // namespace
@@ -148,18 +193,18 @@ vdn_status vdn_get_device_status(const void* ws, void* stream) {
 
 size_t vdn_vda_scan_workspace(const vdn_shape* shape) {
   if (!shape_ok(shape)) return 0;
-  return vda_layout(*shape).total;
+  return vda_plan(*shape).total;
 }
 
 vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
                                  float** P, float** C) {
   if (!shape_ok(shape) || ws == nullptr) return VDN_ERR_INVALID_ARG;
-  const VdaLayout l = vda_layout(*shape);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  if (A) *A = reinterpret_cast<float*>(base + l.A);
-  if (B) *B = reinterpret_cast<float*>(base + l.B);
-  if (P) *P = reinterpret_cast<float*>(base + l.P);
-  if (C) *C = reinterpret_cast<float*>(base + l.C);
+  const VdaPlan pl = vda_plan(*shape);
+  uint8_t* base = static_cast<uint8_t*>(ws) + pl.inner_off;
+  if (A) *A = reinterpret_cast<float*>(base + pl.lay.A);
+  if (B) *B = reinterpret_cast<float*>(base + pl.lay.B);
+  if (P) *P = reinterpret_cast<float*>(base + pl.lay.P);
+  if (C) *C = reinterpret_cast<float*>(base + pl.lay.C);
   return VDN_OK;
 }
 
@@ -178,30 +223,43 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
       !aligned(beta, 4) || !aligned(alpha, 4) || (states_opt && !aligned(states_opt, 16)))
     return VDN_ERR_INVALID_ARG;
   if (!ld_ok(ld, D) || !ld_ok(ld_o, D)) return VDN_ERR_INVALID_ARG;
-  const VdaLayout l = vda_layout(s);
-  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < l.total) return VDN_ERR_WORKSPACE;
+  const VdaPlan pl = vda_plan(s);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < pl.total) return VDN_ERR_WORKSPACE;
 
   uint8_t* base = static_cast<uint8_t*>(ws);
-  float* A = reinterpret_cast<float*>(base + l.A);
-  float* B = reinterpret_cast<float*>(base + l.B);
-  float* P = reinterpret_cast<float*>(base + l.P);
-  float* C = reinterpret_cast<float*>(base + l.C);
-  float* states = states_opt ? states_opt : reinterpret_cast<float*>(base + l.states);
-
-  const int prep_rows = s.d == 128 ? 32 : 64;
-  CUtensorMap kmap, vmap, qmap, omap;
-  if (!make_frame_map(&kmap, k, D, ld, s.N, s.T, prep_rows) ||
-      !make_frame_map(&vmap, v, D, ld, s.N, s.T, prep_rows) ||
-      !make_frame_map(&qmap, q, D, ld, s.N, s.T, 128) ||
-      !make_frame_map(&omap, o_vda, D, ld_o, s.N, s.T, 128))
-    return VDN_ERR_CUDA;
-
+  uint8_t* inner = base + pl.inner_off;
+  float* A = reinterpret_cast<float*>(inner + pl.lay.A);
+  float* B = reinterpret_cast<float*>(inner + pl.lay.B);
+  float* P = reinterpret_cast<float*>(inner + pl.lay.P);
+  float* C = reinterpret_cast<float*>(inner + pl.lay.C);
+  float* states_ws = reinterpret_cast<float*>(inner + pl.lay.states);
   Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
              g_budget_ns.load()};
-  if (launch_vda_prep(ctx, s, kmap, vmap, beta, A, B) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
+  if (!pl.padded)
+    return run_vda(ctx, s, q, k, v, ld, beta, alpha, o_vda, ld_o, A, B, P, C,
+                   states_opt ? states_opt : states_ws);
+
+  // d = 16 or 32: run on a zero-padded 64-wide copy of every head
+  const int L = s.T * s.N, H = s.H, d = s.d;
+  const int64_t D64 = static_cast<int64_t>(H) * 64;
+  uint8_t* qp = base + kStatusBytes;
+  uint8_t* kp = qp + pl.act;
+  uint8_t* vp = kp + pl.act;
+  uint8_t* op = vp + pl.act;
+  cudaStream_t st = ctx.stream;
+  if (launch_repack_bf16(st, qp, D64, q, ld, 1, L, L, H, 64, d) != cudaSuccess ||
+      launch_repack_bf16(st, kp, D64, k, ld, 1, L, L, H, 64, d) != cudaSuccess ||
+      launch_repack_bf16(st, vp, D64, v, ld, 1, L, L, H, 64, d) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  const vdn_status r =
+      run_vda(ctx, pl.inner, qp, kp, vp, D64, beta, alpha, op, D64, A, B, P, C, states_ws);
+  if (r != VDN_OK) return r;
+  if (launch_repack_bf16(st, o_vda, ld_o, op, D64, 1, L, L, H, d, 64) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (states_opt != nullptr &&
+      launch_repack_f32(st, states_opt, d, states_ws, 64, 2 * s.T * H, d, 64, 1, d, 64) !=
+          cudaSuccess)
+    return VDN_ERR_CUDA;
   return VDN_OK;
 }
 

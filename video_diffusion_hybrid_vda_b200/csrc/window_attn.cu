@@ -32,6 +32,7 @@
 #include "common.cuh"
 #include "exp2_fma.cuh"
 #include "ptx.cuh"
+#include "repack.cuh"
 
 namespace vdn {
 
@@ -572,8 +573,15 @@ using namespace vdn;
 
 extern "C" {
 
+// Head dims 16 and 32 run on a zero-padded 64-wide copy of q, k, v and o
+// kept in the workspace after the status word.
+static size_t window_padded_act_bytes(const vdn_shape& s) {
+  return (static_cast<size_t>(s.T) * s.N * s.H * 64 * 2 + 255) / 256 * 256;
+}
+
 size_t vdn_window_attn_workspace(const vdn_shape* shape) {
   if (shape == nullptr || shape->T < 1 || shape->N < 1 || shape->H < 1 || shape->d < 1) return 0;
+  if (shape->d == 16 || shape->d == 32) return kStatusBytes + 4 * window_padded_act_bytes(*shape);
   return kStatusBytes;
 }
 
@@ -591,15 +599,45 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
       (lse_opt && (reinterpret_cast<uintptr_t>(lse_opt) & 3u)))
     return VDN_ERR_INVALID_ARG;
   if (chunk_frames < 1 || window_chunks < 0 || anchors > 3u) return VDN_ERR_INVALID_ARG;
-  if (s.d != 128 && s.d != 64) return VDN_ERR_UNSUPPORTED;
+  const bool padded = s.d == 16 || s.d == 32;
+  if (s.d != 128 && s.d != 64 && !padded) return VDN_ERR_UNSUPPORTED;
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   if (ld < D || ld % 8 || ld_o < D || ld_o % 8) return VDN_ERR_INVALID_ARG;
   if (m_ctx < 0 || m_ctx >= (1 << 30)) return VDN_ERR_INVALID_ARG;
   if (m_ctx > 0 && (ctx_k == nullptr || ctx_v == nullptr || !aligned16(ctx_k) ||
                     !aligned16(ctx_v) || ld_ctx < D || ld_ctx % 8))
     return VDN_ERR_INVALID_ARG;
-  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kStatusBytes)
+  if (m_ctx > 0 && padded) return VDN_ERR_UNSUPPORTED;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      ws_bytes < vdn_window_attn_workspace(shape))
     return VDN_ERR_WORKSPACE;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(s.d));
+  if (padded) {
+    // run on zero-padded 64-wide heads (exact: padded dims add nothing to a
+    // score and give zero output columns), then copy the real columns back
+    const int L = s.T * s.N;
+    const int64_t D64 = static_cast<int64_t>(s.H) * 64;
+    const size_t act = window_padded_act_bytes(s);
+    uint8_t* qp = static_cast<uint8_t*>(ws) + kStatusBytes;
+    uint8_t* kp = qp + act;
+    uint8_t* vp = kp + act;
+    uint8_t* op = vp + act;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (launch_repack_bf16(st, qp, D64, q, ld, 1, L, L, s.H, 64, s.d) != cudaSuccess ||
+        launch_repack_bf16(st, kp, D64, k, ld, 1, L, L, s.H, 64, s.d) != cudaSuccess ||
+        launch_repack_bf16(st, vp, D64, v, ld, 1, L, L, s.H, 64, s.d) != cudaSuccess)
+      return VDN_ERR_CUDA;
+    vdn_shape s64 = s;
+    s64.d = 64;
+    // the inner call sees a workspace that is just this call's status word
+    const vdn_status r = vdn_window_attn_ctx(&s64, qp, kp, vp, D64, nullptr, nullptr, 0, 0,
+                                             chunk_frames, window_chunks, anchors, sc, op, D64,
+                                             lse_opt, ws, kStatusBytes, stream);
+    if (r != VDN_OK) return r;
+    if (launch_repack_bf16(st, o, ld_o, op, D64, 1, L, L, s.H, s.d, 64) != cudaSuccess)
+      return VDN_ERR_CUDA;
+    return VDN_OK;
+  }
   thread_local WinSched sched;  // ~12 KB; copied into the launch's parameters
   if (!build_schedule(s, chunk_frames, window_chunks, anchors, &sched)) return VDN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(sched.total_tiles) * s.H >= (int64_t(1) << 31))
@@ -617,7 +655,6 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
     ckmap = kmap;  // unused
     cvmap = vmap;
   }
-  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(s.d));
   Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
              current_wait_budget_ns()};
   cudaError_t e = s.d == 128 ? launch_window_dh<128>(ctx, s, qmap, kmap, vmap, ckmap, cvmap, m_ctx,

@@ -70,7 +70,7 @@ def lib():
                                       ctypes.c_int, ctypes.c_int, ctypes.c_uint, ctypes.c_float,
                                       _P, _I64, _P, _P, _SZ, _P]
     L.vdn_window_attn_ctx.restype = ctypes.c_int
-    L.vdn_hybrid_fuse_workspace.argtypes = [ctypes.c_int, ctypes.c_int]
+    L.vdn_hybrid_fuse_workspace.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.vdn_hybrid_fuse_workspace.restype = _SZ
     L.vdn_hybrid_fuse.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
                                   _P, ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
@@ -234,8 +234,8 @@ def window_attn(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3,
 
 # ---------------------------------------------------------------- fuse
 
-def hybrid_fuse_workspace(L, D):
-    return int(lib().vdn_hybrid_fuse_workspace(int(L), int(D)))
+def hybrid_fuse_workspace(L, D, H):
+    return int(lib().vdn_hybrid_fuse_workspace(int(L), int(D), int(H)))
 
 
 def hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, H, eps=1e-6, out=None, ws=None,
@@ -246,7 +246,7 @@ def hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, H, eps=1e-6, out=N
     if out is None:
         out = torch.empty((L, D), dtype=torch.bfloat16, device=x.device)
     if ws is None:
-        ws = alloc_workspace(hybrid_fuse_workspace(L, D), x.device)
+        ws = alloc_workspace(hybrid_fuse_workspace(L, D, H), x.device)
     code = lib().vdn_hybrid_fuse(int(L), int(D), int(H), _ptr(x), _ptr(o_s), _ptr(o_vda),
                                  _ptr(W_gs), _ptr(W_gl), _ptr(gamma), float(eps), _ptr(W_os),
                                  _ptr(W_ol), _ptr(out), _ptr(ws), ws.numel(), _stream(stream))
@@ -285,7 +285,7 @@ class HybridLayer:
         self.y = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
         self.ws_vda = alloc_workspace(vda_scan_workspace(T, N, H, d), dev)
         self.ws_win = alloc_workspace(window_attn_workspace(T, N, H, d), dev)
-        self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D), dev)
+        self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D, H), dev)
         self._staging = None
 
     def _to_device(self, tensors, stream):
