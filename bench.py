@@ -40,6 +40,9 @@ WORKLOADS = {
 }
 METRIC = "VDN hybrid attn layer ms & tokens/s at 102 latent frames; % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# FP32 (non-tensor) peak from unit counts and clocks: 148 SMs x 128 FMA/clk x
+# 2 FLOP x 1.965 GHz (clocks.max.sm)
+FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 KERNEL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "window_attn_traffic.json")
 
 
@@ -61,8 +64,9 @@ def work_model(s):
     proj_flop = 4 * 2 * s.L * s.D * s.D                 # gate GEMMs + output GEMMs
     # VDA HBM bytes: prep reads k, v (bf16) and beta; read-out reads q, writes o
     vda_bytes = 2 * s.L * s.D * 2 + s.L * s.H * 4 + 2 * s.L * s.D * 2
-    # FP32 ALU work of the solve (~3 d^3) and the scan (2 x 2 d^3 per frame)
-    vda_alu_flop = s.T * s.H * (3 * s.d ** 3 + 4 * s.d ** 3) * 2
+    # FP32 ALU work in FLOP per (frame, head): Cholesky d^3/3, W = L^-1 d^3/3,
+    # P = W^T W and C = B P 2 d^3 each, and both scans a 2 d^3 product each
+    vda_alu_flop = s.T * s.H * (2 * s.d ** 3 // 3 + 4 * s.d ** 3 + 4 * s.d ** 3)
     return dict(pairs=pairs, softmax_flop=softmax_flop, proj_flop=proj_flop,
                 vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop)
 
@@ -180,6 +184,8 @@ def oracle_sample(shape, seed=0, vda_heads=2, frames=None, rows_per_frame=128):
 
 def run_gpu(args, shape, rank, world):
     from video_diffusion_hybrid_vda_b200 import vdn
+    vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN if args.solver == "gauss-jordan"
+                       else vdn.SOLVER_CHOLESKY)
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(shape, seed=rank, device=dev, with_fuse=True)
@@ -188,20 +194,25 @@ def run_gpu(args, shape, rank, world):
     acts = [inp[k] for k in ("q", "k", "v", "beta", "alpha", "x")]
     stream = torch.cuda.current_stream(dev)
 
-    def step(timed_win=None):
+    def step(ev=None):
+        """One layer pass; ``ev`` = 4 events bracketing the three C-ABI calls."""
         q, k, v, beta, alpha, x = acts
         cf, wc, an = layer.mask
-        if timed_win is not None:
-            timed_win[0].record(stream)
+        if ev is not None:
+            ev[0].record(stream)
         vdn.window_attn(q, k, v, shape.T, shape.N, shape.H, shape.d, cf, wc, an,
                         out=layer.o_s, ws=layer.ws_win, stream=stream)
-        if timed_win is not None:
-            timed_win[1].record(stream)
+        if ev is not None:
+            ev[1].record(stream)
         vdn.vda_scan(q, k, v, beta, alpha, shape.T, shape.N, shape.H, shape.d,
                      out=layer.o_vda, ws=layer.ws_vda, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
         vdn.hybrid_fuse(x, layer.o_s, layer.o_vda, layer.W_gs, layer.W_gl, layer.gamma,
                         layer.W_os, layer.W_ol, shape.H, out=layer.y, ws=layer.ws_fuse,
                         stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -214,19 +225,21 @@ def run_gpu(args, shape, rank, world):
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    win_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                  for _ in range(args.steps)]
+    call_events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+                   for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = clocks_start()
     barrier()
     start.record(stream)
     for i in range(args.steps):
-        step(win_events[i])
+        step(call_events[i])
     end.record(stream)
     barrier()
     clocks = clocks_stop(clk)
     ms = start.elapsed_time(end)
-    win_ms = [a.elapsed_time(b) for a, b in win_events]
+    win_ms = [e[0].elapsed_time(e[1]) for e in call_events]
+    vda_ms = [e[1].elapsed_time(e[2]) for e in call_events]
+    fuse_ms = [e[2].elapsed_time(e[3]) for e in call_events]
     status = layer.status()
     if status != 0:
         raise RuntimeError("device status after timed steps: %d" % status)
@@ -249,13 +262,14 @@ def run_gpu(args, shape, rank, world):
     if layer.status() != 0:
         raise RuntimeError("device status after end-to-end steps")
 
+    t = [ms, e2e_ms, sum(win_ms), sum(vda_ms), sum(fuse_ms)]
     if world > 1:
-        t = torch.tensor([ms, e2e_ms, sum(win_ms)], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms, win_total = t.tolist()
-    else:
-        win_total = sum(win_ms)
-    return dict(ms=ms, win_ms=win_total / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+        tt = torch.tensor(t, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        t = tt.tolist()
+    ms, e2e_ms = t[0], t[1]
+    return dict(ms=ms, win_ms=t[2] / args.steps, vda_ms=t[3] / args.steps,
+                fuse_ms=t[4] / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
                 clocks=clocks, launches=layer.KERNELS_PER_FORWARD * args.steps)
 
 
@@ -267,6 +281,8 @@ def main():
     ap.add_argument("--impl", default="vdn", choices=["vdn", "reference"])
     ap.add_argument("--workload", default="layer102", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
+                    help="solver of (I + A)^-1 in the VDA branch")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -277,6 +293,7 @@ def main():
               "heads": shape.H, "head_dim": shape.d, "hidden": shape.D, "tokens": shape.L,
               "mask": "chunk 5, +-1 chunk, first/last-frame anchors",
               "global_batch": world, "parallelism": f"independent videos x{world}",
+              "vda_solver": args.solver,
               "l2": "inputs larger than L2 (2.5 GB per activation), no flush"}
 
     if args.impl == "reference":
@@ -335,6 +352,20 @@ def main():
         "layer_roofline": {"ms": roof_ms, "frac": roof_ms / ms_step,
                            "terms": "softmax + projections at sustained bf16 peak, VDA bytes "
                                     "at measured HBM"},
+        "rows": {
+            "window_softmax": {"ms": r["win_ms"], "bound": "tensor",
+                               "frac": (work["softmax_flop"] / (peak * 1e12) * 1e3) / r["win_ms"]},
+            "vda_prep_solve_scan_readout": {
+                "ms": r["vda_ms"], "bound": "hbm + fp32 alu",
+                "roofline_ms": (work["vda_bytes"] / (peaks["hbm_gbs"] * 1e9) +
+                                work["vda_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3,
+                "frac": ((work["vda_bytes"] / (peaks["hbm_gbs"] * 1e9) +
+                          work["vda_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3) / r["vda_ms"]},
+            "fuse_gemms": {"ms": r["fuse_ms"], "bound": "tensor",
+                           "achieved_tflops": work["proj_flop"] / (r["fuse_ms"] / 1e3) / 1e12,
+                           "frac": (work["proj_flop"] / (peak * 1e12) * 1e3) / r["fuse_ms"]},
+            "fp32_peak_tflops": FP32_TFLOPS,
+        },
         "e2e": {"value": world * shape.L / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "ms_per_step": r["e2e_ms"]},

@@ -173,3 +173,36 @@ def test_vda_timeout_path_reports_and_recovers(vdn):
     x = {k: host(v) for k, v in inp.items()}
     o_ref, _, _ = oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], *shape_args(shape))
     assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16
+
+
+@pytest.mark.parametrize("T,N,H,d", [(7, 200, 2, 128), (17, 33, 2, 64), (3, 4032, 1, 128)])
+def test_vda_gauss_jordan_solver(vdn, T, N, H, d):
+    """The Gauss-Jordan variant of the solve: P and C against the GPU's own
+    symmetrised A, states and o_vda against the oracle."""
+    shape = synth.Shape(T, N, H, d)
+    inp = _inputs(shape, seed=T * 1000 + N + 1)
+    try:
+        vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN)
+        o, states, ws = _run(vdn, shape, inp)
+    finally:
+        vdn.set_vda_solver(vdn.SOLVER_CHOLESKY)
+    x = {k: host(v) for k, v in inp.items()}
+    A, B, P, C = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
+    for t in range(T):
+        for h in range(H):
+            A_sym = 0.5 * (A[t, h].astype(np.float64) + A[t, h].T.astype(np.float64))
+            P_ref = np.linalg.inv(np.eye(d) + A_sym)
+            assert max_rel(P[t, h], P_ref) <= TOL_SOLVE, ("P", t, h)
+            assert max_rel(C[t, h], B[t, h].astype(np.float64) @ P_ref) <= TOL_SOLVE, ("C", t, h)
+    o_ref, S_fwd, S_bwd = oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], T, N, H, d)
+    st = host(states)
+    for t in range(T):
+        for h in range(H):
+            assert max_rel(st[0, t, h], S_fwd[t, h]) <= TOL_STATE
+            assert max_rel(st[1, t, h], S_bwd[t, h]) <= TOL_STATE
+    assert per_head_max_rel(host(o), o_ref, H, d) <= TOL_BF16
+
+
+def test_vda_solver_rejects_unknown(vdn):
+    with pytest.raises(vdn.VdnError):
+        vdn.set_vda_solver(7)

@@ -62,7 +62,7 @@ def build(force=False, verbose=False, jobs=None):
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))
     tmp = LIB + ".tmp"
-    subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs])
+    subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-ldl"])
     os.replace(tmp, LIB)
     return LIB
 

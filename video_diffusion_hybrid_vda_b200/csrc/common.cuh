@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/vdn.h"
 
 namespace vdn {
@@ -20,6 +22,14 @@ __device__ __forceinline__ void record_status(uint32_t* status, uint32_t bits) {
   if (status != nullptr) atomicOr(status, bits);
 }
 
+// NVTX range around a C-ABI call (a no-op unless a profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Launch context handed to every launcher.
 struct Launch {
   cudaStream_t stream;
@@ -29,6 +39,9 @@ struct Launch {
 
 // Budget (ns) of the bounded device waits, set by vdn_set_wait_budget_ns.
 uint64_t current_wait_budget_ns();
+
+// Solver of the VDA closed form, set by vdn_set_vda_solver.
+int current_vda_solver();
 
 // ---- tensor maps (built on the host with the driver's encoder) ----------
 

@@ -350,6 +350,7 @@ vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const void* o_s,
                            const void* o_vda, const void* W_gs, const void* W_gl,
                            const float* gamma, float eps, const void* W_os, const void* W_ol,
                            void* y, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("vdn_hybrid_fuse");
   if (L < 1 || D < 1 || H < 1 || D % H != 0) return VDN_ERR_INVALID_ARG;
   if (!x || !o_s || !o_vda || !W_gs || !W_gl || !gamma || !W_os || !W_ol || !y)
     return VDN_ERR_INVALID_ARG;

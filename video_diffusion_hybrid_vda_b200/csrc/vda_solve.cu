@@ -56,6 +56,151 @@ __device__ __forceinline__ void publish_row(float (&r)[RA][RG][4], int ka, float
   }
 }
 
+// C = B P for one (frame, head): B staged through shared memory `Bs`, P
+// already in shared memory `Ps` (both [DH][LD2]); each of the 512 threads
+// computes a (DH/32) x (DH/16) tile.  Caller synchronises before the call.
+template <int DH>
+__device__ __forceinline__ void c_equals_b_times_p(const float* __restrict__ Bm, const float* Ps,
+                                                   float* Bs, float* __restrict__ Cm) {
+  using Cfg = SolveCfg<DH>;
+  constexpr int PR = DH / 32, PC = DH / 16;
+  const int i0 = (threadIdx.x >> 4) * PR, c0 = (threadIdx.x & 15) * PC;
+  for (int idx = threadIdx.x; idx < DH * DH / 4; idx += kSolveThreads) {
+    const int rr = idx / (DH / 4), cc = idx % (DH / 4);
+    *reinterpret_cast<float4*>(Bs + rr * Cfg::LD2 + 4 * cc) =
+        __ldg(reinterpret_cast<const float4*>(Bm) + idx);
+  }
+  __syncthreads();
+  float acc[PR][PC];
+#pragma unroll
+  for (int a = 0; a < PR; ++a)
+#pragma unroll
+    for (int b = 0; b < PC; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < DH; k += 4) {
+    float bv[PR][4];
+#pragma unroll
+    for (int a = 0; a < PR; ++a) {
+      const float4 v = *reinterpret_cast<const float4*>(Bs + (i0 + a) * Cfg::LD2 + k);
+      bv[a][0] = v.x; bv[a][1] = v.y; bv[a][2] = v.z; bv[a][3] = v.w;
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      float pc[PC];
+#pragma unroll
+      for (int b = 0; b < PC; b += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(Ps + (k + kk) * Cfg::LD2 + c0 + b);
+        pc[b] = v.x; pc[b + 1] = v.y; pc[b + 2] = v.z; pc[b + 3] = v.w;
+      }
+#pragma unroll
+      for (int a = 0; a < PR; ++a)
+#pragma unroll
+        for (int b = 0; b < PC; ++b) acc[a][b] = fmaf(bv[a][kk], pc[b], acc[a][b]);
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < PR; ++a)
+#pragma unroll
+    for (int b = 0; b < PC; b += 4)
+      *reinterpret_cast<float4*>(Cm + (i0 + a) * DH + c0 + b) =
+          make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+}
+
+// Gauss-Jordan variant (the inverse the pages' own kernels use): one sweep
+// over the pivots p = 0..d-1 of the symmetric positive definite I + A_sym,
+// with the whole matrix in registers (4x8 per thread, d = 128).  Each step
+// publishes pivot row p and pivot column p through shared memory and applies
+//   M[p][p] <- 1/piv,  M[p][k] <- M[p][k]/piv,  M[i][p] <- -M[i][p]/piv,
+//   M[i][k] <- M[i][k] - M[i][p] M[p][k] / piv          (i, k != p),
+// which leaves (I + A)^-1 after the last pivot.  No pivoting is needed: the
+// pivots are Schur-complement diagonals of an SPD matrix with eigenvalues
+// >= 1.  Then C = B P as in the Cholesky kernel.
+template <int DH>
+__global__ void __launch_bounds__(kSolveThreads, 1)
+    vda_solve_gj_kernel(const float* __restrict__ A, const float* __restrict__ B,
+                        float* __restrict__ P, float* __restrict__ Cout, uint32_t* status) {
+  using Cfg = SolveCfg<DH>;
+  extern __shared__ float sm[];
+  float* Ws = sm;                    // [DH][LD2]: B for the C product
+  float* Xs = sm + Cfg::MAT;         // [DH][LD2]: P
+  float* rowb = sm + 2 * Cfg::MAT;   // 2 x [DH] pivot rows
+  float* colb = rowb + 2 * DH;       // 2 x [DH] pivot columns
+  const int tx = threadIdx.x & 15;
+  const int ty = threadIdx.x >> 4;
+  const int64_t mat = static_cast<int64_t>(blockIdx.x) * DH * DH;
+  const float* Am = A + mat;
+  bool bad = false;
+
+  float m[Cfg::RA][Cfg::CB];
+#pragma unroll
+  for (int a = 0; a < Cfg::RA; ++a)
+#pragma unroll
+    for (int b = 0; b < Cfg::CB; ++b) {
+      const int i = ty + 32 * a, k = tx + 16 * b;
+      m[a][b] = 0.5f * (__ldg(Am + i * DH + k) + __ldg(Am + k * DH + i)) + (i == k ? 1.f : 0.f);
+    }
+#pragma unroll 1
+  for (int p = 0; p < DH; ++p) {
+    float* rb = rowb + (p & 1) * DH;
+    float* cb = colb + (p & 1) * DH;
+    if (ty == (p & 31)) {  // owners of row p
+      const int pa = p >> 5;
+#pragma unroll
+      for (int b = 0; b < Cfg::CB; ++b) {
+        float v = m[0][b];
+#pragma unroll
+        for (int a = 1; a < Cfg::RA; ++a) v = (a == pa) ? m[a][b] : v;
+        rb[tx + 16 * b] = v;
+      }
+    }
+    if (tx == (p & 15)) {  // owners of column p
+      const int pb = p >> 4;
+#pragma unroll
+      for (int a = 0; a < Cfg::RA; ++a) {
+        float v = m[a][0];
+#pragma unroll
+        for (int b = 1; b < Cfg::CB; ++b) v = (b == pb) ? m[a][b] : v;
+        cb[ty + 32 * a] = v;
+      }
+    }
+    __syncthreads();
+    float piv = rb[p];
+    if (!(piv > 0.f)) {  // also catches NaN
+      bad = true;
+      piv = 1.f;
+    }
+    const float inv = 1.f / piv;
+    float fi[Cfg::RA], rk[Cfg::CB];
+#pragma unroll
+    for (int a = 0; a < Cfg::RA; ++a) fi[a] = cb[ty + 32 * a] * inv;
+#pragma unroll
+    for (int b = 0; b < Cfg::CB; ++b) rk[b] = rb[tx + 16 * b];
+#pragma unroll
+    for (int a = 0; a < Cfg::RA; ++a) {
+      const int i = ty + 32 * a;
+#pragma unroll
+      for (int b = 0; b < Cfg::CB; ++b) {
+        const int k = tx + 16 * b;
+        const float upd = fmaf(-fi[a], rk[b], m[a][b]);
+        const float rowp = (k == p) ? inv : rk[b] * inv;
+        m[a][b] = (i == p) ? rowp : ((k == p) ? -fi[a] : upd);
+      }
+    }
+    // one barrier per step: the next step writes the other buffer pair
+  }
+#pragma unroll
+  for (int a = 0; a < Cfg::RA; ++a)
+#pragma unroll
+    for (int b = 0; b < Cfg::CB; ++b) {
+      const int i = ty + 32 * a, k = tx + 16 * b;
+      Xs[i * Cfg::LD2 + k] = m[a][b];
+      P[mat + i * DH + k] = m[a][b];
+    }
+  __syncthreads();
+  c_equals_b_times_p<DH>(B + mat, Xs, Ws, Cout + mat);
+  if (bad) record_status(status, kStatusNumeric);
+}
+
 template <int DH>
 __global__ void __launch_bounds__(kSolveThreads, 1)
     vda_solve_kernel(const float* __restrict__ A, const float* __restrict__ B,
@@ -223,61 +368,29 @@ __global__ void __launch_bounds__(kSolveThreads, 1)
   __syncthreads();  // P complete in Xs; W no longer needed: its buffer takes B
 
   // ---------------------------------------------------------------- phase 4
-  // C = B P (B rows staged through shared memory).
-  for (int idx = threadIdx.x; idx < DH * DH / 4; idx += kSolveThreads) {
-    const int rr = idx / (DH / 4), cc = idx % (DH / 4);
-    *reinterpret_cast<float4*>(Ws + rr * Cfg::LD2 + 4 * cc) =
-        __ldg(reinterpret_cast<const float4*>(Bm) + idx);
-  }
-  __syncthreads();
-#pragma unroll
-  for (int a = 0; a < PR; ++a)
-#pragma unroll
-    for (int b = 0; b < PC; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-  for (int k = 0; k < DH; k += 4) {
-    float bv[PR][4];
-#pragma unroll
-    for (int a = 0; a < PR; ++a) {
-      const float4 v = *reinterpret_cast<const float4*>(Ws + (i0 + a) * Cfg::LD2 + k);
-      bv[a][0] = v.x; bv[a][1] = v.y; bv[a][2] = v.z; bv[a][3] = v.w;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      float pc[PC];
-#pragma unroll
-      for (int b = 0; b < PC; b += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(Xs + (k + kk) * Cfg::LD2 + c0 + b);
-        pc[b] = v.x; pc[b + 1] = v.y; pc[b + 2] = v.z; pc[b + 3] = v.w;
-      }
-#pragma unroll
-      for (int a = 0; a < PR; ++a)
-#pragma unroll
-        for (int b = 0; b < PC; ++b) acc[a][b] = fmaf(bv[a][kk], pc[b], acc[a][b]);
-    }
-  }
-  float* Cm = Cout + mat;
-#pragma unroll
-  for (int a = 0; a < PR; ++a)
-#pragma unroll
-    for (int b = 0; b < PC; b += 4)
-      *reinterpret_cast<float4*>(Cm + (i0 + a) * DH + c0 + b) =
-          make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+  c_equals_b_times_p<DH>(Bm, Xs, Ws, Cout + mat);
   if (bad) record_status(status, kStatusNumeric);
 }
 
 template <int DH>
 cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* A,
-                            const float* B, float* P, float* C) {
+                            const float* B, float* P, float* C, int solver) {
   using Cfg = SolveCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(vda_solve_kernel<DH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(vda_solve_gj_kernel<DH>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  vda_solve_kernel<DH><<<s.T * s.H, kSolveThreads, Cfg::SMEM, ctx.stream>>>(A, B, P, C,
+  if (solver == VDN_SOLVER_GAUSS_JORDAN)
+    vda_solve_gj_kernel<DH><<<s.T * s.H, kSolveThreads, Cfg::SMEM, ctx.stream>>>(A, B, P, C,
+                                                                                ctx.status);
+  else
+    vda_solve_kernel<DH><<<s.T * s.H, kSolveThreads, Cfg::SMEM, ctx.stream>>>(A, B, P, C,
                                                                              ctx.status);
   return cudaGetLastError();
 }
@@ -286,8 +399,9 @@ cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* 
 
 cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A,
                              const float* B, float* P, float* C) {
-  if (s.d == 128) return launch_solve_dh<128>(ctx, s, A, B, P, C);
-  if (s.d == 64) return launch_solve_dh<64>(ctx, s, A, B, P, C);
+  const int solver = current_vda_solver();
+  if (s.d == 128) return launch_solve_dh<128>(ctx, s, A, B, P, C, solver);
+  if (s.d == 64) return launch_solve_dh<64>(ctx, s, A, B, P, C, solver);
   return cudaErrorInvalidValue;
 }
 

@@ -19,6 +19,7 @@ namespace vdn {
 namespace {
 
 std::atomic<uint64_t> g_budget_ns{2000000000ull};
+std::atomic<int> g_solver{VDN_SOLVER_CHOLESKY};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -119,6 +120,8 @@ vdn_status run_vda(const Launch& ctx, const vdn_shape& s, const void* q, const v
 
 uint64_t current_wait_budget_ns() { return g_budget_ns.load(); }
 
+int current_vda_solver() { return g_solver.load(); }
+
 bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int N, int T,
                     int box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -170,6 +173,13 @@ const char* vdn_status_string(vdn_status s) {
 
 void vdn_set_wait_budget_ns(uint64_t ns) { g_budget_ns.store(ns); }
 
+vdn_status vdn_set_vda_solver(int solver) {
+  if (solver != VDN_SOLVER_CHOLESKY && solver != VDN_SOLVER_GAUSS_JORDAN)
+    return VDN_ERR_INVALID_ARG;
+  g_solver.store(solver);
+  return VDN_OK;
+}
+
 vdn_status vdn_reset_device_status(void* ws, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return VDN_ERR_WORKSPACE;
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -212,6 +222,7 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
                         int64_t ld, const float* beta, const float* alpha, void* o_vda,
                         int64_t ld_o, float* states_opt, void* ws, size_t ws_bytes,
                         void* stream) {
+  NvtxRange nvtx("vdn_vda_scan");
   if (!shape_ok(shape)) return VDN_ERR_INVALID_ARG;
   const vdn_shape s = *shape;
   if (!head_dim_supported(s.d)) return VDN_ERR_UNSUPPORTED;

@@ -590,6 +590,7 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
                                int64_t ld_ctx, int m_ctx, int chunk_frames, int window_chunks,
                                unsigned anchors, float scale, void* o, int64_t ld_o,
                                float* lse_opt, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("vdn_window_attn_ctx");
   if (shape == nullptr || shape->T < 1 || shape->N < 1 || shape->H < 1 || shape->d < 1)
     return VDN_ERR_INVALID_ARG;
   const vdn_shape s = *shape;

@@ -24,7 +24,11 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_window_attn_workspace", "vdn_window_attn", "vdn_hybrid_fuse_workspace",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
-           "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx"]
+           "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx",
+           "vdn_set_vda_solver"]
+
+SOLVER_CHOLESKY = 0
+SOLVER_GAUSS_JORDAN = 1
 
 
 class VdnError(RuntimeError):
@@ -85,6 +89,8 @@ def lib():
     L.vdn_set_wait_budget_ns.restype = None
     L.vdn_selftest_exp2.argtypes = [_P, _P, _P, ctypes.c_int, _P]
     L.vdn_selftest_exp2.restype = ctypes.c_int
+    L.vdn_set_vda_solver.argtypes = [ctypes.c_int]
+    L.vdn_set_vda_solver.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -142,6 +148,11 @@ def reset_device_status(ws, stream=None):
 
 def set_wait_budget_ns(ns):
     lib().vdn_set_wait_budget_ns(int(ns))
+
+
+def set_vda_solver(solver):
+    """SOLVER_CHOLESKY (default) or SOLVER_GAUSS_JORDAN, process-wide."""
+    _check(lib().vdn_set_vda_solver(int(solver)), "vdn_set_vda_solver")
 
 
 def selftest_exp2(x, stream=None):
