@@ -40,6 +40,15 @@ namespace {
 
 constexpr int kMaxSegs = 256;
 
+// Of every 16 score pairs in a 32-column chunk, this many take the FMA-pipe
+// exponential and the rest the MUFU (measured on B200: see profiles/).
+#ifndef VDN_EXP2_FMA_PAIRS
+#define VDN_EXP2_FMA_PAIRS 0
+#endif
+static_assert(VDN_EXP2_FMA_PAIRS == 0 || VDN_EXP2_FMA_PAIRS == 2 || VDN_EXP2_FMA_PAIRS == 4 ||
+                  VDN_EXP2_FMA_PAIRS == 8,
+              "VDN_EXP2_FMA_PAIRS must divide 16 pairs evenly");
+
 struct WinSeg {
   int q0, q1;      // query token rows [q0, q1)
   int tile_base;   // first CTA tile index of this segment (launch order)
@@ -413,7 +422,9 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
           const uint64_t xs = f32x2_fma(
               (static_cast<uint64_t>(sr[32 * q + 2 * e + 1]) << 32) | sr[32 * q + 2 * e], cc, nm);
           uint64_t pp;
-          if ((e & 3) == 3) {
+          if (VDN_EXP2_FMA_PAIRS > 0 &&
+              (e % (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1))) ==
+                  (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1)) - 1) {
             pp = exp2_fma_x2(xs);
           } else {
             pp = f32x2_pack(exp2_mufu(f32x2_lo(xs)), exp2_mufu(f32x2_hi(xs)));
