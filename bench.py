@@ -125,6 +125,22 @@ def clocks_stop(handle):
             "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def max_over_ranks(values, device, world):
+    """Element-wise max of a list of floats over all ranks (identity at N=1)."""
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def weak_scaling_value(world, tokens_per_rank, ms_per_step):
+    """Whole-job tokens/s: every rank processes its own video per step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- CPU oracle
 
 def oracle_sample(shape, seed=0, vda_heads=2, frames=None, rows_per_frame=128):
@@ -262,11 +278,7 @@ def run_gpu(args, shape, rank, world):
     if layer.status() != 0:
         raise RuntimeError("device status after end-to-end steps")
 
-    t = [ms, e2e_ms, sum(win_ms), sum(vda_ms), sum(fuse_ms)]
-    if world > 1:
-        tt = torch.tensor(t, device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        t = tt.tolist()
+    t = max_over_ranks([ms, e2e_ms, sum(win_ms), sum(vda_ms), sum(fuse_ms)], dev, world)
     ms, e2e_ms = t[0], t[1]
     return dict(ms=ms, win_ms=t[2] / args.steps, vda_ms=t[3] / args.steps,
                 fuse_ms=t[4] / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
@@ -325,7 +337,7 @@ def main():
     r = run_gpu(args, shape, rank, world)
     peaks, peak_kind = load_peaks()
     ms_step = r["ms"] / args.steps
-    tokens_per_s = world * shape.L / (ms_step / 1e3)
+    tokens_per_s = weak_scaling_value(world, shape.L, ms_step)
     win_tflops = work["softmax_flop"] / (r["win_ms"] / 1e3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     traffic = None
@@ -366,7 +378,7 @@ def main():
                            "frac": (work["proj_flop"] / (peak * 1e12) * 1e3) / r["fuse_ms"]},
             "fp32_peak_tflops": FP32_TFLOPS,
         },
-        "e2e": {"value": world * shape.L / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+        "e2e": {"value": weak_scaling_value(world, shape.L, r["e2e_ms"]), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "ms_per_step": r["e2e_ms"]},
         "gpu_launches": r["launches"],
