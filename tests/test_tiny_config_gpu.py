@@ -78,3 +78,24 @@ def test_tiny_layer(vdn, T, N, H, d):
     y2_ref = oracle.hybrid_fuse(x["x"], host(layer.o_s), host(layer.o_vda), x["W_gs"], x["W_gl"],
                                 x["gamma"], 1e-6, x["W_os"], x["W_ol"], H)
     assert max_rel(host(y2), y2_ref) <= TOL_BF16
+
+
+def test_forward_many_pipelined_host_path(vdn):
+    """HybridLayer.forward_many (pinned host in/out, copies overlapping the
+    compute) gives the same y as forward() on device tensors."""
+    s = synth.Shape(12, 96, 2, 128)
+    vids = [synth.make_inputs(s, seed=20 + i, device="cuda", with_fuse=True) for i in range(3)]
+    w = vids[0]
+    layer = vdn.HybridLayer(s.T, s.N, s.H, s.d, w["W_gs"], w["W_gl"], w["W_os"], w["W_ol"],
+                            w["gamma"])
+    names = ("q", "k", "v", "beta", "alpha", "x")
+    refs = []
+    for v in vids:
+        refs.append(layer.forward(*[v[n] for n in names]).clone())
+    batches = [[v[n].to("cpu").pin_memory() for n in names] for v in vids]
+    outs = [torch.empty((s.L, s.D), dtype=torch.bfloat16).pin_memory() for _ in vids]
+    layer.forward_many(batches, outs)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    for o, r in zip(outs, refs):
+        assert torch.equal(o, r.cpu())

@@ -328,6 +328,67 @@ class HybridLayer:
             return out
         return self.y
 
+    def forward_many(self, batches, outs, stream=None, copy_stream=None):
+        """Run the layer over several videos held in (pinned) host memory.
+
+        ``batches`` is a list of (q, k, v, beta, alpha, x) host tuples and
+        ``outs`` a list of host tensors [T*N, D] bf16 that receive y.  Copies
+        run on ``copy_stream`` into two device staging sets, so the input of
+        video i+1 and the result of video i-1 move while video i computes.
+        Returns after enqueueing; synchronise the streams to read ``outs``.
+        """
+        if len(batches) != len(outs):
+            raise ValueError("one output per batch")
+        dev = self.device
+        stream = stream or torch.cuda.current_stream(dev)
+        copy_stream = copy_stream or getattr(self, "_copy_stream", None)
+        if copy_stream is None:
+            copy_stream = self._copy_stream = torch.cuda.Stream(dev)
+        if getattr(self, "_stages", None) is None:
+            b0 = batches[0]
+            self._stages = [[torch.empty(t.shape, dtype=t.dtype, device=dev) for t in b0]
+                            for _ in range(2)]
+            self._ys = [torch.empty((self.L, self.D), dtype=torch.bfloat16, device=dev)
+                        for _ in range(2)]
+        stages, ys = self._stages, self._ys
+        loaded = [torch.cuda.Event() for _ in batches]
+        computed = [torch.cuda.Event() for _ in batches]
+        T, N, H, d = self.T, self.N, self.H, self.d
+        cf, wc, an = self.mask
+
+        def load(i):
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(computed[i - 2])   # stage i % 2 is free
+                for dst, src in zip(stages[i % 2], batches[i]):
+                    dst.copy_(src, non_blocking=True)
+                loaded[i].record(copy_stream)
+
+        copy_stream.wait_stream(stream)  # copies start after work already on `stream`
+        load(0)
+        for i in range(len(batches)):
+            if i + 1 < len(batches):
+                load(i + 1)
+            stream.wait_event(loaded[i])
+            if i >= 2:
+                stream.wait_event(self._read[i - 2])           # y buffer i % 2 is free
+            q, k, v, beta, alpha, x = stages[i % 2]
+            y = ys[i % 2]
+            window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win,
+                        stream=stream)
+            vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
+                     stream=stream)
+            hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
+                        self.W_ol, H, eps=self.eps, out=y, ws=self.ws_fuse, stream=stream)
+            computed[i].record(stream)
+            if i == 0:
+                self._read = [torch.cuda.Event() for _ in batches]
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(computed[i])
+                outs[i].copy_(y, non_blocking=True)
+                self._read[i].record(copy_stream)
+        return outs
+
     def status(self):
         """Worst device status over the layer's workspaces (synchronises)."""
         return max(get_device_status(w) for w in (self.ws_vda, self.ws_win, self.ws_fuse))
