@@ -200,6 +200,26 @@ VDN_API vdn_status vdn_hybrid_fuse(int L, int D, int H, const void* x, const voi
                            const float* gamma, float eps, const void* W_os, const void* W_ol,
                            void* y, void* ws, size_t ws_bytes, void* stream);
 
+/* One head shard of the fuse, for head-parallel multi-GPU runs of one video
+ * (rank r of G owns heads [head0, head0 + H_local)).  The gates are
+ * elementwise, so a shard computes its own hidden columns
+ * c in [head0*d, (head0 + H_local)*d): Z_r = [sigmoid(x W_gs[c]^T) o_s_r |
+ * sigmoid(x W_gl[c]^T) RMSNorm(o_vda_r) gamma[c]], and the partial
+ *   y_partial = Z_r [W_os[:, c] | W_ol[:, c]]^T           (fp32, [L, D])
+ * whose sum over the shards is y (the caller's all-reduce).
+ * x: [L, D] bf16 (full); o_s, o_vda: [L, ld_o] bf16, this shard's heads only
+ * (ld_o == H_local*d); W_*: the full [D, D] bf16 weights; gamma: full [D].
+ * Requires d % 128 == 0 and D % 256 == 0.
+ * ws: >= vdn_hybrid_fuse_shard_workspace(L, D, H_local, d) bytes. */
+VDN_API size_t vdn_hybrid_fuse_shard_workspace(int L, int D, int H_local, int d);
+
+VDN_API vdn_status vdn_hybrid_fuse_shard(int L, int D, int H_local, int d, int head0,
+                                         const void* x, const void* o_s, const void* o_vda,
+                                         int64_t ld_o, const void* W_gs, const void* W_gl,
+                                         const float* gamma, float eps, const void* W_os,
+                                         const void* W_ol, float* y_partial, void* ws,
+                                         size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Status and diagnostics.
  * ------------------------------------------------------------------------ */

@@ -81,3 +81,24 @@ def test_fuse_full_block_sampled(vdn):
     assert max_rel(got, ref) <= TOL_BF16
     del inp, y
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_fuse_head_shards_sum_to_full(vdn, G):
+    """Row-parallel fuse: the fp32 partials of G head shards, summed (the
+    all-reduce of a head-parallel run, done here on one GPU), give y."""
+    shape, inp = _inputs(2, 1000, 8, 128, seed=40 + G)
+    y_full = _fuse(vdn, shape, inp)
+    Hl = shape.H // G
+    acc = torch.zeros((shape.L, shape.D), dtype=torch.float32, device="cuda")
+    for r in range(G):
+        c = slice(r * Hl * 128, (r + 1) * Hl * 128)
+        part, ws = vdn.hybrid_fuse_shard(inp["x"], inp["o_s"][:, c].contiguous(),
+                                         inp["o_vda"][:, c].contiguous(), inp["W_gs"],
+                                         inp["W_gl"], inp["gamma"], inp["W_os"], inp["W_ol"],
+                                         128, r * Hl)
+        assert vdn.get_device_status(ws) == 0
+        acc += part
+    ref = _ref_rows(shape, inp, np.arange(shape.L))
+    assert max_rel(host(acc), ref) <= TOL_BF16
+    assert max_rel(host(acc), host(y_full)) <= TOL_BF16

@@ -25,7 +25,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
            "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx",
-           "vdn_set_vda_solver"]
+           "vdn_set_vda_solver", "vdn_hybrid_fuse_shard_workspace", "vdn_hybrid_fuse_shard"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -89,6 +89,11 @@ def lib():
     L.vdn_set_wait_budget_ns.restype = None
     L.vdn_selftest_exp2.argtypes = [_P, _P, _P, ctypes.c_int, _P]
     L.vdn_selftest_exp2.restype = ctypes.c_int
+    L.vdn_hybrid_fuse_shard_workspace.argtypes = [ctypes.c_int] * 4
+    L.vdn_hybrid_fuse_shard_workspace.restype = _SZ
+    L.vdn_hybrid_fuse_shard.argtypes = [ctypes.c_int] * 5 + [_P, _P, _P, _I64, _P, _P, _P,
+                                                             ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
+    L.vdn_hybrid_fuse_shard.restype = ctypes.c_int
     L.vdn_set_vda_solver.argtypes = [ctypes.c_int]
     L.vdn_set_vda_solver.restype = ctypes.c_int
     L.vdn_version.argtypes = []
@@ -265,6 +270,26 @@ def hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, W_os, W_ol, H, eps=1e-6, out=N
     return out, ws
 
 
+def hybrid_fuse_shard(x, o_s_local, o_vda_local, W_gs, W_gl, gamma, W_os, W_ol, d, head0,
+                      eps=1e-6, out=None, ws=None, stream=None):
+    """This head shard's fp32 partial of y (sum the partials over shards)."""
+    _need_cuda(x, o_s_local, o_vda_local, W_gs, W_gl, gamma, W_os, W_ol, out, ws)
+    L, D = x.shape
+    H_local = o_s_local.shape[1] // d
+    if out is None:
+        out = torch.empty((L, D), dtype=torch.float32, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(int(lib().vdn_hybrid_fuse_shard_workspace(L, D, H_local, d)),
+                             x.device)
+    code = lib().vdn_hybrid_fuse_shard(int(L), int(D), int(H_local), int(d), int(head0),
+                                       _ptr(x), _ptr(o_s_local), _ptr(o_vda_local),
+                                       o_s_local.stride(0), _ptr(W_gs), _ptr(W_gl), _ptr(gamma),
+                                       float(eps), _ptr(W_os), _ptr(W_ol), _ptr(out), _ptr(ws),
+                                       ws.numel(), _stream(stream))
+    _check(code, "vdn_hybrid_fuse_shard")
+    return out, ws
+
+
 # ---------------------------------------------------------------- full layer
 
 class HybridLayer:
@@ -392,3 +417,57 @@ class HybridLayer:
     def status(self):
         """Worst device status over the layer's workspaces (synchronises)."""
         return max(get_device_status(w) for w in (self.ws_vda, self.ws_win, self.ws_fuse))
+
+
+class HeadShardedLayer:
+    """One video's hybrid layer split by heads over a process group.
+
+    Rank r of G owns heads [r H/G, (r+1) H/G).  The window Softmax and VDA
+    branches are per head, so each rank runs them on its own head columns
+    (views into the full [T*N, D] activations) with no communication; the
+    fuse is row-parallel: each rank forms its hidden columns of the gated
+    branch inputs and an fp32 partial of y over the full width
+    (vdn_hybrid_fuse_shard), and the partials are summed across ranks with
+    one all-reduce.  ``ops`` replaces the four compute calls (tests only).
+    """
+
+    def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, group=None,
+                 device=None, ops=None, act_dtype=torch.bfloat16, acc_dtype=torch.float32):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        if H % self.world:
+            raise ValueError("heads must divide evenly over the ranks")
+        self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
+        self.L, self.D = self.T * self.N, self.H * self.d
+        self.Hl = self.H // self.world
+        self.head0 = self.rank * self.Hl
+        self.cols = slice(self.head0 * self.d, (self.head0 + self.Hl) * self.d)
+        self.device = torch.device(device) if device is not None else torch.device("cuda")
+        dev = self.device
+        self.W = [w.to(dev, act_dtype).contiguous() for w in (W_gs, W_gl, W_os, W_ol)]
+        self.gamma = gamma.to(dev, acc_dtype).contiguous()
+        self.eps = float(eps)
+        self.ops = ops or {"window_attn": window_attn, "vda_scan": vda_scan,
+                           "fuse_shard": hybrid_fuse_shard}
+        Dl = self.Hl * self.d
+        self.o_s = torch.empty((self.L, Dl), dtype=act_dtype, device=dev)
+        self.o_vda = torch.empty((self.L, Dl), dtype=act_dtype, device=dev)
+        self.y_partial = torch.empty((self.L, self.D), dtype=acc_dtype, device=dev)
+        self.y = torch.empty((self.L, self.D), dtype=act_dtype, device=dev)
+
+    def forward(self, q, k, v, beta, alpha, x):
+        c, Hl, d = self.cols, self.Hl, self.d
+        h0, h1 = self.head0, self.head0 + self.Hl
+        ql, kl, vl = q[:, c], k[:, c], v[:, c]             # views, row stride D
+        beta_l = beta[:, h0:h1].contiguous()
+        alpha_l = alpha[:, h0:h1].contiguous()
+        self.ops["window_attn"](ql, kl, vl, self.T, self.N, Hl, d, out=self.o_s)
+        self.ops["vda_scan"](ql, kl, vl, beta_l, alpha_l, self.T, self.N, Hl, d, out=self.o_vda)
+        self.ops["fuse_shard"](x, self.o_s, self.o_vda, *self.W[:2], self.gamma, *self.W[2:], d,
+                               h0, eps=self.eps, out=self.y_partial)
+        self.dist.all_reduce(self.y_partial, group=self.group)
+        self.y.copy_(self.y_partial)
+        return self.y
