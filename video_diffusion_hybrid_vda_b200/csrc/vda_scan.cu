@@ -11,8 +11,12 @@
 // state in one direction and runs all T steps; every CTA of the grid is
 // resident at once.  Per step the CTA stages P_t (d x d fp32) into shared
 // memory with one bulk copy, double-buffered so that P_{t+1} lands while
-// step t computes; the state rows stay in shared memory (transposed) and
-// each thread computes a 4 x 8 tile of the new state with packed f32x2 FMA.
+// step t computes; the state rows stay in shared memory (row stride d + 4,
+// so four consecutive k of a row are one float4 and the rows of a warp fall
+// in different banks) and each thread computes 4 rows x 8 columns of the new
+// state with packed f32x2 FMA.  A thread's columns are two interleaved
+// groups of 4 (4c.., d/2 + 4c..), so each quarter warp reads 128 contiguous
+// bytes of P.
 // The scan is serial over T and FP32-ALU bound.
 #include "common.cuh"
 #include "exp2_fma.cuh"
@@ -29,7 +33,8 @@ template <int DH>
 struct ScanCfg {
   static constexpr int THREADS = (kRows / kTR) * (DH / kTC);  // 256 (d=128), 128 (d=64)
   static constexpr int P_BYTES = DH * DH * 4;
-  static constexpr int SMEM = 2 * P_BYTES + DH * kRows * 4 + 64;
+  static constexpr int LDS = DH + 4;  // row stride of the state rows in shared memory
+  static constexpr int SMEM = 2 * P_BYTES + kRows * LDS * 4 + 64;
 };
 
 template <int DH>
@@ -41,8 +46,9 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   constexpr int CG = DH / kTC;  // column groups
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* Pbuf = reinterpret_cast<float*>(smem_raw);                  // 2 x [DH][DH]
-  float* St = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // [DH][kRows]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES + DH * kRows * 4);
+  float* Ss = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // [kRows][LDS]
+  uint64_t* full =
+      reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES + kRows * Cfg::LDS * 4);
 
   const int rb = blockIdx.x;  // row block
   const int h = blockIdx.y;
@@ -51,12 +57,13 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   const int rg = threadIdx.x / CG;
   const int lrow0 = rg * kTR;                  // first local row of the thread's tile
   const int row0 = rb * kRows + lrow0;         // first row of S
-  const int col0 = cg * kTC;
+  // the thread's columns: [colA, colA + 4) and [colB, colB + 4)
+  const int colA = 4 * cg, colB = DH / 2 + 4 * cg;
   const int64_t mat = static_cast<int64_t>(DH) * DH;
   float* out_dir = states + static_cast<int64_t>(dir) * T * H * mat;
   auto frame = [&](int step) { return dir == 0 ? step : T - 1 - step; };
 
-  for (int i = threadIdx.x; i < DH * kRows; i += blockDim.x) St[i] = 0.f;
+  for (int i = threadIdx.x; i < kRows * Cfg::LDS; i += blockDim.x) Ss[i] = 0.f;
   if (threadIdx.x == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
@@ -83,8 +90,8 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     float4 cv[kTR][2];
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
-      cv[r][0] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + col0));
-      cv[r][1] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + col0 + 4));
+      cv[r][0] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colA));
+      cv[r][1] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colB));
     }
     const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
     if (!__syncthreads_and(ok)) {
@@ -92,26 +99,33 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
       break;
     }
     const float* Pt = Pbuf + b * DH * DH;
-    // acc2[r][q] holds columns (col0 + 2q, col0 + 2q + 1) of row r
+    // acc2[r][q]: columns (colA + 2q, +1) for q < 2, (colB + 2(q-2), +1) for q >= 2
     uint64_t acc2[kTR][kTC / 2];
 #pragma unroll
     for (int r = 0; r < kTR; ++r)
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
     if (step > 0) {
-#pragma unroll 4
-      for (int k = 0; k < DH; ++k) {
-        const float4 s4 = *reinterpret_cast<const float4*>(St + k * kRows + lrow0);
-        const ulonglong2 p01 = *reinterpret_cast<const ulonglong2*>(Pt + k * DH + col0);
-        const ulonglong2 p23 = *reinterpret_cast<const ulonglong2*>(Pt + k * DH + col0 + 4);
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll 1
+      for (int k = 0; k < DH; k += 4) {
+        float sr[kTR][4];
 #pragma unroll
         for (int r = 0; r < kTR; ++r) {
-          const uint64_t ss = f32x2_pack(sv[r], sv[r]);
-          acc2[r][0] = f32x2_fma(ss, p01.x, acc2[r][0]);
-          acc2[r][1] = f32x2_fma(ss, p01.y, acc2[r][1]);
-          acc2[r][2] = f32x2_fma(ss, p23.x, acc2[r][2]);
-          acc2[r][3] = f32x2_fma(ss, p23.y, acc2[r][3]);
+          const float4 v = *reinterpret_cast<const float4*>(Ss + (lrow0 + r) * Cfg::LDS + k);
+          sr[r][0] = v.x; sr[r][1] = v.y; sr[r][2] = v.z; sr[r][3] = v.w;
+        }
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const ulonglong2 pa = *reinterpret_cast<const ulonglong2*>(Pt + (k + kk) * DH + colA);
+          const ulonglong2 pb = *reinterpret_cast<const ulonglong2*>(Pt + (k + kk) * DH + colB);
+#pragma unroll
+          for (int r = 0; r < kTR; ++r) {
+            const uint64_t ss = f32x2_pack(sr[r][kk], sr[r][kk]);
+            acc2[r][0] = f32x2_fma(ss, pa.x, acc2[r][0]);
+            acc2[r][1] = f32x2_fma(ss, pa.y, acc2[r][1]);
+            acc2[r][2] = f32x2_fma(ss, pb.x, acc2[r][2]);
+            acc2[r][3] = f32x2_fma(ss, pb.y, acc2[r][3]);
+          }
         }
       }
     }
@@ -128,16 +142,20 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
         snew[r][2 * q + 1] = f32x2_hi(v);
       }
       float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
-                   static_cast<int64_t>(row0 + r) * DH + col0;
-      *reinterpret_cast<float4*>(dst) = make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
-      *reinterpret_cast<float4*>(dst + 4) =
+                   static_cast<int64_t>(row0 + r) * DH;
+      *reinterpret_cast<float4*>(dst + colA) =
+          make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
+      *reinterpret_cast<float4*>(dst + colB) =
           make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
     }
-    __syncthreads();  // every thread has finished reading St (and Pbuf b)
+    __syncthreads();  // every thread has finished reading Ss (and Pbuf b)
 #pragma unroll
-    for (int e = 0; e < kTC; ++e)
-      *reinterpret_cast<float4*>(St + (col0 + e) * kRows + lrow0) =
-          make_float4(snew[0][e], snew[1][e], snew[2][e], snew[3][e]);
+    for (int r = 0; r < kTR; ++r) {
+      *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colA) =
+          make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
+      *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colB) =
+          make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
+    }
     __syncthreads();
   }
   // the bulk copies this CTA started must land before it exits
