@@ -24,6 +24,9 @@ pages' description of the method:
                       the linear branch, separate output projections, summed.
                       Source: same article, 方法概述 item 3.
 
+* ``vda_backward`` -- gradients of the VDA output with respect to q, k, v,
+                      beta and alpha (adjoint scans), for training the branch.
+
 The readings taken where the pages are silent are listed in CONVENTIONS.md
 beside this file.  Parity status of every function is pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``; none is unpinned.
@@ -34,6 +37,7 @@ from .vda import (vda_prep, vda_frame_state, vda_scan, vda_readout, vda,
 from .window_attn import (frame_visible, visible_key_frames, window_attn,
                           window_attn_rows, mask_pair_count)
 from .fuse import sigmoid, rmsnorm_heads, fuse_gates, hybrid_fuse, hybrid_fuse_rows
+from .vda_backward import vda_backward
 
 __all__ = [
     "vda_prep", "vda_frame_state", "vda_scan", "vda_readout", "vda",
@@ -41,4 +45,5 @@ __all__ = [
     "frame_visible", "visible_key_frames", "window_attn", "window_attn_rows",
     "mask_pair_count",
     "sigmoid", "rmsnorm_heads", "fuse_gates", "hybrid_fuse", "hybrid_fuse_rows",
+    "vda_backward",
 ]
