@@ -138,6 +138,48 @@ VDN_API vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q, co
                                        void* stream);
 
 /* ------------------------------------------------------------------------
+ * Gradients of Video Delta Attention, for training the branch (the staged
+ * alignment of 10100.com article, 方法概述 item 3, trains it; the closed form
+ * of item 2 is what is differentiated).
+ *
+ * Given dO = dLoss/do_vda, with G_t = sum_{i in t} dO_i q_i^T and the
+ * adjoint states of the two scans
+ *   D_fwd_t = (alpha_{t+1} D_fwd_{t+1} + G_t) P_t   (t = T-1 .. 0)
+ *   D_bwd_t = (alpha_{t-1} D_bwd_{t-1} + G_t) P_t   (t = 0 .. T-1)
+ * and dB_t = D_fwd_t + D_bwd_t, E_t = dA_t + dA_t^T with
+ * dA_t = -(S_fwd_t^T D_fwd_t + S_bwd_t^T D_bwd_t):
+ *   dq_i     = (S_fwd_t + S_bwd_t)^T dO_i
+ *   dk_i     = beta_i (E_t k_i + dB_t^T v_i)
+ *   dv_i     = beta_i dB_t k_i
+ *   dbeta_i  = k_i . (E_t k_i / 2 + dB_t^T v_i)
+ *   dalpha_t = <D_fwd_t, S_fwd_{t-1}> + <D_bwd_t, S_bwd_{t+1}>
+ *
+ * q, k, v, beta, alpha, ld: the forward's inputs (as for vdn_vda_scan).
+ * d_o       : [L, ld_do] bf16, dLoss/do_vda
+ * dq, dk, dv: [L, ld_g] bf16, outputs (columns past H*d are not written)
+ * dbeta     : [L, H] fp32 output;  dalpha: [T, H] fp32 output
+ * ws        : >= vdn_vda_backward_workspace(shape) bytes.
+ * The call recomputes the forward's A, B, P, C and states in its workspace
+ * (about half of its time at d = 128), so it needs nothing kept from the
+ * forward call.  Errors as for vdn_vda_scan.
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_vda_backward_workspace(const vdn_shape* shape);
+
+VDN_API vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k,
+                                    const void* v, int64_t ld, const float* beta,
+                                    const float* alpha, const void* d_o, int64_t ld_do, void* dq,
+                                    void* dk, void* dv, int64_t ld_g, float* dbeta, float* dalpha,
+                                    void* ws, size_t ws_bytes, void* stream);
+
+/* Pointers into a backward workspace, after vdn_vda_backward on it, to fp32
+ * [2, T, H, d, d] arrays: states ([0] = S_fwd, [1] = S_bwd), adjoint
+ * states ([0] = D_bwd, [1] = D_fwd), and E [T, H, d, d].  For head dims 16
+ * and 32 the arrays are those of the zero-padded 64-wide problem.  Any out
+ * pointer may be NULL.  Pure pointer arithmetic: enqueues nothing. */
+VDN_API vdn_status vdn_vda_backward_debug_buffers(const vdn_shape* shape, void* ws,
+                                                  float** states, float** adj, float** E);
+
+/* ------------------------------------------------------------------------
  * Window-and-anchor Softmax (10100.com article, 方法概述 item 1).
  *
  * Chunk c(t) = floor(t / chunk_frames).  Query frame tq sees key frame tk iff

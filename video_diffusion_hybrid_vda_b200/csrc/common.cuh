@@ -70,4 +70,30 @@ cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* 
 cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                                const CUtensorMap& omap, const float* states);
 
+// ---- gradient pass (see vda_grad.cu) -------------------------------------
+
+// G[t,h] = sum_i dO_i q_i^T (gram mode of the prep kernel; maps as for prep).
+cudaError_t launch_vda_gram(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                            const CUtensorMap& domap, float* G);
+
+// Adjoint scans D_t = (alpha_u D_u + G_t) P_t; adj is [2, T, H, d, d] with
+// direction 0 forward in time (adjoint of the backward scan).
+cudaError_t launch_vda_adjoint_scan(const Launch& ctx, const vdn_shape& s, const float* P,
+                                    const float* G, const float* alpha, float* adj);
+
+// Read-out variants: x (S0 + S1)^T, or x (S0 + S1) when trans_s, rows scaled
+// by row_scale[(t N + i) H + h] when it is non-null.
+cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,
+                                  const CUtensorMap& omap, const float* states, bool trans_s,
+                                  const float* row_scale);
+
+// E = dA + dA^T with dA = -(S_fwd^T D_fwd + S_bwd^T D_bwd), and dalpha.
+cudaError_t launch_vda_grad_combine(const Launch& ctx, const vdn_shape& s, const float* states,
+                                    const float* adj, float* E, float* dalpha);
+
+// dk = beta (K E + V dB) (bf16 through dkmap) and dbeta (fp32 [L, H]).
+cudaError_t launch_vda_grad_k(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, const CUtensorMap& dkmap, const float* E,
+                              const float* adj, const float* beta, float* dbeta);
+
 }  // namespace vdn

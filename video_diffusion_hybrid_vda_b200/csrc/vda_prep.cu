@@ -18,6 +18,10 @@
 //  * the scaler warps then drain TMEM rows to global fp32 A and B.
 // The stage is HBM-bound (k and v are read once); the split doubles the
 // tensor-core work, which stays below the HBM time.
+//
+// Gram mode (kGram) serves the gradient pass: with q in place of k and
+// dL/do in place of v it forms G_t,h = sum_i dO_i q_i^T (no beta, no split:
+// q is already bf16) and writes only that matrix.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -38,7 +42,7 @@ struct PrepCfg {
   static constexpr int CHUNKS_PER_THREAD = TILE_BYTES / 16 / 128;
 };
 
-template <int DH>
+template <int DH, bool kGram>
 __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
     vda_prep_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const float* __restrict__ beta,
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16(128, DH, true, true);
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % C::STAGES;
-        if (!mbar_wait(&scaled[s], (kb / C::STAGES) & 1, budget_ns)) {
+        if (!mbar_wait(kGram ? &full[s] : &scaled[s], (kb / C::STAGES) & 1, budget_ns)) {
           record_status(status, kStatusTimeout);
           break;
         }
@@ -137,7 +141,16 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
           const uint64_t hdesc = sdesc_sw128(hbase + kk * 2048, C::SLAB_BYTES, 1024);
           const uint64_t ldesc = sdesc_sw128(lbase + kk * 2048, C::SLAB_BYTES, 1024);
           const uint64_t kdesc = sdesc_sw128(kbase + kk * 2048, C::SLAB_BYTES, 1024);
-          if constexpr (DH == 128) {
+          if constexpr (kGram) {
+            if constexpr (DH == 128) {
+              // G = dO^T q: dO features along M, q features along N
+              umma_ss(tmem + 128, sdesc_sw128(vbase + kk * 2048, C::SLAB_BYTES, 1024), kdesc,
+                      idesc, acc);
+            } else {
+              // [q | dO] stacked along M against q: rows 64..127 hold G
+              umma_ss(tmem, kdesc, kdesc, idesc, acc);
+            }
+          } else if constexpr (DH == 128) {
             const uint64_t vdesc = sdesc_sw128(vbase + kk * 2048, C::SLAB_BYTES, 1024);
             umma_ss(tmem, kdesc, hdesc, idesc, acc);
             umma_ss(tmem, kdesc, ldesc, idesc, 1);
@@ -157,7 +170,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
     // ------------------------------------------------------------ scalers
     const int tid = threadIdx.x - 64;  // 0..127
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    for (int kb = 0; kb < (kGram ? 0 : nk); ++kb) {
       const int s = kb % C::STAGES;
       // beta for the rows this thread touches in this stage
       float bv[C::CHUNKS_PER_THREAD];
@@ -206,7 +219,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       const int64_t mat = (static_cast<int64_t>(t) * H + h) * DH * DH;
       if constexpr (DH == 128) {
 #pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        for (int half = kGram ? 1 : 0; half < 2; ++half) {
           float* dst = (half == 0 ? A : B) + mat + static_cast<int64_t>(m) * DH;
 #pragma unroll 1
           for (int c = 0; c < DH; c += 32) {
@@ -220,7 +233,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
                               __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
           }
         }
-      } else {
+      } else if (!kGram || quarter >= 2) {  // warp-uniform: rows 0..63 are q^T q
         float* dst = (m < 64 ? A + mat + static_cast<int64_t>(m) * DH
                              : B + mat + static_cast<int64_t>(m - 64) * DH);
 #pragma unroll 1
@@ -251,19 +264,19 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
   }
 }
 
-template <int DH>
+template <int DH, bool kGram>
 cudaError_t launch_prep_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const float* beta, float* A, float* B) {
   using C = PrepCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_prep_kernel<DH>,
+    cudaError_t e = cudaFuncSetAttribute(vda_prep_kernel<DH, kGram>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const int grid = s.T * s.H;
-  vda_prep_kernel<DH><<<grid, C::THREADS, C::SMEM, ctx.stream>>>(
+  vda_prep_kernel<DH, kGram><<<grid, C::THREADS, C::SMEM, ctx.stream>>>(
       kmap, vmap, beta, A, B, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
@@ -272,8 +285,15 @@ cudaError_t launch_prep_dh(const Launch& ctx, const vdn_shape& s, const CUtensor
 
 cudaError_t launch_vda_prep(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                             const CUtensorMap& vmap, const float* beta, float* A, float* B) {
-  if (s.d == 128) return launch_prep_dh<128>(ctx, s, kmap, vmap, beta, A, B);
-  if (s.d == 64) return launch_prep_dh<64>(ctx, s, kmap, vmap, beta, A, B);
+  if (s.d == 128) return launch_prep_dh<128, false>(ctx, s, kmap, vmap, beta, A, B);
+  if (s.d == 64) return launch_prep_dh<64, false>(ctx, s, kmap, vmap, beta, A, B);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_vda_gram(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                            const CUtensorMap& domap, float* G) {
+  if (s.d == 128) return launch_prep_dh<128, true>(ctx, s, qmap, domap, nullptr, nullptr, G);
+  if (s.d == 64) return launch_prep_dh<64, true>(ctx, s, qmap, domap, nullptr, nullptr, G);
   return cudaErrorInvalidValue;
 }
 

@@ -11,6 +11,11 @@
 // swizzled staging tile that a TMA store writes back.  Loads and stores use
 // a 3-D frame view, so the ragged last tile of a frame reads zeros and its
 // extra rows are not written.  HBM-bound: q is read once and o written once.
+//
+// The gradient pass reuses the kernel twice: with kTransS the B operand is
+// read MN-major, giving x (S_fwd + S_bwd) instead of x (S_fwd + S_bwd)^T
+// (dq = dO S), and a non-null row_scale multiplies output row i by
+// row_scale[(t N + i) H + h] (dv = beta k (D_fwd + D_bwd)^T).
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -31,11 +36,12 @@ struct ReadoutCfg {
 };
 
 
-template <int DH>
+template <int DH, bool kTransS>
 __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
     vda_readout_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap omap, const float* __restrict__ states,
-                       int T, int N, int H, uint32_t* status, uint64_t budget_ns) {
+                       const float* __restrict__ row_scale, int T, int N, int H, uint32_t* status,
+                       uint64_t budget_ns) {
   using Cfg = ReadoutCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -124,7 +130,7 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_bf16(128, DH, false, false);
+      constexpr uint32_t idesc = idesc_bf16(128, DH, false, kTransS);
       const uint32_t sb = smem_u32(sbuf);
       for (int j = 0; j < ntiles; ++j) {
         const int s = j % Cfg::STAGES;
@@ -142,9 +148,12 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t soff = (kk >> 2) * (DH * 128) + (kk & 3) * 32;
-          umma_ss(tmem + b * DH, sdesc_sw128(qb + koff, 16, 1024), sdesc_sw128(sb + soff, 16, 1024),
-                  idesc, kk > 0);
+          // K-major: rows of the tile are N, 64-wide K slabs; MN-major: rows
+          // are K (16 per step), 64-wide N slabs DH * 128 bytes apart
+          const uint64_t sdesc = kTransS ? sdesc_sw128(sb + kk * 2048, DH * 128, 1024)
+                                         : sdesc_sw128(sb + (kk >> 2) * (DH * 128) + (kk & 3) * 32,
+                                                       16, 1024);
+          umma_ss(tmem + b * DH, sdesc_sw128(qb + koff, 16, 1024), sdesc, idesc, kk > 0);
         }
         umma_commit(&empty[s]);
         umma_commit(&tfull[b]);
@@ -167,6 +176,10 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
         break;
       }
       tc_fence_after();
+      const int tok = j * 128 + row;
+      const float rs = row_scale == nullptr ? 1.f
+                       : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
+                                 : 0.f;
       uint8_t* ob = obuf + b * Cfg::QTILE_BYTES;
       const uint32_t taddr = tmem + b * DH + ((quarter * 32) << 16);
 #pragma unroll
@@ -177,10 +190,10 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-          u.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-          u.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-          u.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
+          u.x = pack_bf16x2(rs * __uint_as_float(r[8 * q + 0]), rs * __uint_as_float(r[8 * q + 1]));
+          u.y = pack_bf16x2(rs * __uint_as_float(r[8 * q + 2]), rs * __uint_as_float(r[8 * q + 3]));
+          u.z = pack_bf16x2(rs * __uint_as_float(r[8 * q + 4]), rs * __uint_as_float(r[8 * q + 5]));
+          u.w = pack_bf16x2(rs * __uint_as_float(r[8 * q + 6]), rs * __uint_as_float(r[8 * q + 7]));
           const int chunk = ((c & 63) >> 3) + q;  // 16-byte chunk within the 128-byte row
           *reinterpret_cast<uint4*>(ob + (c >> 6) * 16384 + sw128_offset(row, chunk)) = u;
         }
@@ -207,19 +220,20 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
   }
 }
 
-template <int DH>
+template <int DH, bool kTransS>
 cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
-                              const CUtensorMap& omap, const float* states) {
+                              const CUtensorMap& omap, const float* states,
+                              const float* row_scale) {
   using Cfg = ReadoutCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_readout_kernel<DH>,
+    cudaError_t e = cudaFuncSetAttribute(vda_readout_kernel<DH, kTransS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  vda_readout_kernel<DH><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, omap, states, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
+  vda_readout_kernel<DH, kTransS><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, omap, states, row_scale, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
 
@@ -227,8 +241,20 @@ cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUten
 
 cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                                const CUtensorMap& omap, const float* states) {
-  if (s.d == 128) return launch_readout_dh<128>(ctx, s, qmap, omap, states);
-  if (s.d == 64) return launch_readout_dh<64>(ctx, s, qmap, omap, states);
+  if (s.d == 128) return launch_readout_dh<128, false>(ctx, s, qmap, omap, states, nullptr);
+  if (s.d == 64) return launch_readout_dh<64, false>(ctx, s, qmap, omap, states, nullptr);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,
+                                  const CUtensorMap& omap, const float* states, bool trans_s,
+                                  const float* row_scale) {
+  if (s.d == 128)
+    return trans_s ? launch_readout_dh<128, true>(ctx, s, xmap, omap, states, row_scale)
+                   : launch_readout_dh<128, false>(ctx, s, xmap, omap, states, row_scale);
+  if (s.d == 64)
+    return trans_s ? launch_readout_dh<64, true>(ctx, s, xmap, omap, states, row_scale)
+                   : launch_readout_dh<64, false>(ctx, s, xmap, omap, states, row_scale);
   return cudaErrorInvalidValue;
 }
 

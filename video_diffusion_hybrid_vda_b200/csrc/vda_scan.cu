@@ -18,6 +18,16 @@
 // groups of 4 (4c.., d/2 + 4c..), so each quarter warp reads 128 contiguous
 // bytes of P.
 // The scan is serial over T and FP32-ALU bound.
+//
+// Adjoint mode (kAdjoint) runs the two scans of the gradient pass.  With
+// G_t = sum_i dO_i q_i^T, the sensitivity of the loss to the bracket
+// (alpha S_prev + B_t) of each direction obeys
+//   D_t = (alpha_u D_u + G_t) P_t,   u = the frame the same scan visited
+// one step earlier (t - 1 going forward in time, t + 1 going backward).
+// The thread first writes its tile of alpha_u D_u + G_t into the shared
+// rows and then multiplies by P_t, so the step costs the same as the
+// forward's; output direction 0 (forward in time) is the adjoint of the
+// backward scan, direction 1 the adjoint of the forward scan.
 #include "common.cuh"
 #include "exp2_fma.cuh"
 #include "ptx.cuh"
@@ -37,7 +47,7 @@ struct ScanCfg {
   static constexpr int SMEM = 2 * P_BYTES + kRows * LDS * 4 + 64;
 };
 
-template <int DH>
+template <int DH, bool kAdjoint>
 __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     vda_scan_kernel(const float* __restrict__ P, const float* __restrict__ C,
                     const float* __restrict__ alpha, float* __restrict__ states, int T, int H,
@@ -73,6 +83,12 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   }
   __syncthreads();
 
+  float dprev[kTR][kTC];  // adjoint mode: the thread's tile of D from the previous step
+#pragma unroll
+  for (int r = 0; r < kTR; ++r)
+#pragma unroll
+    for (int c = 0; c < kTC; ++c) dprev[r][c] = 0.f;
+
   int issued = 1;
 #pragma unroll 1
   for (int step = 0; step < T; ++step) {
@@ -85,13 +101,31 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
                 Cfg::P_BYTES, &full[b ^ 1]);
       ++issued;
     }
-    const float a = __ldg(alpha + t * H + h);
+    // forward: the decay of the frame being absorbed; adjoint: of the frame
+    // visited one step earlier (unused at step 0, where the carried term is 0)
+    const float a = !kAdjoint ? __ldg(alpha + t * H + h)
+                              : (step > 0 ? __ldg(alpha + frame(step - 1) * H + h) : 0.f);
     const float* Ct = C + (static_cast<int64_t>(t) * H + h) * mat;
     float4 cv[kTR][2];
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
       cv[r][0] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colA));
       cv[r][1] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colB));
+    }
+    if constexpr (kAdjoint) {
+      // U = a D_prev + G_t into the shared rows; every thread left the
+      // previous step's reads behind the barrier that closed it, and the
+      // barrier below publishes U before the multiply
+#pragma unroll
+      for (int r = 0; r < kTR; ++r) {
+        float* srow = Ss + (lrow0 + r) * Cfg::LDS;
+        *reinterpret_cast<float4*>(srow + colA) = make_float4(
+            fmaf(a, dprev[r][0], cv[r][0].x), fmaf(a, dprev[r][1], cv[r][0].y),
+            fmaf(a, dprev[r][2], cv[r][0].z), fmaf(a, dprev[r][3], cv[r][0].w));
+        *reinterpret_cast<float4*>(srow + colB) = make_float4(
+            fmaf(a, dprev[r][4], cv[r][1].x), fmaf(a, dprev[r][5], cv[r][1].y),
+            fmaf(a, dprev[r][6], cv[r][1].z), fmaf(a, dprev[r][7], cv[r][1].w));
+      }
     }
     const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
     if (!__syncthreads_and(ok)) {
@@ -105,7 +139,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     for (int r = 0; r < kTR; ++r)
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
-    if (step > 0) {
+    if (kAdjoint || step > 0) {
 #pragma unroll 1
       for (int k = 0; k < DH; k += 4) {
         float sr[kTR][4];
@@ -137,7 +171,8 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
                            cv[r][1].x, cv[r][1].y, cv[r][1].z, cv[r][1].w};
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) {
-        const uint64_t v = f32x2_fma(aa, acc2[r][q], f32x2_pack(cc[2 * q], cc[2 * q + 1]));
+        const uint64_t v =
+            kAdjoint ? acc2[r][q] : f32x2_fma(aa, acc2[r][q], f32x2_pack(cc[2 * q], cc[2 * q + 1]));
         snew[r][2 * q] = f32x2_lo(v);
         snew[r][2 * q + 1] = f32x2_hi(v);
       }
@@ -149,14 +184,21 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
           make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
     }
     __syncthreads();  // every thread has finished reading Ss (and Pbuf b)
+    if constexpr (kAdjoint) {
 #pragma unroll
-    for (int r = 0; r < kTR; ++r) {
-      *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colA) =
-          make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
-      *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colB) =
-          make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
+      for (int r = 0; r < kTR; ++r)
+#pragma unroll
+        for (int c = 0; c < kTC; ++c) dprev[r][c] = snew[r][c];
+    } else {
+#pragma unroll
+      for (int r = 0; r < kTR; ++r) {
+        *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colA) =
+            make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
+        *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colB) =
+            make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
+      }
+      __syncthreads();
     }
-    __syncthreads();
   }
   // the bulk copies this CTA started must land before it exits
   if (threadIdx.x == 0) {
@@ -165,19 +207,19 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   }
 }
 
-template <int DH>
+template <int DH, bool kAdjoint>
 cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* C,
                            const float* alpha, float* states) {
   using Cfg = ScanCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_scan_kernel<DH>,
+    cudaError_t e = cudaFuncSetAttribute(vda_scan_kernel<DH, kAdjoint>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   dim3 grid(DH / kRows, s.H, 2);
-  vda_scan_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+  vda_scan_kernel<DH, kAdjoint><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       P, C, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
@@ -186,8 +228,15 @@ cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P
 
 cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* P,
                             const float* C, const float* alpha, float* states) {
-  if (s.d == 128) return launch_scan_dh<128>(ctx, s, P, C, alpha, states);
-  if (s.d == 64) return launch_scan_dh<64>(ctx, s, P, C, alpha, states);
+  if (s.d == 128) return launch_scan_dh<128, false>(ctx, s, P, C, alpha, states);
+  if (s.d == 64) return launch_scan_dh<64, false>(ctx, s, P, C, alpha, states);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_vda_adjoint_scan(const Launch& ctx, const vdn_shape& s, const float* P,
+                                    const float* G, const float* alpha, float* adj) {
+  if (s.d == 128) return launch_scan_dh<128, true>(ctx, s, P, G, alpha, adj);
+  if (s.d == 64) return launch_scan_dh<64, true>(ctx, s, P, G, alpha, adj);
   return cudaErrorInvalidValue;
 }
 

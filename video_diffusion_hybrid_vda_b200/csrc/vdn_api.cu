@@ -75,7 +75,9 @@ VdaLayout vda_layout(const vdn_shape& s) {
 }
 
 // Workspace of a VDA call.  Head dims 16 and 32 run through a 64-wide padded
-// copy: [status][q' k' v' o' bf16 L x H*64][A B P C S_fwd S_bwd for d = 64].
+// copy: [status][nact padded activations, bf16 L x H*64][A B P C S_fwd S_bwd
+// for d = 64]; the forward pads q' k' v' o' (4), the gradient pass q' k' v'
+// dO' dq' dk' dv' (7).
 struct VdaPlan {
   bool padded;
   vdn_shape inner;  // shape the kernels run on
@@ -85,14 +87,14 @@ struct VdaPlan {
   size_t total;
 };
 
-VdaPlan vda_plan(const vdn_shape& s) {
+VdaPlan vda_plan(const vdn_shape& s, int nact = 4) {
   VdaPlan p;
   p.padded = head_dim_padded(s.d);
   p.inner = s;
   if (p.padded) p.inner.d = 64;
   p.lay = vda_layout(p.inner);
   p.act = p.padded ? round_up(static_cast<size_t>(s.T) * s.N * s.H * 64 * 2, 256) : 0;
-  p.inner_off = 4 * p.act;
+  p.inner_off = nact * p.act;
   p.total = p.lay.total + p.inner_off;
   return p;
 }
@@ -113,6 +115,47 @@ vdn_status run_vda(const Launch& ctx, const vdn_shape& s, const void* q, const v
   if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
   if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
   if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+// The gradient pass on head dim 64 or 128.  Workspace slots (in memory
+// order A, B, P, C, states) are reused as their contents die: G goes to C
+// (dead after the forward scan), the adjoint states to A and B (dead after
+// the solve; adjacent, so they form one [2, T, H, d, d] array), E to C (G
+// is dead after the adjoint scan).  P is read by both adjoint directions
+// until the adjoint scan ends, so nothing is written there.
+vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q, const void* k,
+                            const void* v, int64_t ld, const float* beta, const float* alpha,
+                            const void* d_o, int64_t ld_do, void* dq, void* dk, void* dv,
+                            int64_t ld_g, float* dbeta, float* dalpha, float* A, float* B,
+                            float* P, float* C, float* states) {
+  const int64_t D = static_cast<int64_t>(s.H) * s.d;
+  const int prep_rows = s.d == 128 ? 32 : 64;
+  CUtensorMap kmap_p, vmap_p, qmap_p, domap_p, domap, dqmap, kmap, vmap, dvmap, dkmap;
+  if (!make_frame_map(&kmap_p, k, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&vmap_p, v, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&qmap_p, q, D, ld, s.N, s.T, prep_rows) ||
+      !make_frame_map(&domap_p, d_o, D, ld_do, s.N, s.T, prep_rows) ||
+      !make_frame_map(&domap, d_o, D, ld_do, s.N, s.T, 128) ||
+      !make_frame_map(&dqmap, dq, D, ld_g, s.N, s.T, 128) ||
+      !make_frame_map(&kmap, k, D, ld, s.N, s.T, 128) ||
+      !make_frame_map(&vmap, v, D, ld, s.N, s.T, 128) ||
+      !make_frame_map(&dvmap, dv, D, ld_g, s.N, s.T, 128) ||
+      !make_frame_map(&dkmap, dk, D, ld_g, s.N, s.T, 128))
+    return VDN_ERR_CUDA;
+  float* G = C;
+  float* adj = A;
+  float* E = C;
+  if (launch_vda_prep(ctx, s, kmap_p, vmap_p, beta, A, B) != cudaSuccess ||
+      launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess ||
+      launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess ||
+      launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
+      launch_vda_adjoint_scan(ctx, s, P, G, alpha, adj) != cudaSuccess ||
+      launch_vda_grad_combine(ctx, s, states, adj, E, dalpha) != cudaSuccess ||
+      launch_vda_readout_ex(ctx, s, domap, dqmap, states, true, nullptr) != cudaSuccess ||
+      launch_vda_readout_ex(ctx, s, kmap, dvmap, adj, false, beta) != cudaSuccess ||
+      launch_vda_grad_k(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta) != cudaSuccess)
+    return VDN_ERR_CUDA;
   return VDN_OK;
 }
 
@@ -271,6 +314,81 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
       launch_repack_f32(st, states_opt, d, states_ws, 64, 2 * s.T * H, d, 64, 1, d, 64) !=
           cudaSuccess)
     return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
+// ----------------------------------------------------------------- VDA gradients
+
+size_t vdn_vda_backward_workspace(const vdn_shape* shape) {
+  if (!shape_ok(shape)) return 0;
+  return vda_plan(*shape, 7).total;
+}
+
+vdn_status vdn_vda_backward_debug_buffers(const vdn_shape* shape, void* ws, float** states,
+                                          float** adj, float** E) {
+  if (!shape_ok(shape) || ws == nullptr) return VDN_ERR_INVALID_ARG;
+  const VdaPlan pl = vda_plan(*shape, 7);
+  uint8_t* base = static_cast<uint8_t*>(ws) + pl.inner_off;
+  if (states) *states = reinterpret_cast<float*>(base + pl.lay.states);
+  if (adj) *adj = reinterpret_cast<float*>(base + pl.lay.A);
+  if (E) *E = reinterpret_cast<float*>(base + pl.lay.C);
+  return VDN_OK;
+}
+
+vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                            int64_t ld, const float* beta, const float* alpha, const void* d_o,
+                            int64_t ld_do, void* dq, void* dk, void* dv, int64_t ld_g,
+                            float* dbeta, float* dalpha, void* ws, size_t ws_bytes,
+                            void* stream) {
+  NvtxRange nvtx("vdn_vda_backward");
+  if (!shape_ok(shape)) return VDN_ERR_INVALID_ARG;
+  const vdn_shape s = *shape;
+  if (!head_dim_supported(s.d)) return VDN_ERR_UNSUPPORTED;
+  const int64_t D = static_cast<int64_t>(s.H) * s.d;
+  if (q == nullptr || k == nullptr || v == nullptr || beta == nullptr || alpha == nullptr ||
+      d_o == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || dbeta == nullptr ||
+      dalpha == nullptr)
+    return VDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_o, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(beta, 4) ||
+      !aligned(alpha, 4) || !aligned(dbeta, 4) || !aligned(dalpha, 4))
+    return VDN_ERR_INVALID_ARG;
+  if (!ld_ok(ld, D) || !ld_ok(ld_do, D) || !ld_ok(ld_g, D)) return VDN_ERR_INVALID_ARG;
+  const VdaPlan pl = vda_plan(s, 7);
+  if (ws == nullptr || !aligned(ws, 256) || ws_bytes < pl.total) return VDN_ERR_WORKSPACE;
+
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* inner = base + pl.inner_off;
+  float* A = reinterpret_cast<float*>(inner + pl.lay.A);
+  float* B = reinterpret_cast<float*>(inner + pl.lay.B);
+  float* P = reinterpret_cast<float*>(inner + pl.lay.P);
+  float* C = reinterpret_cast<float*>(inner + pl.lay.C);
+  float* states = reinterpret_cast<float*>(inner + pl.lay.states);
+  Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
+             g_budget_ns.load()};
+  if (!pl.padded)
+    return run_vda_backward(ctx, s, q, k, v, ld, beta, alpha, d_o, ld_do, dq, dk, dv, ld_g,
+                            dbeta, dalpha, A, B, P, C, states);
+
+  // d = 16 or 32: every head zero-padded to 64 columns (exact, see repack.cu)
+  const int L = s.T * s.N, H = s.H, d = s.d;
+  const int64_t D64 = static_cast<int64_t>(H) * 64;
+  uint8_t* pad[7];
+  for (int i = 0; i < 7; ++i) pad[i] = base + kStatusBytes + i * pl.act;
+  const void* src[4] = {q, k, v, d_o};
+  const int64_t lds[4] = {ld, ld, ld, ld_do};
+  cudaStream_t st = ctx.stream;
+  for (int i = 0; i < 4; ++i)
+    if (launch_repack_bf16(st, pad[i], D64, src[i], lds[i], 1, L, L, H, 64, d) != cudaSuccess)
+      return VDN_ERR_CUDA;
+  const vdn_status r = run_vda_backward(ctx, pl.inner, pad[0], pad[1], pad[2], D64, beta, alpha,
+                                        pad[3], D64, pad[4], pad[5], pad[6], D64, dbeta, dalpha,
+                                        A, B, P, C, states);
+  if (r != VDN_OK) return r;
+  void* dst[3] = {dq, dk, dv};
+  for (int i = 0; i < 3; ++i)
+    if (launch_repack_bf16(st, dst[i], ld_g, pad[4 + i], D64, 1, L, L, H, d, 64) != cudaSuccess)
+      return VDN_ERR_CUDA;
   return VDN_OK;
 }
 

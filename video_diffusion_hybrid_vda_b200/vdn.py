@@ -25,7 +25,8 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_hybrid_fuse", "vdn_status_string", "vdn_get_device_status",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
            "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx",
-           "vdn_set_vda_solver", "vdn_hybrid_fuse_shard_workspace", "vdn_hybrid_fuse_shard"]
+           "vdn_set_vda_solver", "vdn_hybrid_fuse_shard_workspace", "vdn_hybrid_fuse_shard",
+           "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -96,6 +97,13 @@ def lib():
     L.vdn_hybrid_fuse_shard.restype = ctypes.c_int
     L.vdn_set_vda_solver.argtypes = [ctypes.c_int]
     L.vdn_set_vda_solver.restype = ctypes.c_int
+    L.vdn_vda_backward_workspace.argtypes = [S]
+    L.vdn_vda_backward_workspace.restype = _SZ
+    L.vdn_vda_backward.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _P, _I64, _P,
+                                   _P, _P, _SZ, _P]
+    L.vdn_vda_backward.restype = ctypes.c_int
+    L.vdn_vda_backward_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 3
+    L.vdn_vda_backward_debug_buffers.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -208,6 +216,54 @@ def vda_debug_buffers(ws, T, N, H, d):
         off = p.value - base
         out.append(flat[off:off + 4 * n].view(torch.float32).view(T, H, d, d))
     return tuple(out)
+
+
+def vda_backward_workspace(T, N, H, d):
+    return int(lib().vdn_vda_backward_workspace(ctypes.byref(_shape(T, N, H, d))))
+
+
+def vda_backward(q, k, v, beta, alpha, d_o, T, N, H, d, dq=None, dk=None, dv=None, dbeta=None,
+                 dalpha=None, ws=None, stream=None):
+    """Gradients of o_vda with respect to q, k, v, beta and alpha, given
+    d_o = dLoss/do_vda ([T*N, ld] bf16).  Returns (dq, dk, dv, dbeta, dalpha, ws):
+    dq/dk/dv bf16 [T*N, H*d], dbeta fp32 [T*N, H], dalpha fp32 [T, H]."""
+    _need_cuda(q, k, v, beta, alpha, d_o, dq, dk, dv, dbeta, dalpha, ws)
+    shape = _shape(T, N, H, d)
+    dev = q.device
+    L, D = T * N, H * d
+    dq = torch.empty((L, D), dtype=torch.bfloat16, device=dev) if dq is None else dq
+    dk = torch.empty((L, D), dtype=torch.bfloat16, device=dev) if dk is None else dk
+    dv = torch.empty((L, D), dtype=torch.bfloat16, device=dev) if dv is None else dv
+    if not (dq.stride(0) == dk.stride(0) == dv.stride(0)):
+        raise ValueError("dq, dk and dv must share one row stride")
+    dbeta = torch.empty((L, H), dtype=torch.float32, device=dev) if dbeta is None else dbeta
+    dalpha = torch.empty((T, H), dtype=torch.float32, device=dev) if dalpha is None else dalpha
+    if ws is None:
+        ws = alloc_workspace(vda_backward_workspace(T, N, H, d), dev)
+    code = lib().vdn_vda_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
+                                  _ptr(beta), _ptr(alpha), _ptr(d_o), d_o.stride(0), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), dq.stride(0), _ptr(dbeta), _ptr(dalpha),
+                                  _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "vdn_vda_backward")
+    return dq, dk, dv, dbeta, dalpha, ws
+
+
+def vda_backward_debug_buffers(ws, T, N, H, d):
+    """(states [2,T,H,d',d'], adjoint states [2,T,H,d',d'], E [T,H,d',d']) views
+    into a backward workspace; d' = 64 for head dims 16 and 32."""
+    ptrs = [ctypes.c_void_p() for _ in range(3)]
+    _check(lib().vdn_vda_backward_debug_buffers(ctypes.byref(_shape(T, N, H, d)), _ptr(ws),
+                                                *[ctypes.byref(p) for p in ptrs]),
+           "vdn_vda_backward_debug_buffers")
+    dd = 64 if d in (16, 32) else d
+    base = ws.data_ptr()
+    flat = ws.view(torch.uint8)
+    out = []
+    for p, lead in zip(ptrs, (2, 2, 1)):
+        n = lead * T * H * dd * dd
+        off = p.value - base
+        out.append(flat[off:off + 4 * n].view(torch.float32).view(lead, T, H, dd, dd))
+    return out[0], out[1], out[2][0]
 
 
 # ---------------------------------------------------------------- window Softmax
