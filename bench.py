@@ -8,7 +8,12 @@ timed region starts; each activation (2.5 GB) is larger than L2, so no L2
 flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload layer102|layer42|small]
+                    [--workload layer102|layer42|small] [--part all|layer|vda_backward]
+
+The line also carries ``vda_backward``: the VDA gradient pass (dq, dk, dv,
+dbeta, dalpha from dL/do_vda, forward recomputed inside) timed on its own
+on the same inputs; it is not part of the step.  ``--part vda_backward``
+times only that pass (for launch lists and captures).
 
 With N > 1 (torchrun) every rank runs its own video (independent problems,
 no collective on the data path): weak scaling, time = max over ranks.
@@ -67,8 +72,14 @@ def work_model(s):
     # FP32 ALU work in FLOP per (frame, head): Cholesky d^3/3, W = L^-1 d^3/3,
     # P = W^T W and C = B P 2 d^3 each, and both scans a 2 d^3 product each
     vda_alu_flop = s.T * s.H * (2 * s.d ** 3 // 3 + 4 * s.d ** 3 + 4 * s.d ** 3)
+    # VDA gradient pass: reads q, k, v, dO (bf16) and beta, writes dq, dk, dv
+    # (bf16) and dbeta; FP32 ALU: the forward's solve and scans again, the
+    # two adjoint scans (2 d^3 each) and the combine (two d^3 products, 4 d^3)
+    vda_bwd_bytes = 7 * s.L * s.D * 2 + 2 * s.L * s.H * 4
+    vda_bwd_alu_flop = vda_alu_flop + s.T * s.H * (4 * s.d ** 3 + 4 * s.d ** 3)
     return dict(pairs=pairs, softmax_flop=softmax_flop, proj_flop=proj_flop,
-                vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop)
+                vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop, vda_bwd_bytes=vda_bwd_bytes,
+                vda_bwd_alu_flop=vda_bwd_alu_flop)
 
 
 def load_peaks():
@@ -293,6 +304,58 @@ def run_gpu(args, shape, rank, world):
                 clocks=clocks, launches=layer.KERNELS_PER_FORWARD * args.steps)
 
 
+def run_vda_backward(args, shape, rank, world):
+    """Device time of one VDA gradient pass (ms, max over ranks)."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1000 + rank)
+    d_o = torch.randn((shape.L, shape.D), generator=gen, device=dev).to(torch.bfloat16)
+    T, N, H, d = shape.T, shape.N, shape.H, shape.d
+    outs = [torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    dbeta = torch.empty((shape.L, H), dtype=torch.float32, device=dev)
+    dalpha = torch.empty((T, H), dtype=torch.float32, device=dev)
+    ws = vdn.alloc_workspace(vdn.vda_backward_workspace(T, N, H, d), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vdn.vda_backward(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], d_o, T, N, H,
+                         d, dq=outs[0], dk=outs[1], dv=outs[2], dbeta=dbeta, dalpha=dalpha,
+                         ws=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the gradient pass warm-up")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the timed gradient passes")
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    del inp, d_o, outs, ws
+    torch.cuda.empty_cache()
+    return ms
+
+
+def backward_row(work, peaks, ms):
+    roof_ms = (work["vda_bwd_bytes"] / (peaks["hbm_gbs"] * 1e9) +
+               work["vda_bwd_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3
+    return {"ms": ms, "bound": "hbm + fp32 alu", "roofline_ms": roof_ms, "frac": roof_ms / ms,
+            "hbm_bytes": work["vda_bwd_bytes"], "fp32_alu_flop": work["vda_bwd_alu_flop"],
+            "launches_per_pass": 9}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -303,6 +366,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
                     help="solver of (I + A)^-1 in the VDA branch")
+    ap.add_argument("--part", default="all", choices=["all", "layer", "vda_backward"],
+                    help="what to time: the layer step and the VDA gradient pass (all), "
+                         "or one of them")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -342,8 +408,19 @@ def main():
         torch.distributed.init_process_group(
             "nccl", device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
             timeout=__import__("datetime").timedelta(seconds=300))
-    r = run_gpu(args, shape, rank, world)
     peaks, peak_kind = load_peaks()
+    if args.part == "vda_backward":
+        ms = run_vda_backward(args, shape, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "VDA gradient pass ms (dq, dk, dv, dbeta, dalpha)",
+                              "value": ms, "unit": "ms", "higher_is_better": False,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "dtype": "bf16", "data": "synthetic", "config": config,
+                              "vda_backward": backward_row(work, peaks, ms)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    r = run_gpu(args, shape, rank, world)
     ms_step = r["ms"] / args.steps
     tokens_per_s = weak_scaling_value(world, shape.L, ms_step)
     win_tflops = work["softmax_flop"] / (r["win_ms"] / 1e3) / 1e12
@@ -392,6 +469,9 @@ def main():
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    if args.part == "all":
+        line["vda_backward"] = backward_row(work, peaks,
+                                            run_vda_backward(args, shape, rank, world))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(shape)
         line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}

@@ -93,7 +93,7 @@ typedef struct {
  * states_opt: NULL, or fp32 [2, T, H, d, d] output: [0] = S_fwd, [1] = S_bwd,
  *             each state row-major [v_dim][k_dim]
  * ws        : >= vdn_vda_scan_workspace(shape) bytes.  After the call it
- *             also holds A, B, P and C = B P (see vdn_vda_debug_buffers).
+ *             also holds A, B and P (see vdn_vda_debug_buffers).
  * ------------------------------------------------------------------------ */
 VDN_API size_t vdn_vda_scan_workspace(const vdn_shape* shape);
 
@@ -104,10 +104,10 @@ VDN_API vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const voi
 
 /* Pointers into a VDA workspace to the per-(frame, head) fp32 matrices the
  * last vdn_vda_scan on that workspace produced, each [T, H, d, d]:
- * A, B (prep), P = (I + A)^-1 and C = B P (solve).  Any out pointer may be
- * NULL.  Pure pointer arithmetic: enqueues nothing. */
+ * A, B (prep) and P = (I + A)^-1 (solve).  Any out pointer may be NULL.
+ * Pure pointer arithmetic: enqueues nothing. */
 VDN_API vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
-                                 float** P, float** C);
+                                         float** P);
 
 /* vdn_vda_scan without a workspace.  The paper has no counterpart: this
  * entry point exists for callers that cannot allocate device memory (for
@@ -117,8 +117,8 @@ VDN_API vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float
  * arguments minus ws/ws_bytes, and allocates nothing: its scratch is a
  * fixed 64 MiB array of this library's own device memory, present on every
  * GPU that loads the library until the process exits.
- *  - Limit: 256 + 6 * T*H*d*d*4 bytes must fit in 64 MiB (e.g. T*H <= 170
- *    at d = 128, <= 680 at d = 64); larger shapes return VDN_ERR_WORKSPACE
+ *  - Limit: 256 + 5 * T*H*d*d*4 bytes must fit in 64 MiB (e.g. T*H <= 204
+ *    at d = 128, <= 819 at d = 64); larger shapes return VDN_ERR_WORKSPACE
  *    before anything is enqueued.
  *  - The first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before any

@@ -45,7 +45,10 @@ def test_workspace_queries(L):
     lib = L.lib()
     s = L.Shape(102, 4032, 24, 128)
     mat = 102 * 24 * 128 * 128 * 4
-    assert lib.vdn_vda_scan_workspace(ctypes.byref(s)) == 256 + 6 * mat
+    # [status][A][B][P][states x2]; the gradient pass adds one matrix (G, then E)
+    assert lib.vdn_vda_scan_workspace(ctypes.byref(s)) == 256 + 5 * mat
+    assert lib.vdn_vda_backward_workspace(ctypes.byref(s)) == 256 + 6 * mat
+    assert lib.vdn_vda_backward_workspace(None) == 0
     assert lib.vdn_vda_scan_workspace(None) == 0
     assert lib.vdn_vda_scan_workspace(ctypes.byref(L.Shape(0, 1, 1, 64))) == 0
     assert lib.vdn_hybrid_fuse_workspace(411264, 3072, 24) == 256 + 411264 * 2 * 3072 * 2

@@ -1,7 +1,7 @@
 """Parity of vdn_vda_scan (CUDA, through the C ABI) against the CPU oracle.
 
 Small shapes are compared element by element on every intermediate
-(A, B from prep; P, C from the solve; both scans' states; o_vda).  The
+(A, B from prep; P from the solve; both scans' states; o_vda).  The
 full-size shapes (42/102 latent frames x 4032 tokens, the scan sweep) are
 compared on sampled heads (all frames' states) and sampled token rows.
 """
@@ -70,7 +70,7 @@ def test_vda_parity_small(vdn, T, N, H, d):
     o, states, ws = _run(vdn, shape, inp)
     x = {k: host(v) for k, v in inp.items()}
     A_ref, B_ref = oracle.vda_prep(x["k"], x["v"], x["beta"], T, N, H, d)
-    A, B, P, C = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
+    A, B, P = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
     for t in range(T):
         for h in range(H):
             assert max_rel(A[t, h], A_ref[t, h]) <= TOL_PREP, ("A", t, h)
@@ -79,7 +79,6 @@ def test_vda_parity_small(vdn, T, N, H, d):
             A_sym = 0.5 * (A[t, h].astype(np.float64) + A[t, h].T.astype(np.float64))
             P_ref = np.linalg.inv(np.eye(d) + A_sym)
             assert max_rel(P[t, h], P_ref) <= TOL_SOLVE, ("P", t, h)
-            assert max_rel(C[t, h], B[t, h].astype(np.float64) @ P_ref) <= TOL_SOLVE, ("C", t, h)
     S_fwd, S_bwd = oracle.vda_scan(A_ref, B_ref, x["alpha"])
     st = host(states)
     for t in range(T):
@@ -177,7 +176,7 @@ def test_vda_timeout_path_reports_and_recovers(vdn):
 
 @pytest.mark.parametrize("T,N,H,d", [(7, 200, 2, 128), (17, 33, 2, 64), (3, 4032, 1, 128)])
 def test_vda_gauss_jordan_solver(vdn, T, N, H, d):
-    """The Gauss-Jordan variant of the solve: P and C against the GPU's own
+    """The Gauss-Jordan variant of the solve: P against the GPU's own
     symmetrised A, states and o_vda against the oracle."""
     shape = synth.Shape(T, N, H, d)
     inp = _inputs(shape, seed=T * 1000 + N + 1)
@@ -187,13 +186,12 @@ def test_vda_gauss_jordan_solver(vdn, T, N, H, d):
     finally:
         vdn.set_vda_solver(vdn.SOLVER_CHOLESKY)
     x = {k: host(v) for k, v in inp.items()}
-    A, B, P, C = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
+    A, B, P = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
     for t in range(T):
         for h in range(H):
             A_sym = 0.5 * (A[t, h].astype(np.float64) + A[t, h].T.astype(np.float64))
             P_ref = np.linalg.inv(np.eye(d) + A_sym)
             assert max_rel(P[t, h], P_ref) <= TOL_SOLVE, ("P", t, h)
-            assert max_rel(C[t, h], B[t, h].astype(np.float64) @ P_ref) <= TOL_SOLVE, ("C", t, h)
     o_ref, S_fwd, S_bwd = oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], T, N, H, d)
     st = host(states)
     for t in range(T):

@@ -61,11 +61,12 @@ bool make_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld,
 cudaError_t launch_vda_prep(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                             const CUtensorMap& vmap, const float* beta, float* A, float* B);
 
-cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A,
-                             const float* B, float* P, float* C);
+// P = (I + (A + A^T)/2)^-1 per (frame, head).
+cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A, float* P);
 
+// Both scans S_t = (alpha_t S_prev + B_t) P_t into states [2, T, H, d, d].
 cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* P,
-                            const float* C, const float* alpha, float* states);
+                            const float* B, const float* alpha, float* states);
 
 cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                                const CUtensorMap& omap, const float* states);

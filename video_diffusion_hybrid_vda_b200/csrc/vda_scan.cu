@@ -2,32 +2,32 @@
 // DeltaNet", 10100.com article, 方法概述 item 2 and the figure caption under
 // 效率阶梯: a forward and a backward scan over the latent frames):
 //
-//   S_fwd_t = alpha_t S_fwd_{t-1} P_t + C_t      t = 0 .. T-1, S_fwd_{-1} = 0
-//   S_bwd_t = alpha_t S_bwd_{t+1} P_t + C_t      t = T-1 .. 0, S_bwd_T   = 0
+//   S_fwd_t = (alpha_t S_fwd_{t-1} + B_t) P_t    t = 0 .. T-1, S_fwd_{-1} = 0
+//   S_bwd_t = (alpha_t S_bwd_{t+1} + B_t) P_t    t = T-1 .. 0, S_bwd_T   = 0
 //
-// which is (alpha_t S_prev + B_t)(I + A_t)^-1 with P_t = (I + A_t)^-1 and
-// C_t = B_t P_t from the solve.  Rows of S evolve independently (row r of
-// S_t needs only row r of S_{t-1}), so each CTA owns 64 rows of one head's
-// state in one direction and runs all T steps; every CTA of the grid is
-// resident at once.  Per step the CTA stages P_t (d x d fp32) into shared
-// memory with one bulk copy, double-buffered so that P_{t+1} lands while
-// step t computes; the state rows stay in shared memory (row stride d + 4,
-// so four consecutive k of a row are one float4 and the rows of a warp fall
-// in different banks) and each thread computes 4 rows x 8 columns of the new
-// state with packed f32x2 FMA.  A thread's columns are two interleaved
-// groups of 4 (4c.., d/2 + 4c..), so each quarter warp reads 128 contiguous
-// bytes of P.
-// The scan is serial over T and FP32-ALU bound.
+// with P_t = (I + A_t)^-1 from the solve.  Rows of S evolve independently
+// (row r of S_t needs only row r of S_{t-1}), so each CTA owns 64 rows of
+// one head's state in one direction and runs all T steps; every CTA of the
+// grid is resident at once.  Per step the CTA stages P_t (d x d fp32) into
+// shared memory with one bulk copy, double-buffered so that P_{t+1} lands
+// while step t computes.  Each thread first writes its tile of the bracket
+// alpha S_prev + B_t into the shared rows (row stride d + 4, so four
+// consecutive k of a row are one float4 and the rows of a warp fall in
+// different banks), then computes 4 rows x 8 columns of the new state with
+// packed f32x2 FMA.  A thread's columns are two interleaved groups of 4
+// (4c.., d/2 + 4c..), so each quarter warp reads 128 contiguous bytes of P.
+// Multiplying the bracket (rather than adding a precomputed B_t P_t) keeps
+// the d^3 product C = B P out of the solve, at the price of one product at
+// the first step.  The scan is serial over T and FP32-ALU bound.
 //
 // Adjoint mode (kAdjoint) runs the two scans of the gradient pass.  With
-// G_t = sum_i dO_i q_i^T, the sensitivity of the loss to the bracket
-// (alpha S_prev + B_t) of each direction obeys
+// G_t = sum_i dO_i q_i^T, the sensitivity of the loss to the bracket of
+// each direction obeys
 //   D_t = (alpha_u D_u + G_t) P_t,   u = the frame the same scan visited
-// one step earlier (t - 1 going forward in time, t + 1 going backward).
-// The thread first writes its tile of alpha_u D_u + G_t into the shared
-// rows and then multiplies by P_t, so the step costs the same as the
-// forward's; output direction 0 (forward in time) is the adjoint of the
-// backward scan, direction 1 the adjoint of the forward scan.
+// one step earlier (t - 1 going forward in time, t + 1 going backward):
+// the same step with G in place of B and the decay of the previous frame.
+// Output direction 0 (forward in time) is the adjoint of the backward scan,
+// direction 1 the adjoint of the forward scan.
 #include "common.cuh"
 #include "exp2_fma.cuh"
 #include "ptx.cuh"
@@ -49,7 +49,7 @@ struct ScanCfg {
 
 template <int DH, bool kAdjoint>
 __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
-    vda_scan_kernel(const float* __restrict__ P, const float* __restrict__ C,
+    vda_scan_kernel(const float* __restrict__ P, const float* __restrict__ X,
                     const float* __restrict__ alpha, float* __restrict__ states, int T, int H,
                     uint32_t* status, uint64_t budget_ns) {
   using Cfg = ScanCfg<DH>;
@@ -83,11 +83,11 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   }
   __syncthreads();
 
-  float dprev[kTR][kTC];  // adjoint mode: the thread's tile of D from the previous step
+  float sprev[kTR][kTC];  // the thread's tile of the previous step's state
 #pragma unroll
   for (int r = 0; r < kTR; ++r)
 #pragma unroll
-    for (int c = 0; c < kTC; ++c) dprev[r][c] = 0.f;
+    for (int c = 0; c < kTC; ++c) sprev[r][c] = 0.f;
 
   int issued = 1;
 #pragma unroll 1
@@ -105,27 +105,21 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     // visited one step earlier (unused at step 0, where the carried term is 0)
     const float a = !kAdjoint ? __ldg(alpha + t * H + h)
                               : (step > 0 ? __ldg(alpha + frame(step - 1) * H + h) : 0.f);
-    const float* Ct = C + (static_cast<int64_t>(t) * H + h) * mat;
-    float4 cv[kTR][2];
+    const float* Xt = X + (static_cast<int64_t>(t) * H + h) * mat;
+    // U = a S_prev + X_t into the shared rows; every thread left the previous
+    // step's reads behind the barrier that closed it, and the barrier below
+    // publishes U before the multiply
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
-      cv[r][0] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colA));
-      cv[r][1] = __ldg(reinterpret_cast<const float4*>(Ct + (row0 + r) * DH + colB));
-    }
-    if constexpr (kAdjoint) {
-      // U = a D_prev + G_t into the shared rows; every thread left the
-      // previous step's reads behind the barrier that closed it, and the
-      // barrier below publishes U before the multiply
-#pragma unroll
-      for (int r = 0; r < kTR; ++r) {
-        float* srow = Ss + (lrow0 + r) * Cfg::LDS;
-        *reinterpret_cast<float4*>(srow + colA) = make_float4(
-            fmaf(a, dprev[r][0], cv[r][0].x), fmaf(a, dprev[r][1], cv[r][0].y),
-            fmaf(a, dprev[r][2], cv[r][0].z), fmaf(a, dprev[r][3], cv[r][0].w));
-        *reinterpret_cast<float4*>(srow + colB) = make_float4(
-            fmaf(a, dprev[r][4], cv[r][1].x), fmaf(a, dprev[r][5], cv[r][1].y),
-            fmaf(a, dprev[r][6], cv[r][1].z), fmaf(a, dprev[r][7], cv[r][1].w));
-      }
+      const float4 xa = __ldg(reinterpret_cast<const float4*>(Xt + (row0 + r) * DH + colA));
+      const float4 xb = __ldg(reinterpret_cast<const float4*>(Xt + (row0 + r) * DH + colB));
+      float* srow = Ss + (lrow0 + r) * Cfg::LDS;
+      *reinterpret_cast<float4*>(srow + colA) =
+          make_float4(fmaf(a, sprev[r][0], xa.x), fmaf(a, sprev[r][1], xa.y),
+                      fmaf(a, sprev[r][2], xa.z), fmaf(a, sprev[r][3], xa.w));
+      *reinterpret_cast<float4*>(srow + colB) =
+          make_float4(fmaf(a, sprev[r][4], xb.x), fmaf(a, sprev[r][5], xb.y),
+                      fmaf(a, sprev[r][6], xb.z), fmaf(a, sprev[r][7], xb.w));
     }
     const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
     if (!__syncthreads_and(ok)) {
@@ -139,7 +133,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     for (int r = 0; r < kTR; ++r)
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
-    if (kAdjoint || step > 0) {
+    {
 #pragma unroll 1
       for (int k = 0; k < DH; k += 4) {
         float sr[kTR][4];
@@ -164,17 +158,12 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
       }
     }
     float snew[kTR][kTC];
-    const uint64_t aa = f32x2_pack(a, a);
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
-      const float cc[8] = {cv[r][0].x, cv[r][0].y, cv[r][0].z, cv[r][0].w,
-                           cv[r][1].x, cv[r][1].y, cv[r][1].z, cv[r][1].w};
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) {
-        const uint64_t v =
-            kAdjoint ? acc2[r][q] : f32x2_fma(aa, acc2[r][q], f32x2_pack(cc[2 * q], cc[2 * q + 1]));
-        snew[r][2 * q] = f32x2_lo(v);
-        snew[r][2 * q + 1] = f32x2_hi(v);
+        snew[r][2 * q] = f32x2_lo(acc2[r][q]);
+        snew[r][2 * q + 1] = f32x2_hi(acc2[r][q]);
       }
       float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
                    static_cast<int64_t>(row0 + r) * DH;
@@ -184,21 +173,10 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
           make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
     }
     __syncthreads();  // every thread has finished reading Ss (and Pbuf b)
-    if constexpr (kAdjoint) {
 #pragma unroll
-      for (int r = 0; r < kTR; ++r)
+    for (int r = 0; r < kTR; ++r)
 #pragma unroll
-        for (int c = 0; c < kTC; ++c) dprev[r][c] = snew[r][c];
-    } else {
-#pragma unroll
-      for (int r = 0; r < kTR; ++r) {
-        *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colA) =
-            make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
-        *reinterpret_cast<float4*>(Ss + (lrow0 + r) * Cfg::LDS + colB) =
-            make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
-      }
-      __syncthreads();
-    }
+      for (int c = 0; c < kTC; ++c) sprev[r][c] = snew[r][c];
   }
   // the bulk copies this CTA started must land before it exits
   if (threadIdx.x == 0) {
@@ -208,7 +186,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
 }
 
 template <int DH, bool kAdjoint>
-cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* C,
+cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* X,
                            const float* alpha, float* states) {
   using Cfg = ScanCfg<DH>;
   static bool attr_set = false;
@@ -220,16 +198,16 @@ cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P
   }
   dim3 grid(DH / kRows, s.H, 2);
   vda_scan_kernel<DH, kAdjoint><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      P, C, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
+      P, X, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* P,
-                            const float* C, const float* alpha, float* states) {
-  if (s.d == 128) return launch_scan_dh<128, false>(ctx, s, P, C, alpha, states);
-  if (s.d == 64) return launch_scan_dh<64, false>(ctx, s, P, C, alpha, states);
+                            const float* B, const float* alpha, float* states) {
+  if (s.d == 128) return launch_scan_dh<128, false>(ctx, s, P, B, alpha, states);
+  if (s.d == 64) return launch_scan_dh<64, false>(ctx, s, P, B, alpha, states);
   return cudaErrorInvalidValue;
 }
 

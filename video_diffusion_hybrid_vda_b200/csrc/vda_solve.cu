@@ -3,7 +3,7 @@
 //
 // Per (frame t, head h) one CTA of 256 threads (two CTAs per SM, so two
 // problems hide each other's barrier latency) produces
-//   P_t = (I + A_sym)^-1  and  C_t = B_t P_t,   A_sym = (A + A^T) / 2
+//   P_t = (I + A_sym)^-1,   A_sym = (A + A^T) / 2
 // (the tensor-core product in the prep rounds beta*k on one operand only, so
 // A is symmetric up to that rounding).  Two solvers:
 //
@@ -13,11 +13,12 @@
 //      through shared memory each step and L is kept in shared memory;
 //   2. W = L^-1 by forward substitution against I (row k of W is published
 //      each step; column blocks that are still zero are skipped);
-//   3. P = W^T W as a shared-memory product (no barriers inside the loop).
+//   3. P = W^T W as a shared-memory product (no barriers inside the loop);
+//      W is lower triangular, so entry (i, c) sums rows k >= max(i, c) only.
 //  Gauss-Jordan (the inverse the pages' own kernels use):
 //   one in-register sweep over the pivots, publishing the pivot row and
 //   column each step, leaves (I + A_sym)^-1.
-//  Both: 4. C = B P with P in shared memory and B read through L2.
+// The scan multiplies (alpha S + B_t) by P_t itself, so no B P is formed here.
 //
 // I + A_sym is symmetric positive definite with eigenvalues >= 1 (beta >= 0),
 // so neither solver pivots; a non-positive or NaN pivot is reported as
@@ -78,55 +79,11 @@ __device__ __forceinline__ void load_spd(const float* __restrict__ Am,
     }
 }
 
-// C = B P for one problem: P in shared memory ([DH][LD2]), B through L2.
-// Thread tile TR x TR at rows i0 = TR * (tid / 16), columns c0 = TR * (tid % 16).
-template <int DH>
-__device__ __forceinline__ void c_equals_b_times_p(const float* __restrict__ Bm, const float* Ps,
-                                                   float* __restrict__ Cm) {
-  using Cfg = SolveCfg<DH>;
-  constexpr int TR = Cfg::TR;
-  const int i0 = (threadIdx.x >> 4) * TR, c0 = (threadIdx.x & 15) * TR;
-  float acc[TR][TR];
-#pragma unroll
-  for (int a = 0; a < TR; ++a)
-#pragma unroll
-    for (int b = 0; b < TR; ++b) acc[a][b] = 0.f;
-#pragma unroll 1
-  for (int k = 0; k < DH; k += 4) {
-    float bv[TR][4];
-#pragma unroll
-    for (int a = 0; a < TR; ++a) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(Bm + (i0 + a) * DH + k));
-      bv[a][0] = v.x; bv[a][1] = v.y; bv[a][2] = v.z; bv[a][3] = v.w;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      float pc[TR];
-#pragma unroll
-      for (int b = 0; b < TR; b += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(Ps + (k + kk) * Cfg::LD2 + c0 + b);
-        pc[b] = v.x; pc[b + 1] = v.y; pc[b + 2] = v.z; pc[b + 3] = v.w;
-      }
-#pragma unroll
-      for (int a = 0; a < TR; ++a)
-#pragma unroll
-        for (int b = 0; b < TR; ++b) acc[a][b] = fmaf(bv[a][kk], pc[b], acc[a][b]);
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < TR; ++a)
-#pragma unroll
-    for (int b = 0; b < TR; b += 4)
-      *reinterpret_cast<float4*>(Cm + (i0 + a) * DH + c0 + b) =
-          make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
-}
-
 // ---------------------------------------------------------------- Cholesky
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2)
-    vda_solve_kernel(const float* __restrict__ A, const float* __restrict__ B,
-                     float* __restrict__ P, float* __restrict__ Cout, uint32_t* status) {
+    vda_solve_kernel(const float* __restrict__ A, float* __restrict__ P, uint32_t* status) {
   using Cfg = SolveCfg<DH>;
   extern __shared__ float sm[];
   float* Ls = sm;                    // [DH][LD]: L, later W and P ([DH][LD2])
@@ -237,8 +194,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int a = 0; a < TR; ++a)
 #pragma unroll
       for (int b = 0; b < TR; ++b) acc[a][b] = 0.f;
+    // W[k][i] = 0 for k < i: rows below max(i0, c0) add nothing to the tile
 #pragma unroll 2
-    for (int k = 0; k < DH; ++k) {
+    for (int k = max(i0, c0); k < DH; ++k) {
       const float* wk = sm + k * Cfg::LD2;
       float wi[TR], wc[TR];
 #pragma unroll
@@ -256,21 +214,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int b = 0; b < TR; ++b) acc[a][b] = fmaf(wi[a], wc[b], acc[a][b]);
     }
-    __syncthreads();  // all reads of W done: the buffer now takes P
     float* Pm = P + mat;
 #pragma unroll
     for (int a = 0; a < TR; ++a)
 #pragma unroll
-      for (int b = 0; b < TR; b += 4) {
-        const float4 v = make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
-        *reinterpret_cast<float4*>(sm + (i0 + a) * Cfg::LD2 + c0 + b) = v;
-        *reinterpret_cast<float4*>(Pm + (i0 + a) * DH + c0 + b) = v;
-      }
+      for (int b = 0; b < TR; b += 4)
+        *reinterpret_cast<float4*>(Pm + (i0 + a) * DH + c0 + b) =
+            make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
   }
-  __syncthreads();
-
-  // ---------------------------------------------------------------- 4. C = B P
-  c_equals_b_times_p<DH>(B + mat, sm, Cout + mat);
   if (bad) record_status(status, kStatusNumeric);
 }
 
@@ -281,8 +232,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // diagonals of an SPD matrix with eigenvalues >= 1.
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2)
-    vda_solve_gj_kernel(const float* __restrict__ A, const float* __restrict__ B,
-                        float* __restrict__ P, float* __restrict__ Cout, uint32_t* status) {
+    vda_solve_gj_kernel(const float* __restrict__ A, float* __restrict__ P, uint32_t* status) {
   using Cfg = SolveCfg<DH>;
   extern __shared__ float sm[];
   float* rowb = sm + Cfg::MAT;   // 2 x [DH] pivot rows
@@ -347,19 +297,13 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
   for (int a = 0; a < Cfg::RA; ++a)
 #pragma unroll
-    for (int b = 0; b < Cfg::CB; ++b) {
-      const int i = ty + 16 * a, k = tx + 16 * b;
-      sm[i * Cfg::LD2 + k] = m[a][b];
-      Pm[i * DH + k] = m[a][b];
-    }
-  __syncthreads();
-  c_equals_b_times_p<DH>(B + mat, sm, Cout + mat);
+    for (int b = 0; b < Cfg::CB; ++b) Pm[(ty + 16 * a) * DH + tx + 16 * b] = m[a][b];
   if (bad) record_status(status, kStatusNumeric);
 }
 
 template <int DH>
-cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* A,
-                            const float* B, float* P, float* C, int solver) {
+cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* A, float* P,
+                            int solver) {
   using Cfg = SolveCfg<DH>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -372,20 +316,18 @@ cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* 
     attr_set = true;
   }
   if (solver == VDN_SOLVER_GAUSS_JORDAN)
-    vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, B, P, C,
-                                                                           ctx.status);
+    vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
   else
-    vda_solve_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, B, P, C, ctx.status);
+    vda_solve_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A,
-                             const float* B, float* P, float* C) {
+cudaError_t launch_vda_solve(const Launch& ctx, const vdn_shape& s, const float* A, float* P) {
   const int solver = current_vda_solver();
-  if (s.d == 128) return launch_solve_dh<128>(ctx, s, A, B, P, C, solver);
-  if (s.d == 64) return launch_solve_dh<64>(ctx, s, A, B, P, C, solver);
+  if (s.d == 128) return launch_solve_dh<128>(ctx, s, A, P, solver);
+  if (s.d == 64) return launch_solve_dh<64>(ctx, s, A, P, solver);
   return cudaErrorInvalidValue;
 }
 

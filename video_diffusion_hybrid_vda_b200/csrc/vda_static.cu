@@ -4,7 +4,7 @@
 // inside a host framework which owns every device allocation, or a loop with
 // a fixed memory budget where a cudaMalloc (and the device synchronisation
 // it can imply) is not allowed.  For them, vdn_vda_scan_static keeps its
-// scratch (the per-(frame, head) A, B, P, C matrices and both scans' states)
+// scratch (the per-(frame, head) A, B, P matrices and both scans' states)
 // in a fixed-size array of this library's own device memory instead of a
 // caller-provided workspace.  The array exists on every GPU that loads the
 // library, until the process exits.
@@ -15,8 +15,8 @@
 namespace vdn {
 namespace {
 
-// 64 MiB: room for T*H*d*d*4*6 bytes of scratch plus the status word, e.g.
-// 170 (frame, head) pairs at d = 128 or 680 pairs at d = 64.
+// 64 MiB: room for T*H*d*d*4*5 bytes of scratch plus the status word, e.g.
+// 204 (frame, head) pairs at d = 128 or 819 pairs at d = 64.
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;
 
 static __device__ __align__(256) uint8_t g_vda_scratch[kStaticScratchBytes];
@@ -72,9 +72,9 @@ extern "C" vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q,
       (dev_status_opt && !ptr_aligned(dev_status_opt, 4)))
     return VDN_ERR_INVALID_ARG;
   if (ld < D || ld % 8 || ld_o < D || ld_o % 8) return VDN_ERR_INVALID_ARG;
-  // scratch: [status 256 B][A][B][P][C][states x2], as in the workspace path
+  // scratch: [status 256 B][A][B][P][states x2], as in the workspace path
   const size_t mat = round_up256(static_cast<size_t>(s.T) * s.H * s.d * s.d * sizeof(float));
-  const size_t need = kStatusBytes + 6 * mat;
+  const size_t need = kStatusBytes + 5 * mat;
   if (need > kStaticScratchBytes) return VDN_ERR_WORKSPACE;  // beyond the fixed maximum
 
   uint8_t* base = nullptr;
@@ -82,9 +82,8 @@ extern "C" vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q,
   float* A = reinterpret_cast<float*>(base + kStatusBytes);
   float* B = reinterpret_cast<float*>(base + kStatusBytes + mat);
   float* P = reinterpret_cast<float*>(base + kStatusBytes + 2 * mat);
-  float* C = reinterpret_cast<float*>(base + kStatusBytes + 3 * mat);
   float* states =
-      states_opt ? states_opt : reinterpret_cast<float*>(base + kStatusBytes + 4 * mat);
+      states_opt ? states_opt : reinterpret_cast<float*>(base + kStatusBytes + 3 * mat);
 
   CUtensorMap kmap, vmap, qmap, omap;
   const int prep_rows = s.d == 128 ? 32 : 64;
@@ -99,8 +98,8 @@ extern "C" vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q,
   if (cudaMemsetAsync(base, 0, sizeof(uint32_t), st) != cudaSuccess) return VDN_ERR_CUDA;
   Launch ctx{st, reinterpret_cast<uint32_t*>(base), current_wait_budget_ns()};
   if (launch_vda_prep(ctx, s, kmap, vmap, beta, A, B) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_solve(ctx, s, A, P) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
   if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
   if (dev_status_opt != nullptr &&
       cudaMemcpyAsync(dev_status_opt, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) !=

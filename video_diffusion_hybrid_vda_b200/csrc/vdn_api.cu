@@ -56,26 +56,27 @@ bool head_dim_padded(int d) { return d == 16 || d == 32; }
 
 bool ld_ok(int64_t ld, int64_t D) { return ld >= D && ld % 8 == 0; }
 
-// VDA workspace: [status 256 B][A][B][P][C][states (2x)], each region
-// 256-byte aligned, every matrix fp32 [T, H, d, d].
+// VDA workspace: [status 256 B][A][B][P]([X])[states (2x)], each region
+// 256-byte aligned, every matrix fp32 [T, H, d, d]; the gradient pass adds
+// the slot X (for G, then E).
 struct VdaLayout {
-  size_t mat_bytes, A, B, P, C, states, total;
+  size_t mat_bytes, A, B, P, X, states, total;
 };
 
-VdaLayout vda_layout(const vdn_shape& s) {
+VdaLayout vda_layout(const vdn_shape& s, bool with_x) {
   VdaLayout l;
   l.mat_bytes = round_up(static_cast<size_t>(s.T) * s.H * s.d * s.d * sizeof(float), 256);
   l.A = kStatusBytes;
   l.B = l.A + l.mat_bytes;
   l.P = l.B + l.mat_bytes;
-  l.C = l.P + l.mat_bytes;
-  l.states = l.C + l.mat_bytes;
+  l.X = l.P + l.mat_bytes;
+  l.states = l.X + (with_x ? l.mat_bytes : 0);
   l.total = l.states + 2 * l.mat_bytes;
   return l;
 }
 
 // Workspace of a VDA call.  Head dims 16 and 32 run through a 64-wide padded
-// copy: [status][nact padded activations, bf16 L x H*64][A B P C S_fwd S_bwd
+// copy: [status][nact padded activations, bf16 L x H*64][the layout above
 // for d = 64]; the forward pads q' k' v' o' (4), the gradient pass q' k' v'
 // dO' dq' dk' dv' (7).
 struct VdaPlan {
@@ -87,12 +88,13 @@ struct VdaPlan {
   size_t total;
 };
 
-VdaPlan vda_plan(const vdn_shape& s, int nact = 4) {
+VdaPlan vda_plan(const vdn_shape& s, bool backward = false) {
+  const int nact = backward ? 7 : 4;
   VdaPlan p;
   p.padded = head_dim_padded(s.d);
   p.inner = s;
   if (p.padded) p.inner.d = 64;
-  p.lay = vda_layout(p.inner);
+  p.lay = vda_layout(p.inner, backward);
   p.act = p.padded ? round_up(static_cast<size_t>(s.T) * s.N * s.H * 64 * 2, 256) : 0;
   p.inner_off = nact * p.act;
   p.total = p.lay.total + p.inner_off;
@@ -102,7 +104,7 @@ VdaPlan vda_plan(const vdn_shape& s, int nact = 4) {
 // The four VDA kernels on head dim 64 or 128.
 vdn_status run_vda(const Launch& ctx, const vdn_shape& s, const void* q, const void* k,
                    const void* v, int64_t ld, const float* beta, const float* alpha, void* o,
-                   int64_t ld_o, float* A, float* B, float* P, float* C, float* states) {
+                   int64_t ld_o, float* A, float* B, float* P, float* states) {
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   const int prep_rows = s.d == 128 ? 32 : 64;
   CUtensorMap kmap, vmap, qmap, omap;
@@ -112,23 +114,23 @@ vdn_status run_vda(const Launch& ctx, const vdn_shape& s, const void* q, const v
       !make_frame_map(&omap, o, D, ld_o, s.N, s.T, 128))
     return VDN_ERR_CUDA;
   if (launch_vda_prep(ctx, s, kmap, vmap, beta, A, B) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess) return VDN_ERR_CUDA;
-  if (launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_solve(ctx, s, A, P) != cudaSuccess) return VDN_ERR_CUDA;
+  if (launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess) return VDN_ERR_CUDA;
   if (launch_vda_readout(ctx, s, qmap, omap, states) != cudaSuccess) return VDN_ERR_CUDA;
   return VDN_OK;
 }
 
 // The gradient pass on head dim 64 or 128.  Workspace slots (in memory
-// order A, B, P, C, states) are reused as their contents die: G goes to C
-// (dead after the forward scan), the adjoint states to A and B (dead after
-// the solve; adjacent, so they form one [2, T, H, d, d] array), E to C (G
-// is dead after the adjoint scan).  P is read by both adjoint directions
-// until the adjoint scan ends, so nothing is written there.
+// order A, B, P, X, states) are reused as their contents die: G goes to X,
+// the adjoint states to A and B (dead after the forward scan; adjacent, so
+// they form one [2, T, H, d, d] array), E to X (G is dead after the adjoint
+// scan).  P is read by both adjoint directions until the adjoint scan ends,
+// so nothing is written there.
 vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q, const void* k,
                             const void* v, int64_t ld, const float* beta, const float* alpha,
                             const void* d_o, int64_t ld_do, void* dq, void* dk, void* dv,
                             int64_t ld_g, float* dbeta, float* dalpha, float* A, float* B,
-                            float* P, float* C, float* states) {
+                            float* P, float* X, float* states) {
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   const int prep_rows = s.d == 128 ? 32 : 64;
   CUtensorMap kmap_p, vmap_p, qmap_p, domap_p, domap, dqmap, kmap, vmap, dvmap, dkmap;
@@ -143,12 +145,12 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
       !make_frame_map(&dvmap, dv, D, ld_g, s.N, s.T, 128) ||
       !make_frame_map(&dkmap, dk, D, ld_g, s.N, s.T, 128))
     return VDN_ERR_CUDA;
-  float* G = C;
+  float* G = X;
   float* adj = A;
-  float* E = C;
+  float* E = X;
   if (launch_vda_prep(ctx, s, kmap_p, vmap_p, beta, A, B) != cudaSuccess ||
-      launch_vda_solve(ctx, s, A, B, P, C) != cudaSuccess ||
-      launch_vda_scan(ctx, s, P, C, alpha, states) != cudaSuccess ||
+      launch_vda_solve(ctx, s, A, P) != cudaSuccess ||
+      launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess ||
       launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
       launch_vda_adjoint_scan(ctx, s, P, G, alpha, adj) != cudaSuccess ||
       launch_vda_grad_combine(ctx, s, states, adj, E, dalpha) != cudaSuccess ||
@@ -250,14 +252,13 @@ size_t vdn_vda_scan_workspace(const vdn_shape* shape) {
 }
 
 vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float** A, float** B,
-                                 float** P, float** C) {
+                                 float** P) {
   if (!shape_ok(shape) || ws == nullptr) return VDN_ERR_INVALID_ARG;
   const VdaPlan pl = vda_plan(*shape);
   uint8_t* base = static_cast<uint8_t*>(ws) + pl.inner_off;
   if (A) *A = reinterpret_cast<float*>(base + pl.lay.A);
   if (B) *B = reinterpret_cast<float*>(base + pl.lay.B);
   if (P) *P = reinterpret_cast<float*>(base + pl.lay.P);
-  if (C) *C = reinterpret_cast<float*>(base + pl.lay.C);
   return VDN_OK;
 }
 
@@ -285,12 +286,11 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
   float* A = reinterpret_cast<float*>(inner + pl.lay.A);
   float* B = reinterpret_cast<float*>(inner + pl.lay.B);
   float* P = reinterpret_cast<float*>(inner + pl.lay.P);
-  float* C = reinterpret_cast<float*>(inner + pl.lay.C);
   float* states_ws = reinterpret_cast<float*>(inner + pl.lay.states);
   Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
              g_budget_ns.load()};
   if (!pl.padded)
-    return run_vda(ctx, s, q, k, v, ld, beta, alpha, o_vda, ld_o, A, B, P, C,
+    return run_vda(ctx, s, q, k, v, ld, beta, alpha, o_vda, ld_o, A, B, P,
                    states_opt ? states_opt : states_ws);
 
   // d = 16 or 32: run on a zero-padded 64-wide copy of every head
@@ -306,7 +306,7 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
       launch_repack_bf16(st, vp, D64, v, ld, 1, L, L, H, 64, d) != cudaSuccess)
     return VDN_ERR_CUDA;
   const vdn_status r =
-      run_vda(ctx, pl.inner, qp, kp, vp, D64, beta, alpha, op, D64, A, B, P, C, states_ws);
+      run_vda(ctx, pl.inner, qp, kp, vp, D64, beta, alpha, op, D64, A, B, P, states_ws);
   if (r != VDN_OK) return r;
   if (launch_repack_bf16(st, o_vda, ld_o, op, D64, 1, L, L, H, d, 64) != cudaSuccess)
     return VDN_ERR_CUDA;
@@ -321,17 +321,17 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
 
 size_t vdn_vda_backward_workspace(const vdn_shape* shape) {
   if (!shape_ok(shape)) return 0;
-  return vda_plan(*shape, 7).total;
+  return vda_plan(*shape, true).total;
 }
 
 vdn_status vdn_vda_backward_debug_buffers(const vdn_shape* shape, void* ws, float** states,
                                           float** adj, float** E) {
   if (!shape_ok(shape) || ws == nullptr) return VDN_ERR_INVALID_ARG;
-  const VdaPlan pl = vda_plan(*shape, 7);
+  const VdaPlan pl = vda_plan(*shape, true);
   uint8_t* base = static_cast<uint8_t*>(ws) + pl.inner_off;
   if (states) *states = reinterpret_cast<float*>(base + pl.lay.states);
   if (adj) *adj = reinterpret_cast<float*>(base + pl.lay.A);
-  if (E) *E = reinterpret_cast<float*>(base + pl.lay.C);
+  if (E) *E = reinterpret_cast<float*>(base + pl.lay.X);
   return VDN_OK;
 }
 
@@ -354,7 +354,7 @@ vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k
       !aligned(alpha, 4) || !aligned(dbeta, 4) || !aligned(dalpha, 4))
     return VDN_ERR_INVALID_ARG;
   if (!ld_ok(ld, D) || !ld_ok(ld_do, D) || !ld_ok(ld_g, D)) return VDN_ERR_INVALID_ARG;
-  const VdaPlan pl = vda_plan(s, 7);
+  const VdaPlan pl = vda_plan(s, true);
   if (ws == nullptr || !aligned(ws, 256) || ws_bytes < pl.total) return VDN_ERR_WORKSPACE;
 
   uint8_t* base = static_cast<uint8_t*>(ws);
@@ -362,13 +362,13 @@ vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k
   float* A = reinterpret_cast<float*>(inner + pl.lay.A);
   float* B = reinterpret_cast<float*>(inner + pl.lay.B);
   float* P = reinterpret_cast<float*>(inner + pl.lay.P);
-  float* C = reinterpret_cast<float*>(inner + pl.lay.C);
+  float* X = reinterpret_cast<float*>(inner + pl.lay.X);
   float* states = reinterpret_cast<float*>(inner + pl.lay.states);
   Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
              g_budget_ns.load()};
   if (!pl.padded)
     return run_vda_backward(ctx, s, q, k, v, ld, beta, alpha, d_o, ld_do, dq, dk, dv, ld_g,
-                            dbeta, dalpha, A, B, P, C, states);
+                            dbeta, dalpha, A, B, P, X, states);
 
   // d = 16 or 32: every head zero-padded to 64 columns (exact, see repack.cu)
   const int L = s.T * s.N, H = s.H, d = s.d;
@@ -383,7 +383,7 @@ vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k
       return VDN_ERR_CUDA;
   const vdn_status r = run_vda_backward(ctx, pl.inner, pad[0], pad[1], pad[2], D64, beta, alpha,
                                         pad[3], D64, pad[4], pad[5], pad[6], D64, dbeta, dalpha,
-                                        A, B, P, C, states);
+                                        A, B, P, X, states);
   if (r != VDN_OK) return r;
   void* dst[3] = {dq, dk, dv};
   for (int i = 0; i < 3; ++i)

@@ -64,7 +64,7 @@ def lib():
     L.vdn_vda_scan_workspace.restype = _SZ
     L.vdn_vda_scan.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]
     L.vdn_vda_scan.restype = ctypes.c_int
-    L.vdn_vda_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 4
+    L.vdn_vda_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 3
     L.vdn_vda_debug_buffers.restype = ctypes.c_int
     L.vdn_window_attn_workspace.argtypes = [S]
     L.vdn_window_attn_workspace.restype = _SZ
@@ -204,8 +204,8 @@ def vda_scan(q, k, v, beta, alpha, T, N, H, d, out=None, states=None, ws=None, s
 
 
 def vda_debug_buffers(ws, T, N, H, d):
-    """(A, B, P, C) views into a VDA workspace, each fp32 [T, H, d, d]."""
-    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    """(A, B, P) views into a VDA workspace, each fp32 [T, H, d, d]."""
+    ptrs = [ctypes.c_void_p() for _ in range(3)]
     _check(lib().vdn_vda_debug_buffers(ctypes.byref(_shape(T, N, H, d)), _ptr(ws),
                                        *[ctypes.byref(p) for p in ptrs]), "vdn_vda_debug_buffers")
     base = ws.data_ptr()
