@@ -7,14 +7,10 @@
 // (the tensor-core product in the prep rounds beta*k on one operand only, so
 // A is symmetric up to that rounding).  Two solvers:
 //
-//  Cholesky (default):
-//   1. L L^T = I + A_sym, right-looking; the matrix lives in registers
-//      (8x8 per thread at d = 128), the scaled pivot column is published
-//      through shared memory each step and L is kept in shared memory;
-//   2. W = L^-1 by forward substitution against I (row k of W is published
-//      each step; column blocks that are still zero are skipped);
-//   3. P = W^T W as a shared-memory product (no barriers inside the loop);
-//      W is lower triangular, so entry (i, c) sums rows k >= max(i, c) only.
+//  Cholesky (default): blocked in 16 x 16 blocks; one warp factors and
+//   inverts each diagonal block with shuffles, every thread takes part in
+//   the panel and trailing block products; then W = L^-1 by blocked forward
+//   substitution and P = W^T W (see the kernel's own comment).
 //  Gauss-Jordan (the inverse the pages' own kernels use):
 //   one in-register sweep over the pivots, publishing the pivot row and
 //   column each step, leaves (I + A_sym)^-1.
@@ -24,6 +20,7 @@
 // so neither solver pivots; a non-positive or NaN pivot is reported as
 // VDN_ERR_NUMERIC.  This step is FP32-ALU and latency bound.
 #include "common.cuh"
+#include "exp2_fma.cuh"
 #include "ptx.cuh"
 
 namespace vdn {
@@ -43,28 +40,6 @@ struct SolveCfg {
   static constexpr int SMEM = MAT * 4 + 4 * DH * 4;
 };
 
-// Scale row group `ka` of the register tile by `dinv`, write it back and
-// publish it (4 floats per 64-column group) to shared memory.  Predicated
-// selects keep the tile in registers.
-template <int RA, int RG>
-__device__ __forceinline__ void publish_row(float (&r)[RA][RG][4], int ka, float dinv,
-                                            float* dst) {
-#pragma unroll
-  for (int g = 0; g < RG; ++g) {
-    float y[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float v = r[0][g][e];
-#pragma unroll
-      for (int a = 1; a < RA; ++a) v = (a == ka) ? r[a][g][e] : v;
-      y[e] = v * dinv;
-#pragma unroll
-      for (int a = 0; a < RA; ++a) r[a][g][e] = (a == ka) ? y[e] : r[a][g][e];
-    }
-    *reinterpret_cast<float4*>(dst + 64 * g) = make_float4(y[0], y[1], y[2], y[3]);
-  }
-}
-
 // Load (I + A_sym) into the register tile m (rows ty + 16 a, cols tx + 16 b).
 template <int DH>
 __device__ __forceinline__ void load_spd(const float* __restrict__ Am,
@@ -80,147 +55,255 @@ __device__ __forceinline__ void load_spd(const float* __restrict__ Am,
 }
 
 // ---------------------------------------------------------------- Cholesky
+//
+// Blocked in 16 x 16 blocks (NB = DH / 16 block rows).  Thread (ty, tx)
+// holds element (ty, tx) of every block, so block products need no
+// reshuffling: a block (a, b) of the register tile is m[a][b].
+//
+//  1. factor, for p = 0 .. NB-1:
+//     a. every thread stages block column p (rows >= 16p) in Apan;
+//     b. warp 0 factors the diagonal block with shuffles (lane j holds
+//        column j; the pivot column is broadcast row by row) into L_pp and
+//        inverts it, W_pp = L_pp^-1 (one column per lane); both to smem;
+//     c. L_ip = A_ip W_pp^T for the blocks below (16-term dot products);
+//     d. trailing update A_ab -= L_ap L_bp^T for p < b <= a (packed f32x2);
+//  2. W = L^-1 in place, block row by block row:
+//     W_ij = -W_ii sum_{k=j}^{i-1} L_ik W_kj   (j < i);
+//  3. P = W^T W over the rows where W can be nonzero (k >= max(i, c)).
+// About 54 barriers in all (the unblocked form needs two per column).
+template <int DH>
+struct CholCfg {
+  static constexpr int NB = DH / 16;
+  static constexpr int LDL = DH + 4;   // row stride of L / W (float4 rows)
+  static constexpr int LDP = 20;       // row stride of the 16-wide staging blocks
+  static constexpr int SMEM = (DH * LDL + DH * LDP + NB * 16 * LDP) * 4;
+};
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2)
     vda_solve_kernel(const float* __restrict__ A, float* __restrict__ P, uint32_t* status) {
-  using Cfg = SolveCfg<DH>;
-  extern __shared__ float sm[];
-  float* Ls = sm;                    // [DH][LD]: L, later W and P ([DH][LD2])
-  float* buf0 = sm + Cfg::MAT;       // two 2*DH broadcast buffers
-  float* buf1 = buf0 + 2 * DH;
+  using Cfg = CholCfg<DH>;
+  constexpr int NB = Cfg::NB;
+  constexpr int LDL = Cfg::LDL;
+  constexpr int LDP = Cfg::LDP;
+  extern __shared__ __align__(16) float sm[];
+  float* Ls = sm;                       // [DH][LDL]: L (lower blocks), then W
+  float* Apan = Ls + DH * LDL;          // [DH][LDP]: block column p before scaling
+  float* Wd = Apan + DH * LDP;          // [NB][16][LDP]: W_pp = L_pp^-1
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
   const int64_t mat = static_cast<int64_t>(blockIdx.x) * DH * DH;
+  const float* Am = A + mat;
   bool bad = false;
 
-  // ---------------------------------------------------------------- 1. Cholesky
-  {
-    float m[Cfg::RA][Cfg::CB];
-    load_spd<DH>(A + mat, m, ty, tx);
-#pragma unroll 1
-    for (int j = 0; j < DH; ++j) {
-      float* col = (j & 1) ? buf1 : buf0;
-      if (tx == (j & 15)) {  // owners of column j publish it
-        const int jb = j >> 4;
+  // strictly upper blocks of L / W stay zero (the product in 3 reads them)
+  for (int e = threadIdx.x; e < DH * DH; e += kThreads) {
+    const int r = e / DH, c = e % DH;
+    if ((c >> 4) > (r >> 4)) Ls[r * LDL + c] = 0.f;
+  }
+
+  // lower blocks of I + (A + A^T) / 2 into registers
+  float m[NB][NB];
 #pragma unroll
-        for (int a = 0; a < Cfg::RA; ++a) {
-          float v = m[a][0];
+  for (int a = 0; a < NB; ++a)
 #pragma unroll
-          for (int b = 1; b < Cfg::CB; ++b) v = (b == jb) ? m[a][b] : v;
-          col[ty + 16 * a] = v;
+    for (int b = 0; b <= a; ++b) {
+      const int i = 16 * a + ty, k = 16 * b + tx;
+      m[a][b] = 0.5f * (__ldg(Am + i * DH + k) + __ldg(Am + k * DH + i)) + (i == k ? 1.f : 0.f);
+    }
+
+  // ---------------------------------------------------------------- 1. factor
+#pragma unroll
+  for (int p = 0; p < NB; ++p) {
+#pragma unroll
+    for (int a = p; a < NB; ++a) Apan[(16 * a + ty) * LDP + tx] = m[a][p];
+    __syncthreads();
+
+    if (threadIdx.x < 32) {
+      // lane j (mod 16) holds column j of the diagonal block
+      const int j = threadIdx.x & 15;
+      float dc[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) dc[r] = Apan[(16 * p + r) * LDP + j];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        float piv = __shfl_sync(0xffffffffu, dc[c], c);
+        if (!(piv > 0.f)) {  // also catches NaN
+          bad = true;
+          piv = 1.f;
         }
+        const float f = dc[c] / piv;  // D[c][j] / D[c][c]
+#pragma unroll
+        for (int r = c + 1; r < 16; ++r) {
+          const float v = __shfl_sync(0xffffffffu, dc[r], c);  // D[r][c]
+          if (j > c) dc[r] = fmaf(-v, f, dc[r]);
+        }
+        if (j == c) {
+          const float sq = sqrtf(piv);
+          const float is = 1.f / sq;
+#pragma unroll
+          for (int r = c + 1; r < 16; ++r) dc[r] *= is;
+          dc[c] = sq;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (r < j) dc[r] = 0.f;
+      if (threadIdx.x < 16)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Ls[(16 * p + r) * LDL + 16 * p + j] = dc[r];
+      __syncwarp();
+      // column j of W_pp by forward substitution (rows above j come out 0)
+      float w[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const float* lr = Ls + (16 * p + r) * LDL + 16 * p;
+        float acc = (r == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int k = 0; k < r; ++k) acc = fmaf(-lr[k], w[k], acc);
+        w[r] = acc / lr[r];
+      }
+      if (threadIdx.x < 16)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Wd[(p * 16 + r) * LDP + j] = w[r];
+    }
+    __syncthreads();
+
+    if (p + 1 < NB) {
+      // L_ip = A_ip W_pp^T: row ty of A_ip against row tx of W_pp
+      uint64_t wr[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(Wd + (p * 16 + tx) * LDP + 4 * q);
+        wr[2 * q] = v.x;
+        wr[2 * q + 1] = v.y;
+      }
+#pragma unroll
+      for (int i = p + 1; i < NB; ++i) {
+        uint64_t acc = 0ull;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(Apan + (16 * i + ty) * LDP + 4 * q);
+          acc = f32x2_fma(v.x, wr[2 * q], acc);
+          acc = f32x2_fma(v.y, wr[2 * q + 1], acc);
+        }
+        Ls[(16 * i + ty) * LDL + 16 * p + tx] = f32x2_lo(acc) + f32x2_hi(acc);
       }
       __syncthreads();
-      float piv = col[j];
-      if (!(piv > 0.f)) {  // also catches NaN
-        bad = true;
-        piv = 1.f;
-      }
-      const float s = sqrtf(piv);
-      const float inv = 1.f / s;
-      if (threadIdx.x < DH) {
-        const int i = threadIdx.x;
-        Ls[i * Cfg::LD + j] = i > j ? col[i] * inv : (i == j ? s : 0.f);
-      }
-      float li[Cfg::RA], lk[Cfg::CB];
+      // trailing update of the lower blocks right of panel p
 #pragma unroll
-      for (int a = 0; a < Cfg::RA; ++a) li[a] = col[ty + 16 * a] * inv;
+      for (int a = p + 1; a < NB; ++a) {
+        uint64_t la[8];
 #pragma unroll
-      for (int b = 0; b < Cfg::CB; ++b) lk[b] = col[tx + 16 * b] * inv;
+        for (int q = 0; q < 4; ++q) {
+          const ulonglong2 v =
+              *reinterpret_cast<const ulonglong2*>(Ls + (16 * a + ty) * LDL + 16 * p + 4 * q);
+          la[2 * q] = v.x;
+          la[2 * q + 1] = v.y;
+        }
 #pragma unroll
-      for (int a = 0; a < Cfg::RA; ++a) {
-        if (16 * a + 15 <= j) continue;  // whole row group already factored
+        for (int b = p + 1; b <= a; ++b) {
+          uint64_t acc = 0ull;
 #pragma unroll
-        for (int b = 0; b < Cfg::CB; ++b) {
-          if (16 * b + 15 <= j) continue;
-          const int i = ty + 16 * a, k = tx + 16 * b;
-          if (i > j && k > j) m[a][b] = fmaf(-li[a], lk[b], m[a][b]);
+          for (int q = 0; q < 4; ++q) {
+            const ulonglong2 v =
+                *reinterpret_cast<const ulonglong2*>(Ls + (16 * b + tx) * LDL + 16 * p + 4 * q);
+            acc = f32x2_fma(la[2 * q], v.x, acc);
+            acc = f32x2_fma(la[2 * q + 1], v.y, acc);
+          }
+          m[a][b] -= f32x2_lo(acc) + f32x2_hi(acc);
         }
       }
-      // one barrier per step: the next step writes the other buffer
     }
   }
-  __syncthreads();  // L complete in shared memory
 
   // ---------------------------------------------------------------- 2. W = L^-1
-  // forward substitution against I; columns c = 64 g + 4 tx + e, rows ty + 16 a
-  {
-    float r[Cfg::RA][Cfg::RG][4];
-#pragma unroll
-    for (int a = 0; a < Cfg::RA; ++a)
-#pragma unroll
-      for (int g = 0; g < Cfg::RG; ++g)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) r[a][g][e] = (ty + 16 * a == 64 * g + 4 * tx + e) ? 1.f : 0.f;
-#pragma unroll 1
-    for (int k = 0; k < DH; ++k) {
-      float* row = (k & 1) ? buf1 : buf0;
-      const float dinv = 1.f / Ls[k * Cfg::LD + k];
-      if (ty == (k & 15)) publish_row<Cfg::RA, Cfg::RG>(r, k >> 4, dinv, row + 4 * tx);
-      __syncthreads();
-#pragma unroll
-      for (int a = 0; a < Cfg::RA; ++a) {
-        if (16 * a + 15 <= k) continue;
-        const int i = ty + 16 * a;
-        const float lik = i > k ? Ls[i * Cfg::LD + k] : 0.f;
-#pragma unroll
-        for (int g = 0; g < Cfg::RG; ++g) {
-          if (64 * g > k) continue;  // W[k][c] = 0 for c > k
-          const float4 y = *reinterpret_cast<const float4*>(row + 64 * g + 4 * tx);
-          r[a][g][0] = fmaf(-lik, y.x, r[a][g][0]);
-          r[a][g][1] = fmaf(-lik, y.y, r[a][g][1]);
-          r[a][g][2] = fmaf(-lik, y.z, r[a][g][2]);
-          r[a][g][3] = fmaf(-lik, y.w, r[a][g][3]);
-        }
-      }
-    }
-    __syncthreads();  // all reads of L done: the buffer now takes W
-#pragma unroll
-    for (int a = 0; a < Cfg::RA; ++a)
-#pragma unroll
-      for (int g = 0; g < Cfg::RG; ++g)
-        *reinterpret_cast<float4*>(sm + (ty + 16 * a) * Cfg::LD2 + 64 * g + 4 * tx) =
-            make_float4(r[a][g][0], r[a][g][1], r[a][g][2], r[a][g][3]);
-  }
+  // (the barrier closing the last factor step made L complete)
+  Ls[ty * LDL + tx] = Wd[ty * LDP + tx];  // W_00
   __syncthreads();
+#pragma unroll
+  for (int i = 1; i < NB; ++i) {
+    float t[NB];
+#pragma unroll
+    for (int j = 0; j < i; ++j) t[j] = 0.f;
+#pragma unroll
+    for (int k = 0; k < i; ++k) {
+      float lr[16];  // row ty of L_ik
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(Ls + (16 * i + ty) * LDL + 16 * k + 4 * q);
+        lr[4 * q] = v.x; lr[4 * q + 1] = v.y; lr[4 * q + 2] = v.z; lr[4 * q + 3] = v.w;
+      }
+#pragma unroll
+      for (int j = 0; j <= k; ++j)
+#pragma unroll
+        for (int n = 0; n < 16; ++n) t[j] = fmaf(lr[n], Ls[(16 * k + n) * LDL + 16 * j + tx], t[j]);
+    }
+    __syncthreads();  // every read of L_i* is done
+#pragma unroll
+    for (int j = 0; j < i; ++j) Ls[(16 * i + ty) * LDL + 16 * j + tx] = t[j];
+    __syncthreads();
+    float wi[16];  // row ty of W_ii
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(Wd + (i * 16 + ty) * LDP + 4 * q);
+      wi[4 * q] = v.x; wi[4 * q + 1] = v.y; wi[4 * q + 2] = v.z; wi[4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < i; ++j) {
+      float acc = 0.f;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) acc = fmaf(wi[n], Ls[(16 * i + n) * LDL + 16 * j + tx], acc);
+      t[j] = -acc;
+    }
+    __syncthreads();  // every read of T_i* is done
+#pragma unroll
+    for (int j = 0; j < i; ++j) Ls[(16 * i + ty) * LDL + 16 * j + tx] = t[j];
+    Ls[(16 * i + ty) * LDL + 16 * i + tx] = Wd[(i * 16 + ty) * LDP + tx];
+    __syncthreads();
+  }
 
   // ---------------------------------------------------------------- 3. P = W^T W
   {
-    constexpr int TR = Cfg::TR;
+    constexpr int TR = DH / 16;
     const int i0 = (threadIdx.x >> 4) * TR, c0 = (threadIdx.x & 15) * TR;
-    float acc[TR][TR];
+    uint64_t acc[TR][TR / 2];
 #pragma unroll
     for (int a = 0; a < TR; ++a)
 #pragma unroll
-      for (int b = 0; b < TR; ++b) acc[a][b] = 0.f;
+      for (int b = 0; b < TR / 2; ++b) acc[a][b] = 0ull;
     // W[k][i] = 0 for k < i: rows below max(i0, c0) add nothing to the tile
 #pragma unroll 2
     for (int k = max(i0, c0); k < DH; ++k) {
-      const float* wk = sm + k * Cfg::LD2;
-      float wi[TR], wc[TR];
+      const float* wk = Ls + k * LDL;
+      float wi[TR];
+      uint64_t wc[TR / 2];
 #pragma unroll
       for (int a = 0; a < TR; a += 4) {
         const float4 v = *reinterpret_cast<const float4*>(wk + i0 + a);
         wi[a] = v.x; wi[a + 1] = v.y; wi[a + 2] = v.z; wi[a + 3] = v.w;
       }
 #pragma unroll
-      for (int b = 0; b < TR; b += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(wk + c0 + b);
-        wc[b] = v.x; wc[b + 1] = v.y; wc[b + 2] = v.z; wc[b + 3] = v.w;
+      for (int b = 0; b < TR / 2; b += 2) {
+        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(wk + c0 + 2 * b);
+        wc[b] = v.x;
+        wc[b + 1] = v.y;
       }
 #pragma unroll
-      for (int a = 0; a < TR; ++a)
+      for (int a = 0; a < TR; ++a) {
+        const uint64_t aa = f32x2_pack(wi[a], wi[a]);
 #pragma unroll
-        for (int b = 0; b < TR; ++b) acc[a][b] = fmaf(wi[a], wc[b], acc[a][b]);
+        for (int b = 0; b < TR / 2; ++b) acc[a][b] = f32x2_fma(aa, wc[b], acc[a][b]);
+      }
     }
     float* Pm = P + mat;
 #pragma unroll
     for (int a = 0; a < TR; ++a)
 #pragma unroll
-      for (int b = 0; b < TR; b += 4)
-        *reinterpret_cast<float4*>(Pm + (i0 + a) * DH + c0 + b) =
-            make_float4(acc[a][b], acc[a][b + 1], acc[a][b + 2], acc[a][b + 3]);
+      for (int b = 0; b < TR / 2; b += 2)
+        *reinterpret_cast<float4*>(Pm + (i0 + a) * DH + c0 + 2 * b) =
+            make_float4(f32x2_lo(acc[a][b]), f32x2_hi(acc[a][b]), f32x2_lo(acc[a][b + 1]),
+                        f32x2_hi(acc[a][b + 1]));
   }
   if (bad) record_status(status, kStatusNumeric);
 }
@@ -308,7 +391,8 @@ cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* 
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(vda_solve_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         CholCfg<DH>::SMEM);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(vda_solve_gj_kernel<DH>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
@@ -318,7 +402,8 @@ cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* 
   if (solver == VDN_SOLVER_GAUSS_JORDAN)
     vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
   else
-    vda_solve_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
+    vda_solve_kernel<DH><<<s.T * s.H, kThreads, CholCfg<DH>::SMEM, ctx.stream>>>(A, P,
+                                                                                 ctx.status);
   return cudaGetLastError();
 }
 
