@@ -56,28 +56,44 @@ __device__ __forceinline__ void load_spd(const float* __restrict__ Am,
 
 // ---------------------------------------------------------------- Cholesky
 //
-// Blocked in 16 x 16 blocks (NB = DH / 16 block rows).  Thread (ty, tx)
-// holds element (ty, tx) of every block, so block products need no
-// reshuffling: a block (a, b) of the register tile is m[a][b].
-//
+// Blocked in 16 x 16 blocks (NB = DH / 16 block rows), the matrix in shared
+// memory (lower blocks; strictly upper blocks held at zero), thread (ty, tx)
+// working on element (ty, tx) of every block it touches:
 //  1. factor, for p = 0 .. NB-1:
-//     a. every thread stages block column p (rows >= 16p) in Apan;
-//     b. warp 0 factors the diagonal block with shuffles (lane j holds
-//        column j; the pivot column is broadcast row by row) into L_pp and
-//        inverts it, W_pp = L_pp^-1 (one column per lane); both to smem;
-//     c. L_ip = A_ip W_pp^T for the blocks below (16-term dot products);
-//     d. trailing update A_ab -= L_ap L_bp^T for p < b <= a (packed f32x2);
+//     a. warp 0 factors the diagonal block with shuffles (lane j holds
+//        column j; the pivot column is broadcast row by row) and inverts it,
+//        W_pp = L_pp^-1 (one column per lane), which replaces the block;
+//     b. L_ip = A_ip W_pp^T for the blocks below, into a panel buffer;
+//     c. trailing update A_ab -= L_ap L_bp^T (p < b <= a, packed f32x2),
+//        and L_ip copied into block column p;
 //  2. W = L^-1 in place, block row by block row:
 //     W_ij = -W_ii sum_{k=j}^{i-1} L_ik W_kj   (j < i);
 //  3. P = W^T W over the rows where W can be nonzero (k >= max(i, c)).
-// About 54 barriers in all (the unblocked form needs two per column).
+// The block loops are runtime loops, so the program stays small (each
+// step's code is fetched once and reused); only the 16-step factorization
+// of a diagonal block is unrolled.  About 40 barriers in all.
 template <int DH>
 struct CholCfg {
   static constexpr int NB = DH / 16;
-  static constexpr int LDL = DH + 4;   // row stride of L / W (float4 rows)
-  static constexpr int LDP = 20;       // row stride of the 16-wide staging blocks
-  static constexpr int SMEM = (DH * LDL + DH * LDP + NB * 16 * LDP) * 4;
+  static constexpr int LDL = DH + 4;   // row stride of the matrix (float4 rows)
+  static constexpr int LDP = 20;       // row stride of the 16-wide panel buffer
+  static constexpr int LDT = DH + 4;   // row stride of the 16-row T buffer (aliases the panel)
+  static constexpr int PANEL = (DH * LDP > 16 * LDT) ? DH * LDP : 16 * LDT;
+  static constexpr int SMEM = (DH * LDL + PANEL + 16) * 4;
 };
+
+// 16-term dot product of two 16-float rows in shared memory (16-byte aligned)
+__device__ __forceinline__ float dot16(const float* x, const float* y) {
+  uint64_t acc = 0ull;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(x + 4 * q);
+    const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(y + 4 * q);
+    acc = f32x2_fma(a.x, b.x, acc);
+    acc = f32x2_fma(a.y, b.y, acc);
+  }
+  return f32x2_lo(acc) + f32x2_hi(acc);
+}
 
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -86,45 +102,55 @@ __global__ void __launch_bounds__(kThreads, 2)
   constexpr int NB = Cfg::NB;
   constexpr int LDL = Cfg::LDL;
   constexpr int LDP = Cfg::LDP;
+  constexpr int LDT = Cfg::LDT;
   extern __shared__ __align__(16) float sm[];
-  float* Ls = sm;                       // [DH][LDL]: L (lower blocks), then W
-  float* Apan = Ls + DH * LDL;          // [DH][LDP]: block column p before scaling
-  float* Wd = Apan + DH * LDP;          // [NB][16][LDP]: W_pp = L_pp^-1
+  float* Ls = sm;                   // [DH][LDL]: the matrix, then L / W blocks
+  float* Pan = Ls + DH * LDL;       // [DH][LDP] panel L_ip; in step 2 [16][LDT] T rows
+  float* idg = Pan + Cfg::PANEL;    // [16] 1 / L_pp[r][r]
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
   const int64_t mat = static_cast<int64_t>(blockIdx.x) * DH * DH;
   const float* Am = A + mat;
   bool bad = false;
 
-  // strictly upper blocks of L / W stay zero (the product in 3 reads them)
-  for (int e = threadIdx.x; e < DH * DH; e += kThreads) {
-    const int r = e / DH, c = e % DH;
-    if ((c >> 4) > (r >> 4)) Ls[r * LDL + c] = 0.f;
+  // ---------------------------------------------------------------- load
+  // A row-major into shared memory (coalesced), then I + (A + A^T) / 2 on
+  // the lower blocks and zero on the strictly upper ones
+  for (int e = threadIdx.x; e < DH * DH / 4; e += kThreads) {
+    const int r = e / (DH / 4), c4 = e % (DH / 4);
+    *reinterpret_cast<float4*>(Ls + r * LDL + 4 * c4) =
+        __ldg(reinterpret_cast<const float4*>(Am + r * DH + 4 * c4));
   }
-
-  // lower blocks of I + (A + A^T) / 2 into registers
-  float m[NB][NB];
+  __syncthreads();
+  {
+    constexpr int PER = DH * DH / kThreads;
+    float v[PER];
 #pragma unroll
-  for (int a = 0; a < NB; ++a)
-#pragma unroll
-    for (int b = 0; b <= a; ++b) {
-      const int i = 16 * a + ty, k = 16 * b + tx;
-      m[a][b] = 0.5f * (__ldg(Am + i * DH + k) + __ldg(Am + k * DH + i)) + (i == k ? 1.f : 0.f);
+    for (int q = 0; q < PER; ++q) {
+      const int e = threadIdx.x + kThreads * q;
+      const int r = e / DH, c = e % DH;
+      v[q] = (c >> 4) > (r >> 4) ? 0.f
+                                 : 0.5f * (Ls[r * LDL + c] + Ls[c * LDL + r]) + (r == c ? 1.f : 0.f);
     }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+      const int e = threadIdx.x + kThreads * q;
+      Ls[(e / DH) * LDL + e % DH] = v[q];
+    }
+  }
+  __syncthreads();
 
   // ---------------------------------------------------------------- 1. factor
-#pragma unroll
+#pragma unroll 1
   for (int p = 0; p < NB; ++p) {
-#pragma unroll
-    for (int a = p; a < NB; ++a) Apan[(16 * a + ty) * LDP + tx] = m[a][p];
-    __syncthreads();
-
+    float* Dg = Ls + (16 * p) * LDL + 16 * p;  // diagonal block (p, p)
     if (threadIdx.x < 32) {
       // lane j (mod 16) holds column j of the diagonal block
       const int j = threadIdx.x & 15;
       float dc[16];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) dc[r] = Apan[(16 * p + r) * LDP + j];
+      for (int r = 0; r < 16; ++r) dc[r] = Dg[r * LDL + j];
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         float piv = __shfl_sync(0xffffffffu, dc[c], c);
@@ -132,135 +158,97 @@ __global__ void __launch_bounds__(kThreads, 2)
           bad = true;
           piv = 1.f;
         }
-        const float f = dc[c] / piv;  // D[c][j] / D[c][c]
+        const float f = (j > c) ? dc[c] * __frcp_rn(piv) : 0.f;  // D[c][j] / D[c][c]
+        const float sq = sqrtf(piv);
+        const float is = __frcp_rn(sq);
 #pragma unroll
-        for (int r = c + 1; r < 16; ++r) {
-          const float v = __shfl_sync(0xffffffffu, dc[r], c);  // D[r][c]
-          if (j > c) dc[r] = fmaf(-v, f, dc[r]);
+        for (int r = 0; r < 16; ++r) {
+          if (r > c) {
+            const float v = __shfl_sync(0xffffffffu, dc[r], c);  // D[r][c]
+            dc[r] = (j == c) ? dc[r] * is : fmaf(-v, f, dc[r]);
+          }
         }
-        if (j == c) {
-          const float sq = sqrtf(piv);
-          const float is = 1.f / sq;
-#pragma unroll
-          for (int r = c + 1; r < 16; ++r) dc[r] *= is;
-          dc[c] = sq;
-        }
+        if (j == c) dc[c] = sq;
+        if (threadIdx.x == c) idg[c] = is;
       }
-#pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r < j) dc[r] = 0.f;
+      // L_pp (zero above the diagonal) into the panel rows 16p.. (free now)
+      float* Lp = Pan + (16 * p) * LDP;
       if (threadIdx.x < 16)
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Ls[(16 * p + r) * LDL + 16 * p + j] = dc[r];
+        for (int r = 0; r < 16; ++r) Lp[r * LDP + j] = r < j ? 0.f : dc[r];
       __syncwarp();
       // column j of W_pp by forward substitution (rows above j come out 0)
       float w[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
-        const float* lr = Ls + (16 * p + r) * LDL + 16 * p;
+        const float* lr = Lp + r * LDP;
         float acc = (r == j) ? 1.f : 0.f;
 #pragma unroll
         for (int k = 0; k < r; ++k) acc = fmaf(-lr[k], w[k], acc);
-        w[r] = acc / lr[r];
+        w[r] = acc * idg[r];
       }
       if (threadIdx.x < 16)
 #pragma unroll
-        for (int r = 0; r < 16; ++r) Wd[(p * 16 + r) * LDP + j] = w[r];
+        for (int r = 0; r < 16; ++r) Dg[r * LDL + j] = w[r];
     }
     __syncthreads();
+    if (p + 1 == NB) break;
 
-    if (p + 1 < NB) {
-      // L_ip = A_ip W_pp^T: row ty of A_ip against row tx of W_pp
-      uint64_t wr[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(Wd + (p * 16 + tx) * LDP + 4 * q);
-        wr[2 * q] = v.x;
-        wr[2 * q + 1] = v.y;
-      }
-#pragma unroll
-      for (int i = p + 1; i < NB; ++i) {
-        uint64_t acc = 0ull;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const ulonglong2 v = *reinterpret_cast<const ulonglong2*>(Apan + (16 * i + ty) * LDP + 4 * q);
-          acc = f32x2_fma(v.x, wr[2 * q], acc);
-          acc = f32x2_fma(v.y, wr[2 * q + 1], acc);
-        }
-        Ls[(16 * i + ty) * LDL + 16 * p + tx] = f32x2_lo(acc) + f32x2_hi(acc);
-      }
-      __syncthreads();
-      // trailing update of the lower blocks right of panel p
-#pragma unroll
-      for (int a = p + 1; a < NB; ++a) {
-        uint64_t la[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const ulonglong2 v =
-              *reinterpret_cast<const ulonglong2*>(Ls + (16 * a + ty) * LDL + 16 * p + 4 * q);
-          la[2 * q] = v.x;
-          la[2 * q + 1] = v.y;
-        }
-#pragma unroll
-        for (int b = p + 1; b <= a; ++b) {
-          uint64_t acc = 0ull;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const ulonglong2 v =
-                *reinterpret_cast<const ulonglong2*>(Ls + (16 * b + tx) * LDL + 16 * p + 4 * q);
-            acc = f32x2_fma(la[2 * q], v.x, acc);
-            acc = f32x2_fma(la[2 * q + 1], v.y, acc);
-          }
-          m[a][b] -= f32x2_lo(acc) + f32x2_hi(acc);
-        }
-      }
+    // L_ip = A_ip W_pp^T: row ty of A_ip against row tx of W_pp
+#pragma unroll 1
+    for (int i = p + 1; i < NB; ++i)
+      Pan[(16 * i + ty) * LDP + tx] = dot16(Ls + (16 * i + ty) * LDL + 16 * p, Dg + tx * LDL);
+    __syncthreads();
+
+    // trailing update of the lower blocks right of panel p; L_ip into place
+#pragma unroll 1
+    for (int a = p + 1; a < NB; ++a) {
+      const float* la = Pan + (16 * a + ty) * LDP;
+#pragma unroll 1
+      for (int b = p + 1; b <= a; ++b)
+        Ls[(16 * a + ty) * LDL + 16 * b + tx] -= dot16(la, Pan + (16 * b + tx) * LDP);
+      Ls[(16 * a + ty) * LDL + 16 * p + tx] = Pan[(16 * a + ty) * LDP + tx];
     }
+    __syncthreads();
   }
 
   // ---------------------------------------------------------------- 2. W = L^-1
-  // (the barrier closing the last factor step made L complete)
-  Ls[ty * LDL + tx] = Wd[ty * LDP + tx];  // W_00
-  __syncthreads();
-#pragma unroll
+  // block row 0 holds W_00 already; the diagonal blocks hold W_ii
+#pragma unroll 1
   for (int i = 1; i < NB; ++i) {
-    float t[NB];
+    const float* li = Ls + (16 * i + ty) * LDL;  // row ty of block row i
+#pragma unroll 1
+    for (int j = 0; j < i; ++j) {
+      float t = 0.f;
+#pragma unroll 1
+      for (int k = j; k < i; ++k) {
+        const float* wkj = Ls + (16 * k) * LDL + 16 * j + tx;  // column tx of W_kj
+        float lr[16];
 #pragma unroll
-    for (int j = 0; j < i; ++j) t[j] = 0.f;
+        for (int q = 0; q < 4; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(li + 16 * k + 4 * q);
+          lr[4 * q] = v.x; lr[4 * q + 1] = v.y; lr[4 * q + 2] = v.z; lr[4 * q + 3] = v.w;
+        }
 #pragma unroll
-    for (int k = 0; k < i; ++k) {
-      float lr[16];  // row ty of L_ik
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(Ls + (16 * i + ty) * LDL + 16 * k + 4 * q);
-        lr[4 * q] = v.x; lr[4 * q + 1] = v.y; lr[4 * q + 2] = v.z; lr[4 * q + 3] = v.w;
+        for (int n = 0; n < 16; ++n) t = fmaf(lr[n], wkj[n * LDL], t);
       }
-#pragma unroll
-      for (int j = 0; j <= k; ++j)
-#pragma unroll
-        for (int n = 0; n < 16; ++n) t[j] = fmaf(lr[n], Ls[(16 * k + n) * LDL + 16 * j + tx], t[j]);
+      Pan[ty * LDT + 16 * j + tx] = t;  // T_ij
     }
-    __syncthreads();  // every read of L_i* is done
-#pragma unroll
-    for (int j = 0; j < i; ++j) Ls[(16 * i + ty) * LDL + 16 * j + tx] = t[j];
-    __syncthreads();
-    float wi[16];  // row ty of W_ii
+    __syncthreads();  // T complete; every read of L_i* is done
+    float wi[16];     // row ty of W_ii
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 v = *reinterpret_cast<const float4*>(Wd + (i * 16 + ty) * LDP + 4 * q);
+      const float4 v = *reinterpret_cast<const float4*>(li + 16 * i + 4 * q);
       wi[4 * q] = v.x; wi[4 * q + 1] = v.y; wi[4 * q + 2] = v.z; wi[4 * q + 3] = v.w;
     }
-#pragma unroll
+#pragma unroll 1
     for (int j = 0; j < i; ++j) {
       float acc = 0.f;
 #pragma unroll
-      for (int n = 0; n < 16; ++n) acc = fmaf(wi[n], Ls[(16 * i + n) * LDL + 16 * j + tx], acc);
-      t[j] = -acc;
+      for (int n = 0; n < 16; ++n) acc = fmaf(wi[n], Pan[n * LDT + 16 * j + tx], acc);
+      Ls[(16 * i + ty) * LDL + 16 * j + tx] = -acc;
     }
-    __syncthreads();  // every read of T_i* is done
-#pragma unroll
-    for (int j = 0; j < i; ++j) Ls[(16 * i + ty) * LDL + 16 * j + tx] = t[j];
-    Ls[(16 * i + ty) * LDL + 16 * i + tx] = Wd[(i * 16 + ty) * LDP + tx];
-    __syncthreads();
+    __syncthreads();  // W_i* complete; T free again
   }
 
   // ---------------------------------------------------------------- 3. P = W^T W
