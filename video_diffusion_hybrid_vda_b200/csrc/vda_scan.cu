@@ -8,14 +8,18 @@
 // with P_t = (I + A_t)^-1 from the solve.  Rows of S evolve independently
 // (row r of S_t needs only row r of S_{t-1}), so each CTA owns 64 rows of
 // one head's state in one direction and runs all T steps; every CTA of the
-// grid is resident at once.  Per step the CTA stages P_t (d x d fp32) into
-// shared memory with one bulk copy, double-buffered so that P_{t+1} lands
-// while step t computes.  Each thread first writes its tile of the bracket
-// alpha S_prev + B_t into the shared rows (row stride d + 4, so four
-// consecutive k of a row are one float4 and the rows of a warp fall in
-// different banks), then computes 4 rows x 8 columns of the new state with
-// packed f32x2 FMA.  A thread's columns are two interleaved groups of 4
-// (4c.., d/2 + 4c..), so each quarter warp reads 128 contiguous bytes of P.
+// grid is resident at once.  Per step the CTA stages P_t (d x d fp32) and
+// its 64 rows of B_t (one contiguous block) into shared memory with bulk
+// copies, double-buffered so that step t+1's operands land while step t
+// computes (nothing on a step's critical path waits on global memory).
+// Each thread first writes its tile of the bracket alpha S_prev + B_t into
+// the shared rows (row stride d + 4, so four consecutive k of a row are one
+// float4 and the rows of a warp fall in different banks), then computes 8
+// rows x 8 columns of the new state with packed f32x2 FMA: per k it loads 8
+// state and 8 P values for 64 FMA, the ratio at which shared-memory
+// bandwidth (32 floats per clock per SM) keeps up with the FMA pipes.  A
+// thread's columns are two interleaved groups of 4 (4c.., d/2 + 4c..), so
+// each quarter warp reads 128 contiguous bytes of P.
 // Multiplying the bracket (rather than adding a precomputed B_t P_t) keeps
 // the d^3 product C = B P out of the solve, at the price of one product at
 // the first step.  The scan is serial over T and FP32-ALU bound.
@@ -36,15 +40,16 @@ namespace vdn {
 namespace {
 
 constexpr int kRows = 64;   // rows of S per CTA
-constexpr int kTR = 4;      // rows per thread
+constexpr int kTR = 8;      // rows per thread
 constexpr int kTC = 8;      // columns per thread
 
 template <int DH>
 struct ScanCfg {
-  static constexpr int THREADS = (kRows / kTR) * (DH / kTC);  // 256 (d=128), 128 (d=64)
+  static constexpr int THREADS = (kRows / kTR) * (DH / kTC);  // 128 (d=128), 64 (d=64)
   static constexpr int P_BYTES = DH * DH * 4;
+  static constexpr int X_BYTES = kRows * DH * 4;  // the CTA's rows of B_t (or G_t)
   static constexpr int LDS = DH + 4;  // row stride of the state rows in shared memory
-  static constexpr int SMEM = 2 * P_BYTES + kRows * LDS * 4 + 64;
+  static constexpr int SMEM = 2 * P_BYTES + 2 * X_BYTES + kRows * LDS * 4 + 64;
 };
 
 template <int DH, bool kAdjoint>
@@ -56,9 +61,10 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   constexpr int CG = DH / kTC;  // column groups
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* Pbuf = reinterpret_cast<float*>(smem_raw);                  // 2 x [DH][DH]
-  float* Ss = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // [kRows][LDS]
-  uint64_t* full =
-      reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES + kRows * Cfg::LDS * 4);
+  float* Xbuf = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // 2 x [kRows][DH]
+  float* Ss = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES + 2 * Cfg::X_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES +
+                                               2 * Cfg::X_BYTES + kRows * Cfg::LDS * 4);
 
   const int rb = blockIdx.x;  // row block
   const int h = blockIdx.y;
@@ -72,14 +78,21 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   const int64_t mat = static_cast<int64_t>(DH) * DH;
   float* out_dir = states + static_cast<int64_t>(dir) * T * H * mat;
   auto frame = [&](int step) { return dir == 0 ? step : T - 1 - step; };
+  // both operands of the step that visits frame(step), into buffer `buf`
+  auto stage = [&](int step, int buf) {
+    const int64_t th = static_cast<int64_t>(frame(step)) * H + h;
+    mbar_arrive_expect_tx(&full[buf], Cfg::P_BYTES + Cfg::X_BYTES);
+    bulk_load(Pbuf + buf * DH * DH, P + th * mat, Cfg::P_BYTES, &full[buf]);
+    bulk_load(Xbuf + buf * kRows * DH, X + th * mat + static_cast<int64_t>(rb) * kRows * DH,
+              Cfg::X_BYTES, &full[buf]);
+  };
 
   for (int i = threadIdx.x; i < kRows * Cfg::LDS; i += blockDim.x) Ss[i] = 0.f;
   if (threadIdx.x == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&full[0], Cfg::P_BYTES);
-    bulk_load(Pbuf, P + (static_cast<int64_t>(frame(0)) * H + h) * mat, Cfg::P_BYTES, &full[0]);
+    stage(0, 0);
   }
   __syncthreads();
 
@@ -89,6 +102,15 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
 #pragma unroll
     for (int c = 0; c < kTC; ++c) sprev[r][c] = 0.f;
 
+  // forward: the decay of the frame being absorbed; adjoint: of the frame
+  // visited one step earlier (unused at step 0, where the carried term is 0).
+  // Read one step ahead, so no step waits on it.
+  auto decay = [&](int step) {
+    return !kAdjoint ? __ldg(alpha + frame(step) * H + h)
+                     : (step > 0 ? __ldg(alpha + frame(step - 1) * H + h) : 0.f);
+  };
+  float a_next = decay(0);
+
   int issued = 1;
 #pragma unroll 1
   for (int step = 0; step < T; ++step) {
@@ -96,23 +118,20 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     const int b = step & 1;
     if (threadIdx.x == 0 && step + 1 < T) {
       // buffer b^1 was last read in step-1, which every thread has left
-      mbar_arrive_expect_tx(&full[b ^ 1], Cfg::P_BYTES);
-      bulk_load(Pbuf + (b ^ 1) * DH * DH, P + (static_cast<int64_t>(frame(step + 1)) * H + h) * mat,
-                Cfg::P_BYTES, &full[b ^ 1]);
+      stage(step + 1, b ^ 1);
       ++issued;
     }
-    // forward: the decay of the frame being absorbed; adjoint: of the frame
-    // visited one step earlier (unused at step 0, where the carried term is 0)
-    const float a = !kAdjoint ? __ldg(alpha + t * H + h)
-                              : (step > 0 ? __ldg(alpha + frame(step - 1) * H + h) : 0.f);
-    const float* Xt = X + (static_cast<int64_t>(t) * H + h) * mat;
+    const float a = a_next;
+    if (step + 1 < T) a_next = decay(step + 1);
     // U = a S_prev + X_t into the shared rows; every thread left the previous
     // step's reads behind the barrier that closed it, and the barrier below
     // publishes U before the multiply
+    const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
+    const float* Xt = Xbuf + b * kRows * DH;
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
-      const float4 xa = __ldg(reinterpret_cast<const float4*>(Xt + (row0 + r) * DH + colA));
-      const float4 xb = __ldg(reinterpret_cast<const float4*>(Xt + (row0 + r) * DH + colB));
+      const float4 xa = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colA);
+      const float4 xb = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colB);
       float* srow = Ss + (lrow0 + r) * Cfg::LDS;
       *reinterpret_cast<float4*>(srow + colA) =
           make_float4(fmaf(a, sprev[r][0], xa.x), fmaf(a, sprev[r][1], xa.y),
@@ -121,7 +140,6 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
           make_float4(fmaf(a, sprev[r][4], xb.x), fmaf(a, sprev[r][5], xb.y),
                       fmaf(a, sprev[r][6], xb.z), fmaf(a, sprev[r][7], xb.w));
     }
-    const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
     if (!__syncthreads_and(ok)) {
       if (threadIdx.x == 0) record_status(status, kStatusTimeout);
       break;
