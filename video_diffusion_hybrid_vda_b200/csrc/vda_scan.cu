@@ -17,7 +17,10 @@
 // float4 and the rows of a warp fall in different banks), then computes 8
 // rows x 8 columns of the new state with packed f32x2 FMA: per k it loads 8
 // state and 8 P values for 64 FMA, the ratio at which shared-memory
-// bandwidth (32 floats per clock per SM) keeps up with the FMA pipes.  A
+// bandwidth (32 floats per clock per SM) keeps up with the FMA pipes.  The
+// CTA's two halves split the k range of the product (two warps per SM
+// sub-partition keep the packed FMAs issuing); the upper half hands its
+// partial sums over through the step's B buffer, already consumed.  A
 // thread's columns are two interleaved groups of 4 (4c.., d/2 + 4c..), so
 // each quarter warp reads 128 contiguous bytes of P.
 // Multiplying the bracket (rather than adding a precomputed B_t P_t) keeps
@@ -45,7 +48,8 @@ constexpr int kTC = 8;      // columns per thread
 
 template <int DH>
 struct ScanCfg {
-  static constexpr int THREADS = (kRows / kTR) * (DH / kTC);  // 128 (d=128), 64 (d=64)
+  static constexpr int HALF = (kRows / kTR) * (DH / kTC);  // threads per k half
+  static constexpr int THREADS = 2 * HALF;                   // 256 (d=128), 128 (d=64)
   static constexpr int P_BYTES = DH * DH * 4;
   static constexpr int X_BYTES = kRows * DH * 4;  // the CTA's rows of B_t (or G_t)
   static constexpr int LDS = DH + 4;  // row stride of the state rows in shared memory
@@ -69,8 +73,10 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   const int rb = blockIdx.x;  // row block
   const int h = blockIdx.y;
   const int dir = blockIdx.z;  // 0 forward, 1 backward
-  const int cg = threadIdx.x % CG;
-  const int rg = threadIdx.x / CG;
+  const int half = threadIdx.x / Cfg::HALF;  // which half of the k range
+  const int lt = threadIdx.x % Cfg::HALF;
+  const int cg = lt % CG;
+  const int rg = lt / CG;
   const int lrow0 = rg * kTR;                  // first local row of the thread's tile
   const int row0 = rb * kRows + lrow0;         // first row of S
   // the thread's columns: [colA, colA + 4) and [colB, colB + 4)
@@ -127,9 +133,10 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     // step's reads behind the barrier that closed it, and the barrier below
     // publishes U before the multiply
     const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
-    const float* Xt = Xbuf + b * kRows * DH;
+    float* Xt = Xbuf + b * kRows * DH;
 #pragma unroll
     for (int r = 0; r < kTR; ++r) {
+      if (half != 0) break;  // the lower half holds the state
       const float4 xa = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colA);
       const float4 xb = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colB);
       float* srow = Ss + (lrow0 + r) * Cfg::LDS;
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
       for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
     {
 #pragma unroll 1
-      for (int k = 0; k < DH; k += 4) {
+      for (int k = half * (DH / 2); k < (half + 1) * (DH / 2); k += 4) {
         float sr[kTR][4];
 #pragma unroll
         for (int r = 0; r < kTR; ++r) {
@@ -175,26 +182,38 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
         }
       }
     }
-    float snew[kTR][kTC];
+    // the upper half's partial sums, through the consumed B buffer
+    if (half != 0) {
 #pragma unroll
-    for (int r = 0; r < kTR; ++r) {
-#pragma unroll
-      for (int q = 0; q < kTC / 2; ++q) {
-        snew[r][2 * q] = f32x2_lo(acc2[r][q]);
-        snew[r][2 * q + 1] = f32x2_hi(acc2[r][q]);
+      for (int r = 0; r < kTR; ++r) {
+        *reinterpret_cast<ulonglong2*>(Xt + (lrow0 + r) * DH + colA) =
+            make_ulonglong2(acc2[r][0], acc2[r][1]);
+        *reinterpret_cast<ulonglong2*>(Xt + (lrow0 + r) * DH + colB) =
+            make_ulonglong2(acc2[r][2], acc2[r][3]);
       }
-      float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
-                   static_cast<int64_t>(row0 + r) * DH;
-      *reinterpret_cast<float4*>(dst + colA) =
-          make_float4(snew[r][0], snew[r][1], snew[r][2], snew[r][3]);
-      *reinterpret_cast<float4*>(dst + colB) =
-          make_float4(snew[r][4], snew[r][5], snew[r][6], snew[r][7]);
     }
-    __syncthreads();  // every thread has finished reading Ss (and Pbuf b)
+    __syncthreads();  // partials visible; every read of Ss and Pbuf b is done
+    if (half == 0) {
 #pragma unroll
-    for (int r = 0; r < kTR; ++r)
+      for (int r = 0; r < kTR; ++r) {
+        const ulonglong2 ua = *reinterpret_cast<const ulonglong2*>(Xt + (lrow0 + r) * DH + colA);
+        const ulonglong2 ub = *reinterpret_cast<const ulonglong2*>(Xt + (lrow0 + r) * DH + colB);
+        const uint64_t v[4] = {f32x2_add(acc2[r][0], ua.x), f32x2_add(acc2[r][1], ua.y),
+                               f32x2_add(acc2[r][2], ub.x), f32x2_add(acc2[r][3], ub.y)};
 #pragma unroll
-      for (int c = 0; c < kTC; ++c) sprev[r][c] = snew[r][c];
+        for (int q = 0; q < kTC / 2; ++q) {
+          sprev[r][2 * q] = f32x2_lo(v[q]);
+          sprev[r][2 * q + 1] = f32x2_hi(v[q]);
+        }
+        float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
+                     static_cast<int64_t>(row0 + r) * DH;
+        *reinterpret_cast<float4*>(dst + colA) =
+            make_float4(sprev[r][0], sprev[r][1], sprev[r][2], sprev[r][3]);
+        *reinterpret_cast<float4*>(dst + colB) =
+            make_float4(sprev[r][4], sprev[r][5], sprev[r][6], sprev[r][7]);
+      }
+    }
+    __syncthreads();  // the partials are read: buffer b may be refilled
   }
   // the bulk copies this CTA started must land before it exits
   if (threadIdx.x == 0) {
