@@ -26,6 +26,8 @@ pages' description of the method:
 
 * ``vda_backward`` -- gradients of the VDA output with respect to q, k, v,
                       beta and alpha (adjoint scans), for training the branch.
+* ``mxfp8``        -- MXFP8 quantization (E4M3 elements, UE8M0 block scales)
+                      and the fuse with MXFP8 projections.
 
 The readings taken where the pages are silent are listed in CONVENTIONS.md
 beside this file.  Parity status of every function is pinned by the
@@ -38,6 +40,7 @@ from .window_attn import (frame_visible, visible_key_frames, window_attn,
                           window_attn_rows, mask_pair_count)
 from .fuse import sigmoid, rmsnorm_heads, fuse_gates, hybrid_fuse, hybrid_fuse_rows
 from .vda_backward import vda_backward
+from . import mxfp8
 
 __all__ = [
     "vda_prep", "vda_frame_state", "vda_scan", "vda_readout", "vda",
@@ -45,5 +48,5 @@ __all__ = [
     "frame_visible", "visible_key_frames", "window_attn", "window_attn_rows",
     "mask_pair_count",
     "sigmoid", "rmsnorm_heads", "fuse_gates", "hybrid_fuse", "hybrid_fuse_rows",
-    "vda_backward",
+    "vda_backward", "mxfp8",
 ]

@@ -1,0 +1,104 @@
+"""Pins of the MXFP8 oracle: the E4M3 value table against its defining
+constants, encoding against torch's independent float8_e4m3fn conversion,
+round-to-nearest-even ties, saturation, the block-scale rule on blocks with
+known maxima, the quantization error bound, and the tile layout of the
+scale bytes on hand-computed offsets."""
+
+import numpy as np
+import torch
+
+from oracle import mxfp8
+
+
+def test_e4m3_table_constants():
+    v = mxfp8.E4M3_VALUES
+    assert v.shape == (127,)
+    assert np.all(np.diff(v) > 0)
+    assert v[0x7E] == 448.0                    # largest finite
+    assert v[0x38] == 1.0                      # exponent field 7 = bias
+    assert v[0x08] == 2.0 ** -6                # smallest normal
+    assert v[0x01] == 2.0 ** -9                # smallest subnormal
+    assert v[0x07] == 7 * 2.0 ** -9            # largest subnormal
+
+
+def test_encode_matches_torch_float8_on_the_rounding_range():
+    rng = np.random.default_rng(0)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.uniform(-4, 2.6, 20000),
+                        mxfp8.E4M3_VALUES, -mxfp8.E4M3_VALUES,
+                        (mxfp8.E4M3_VALUES[1:] + mxfp8.E4M3_VALUES[:-1]) / 2])  # every tie
+    x = x[np.abs(x) <= 464.0].astype(np.float32)
+    ours = mxfp8.e4m3_encode(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_round_trip_ties_and_saturation():
+    v = mxfp8.E4M3_VALUES
+    np.testing.assert_array_equal(mxfp8.e4m3_decode(mxfp8.e4m3_encode(v)), v)
+    np.testing.assert_array_equal(mxfp8.e4m3_decode(mxfp8.e4m3_encode(-v[1:])), -v[1:])
+    assert mxfp8.e4m3_encode(1.0625) == 0x38      # tie between 1.0 and 1.125 -> even code
+    assert mxfp8.e4m3_encode(1.1875) == 0x3A      # tie between 1.125 and 1.25 -> even code
+    assert mxfp8.e4m3_encode(2.0 ** -10) == 0x00  # tie between 0 and 2^-9
+    assert mxfp8.e4m3_encode(1000.0) == 0x7E
+    assert mxfp8.e4m3_encode(-1e9) == 0xFE
+    assert mxfp8.e4m3_encode(-2.0 ** -12) == 0x80  # negative, rounds to -0
+
+
+def test_block_scale_rule():
+    blk = np.zeros((5, 32))
+    blk[0, 3] = 1.0            # max 1      -> e = 0 - 8
+    blk[1, 7] = -3.5           # max 3.5    -> e = 1 - 8
+    blk[2, 0] = 2.0 ** -20     # max 2^-20  -> e = -28
+    blk[3, 0] = 1e38           # e = 126 - 8 = 118
+    codes, sb = mxfp8.mx_quantize(blk)
+    assert list(sb[:, 0].astype(int) - 127) == [-8, -7, -28, 118, -127]
+    assert np.all(codes[4] == 0)                           # a zero block
+    # the scaled block maximum lies in [256, 512) and saturates above 448
+    assert mxfp8.e4m3_decode(codes[0, 3]) * 2.0 ** -8 == 1.0
+    assert mxfp8.e4m3_decode(codes[1, 7]) * 2.0 ** -7 == -3.5
+    big = np.full((1, 32), 1.0)
+    big[0, 0] = 1.99                                        # 1.99 * 2^8 = 509 -> 448
+    c, s = mxfp8.mx_quantize(big)
+    assert mxfp8.mx_dequantize(c, s)[0, 0] == 448 * 2.0 ** -8
+
+
+def test_quantization_error_bound():
+    """Every element within half an E4M3 step of its value (relative 2^-4 of
+    the element for the normal range, 2^-10 of the block scale's 2^8 for the
+    subnormal range), except a saturated block maximum (at most 1/8 low)."""
+    rng = np.random.default_rng(1)
+    v = rng.standard_normal((64, 256)) * np.exp(rng.uniform(-6, 6, (64, 1)))
+    c, s = mxfp8.mx_quantize(v)
+    dq = mxfp8.mx_dequantize(c, s)
+    scale = np.repeat(np.ldexp(1.0, s.astype(int) - 127), 32, axis=1)
+    x = v / scale
+    err = np.abs(dq / scale - x)
+    ok = (err <= np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10)) | \
+         ((np.abs(x) > 448) & (err <= np.abs(x) / 8))
+    assert ok.all()
+
+
+def test_scale_tile_layout_offsets():
+    R, K = 300, 512
+    sb = np.arange(R * (K // 32), dtype=np.int64).reshape(R, K // 32) % 251
+    t = mxfp8.sf_tiled(sb.astype(np.uint8))
+    assert t.size == 3 * 4 * 512                       # ceil(300/128) x (512/128) tiles
+    # row 33, k-block 5: tile (0, 1), row 1 of the 32-row group 1, byte 1
+    assert t[512 + 1 * 16 + 1 * 4 + 1] == sb[33, 5]
+    # row 299, k-block 15: tile (2, 3); 299 % 128 = 43 -> group 1, row 11
+    assert t[(2 * 4 + 3) * 512 + 11 * 16 + 1 * 4 + 3] == sb[299, 15]
+    # padding rows hold the unit scale
+    assert t[(2 * 4 + 0) * 512 + 31 * 16 + 3 * 4] == 127
+
+
+def test_gemm_mx_is_the_product_of_dequantized_operands():
+    rng = np.random.default_rng(2)
+    a, b = rng.standard_normal((7, 64)), rng.standard_normal((5, 64))
+    aq, bq = mxfp8.mx_quantize(a), mxfp8.mx_quantize(b)
+    c = mxfp8.gemm_mx(*aq, *bq)
+    A, B = mxfp8.mx_dequantize(*aq), mxfp8.mx_dequantize(*bq)
+    for i in range(7):
+        for j in range(5):
+            assert abs(c[i, j] - sum(A[i, k] * B[j, k] for k in range(64))) < 1e-12
+    # and close to the unquantized product (E4M3 keeps ~2 significant digits)
+    assert np.abs(c - a @ b.T).max() < 0.1 * np.abs(a @ b.T).max()
