@@ -180,6 +180,55 @@ VDN_API vdn_status vdn_vda_backward_debug_buffers(const vdn_shape* shape, void* 
                                                   float** states, float** adj, float** E);
 
 /* ------------------------------------------------------------------------
+ * MXFP8 projections (10100.com article, 实验结果 / 效率阶梯 times the
+ * denoiser under MXFP8; the format is the OCP Microscaling one).
+ *
+ * An MXFP8 operand [R, K] (K-major, K a multiple of 128) is a pair:
+ *  - codes: R x K bytes, row-major, E4M3 (bias 7, no infinities, +-448 max);
+ *  - scales: vdn_mxfp8_scale_bytes(R, K) bytes of UE8M0 (2^(byte - 127)),
+ *    one per 32 consecutive elements of a row, in the tile layout the
+ *    block-scaled tensor-core MMA reads: per 128-row x 128-column tile one
+ *    512-byte block; the scale of (row r, column block kb = k / 32) is byte
+ *    (r % 32) * 16 + ((r % 128) / 32) * 4 + kb % 4 of block number
+ *    (r / 128) * (K / 128) + k / 128; rows past R up to the next multiple
+ *    of 128 hold 127 (scale 1).
+ * Quantization: per block e = floor(log2(max|v|)) - 8 clamped to
+ * [-127, 127] (-127 for a zero block); code = E4M3(v * 2^-e), round to
+ * nearest even, saturated at +-448; scale byte = e + 127.
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_mxfp8_scale_bytes(int64_t rows, int64_t cols);
+
+/* x bf16 [rows, ld] -> q codes [rows, cols] and sf scales (sizes above).
+ * cols a multiple of 128, ld >= cols and a multiple of 8; x, q 16-byte
+ * aligned.  One kernel on `stream`. */
+VDN_API vdn_status vdn_mxfp8_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld,
+                                      void* q, void* sf, void* stream);
+
+/* C [M, N] = A [M, K] B [N, K]^T on MXFP8 operands (codes and scales as
+ * above, row stride K bytes), fp32 accumulation; C row-major with row
+ * stride N, bf16 (c_is_f32 = 0) or fp32 (c_is_f32 != 0).  K a multiple of
+ * 128, N a multiple of 32; pointers 16-byte aligned; ws >= 256 bytes
+ * (status word).  VDN_ERR_UNSUPPORTED for other shapes. */
+VDN_API vdn_status vdn_gemm_mxfp8(int M, int N, int K, const void* a, const void* a_sf,
+                                  const void* b, const void* b_sf, void* c, int c_is_f32,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* vdn_hybrid_fuse with both projection GEMMs in MXFP8: x is quantized on
+ * the device; the gate GEMM's epilogue forms Z = [g_s o_s | g_l RMSNorm(o_vda)
+ * gamma] in fp32 and writes it quantized; y = Z [W_os | W_ol]^T.
+ * wg_q / wg_sf: MXFP8 of the stacked gate weights [W_gs; W_gl] ([2D, D]);
+ * wo_q / wo_sf: MXFP8 of [W_os | W_ol] ([D, 2D]) (vdn_mxfp8_quantize).
+ * Shapes: D a multiple of 128, head dim d = D / H a multiple of 32 that
+ * divides 128.  ws >= vdn_hybrid_fuse_mxfp8_workspace(L, D, H). */
+VDN_API size_t vdn_hybrid_fuse_mxfp8_workspace(int L, int D, int H);
+
+VDN_API vdn_status vdn_hybrid_fuse_mxfp8(int L, int D, int H, const void* x, const void* o_s,
+                                         const void* o_vda, const void* wg_q, const void* wg_sf,
+                                         const float* gamma, float eps, const void* wo_q,
+                                         const void* wo_sf, void* y, void* ws, size_t ws_bytes,
+                                         void* stream);
+
+/* ------------------------------------------------------------------------
  * Window-and-anchor Softmax (10100.com article, 方法概述 item 1).
  *
  * Chunk c(t) = floor(t / chunk_frames).  Query frame tq sees key frame tk iff

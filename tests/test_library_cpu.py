@@ -25,6 +25,29 @@ def _declared():
     return sorted(set(re.findall(r"^VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(", src, re.M)))
 
 
+def _declared_param_counts():
+    """Number of parameters of every VDN_API function in include/vdn.h."""
+    src = open(os.path.join(ROOT, "include", "vdn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(([^)]*)\)", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(L):
+    """Every ctypes prototype in the binding has as many arguments as the C
+    declaration (a mismatch would pass wrong values at call time)."""
+    lib = L.lib()
+    counts = _declared_param_counts()
+    assert sorted(counts) == _declared()
+    for name, n in counts.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
 def test_exports_every_declared_symbol(L):
     names = _declared()
     assert len(names) >= 12

@@ -25,11 +25,6 @@ pytestmark = pytest.mark.gpu
 def vdn():
     ensure_built()
     from video_diffusion_hybrid_vda_b200 import vdn as _vdn
-    L = _vdn.lib()
-    P = ctypes.c_void_p
-    L.vdn_vda_scan_static.argtypes = [ctypes.POINTER(_vdn.Shape), P, P, P, ctypes.c_int64, P, P,
-                                      P, ctypes.c_int64, P, P, P]
-    L.vdn_vda_scan_static.restype = ctypes.c_int
     return _vdn
 
 

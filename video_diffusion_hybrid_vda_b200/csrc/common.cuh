@@ -56,6 +56,11 @@ bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld
 bool make_rows_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int64_t rows,
                    int box_rows);
 
+// 2-D byte map over a row-major [rows, ld] matrix of 8-bit codes with box
+// {128 bytes, box_rows}, 128-byte swizzle.
+bool make_rows_map_u8(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int64_t rows,
+                      int box_rows);
+
 // ---- kernel launchers (return cudaSuccess or the launch error) ----------
 
 cudaError_t launch_vda_prep(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
@@ -70,6 +75,11 @@ cudaError_t launch_vda_scan(const Launch& ctx, const vdn_shape& s, const float* 
 
 cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                                const CUtensorMap& omap, const float* states);
+
+// MXFP8 quantization of a bf16 [R, ld] operand (K = cols, a multiple of 128):
+// codes [R, K] row-major and scale bytes in the MMA tile layout (mxfp8.cuh).
+cudaError_t launch_mx_quantize(cudaStream_t st, const void* x, int64_t ld, int R, int K,
+                               uint8_t* q, uint8_t* sf);
 
 // ---- gradient pass (see vda_grad.cu) -------------------------------------
 

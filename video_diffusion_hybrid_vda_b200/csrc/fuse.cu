@@ -17,7 +17,10 @@
 // rows are reused from L2 and the weights stay L2-resident.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
+#include "mxfp8.cuh"
 #include "ptx.cuh"
 #include "repack.cuh"
 
@@ -83,10 +86,12 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float (&f)
                       pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
 }
 
-// Epilogue for GEMM 1 on one 32-column chunk of row r starting at column n.
-__device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
-                                           const uint32_t (&acc)[32], float& rinv) {
-  float z[32];
+// Gated branch inputs z for one 32-column chunk of row r starting at
+// column n of GEMM 1's output (gate logits in acc); rinv carries the head's
+// 1 / RMS from its first chunk to the next ones.
+template <class A>
+__device__ __forceinline__ void gate_values(const A& a, int64_t r, int n, const uint32_t (&acc)[32],
+                                            float& rinv, float (&z)[32]) {
   if (n < a.D) {
     float os[32];
     load_bf16x32(a.o_s + r * a.D + n, os);
@@ -111,6 +116,13 @@ __device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
     for (int e = 0; e < 32; ++e)
       z[e] = sigmoidf_fast(__uint_as_float(acc[e])) * (ov[e] * rinv * __ldg(a.gamma + c + e));
   }
+}
+
+// Epilogue for GEMM 1 on one 32-column chunk of row r starting at column n.
+__device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
+                                           const uint32_t (&acc)[32], float& rinv) {
+  float z[32];
+  gate_values(a, r, n, acc, rinv, z);
   store_bf16x32(a.Z + r * (2 * static_cast<int64_t>(a.D)) + n, z);
 }
 
@@ -307,6 +319,231 @@ cudaError_t launch_gemm(const Launch& ctx, const CUtensorMap& a, const CUtensorM
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- MXFP8 GEMM
+//
+// C[M, N] = A[M, K] B[N, K]^T with both operands MXFP8 (E4M3 codes, K-major,
+// one UE8M0 scale per 32 elements of K in the tile layout of mxfp8.cuh).
+// Same persistent structure as gemm_kernel, with 128 x 128 output tiles: a
+// 6-stage ring of [128 x 128]-byte A and B tiles (TMA, 128B swizzle) plus
+// the two 512-byte scale blocks of the stage (bulk copies); the MMA thread
+// copies a stage's scales into TMEM (tcgen05.cp, replicated into all lane
+// quarters) and issues four block-scaled MMAs (K = 32 each, the scale byte
+// chosen by the instruction's scale id).  TMEM: two 128-column accumulators
+// and 8 scale columns per stage.
+constexpr int MX_BM = 128, MX_BN = 128, MX_BK = 128, MX_STAGES = 6;
+constexpr int MX_TILE = 128 * MX_BK;                 // 16 KB of codes
+constexpr int MX_STAGE = 2 * MX_TILE + 1024;         // A, B, their scale blocks
+constexpr int MX_SMEM = 1024 + MX_STAGES * MX_STAGE + 256;
+constexpr int MX_SF_COL = 2 * MX_BN;                 // first scale column in TMEM
+
+struct GateMXArgs {
+  const __nv_bfloat16* o_s;
+  const __nv_bfloat16* o_vda;
+  const float* gamma;
+  float eps;
+  int D, d;
+  float inv_d;
+  uint8_t* zq;   // [M, 2D] E4M3 codes
+  uint8_t* zsf;  // scales of Z, tile layout (2D / 128 column tiles)
+};
+
+template <class Args>
+__global__ void __launch_bounds__(GEMM_THREADS, 1)
+    gemm_mx_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                   const uint8_t* __restrict__ a_sf, const uint8_t* __restrict__ b_sf, int M, int N,
+                   int K, Args args, uint32_t* status, uint64_t budget_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + MX_STAGES * MX_STAGE);
+  uint64_t* empty = full + MX_STAGES;
+  uint64_t* tfull = empty + MX_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int mblocks = (M + MX_BM - 1) / MX_BM;
+  const int nblocks = (N + MX_BN - 1) / MX_BN;
+  const int ntiles = mblocks * nblocks;
+  const int nk = K / MX_BK;
+  const uint32_t warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < MX_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 128);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&bmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int mb = tile / nblocks, nb = tile % nblocks;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % MX_STAGES;
+          if (it >= MX_STAGES && !mbar_wait(&empty[s], ((it / MX_STAGES) & 1) ^ 1, budget_ns)) {
+            record_status(status, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * MX_STAGE;
+          mbar_arrive_expect_tx(&full[s], MX_STAGE);
+          tma_load_2d(st, &amap, &full[s], kb * MX_BK, mb * MX_BM);
+          tma_load_2d(st + MX_TILE, &bmap, &full[s], kb * MX_BK, nb * MX_BN);
+          bulk_load(st + 2 * MX_TILE, a_sf + (static_cast<int64_t>(mb) * nk + kb) * 512, 512,
+                    &full[s]);
+          bulk_load(st + 2 * MX_TILE + 512, b_sf + (static_cast<int64_t>(nb) * nk + kb) * 512, 512,
+                    &full[s]);
+        }
+      }
+      const uint32_t first = it > MX_STAGES ? it - MX_STAGES : 0;
+      for (uint32_t j = first; j < it; ++j)
+        if (!mbar_wait(&full[j % MX_STAGES], (j / MX_STAGES) & 1, 200000000ull))
+          record_status(status, kStatusTimeout);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      constexpr uint32_t idesc = idesc_mxf8(MX_BM, MX_BN);
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++lt) {
+        const int b = lt & 1;
+        if (lt >= 2 && !mbar_wait(&tempty[b], ((lt >> 1) & 1) ^ 1, budget_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc_addr = tmem + b * MX_BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % MX_STAGES;
+          if (!mbar_wait(&full[s], (it / MX_STAGES) & 1, budget_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + s * MX_STAGE);
+          const uint32_t sfa = tmem + MX_SF_COL + 8 * s;
+          const uint32_t sfb = sfa + 4;
+          // 32 rows x 16 bytes per block: 8-row groups 128 bytes apart
+          tmem_cp_32x128b_x4(sfa, sdesc_none(st + 2 * MX_TILE, 16, 128));
+          tmem_cp_32x128b_x4(sfb, sdesc_none(st + 2 * MX_TILE + 512, 16, 128));
+#pragma unroll
+          for (int j = 0; j < MX_BK / 32; ++j) {
+            const uint32_t id = idesc | (static_cast<uint32_t>(j) << 29) | (static_cast<uint32_t>(j) << 4);
+            umma_mx_ss(acc_addr, sdesc_sw128(st + j * 32, 16, 1024),
+                       sdesc_sw128(st + MX_TILE + j * 32, 16, 1024), id,
+                       sfa | (static_cast<uint32_t>(j) << 30), sfb | (static_cast<uint32_t>(j) << 30),
+                       (kb | j) != 0);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[b]);
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+      umma_commit(mma_done);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t quarter = warp & 3;
+    const int row = quarter * 32 + lane_id();
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      // warp-uniform: the TMEM loads below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[b], (lt >> 1) & 1, budget_ns))) {
+        record_status(status, kStatusTimeout);
+        break;
+      }
+      tc_fence_after();
+      const int mb = tile / nblocks, nb = tile % nblocks;
+      const int64_t r = static_cast<int64_t>(mb) * MX_BM + row;
+      const uint32_t taddr = tmem + b * MX_BN + ((quarter * 32) << 16);
+      float rinv = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < MX_BN; c += 32) {
+        uint32_t acc[32];
+        tmem_ld32(taddr + c, acc);
+        tmem_ld_wait();
+        const int n = nb * MX_BN + c;
+        if (r < M && n < N) {
+          if constexpr (std::is_same<Args, GateMXArgs>::value) {
+            float z[32];
+            gate_values(args, r, n, acc, rinv, z);
+            uint4 codes[2];
+            const uint8_t sb = mx_quantize_block(z, codes);
+            const int64_t ldz = 2 * static_cast<int64_t>(args.D);
+            uint4* dst = reinterpret_cast<uint4*>(args.zq + r * ldz + n);
+            dst[0] = codes[0];
+            dst[1] = codes[1];
+            args.zsf[mx_sf_offset(r, n / 32, static_cast<int>(ldz / 128))] = sb;
+          } else if constexpr (sizeof(args.y[0]) == 4) {
+            float4* dst = reinterpret_cast<float4*>(args.y + r * N + n);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(acc[4 * e]), __uint_as_float(acc[4 * e + 1]),
+                                   __uint_as_float(acc[4 * e + 2]),
+                                   __uint_as_float(acc[4 * e + 3]));
+          } else {
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(acc[e]);
+            store_bf16x32(args.y + r * N + n, f);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    mbar_wait(mma_done, 0, 200000000ull);
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <class Args>
+cudaError_t launch_gemm_mx(const Launch& ctx, const CUtensorMap& a, const CUtensorMap& b,
+                           const uint8_t* a_sf, const uint8_t* b_sf, int M, int N, int K,
+                           const Args& args, int sm_count) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_mx_kernel<Args>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, MX_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int ntiles = ((M + MX_BM - 1) / MX_BM) * ((N + MX_BN - 1) / MX_BN);
+  const int grid = ntiles < sm_count ? ntiles : sm_count;
+  gemm_mx_kernel<Args><<<grid, GEMM_THREADS, MX_SMEM, ctx.stream>>>(
+      a, b, a_sf, b_sf, M, N, K, args, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
 bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int sm_count_of_current_device() {
@@ -494,4 +731,106 @@ vdn_status vdn_hybrid_fuse_shard(int L, int D, int H_local, int d, int head0, co
   return VDN_OK;
 }
 
+// ----------------------------------------------------------------- MXFP8
+
+vdn_status vdn_gemm_mxfp8(int M, int N, int K, const void* a, const void* a_sf, const void* b,
+                          const void* b_sf, void* c, int c_is_f32, void* ws, size_t ws_bytes,
+                          void* stream) {
+  NvtxRange nvtx("vdn_gemm_mxfp8");
+  if (M < 1 || N < 1 || K < 1 || !a || !a_sf || !b || !b_sf || !c) return VDN_ERR_INVALID_ARG;
+  if (K % 128 != 0 || N % 32 != 0) return VDN_ERR_UNSUPPORTED;
+  if (!a16(a) || !a16(a_sf) || !a16(b) || !a16(b_sf) || !a16(c)) return VDN_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < kStatusBytes)
+    return VDN_ERR_WORKSPACE;
+  CUtensorMap amap, bmap;
+  if (!make_rows_map_u8(&amap, a, K, K, M, MX_BM) || !make_rows_map_u8(&bmap, b, K, K, N, MX_BN))
+    return VDN_ERR_CUDA;
+  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
+             current_wait_budget_ns()};
+  const int sms = sm_count_of_current_device();
+  const uint8_t* asf = static_cast<const uint8_t*>(a_sf);
+  const uint8_t* bsf = static_cast<const uint8_t*>(b_sf);
+  cudaError_t e;
+  if (c_is_f32)
+    e = launch_gemm_mx(ctx, amap, bmap, asf, bsf, M, N, K, StoreF32Args{static_cast<float*>(c)},
+                       sms);
+  else
+    e = launch_gemm_mx(ctx, amap, bmap, asf, bsf, M, N, K,
+                       StoreArgs{static_cast<__nv_bfloat16*>(c)}, sms);
+  return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
+}
+
+namespace {
+
+// MXFP8 fuse workspace: [status][x codes L x D][x scales][Z codes L x 2D][Z scales]
+struct MxFusePlan {
+  size_t xq, xsf, zq, zsf, total;
+};
+
+MxFusePlan mx_fuse_plan(int L, int D) {
+  MxFusePlan p;
+  p.xq = kStatusBytes;
+  p.xsf = p.xq + r256(static_cast<size_t>(L) * D);
+  p.zq = p.xsf + r256(vdn_mxfp8_scale_bytes(L, D));
+  p.zsf = p.zq + r256(static_cast<size_t>(L) * 2 * D);
+  p.total = p.zsf + r256(vdn_mxfp8_scale_bytes(L, 2 * static_cast<int64_t>(D)));
+  return p;
+}
+
+}  // namespace
+
+size_t vdn_hybrid_fuse_mxfp8_workspace(int L, int D, int H) {
+  if (L < 1 || D < 128 || H < 1 || D % H != 0 || D % 128 != 0) return 0;
+  return mx_fuse_plan(L, D).total;
+}
+
+vdn_status vdn_hybrid_fuse_mxfp8(int L, int D, int H, const void* x, const void* o_s,
+                                 const void* o_vda, const void* wg_q, const void* wg_sf,
+                                 const float* gamma, float eps, const void* wo_q,
+                                 const void* wo_sf, void* y, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  NvtxRange nvtx("vdn_hybrid_fuse_mxfp8");
+  if (L < 1 || D < 1 || H < 1 || D % H != 0) return VDN_ERR_INVALID_ARG;
+  if (!x || !o_s || !o_vda || !wg_q || !wg_sf || !gamma || !wo_q || !wo_sf || !y)
+    return VDN_ERR_INVALID_ARG;
+  if (!a16(x) || !a16(o_s) || !a16(o_vda) || !a16(wg_q) || !a16(wg_sf) || !a16(wo_q) ||
+      !a16(wo_sf) || !a16(y) || (reinterpret_cast<uintptr_t>(gamma) & 3u) || !(eps >= 0.f))
+    return VDN_ERR_INVALID_ARG;
+  const int d = D / H;
+  // 128-column tiles: heads must not cross a tile (d divides 128) and the
+  // RMSNorm reads whole 32-column chunks
+  if (D % 128 != 0 || d % 32 != 0 || 128 % d != 0) return VDN_ERR_UNSUPPORTED;
+  const MxFusePlan pl = mx_fuse_plan(L, D);
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) || ws_bytes < pl.total)
+    return VDN_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* xq = base + pl.xq;
+  uint8_t* xsf = base + pl.xsf;
+  uint8_t* zq = base + pl.zq;
+  uint8_t* zsf = base + pl.zsf;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (launch_mx_quantize(st, x, D, L, D, xq, xsf) != cudaSuccess) return VDN_ERR_CUDA;
+
+  CUtensorMap xmap, gmap, zmap, omap;
+  if (!make_rows_map_u8(&xmap, xq, D, D, L, MX_BM) ||
+      !make_rows_map_u8(&gmap, wg_q, D, D, 2 * static_cast<int64_t>(D), MX_BN) ||
+      !make_rows_map_u8(&zmap, zq, 2 * static_cast<int64_t>(D), 2 * static_cast<int64_t>(D), L,
+                        MX_BM) ||
+      !make_rows_map_u8(&omap, wo_q, 2 * static_cast<int64_t>(D), 2 * static_cast<int64_t>(D), D,
+                        MX_BN))
+    return VDN_ERR_CUDA;
+  Launch ctx{st, static_cast<uint32_t*>(ws), current_wait_budget_ns()};
+  const int sms = sm_count_of_current_device();
+  GateMXArgs g{static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_vda),
+               gamma, eps, D, d, 1.f / static_cast<float>(d), zq, zsf};
+  if (launch_gemm_mx(ctx, xmap, gmap, xsf, static_cast<const uint8_t*>(wg_sf), L, 2 * D, D, g,
+                     sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (launch_gemm_mx(ctx, zmap, omap, zsf, static_cast<const uint8_t*>(wo_sf), L, D, 2 * D,
+                     StoreArgs{static_cast<__nv_bfloat16*>(y)}, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
 }  // extern "C"
+

@@ -207,6 +207,30 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with MX block scales (E4M3 operands, one
+// UE8M0 scale per 32 elements of K; K = 32 per instruction).  sfa / sfb are
+// TMEM addresses of the scale columns; their top two bits select the byte of
+// each 32-bit cell (and must equal the scale ids in idesc).
+__device__ __forceinline__ void umma_mx_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Shared memory -> TMEM copy of a 32-row x 16-byte block into TMEM lanes
+// 0..31 of four columns, replicated into every lane quarter (the layout of
+// MX scale factors).  Asynchronous; ordered with the MMAs this thread
+// issues after it.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.
 __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                         uint32_t idesc, uint32_t accumulate) {
@@ -291,6 +315,27 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100)
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
+}
+
+// Shared-memory descriptor without swizzle, K-major: 8-row core matrices of
+// 16-byte rows, 8-row groups sbo bytes apart (lbo: between core matrices
+// along K, unused for one 16-byte column).
+__device__ __forceinline__ uint64_t sdesc_none(uint32_t saddr, uint32_t lbo_bytes,
+                                               uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm_100); layout 0 = no swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::mxf8f6f4 with block scales: E4M3 A and B
+// (format 0), UE8M0 scales (bit 23), both K-major, fp32 accumulator; the
+// scale ids (bits 29-30 for A, 4-5 for B) are added per instruction.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N) {
+  return (0u << 7) | (0u << 10) | (1u << 23) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator.

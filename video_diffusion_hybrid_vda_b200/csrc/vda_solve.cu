@@ -32,11 +32,8 @@ template <int DH>
 struct SolveCfg {
   static constexpr int RA = DH / 16;   // rows per thread (rows ty + 16 a)
   static constexpr int CB = DH / 16;   // columns per thread (cols tx + 16 b)
-  static constexpr int RG = DH / 64;   // 4-wide column groups of W per thread
-  static constexpr int LD = DH + 1;    // row stride of L (column accesses)
-  static constexpr int LD2 = DH + 4;   // row stride of W / P (float4 rows)
-  static constexpr int MAT = DH * LD2; // floats of the matrix buffer (>= DH * LD)
-  static constexpr int TR = DH / 16;   // products: TR x TR tile per thread
+  static constexpr int LD2 = DH + 4;   // row stride of the matrix buffer (float4 rows)
+  static constexpr int MAT = DH * LD2; // floats of the matrix buffer
   static constexpr int SMEM = MAT * 4 + 4 * DH * 4;
 };
 

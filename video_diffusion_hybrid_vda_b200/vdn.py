@@ -26,7 +26,9 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_reset_device_status", "vdn_set_wait_budget_ns", "vdn_version",
            "vdn_vda_scan_static", "vdn_selftest_exp2", "vdn_window_attn_ctx",
            "vdn_set_vda_solver", "vdn_hybrid_fuse_shard_workspace", "vdn_hybrid_fuse_shard",
-           "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers"]
+           "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers",
+           "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
+           "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -104,6 +106,19 @@ def lib():
     L.vdn_vda_backward.restype = ctypes.c_int
     L.vdn_vda_backward_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 3
     L.vdn_vda_backward_debug_buffers.restype = ctypes.c_int
+    L.vdn_vda_scan_static.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _P]
+    L.vdn_vda_scan_static.restype = ctypes.c_int
+    L.vdn_mxfp8_scale_bytes.argtypes = [_I64, _I64]
+    L.vdn_mxfp8_scale_bytes.restype = _SZ
+    L.vdn_mxfp8_quantize.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P]
+    L.vdn_mxfp8_quantize.restype = ctypes.c_int
+    L.vdn_gemm_mxfp8.argtypes = [ctypes.c_int] * 3 + [_P] * 5 + [ctypes.c_int, _P, _SZ, _P]
+    L.vdn_gemm_mxfp8.restype = ctypes.c_int
+    L.vdn_hybrid_fuse_mxfp8_workspace.argtypes = [ctypes.c_int] * 3
+    L.vdn_hybrid_fuse_mxfp8_workspace.restype = _SZ
+    L.vdn_hybrid_fuse_mxfp8.argtypes = [ctypes.c_int] * 3 + [_P] * 6 + [ctypes.c_float, _P, _P,
+                                                                         _P, _P, _SZ, _P]
+    L.vdn_hybrid_fuse_mxfp8.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -264,6 +279,64 @@ def vda_backward_debug_buffers(ws, T, N, H, d):
         off = p.value - base
         out.append(flat[off:off + 4 * n].view(torch.float32).view(lead, T, H, dd, dd))
     return out[0], out[1], out[2][0]
+
+
+# ---------------------------------------------------------------- MXFP8
+
+def mxfp8_scale_bytes(rows, cols):
+    return int(lib().vdn_mxfp8_scale_bytes(int(rows), int(cols)))
+
+
+def mxfp8_quantize(x, stream=None):
+    """bf16 [R, K] (K a multiple of 128) -> (E4M3 codes uint8 [R, K], scale
+    bytes uint8 in the GEMM's tile layout)."""
+    _need_cuda(x)
+    R, K = x.shape
+    q = torch.empty((R, K), dtype=torch.uint8, device=x.device)
+    sf = torch.empty(max(mxfp8_scale_bytes(R, K), 16), dtype=torch.uint8, device=x.device)
+    _check(lib().vdn_mxfp8_quantize(_ptr(x), R, K, x.stride(0), _ptr(q), _ptr(sf), _stream(stream)),
+           "vdn_mxfp8_quantize")
+    return q, sf
+
+
+def gemm_mxfp8(a, b, out_f32=False, ws=None, stream=None):
+    """C = A B^T for MXFP8 operands a = (codes [M, K], scales), b = (codes [N, K], scales)."""
+    (aq, asf), (bq, bsf) = a, b
+    _need_cuda(aq, asf, bq, bsf)
+    M, K = aq.shape
+    N = bq.shape[0]
+    c = torch.empty((M, N), dtype=torch.float32 if out_f32 else torch.bfloat16, device=aq.device)
+    if ws is None:
+        ws = alloc_workspace(256, aq.device)
+    _check(lib().vdn_gemm_mxfp8(M, N, K, _ptr(aq), _ptr(asf), _ptr(bq), _ptr(bsf), _ptr(c),
+                                int(bool(out_f32)), _ptr(ws), ws.numel(), _stream(stream)),
+           "vdn_gemm_mxfp8")
+    return c, ws
+
+
+def mxfp8_fuse_weights(W_gs, W_gl, W_os, W_ol, stream=None):
+    """MXFP8 weights of the fuse: the stacked gate weights [W_gs; W_gl] and
+    the side-by-side output weights [W_os | W_ol], each (codes, scales)."""
+    wg = mxfp8_quantize(torch.cat([W_gs, W_gl], dim=0).contiguous(), stream)
+    wo = mxfp8_quantize(torch.cat([W_os, W_ol], dim=1).contiguous(), stream)
+    return wg, wo
+
+
+def hybrid_fuse_mxfp8(x, o_s, o_vda, wg, gamma, wo, H, eps=1e-6, out=None, ws=None, stream=None):
+    """The fuse with MXFP8 projections (wg, wo from mxfp8_fuse_weights).
+    Returns (y bf16 [L, D], ws)."""
+    _need_cuda(x, o_s, o_vda, gamma, out, ws)
+    L, D = x.shape
+    if out is None:
+        out = torch.empty((L, D), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(int(lib().vdn_hybrid_fuse_mxfp8_workspace(L, D, H)), x.device)
+    _check(lib().vdn_hybrid_fuse_mxfp8(L, D, H, _ptr(x), _ptr(o_s), _ptr(o_vda), _ptr(wg[0]),
+                                       _ptr(wg[1]), _ptr(gamma), float(eps), _ptr(wo[0]),
+                                       _ptr(wo[1]), _ptr(out), _ptr(ws), ws.numel(),
+                                       _stream(stream)),
+           "vdn_hybrid_fuse_mxfp8")
+    return out, ws
 
 
 # ---------------------------------------------------------------- window Softmax
