@@ -10,10 +10,13 @@ flush is needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload layer102|layer42|small] [--part all|layer|vda_backward]
 
-The line also carries ``vda_backward``: the VDA gradient pass (dq, dk, dv,
-dbeta, dalpha from dL/do_vda, forward recomputed inside) timed on its own
-on the same inputs; it is not part of the step.  ``--part vda_backward``
-times only that pass (for launch lists and captures).
+The line also carries two rows timed on their own, not part of the step:
+``vda_backward``, the VDA gradient pass (dq, dk, dv, dbeta, dalpha from
+dL/do_vda, forward recomputed inside), and ``fuse_mxfp8``, the fuse with
+both projection GEMMs in MXFP8 (x quantized inside the timed call, weights
+quantized beforehand), against the FP8 peak and beside the bf16 fuse's
+output.  ``--part vda_backward`` / ``--part fuse_mxfp8`` time only that
+row (for launch lists and captures).
 
 With N > 1 (torchrun) every rank runs its own video (independent problems,
 no collective on the data path): weak scaling, time = max over ranks.
@@ -348,6 +351,60 @@ def run_vda_backward(args, shape, rank, world):
     return ms
 
 
+def run_fuse_mxfp8(args, shape, rank, world):
+    """Device time of the MXFP8 fuse (ms, max over ranks) and the max
+    relative deviation of its output from the bf16 fuse's on the same inputs."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev, with_fuse=True)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2000 + rank)
+    o_s = torch.randn((shape.L, shape.D), generator=gen, device=dev).to(torch.bfloat16)
+    o_vda = torch.randn((shape.L, shape.D), generator=gen, device=dev).to(torch.bfloat16)
+    wg, wo = vdn.mxfp8_fuse_weights(inp["W_gs"], inp["W_gl"], inp["W_os"], inp["W_ol"])
+    y = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
+    ws = vdn.alloc_workspace(vdn.lib().vdn_hybrid_fuse_mxfp8_workspace(shape.L, shape.D, shape.H),
+                             dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vdn.hybrid_fuse_mxfp8(inp["x"], o_s, o_vda, wg, inp["gamma"], wo, shape.H, out=y, ws=ws,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the MXFP8 fuse warm-up")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    y_bf16, _ = vdn.hybrid_fuse(inp["x"], o_s, o_vda, inp["W_gs"], inp["W_gl"], inp["gamma"],
+                                inp["W_os"], inp["W_ol"], shape.H)
+    dev_rel = float(((y.float() - y_bf16.float()).abs().max() / y_bf16.float().abs().max()).item())
+    del inp, o_s, o_vda, wg, wo, y, ws, y_bf16
+    torch.cuda.empty_cache()
+    return ms, dev_rel
+
+
+def mxfp8_row(work, peaks, ms, dev_rel):
+    peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    tf = work["proj_flop"] / (ms / 1e3) / 1e12
+    return {"ms": ms, "bound": "tensor", "achieved_tflops": tf, "peak_tflops": peak,
+            "frac": tf / peak, "peak_source": "measured bf16_tflops_sustained x 2 (nominal "
+                                              "fp8 / bf16 dense ratio)",
+            "max_rel_vs_bf16_fuse": dev_rel, "launches_per_call": 3}
+
+
 def backward_row(work, peaks, ms):
     roof_ms = (work["vda_bwd_bytes"] / (peaks["hbm_gbs"] * 1e9) +
                work["vda_bwd_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3
@@ -366,9 +423,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
                     help="solver of (I + A)^-1 in the VDA branch")
-    ap.add_argument("--part", default="all", choices=["all", "layer", "vda_backward"],
-                    help="what to time: the layer step and the VDA gradient pass (all), "
-                         "or one of them")
+    ap.add_argument("--part", default="all",
+                    choices=["all", "layer", "vda_backward", "fuse_mxfp8"],
+                    help="what to time: the layer step and the two side rows (all), or one "
+                         "of them")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -417,6 +475,18 @@ def main():
                               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                               "dtype": "bf16", "data": "synthetic", "config": config,
                               "vda_backward": backward_row(work, peaks, ms)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if args.part == "fuse_mxfp8":
+        ms, dev_rel = run_fuse_mxfp8(args, shape, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "MXFP8 fuse ms (both projection GEMMs in MXFP8)",
+                              "value": ms, "unit": "ms", "higher_is_better": False,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "dtype": "mxfp8 (e4m3, ue8m0 / 32)", "data": "synthetic",
+                              "config": config,
+                              "fuse_mxfp8": mxfp8_row(work, peaks, ms, dev_rel)}))
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -472,6 +542,7 @@ def main():
     if args.part == "all":
         line["vda_backward"] = backward_row(work, peaks,
                                             run_vda_backward(args, shape, rank, world))
+        line["fuse_mxfp8"] = mxfp8_row(work, peaks, *run_fuse_mxfp8(args, shape, rank, world))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(shape)
         line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
