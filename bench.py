@@ -304,7 +304,7 @@ def run_gpu(args, shape, rank, world):
     ms, e2e_ms = t[0], t[1]
     return dict(ms=ms, win_ms=t[2] / args.steps, vda_ms=t[3] / args.steps,
                 fuse_ms=t[4] / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
-                clocks=clocks, launches=layer.KERNELS_PER_FORWARD * args.steps)
+                clocks=clocks, launches=layer.kernels_per_forward * args.steps)
 
 
 def run_vda_backward(args, shape, rank, world):

@@ -124,3 +124,25 @@ def test_fuse_mxfp8_full_block_sampled(vdn):
     assert max_rel(host(y[torch.as_tensor(rows, device="cuda")]), ref) <= TOL_BF16
     del inp, y, ws
     torch.cuda.empty_cache()
+
+
+def test_hybrid_layer_with_mxfp8_projections(vdn):
+    """HybridLayer(projections="mxfp8"): y against the oracle's MXFP8 fuse
+    on the layer's own branch outputs, and the host-copy path (forward_many)
+    giving the same y."""
+    shape = synth.Shape(12, 96, 2, 128)
+    inp = synth.make_inputs(shape, seed=4, device="cuda", with_fuse=True)
+    layer = vdn.HybridLayer(shape.T, shape.N, shape.H, shape.d, inp["W_gs"], inp["W_gl"],
+                            inp["W_os"], inp["W_ol"], inp["gamma"], projections="mxfp8")
+    acts = [inp[k] for k in ("q", "k", "v", "beta", "alpha", "x")]
+    y = layer.forward(*acts).clone()
+    assert layer.status() == 0
+    ref = omx.hybrid_fuse_mxfp8(host(inp["x"]), host(layer.o_s), host(layer.o_vda),
+                                host(inp["W_gs"]), host(inp["W_gl"]), host(inp["gamma"]), 1e-6,
+                                host(inp["W_os"]), host(inp["W_ol"]), shape.H)
+    assert max_rel(host(y), ref) <= TOL_BF16
+    hosts = [[t.cpu().pin_memory() for t in acts]]
+    outs = [torch.empty((shape.L, shape.D), dtype=torch.bfloat16).pin_memory()]
+    layer.forward_many(hosts, outs)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], y.cpu())

@@ -31,7 +31,10 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;  // 16 KB
 constexpr int B_BYTES = BN * BK * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int GEMM_THREADS = 192;  // warp0 TMA, warp1 MMA, warps2-5 epilogue
+// warp 0 TMA, warp 1 MMA, warps 2-9 epilogue: two warps per TMEM lane quarter,
+// each draining half of the tile's columns
+constexpr int EPI_THREADS = 256;
+constexpr int GEMM_THREADS = 64 + EPI_THREADS;
 constexpr int GEMM_SMEM = 1024 + STAGES * STAGE_BYTES + 256;
 
 enum class BSplit { kByN, kByK };
@@ -88,10 +91,11 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* p, const float (&f)
 
 // Gated branch inputs z for one 32-column chunk of row r starting at
 // column n of GEMM 1's output (gate logits in acc); rinv carries the head's
-// 1 / RMS from its first chunk to the next ones.
+// 1 / RMS from its first chunk to the next ones (fresh: the thread's first
+// chunk of a tile, which may start inside a head).
 template <class A>
 __device__ __forceinline__ void gate_values(const A& a, int64_t r, int n, const uint32_t (&acc)[32],
-                                            float& rinv, float (&z)[32]) {
+                                            float& rinv, float (&z)[32], bool fresh) {
   if (n < a.D) {
     float os[32];
     load_bf16x32(a.o_s + r * a.D + n, os);
@@ -100,11 +104,12 @@ __device__ __forceinline__ void gate_values(const A& a, int64_t r, int n, const 
   } else {
     const int c = n - a.D;
     const __nv_bfloat16* orow = a.o_vda + r * a.D;
-    if (c % a.d == 0) {  // first chunk of a head: its RMS over d channels
+    if (fresh || c % a.d == 0) {  // the head's RMS over its d channels
+      const int hs = c - c % a.d;
       float ss = 0.f;
       for (int k = 0; k < a.d; k += 32) {
         float f[32];
-        load_bf16x32(orow + c + k, f);
+        load_bf16x32(orow + hs + k, f);
 #pragma unroll
         for (int e = 0; e < 32; ++e) ss = fmaf(f[e], f[e], ss);
       }
@@ -120,9 +125,9 @@ __device__ __forceinline__ void gate_values(const A& a, int64_t r, int n, const 
 
 // Epilogue for GEMM 1 on one 32-column chunk of row r starting at column n.
 __device__ __forceinline__ void gate_chunk(const GateArgs& a, int64_t r, int n,
-                                           const uint32_t (&acc)[32], float& rinv) {
+                                           const uint32_t (&acc)[32], float& rinv, bool fresh) {
   float z[32];
-  gate_values(a, r, n, acc, rinv, z);
+  gate_values(a, r, n, acc, rinv, z, fresh);
   store_bf16x32(a.Z + r * (2 * static_cast<int64_t>(a.D)) + n, z);
 }
 
@@ -154,7 +159,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], EPI_THREADS);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -250,6 +255,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane_id();
+    const int c0 = static_cast<int>((warp - 2) >> 2) * (BN / 2);  // this warp's column half
     int lt = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
       const int b = lt & 1;
@@ -264,14 +270,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t taddr = tmem + b * BN + ((quarter * 32) << 16);
       float rinv = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = c0; c < c0 + BN / 2; c += 32) {
         uint32_t acc[32];
         tmem_ld32(taddr + c, acc);
         tmem_ld_wait();
         const int n = nb * BN + c;
         if (r < M && n < N) {
           if constexpr (SPLIT == BSplit::kByN) {
-            gate_chunk(args, r, n, acc, rinv);
+            gate_chunk(args, r, n, acc, rinv, c == c0);
           } else if constexpr (sizeof(args.y[0]) == 4) {
             float4* dst = reinterpret_cast<float4*>(args.y + r * N + n);
 #pragma unroll
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
+      mbar_init(&tempty[b], EPI_THREADS);
     }
     mbar_init(mma_done, 1);
     fence_mbar_init();
@@ -467,6 +473,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     // ------------------------------------------------------------ epilogue
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane_id();
+    const int c0 = static_cast<int>((warp - 2) >> 2) * (MX_BN / 2);  // this warp's column half
     int lt = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++lt) {
       const int b = lt & 1;
@@ -481,7 +488,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t taddr = tmem + b * MX_BN + ((quarter * 32) << 16);
       float rinv = 0.f;
 #pragma unroll 1
-      for (int c = 0; c < MX_BN; c += 32) {
+      for (int c = c0; c < c0 + MX_BN / 2; c += 32) {
         uint32_t acc[32];
         tmem_ld32(taddr + c, acc);
         tmem_ld_wait();
@@ -489,7 +496,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (r < M && n < N) {
           if constexpr (std::is_same<Args, GateMXArgs>::value) {
             float z[32];
-            gate_values(args, r, n, acc, rinv, z);
+            gate_values(args, r, n, acc, rinv, z, c == c0);
             uint4 codes[2];
             const uint8_t sb = mx_quantize_block(z, codes);
             const int64_t ldz = 2 * static_cast<int64_t>(args.D);

@@ -429,12 +429,14 @@ class HybridLayer:
     Inputs may be CUDA tensors, or host tensors (pinned for asynchronous
     copies): host inputs are copied into device buffers owned by the layer
     and, when ``out`` is a host tensor, y is copied back into it.
+    ``projections="mxfp8"`` runs both fuse GEMMs on MXFP8 operands (weights
+    quantized once here, x on every call).
     """
 
     KERNELS_PER_FORWARD = 7   # prep, solve, scan, read-out, window Softmax, 2 GEMMs
 
     def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, chunk_frames=5,
-                 window_chunks=1, anchors=3, device=None):
+                 window_chunks=1, anchors=3, device=None, projections="bf16"):
         self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
         self.L, self.D = self.T * self.N, self.H * self.d
         self.device = torch.device(device or "cuda")
@@ -450,8 +452,26 @@ class HybridLayer:
         self.y = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
         self.ws_vda = alloc_workspace(vda_scan_workspace(T, N, H, d), dev)
         self.ws_win = alloc_workspace(window_attn_workspace(T, N, H, d), dev)
-        self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D, H), dev)
+        if projections not in ("bf16", "mxfp8"):
+            raise ValueError("projections: 'bf16' or 'mxfp8'")
+        self.projections = projections
+        if projections == "mxfp8":
+            self.wg, self.wo = mxfp8_fuse_weights(self.W_gs, self.W_gl, self.W_os, self.W_ol)
+            self.ws_fuse = alloc_workspace(
+                int(lib().vdn_hybrid_fuse_mxfp8_workspace(L, D, H)), dev)
+            self.kernels_per_forward = self.KERNELS_PER_FORWARD + 1  # + quantize x
+        else:
+            self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D, H), dev)
+            self.kernels_per_forward = self.KERNELS_PER_FORWARD
         self._staging = None
+
+    def _fuse(self, x, y, stream):
+        if self.projections == "mxfp8":
+            hybrid_fuse_mxfp8(x, self.o_s, self.o_vda, self.wg, self.gamma, self.wo, self.H,
+                              eps=self.eps, out=y, ws=self.ws_fuse, stream=stream)
+        else:
+            hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
+                        self.W_ol, self.H, eps=self.eps, out=y, ws=self.ws_fuse, stream=stream)
 
     def _to_device(self, tensors, stream):
         if all(t.is_cuda for t in tensors):
@@ -474,8 +494,7 @@ class HybridLayer:
         window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win, stream=stream,
                     ctx_k=ctx_k, ctx_v=ctx_v)
         vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda, stream=stream)
-        hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
-                    self.W_ol, H, eps=self.eps, out=self.y, ws=self.ws_fuse, stream=stream)
+        self._fuse(x, self.y, stream)
         if out is not None and not out.is_cuda:
             with torch.cuda.stream(stream):
                 out.copy_(self.y, non_blocking=True)
@@ -532,8 +551,7 @@ class HybridLayer:
                         stream=stream)
             vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
                      stream=stream)
-            hybrid_fuse(x, self.o_s, self.o_vda, self.W_gs, self.W_gl, self.gamma, self.W_os,
-                        self.W_ol, H, eps=self.eps, out=y, ws=self.ws_fuse, stream=stream)
+            self._fuse(x, y, stream)
             computed[i].record(stream)
             if i == 0:
                 self._read = [torch.cuda.Event() for _ in batches]
