@@ -311,6 +311,27 @@ VDN_API vdn_status vdn_hybrid_fuse_shard(int L, int D, int H_local, int d, int h
                                          const void* W_ol, float* y_partial, void* ws,
                                          size_t ws_bytes, void* stream);
 
+/* vdn_hybrid_fuse_shard with the reduce-scatter fused into the output
+ * GEMM: instead of writing an fp32 partial, the GEMM's epilogue adds row r
+ * of this shard's partial into y_owners[r / R] at row r % R, R = ceil(L / G),
+ * with system-scope atomic adds (so the owners may be other GPUs' memory
+ * reached through a peer mapping: CUDA IPC, a symmetric-memory allocation).
+ * After every shard's call the owners hold the summed rows of y.
+ *  - y_owners: host array of G device pointers (1 <= G <= 8), each fp32
+ *    [R, D] (the last [L - (G-1) R, D]), 16-byte aligned.
+ *  - The caller zeroes the owners' buffers before any shard's call and reads
+ *    them only after every shard's call has finished (a barrier across the
+ *    ranks' streams on both sides).  The sum's order is not fixed.
+ *  - Other arguments, shapes and errors as for vdn_hybrid_fuse_shard.
+ * Head-parallel runs were not possible here (one GPU); the single-GPU test
+ * runs G shards into G owner buffers on one device. */
+VDN_API vdn_status vdn_hybrid_fuse_shard_rs(int L, int D, int H_local, int d, int head0,
+                                            const void* x, const void* o_s, const void* o_vda,
+                                            int64_t ld_o, const void* W_gs, const void* W_gl,
+                                            const float* gamma, float eps, const void* W_os,
+                                            const void* W_ol, float* const* y_owners, int G,
+                                            void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Status and diagnostics.
  * ------------------------------------------------------------------------ */

@@ -102,3 +102,29 @@ def test_fuse_head_shards_sum_to_full(vdn, G):
     ref = _ref_rows(shape, inp, np.arange(shape.L))
     assert max_rel(host(acc), ref) <= TOL_BF16
     assert max_rel(host(acc), host(y_full)) <= TOL_BF16
+
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_fuse_shards_reduce_scatter_into_owners(vdn, G):
+    """The output GEMM fused with the reduce-scatter: G shards (each a
+    separate launch, as G ranks would run them) add their partials into G
+    owner buffers; the owners' row blocks, stacked, equal the full fuse.
+    No launch waits on another, so they may share one GPU."""
+    shape, inp = _inputs(2, 1000, 8, 128, seed=50 + G)
+    y_full = _fuse(vdn, shape, inp)
+    Hl = shape.H // G
+    R = -(-shape.L // G)
+    owners = [torch.zeros((min(R, shape.L - o * R), shape.D), dtype=torch.float32, device="cuda")
+              for o in range(G)]
+    for r in range(G):
+        c = slice(r * Hl * 128, (r + 1) * Hl * 128)
+        ws = vdn.hybrid_fuse_shard_rs(inp["x"], inp["o_s"][:, c].contiguous(),
+                                      inp["o_vda"][:, c].contiguous(), inp["W_gs"], inp["W_gl"],
+                                      inp["gamma"], inp["W_os"], inp["W_ol"], 128, r * Hl,
+                                      owners)
+        assert vdn.get_device_status(ws) == 0
+    y = torch.cat(owners, dim=0)
+    ref = _ref_rows(shape, inp, np.arange(shape.L))
+    assert max_rel(host(y), ref) <= TOL_BF16
+    assert max_rel(host(y), host(y_full)) <= TOL_BF16
+

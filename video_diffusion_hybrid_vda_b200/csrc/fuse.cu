@@ -57,6 +57,15 @@ struct StoreF32Args {
   float* y;  // [M, N] fp32 (partial sums of a head shard)
 };
 
+// GEMM fused with a reduce-scatter: row r of the fp32 partial is added into
+// owner[r / rows] at row r % rows (peer memory of the rank that owns the
+// row block), with system-scope atomics, so the partials of all shards
+// arrive summed in their owners' buffers without a separate collective.
+struct RedScatterArgs {
+  float* owner[8];
+  int rows;
+};
+
 __device__ __forceinline__ float sigmoidf_fast(float x) {
   float e;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-x * 1.4426950408889634f));
@@ -278,6 +287,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (r < M && n < N) {
           if constexpr (SPLIT == BSplit::kByN) {
             gate_chunk(args, r, n, acc, rinv, c == c0);
+          } else if constexpr (std::is_same<Args, RedScatterArgs>::value) {
+            const int o = static_cast<int>(r / args.rows);
+            float4* dst = reinterpret_cast<float4*>(
+                args.owner[o] + (r - static_cast<int64_t>(o) * args.rows) * N + n);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              atomicAdd_system(dst + e, make_float4(__uint_as_float(acc[4 * e]),
+                                                    __uint_as_float(acc[4 * e + 1]),
+                                                    __uint_as_float(acc[4 * e + 2]),
+                                                    __uint_as_float(acc[4 * e + 3])));
           } else if constexpr (sizeof(args.y[0]) == 4) {
             float4* dst = reinterpret_cast<float4*>(args.y + r * N + n);
 #pragma unroll
@@ -560,6 +579,58 @@ int sm_count_of_current_device() {
   return n > 0 ? n : 148;
 }
 
+// The head shard's fuse; Out is the output GEMM's epilogue (an fp32
+// partial, or the reduce-scatter into the owners' buffers).
+template <class Out>
+vdn_status fuse_shard_impl(int L, int D, int H_local, int d, int head0, const void* x,
+                           const void* o_s, const void* o_vda, int64_t ld_o, const void* W_gs,
+                           const void* W_gl, const float* gamma, float eps, const void* W_os,
+                           const void* W_ol, const Out& out, const void* out_ptr, void* ws,
+                           size_t ws_bytes, void* stream) {
+  const int64_t Dl = static_cast<int64_t>(H_local) * d;
+  if (L < 1 || D < 1 || H_local < 1 || d < 1 || head0 < 0) return VDN_ERR_INVALID_ARG;
+  if (D % d != 0 || static_cast<int64_t>(head0 + H_local) * d > D) return VDN_ERR_INVALID_ARG;
+  if (!x || !o_s || !o_vda || !W_gs || !W_gl || !gamma || !W_os || !W_ol || !out_ptr)
+    return VDN_ERR_INVALID_ARG;
+  if (!a16(x) || !a16(o_s) || !a16(o_vda) || !a16(W_gs) || !a16(W_gl) || !a16(W_os) ||
+      !a16(W_ol) || !a16(out_ptr) || (reinterpret_cast<uintptr_t>(gamma) & 3u))
+    return VDN_ERR_INVALID_ARG;
+  if (ld_o < Dl || ld_o % 8 || !(eps >= 0.f)) return VDN_ERR_INVALID_ARG;
+  // row-parallel fuse: full-D reduction for the gates, local head columns in
+  // Z, a partial y over the full output width
+  if (d % 128 != 0 || D % 256 != 0 || Dl % 128 != 0) return VDN_ERR_UNSUPPORTED;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
+      ws_bytes < vdn_hybrid_fuse_shard_workspace(L, D, H_local, d))
+    return VDN_ERR_WORKSPACE;
+  __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+  const int64_t c0 = static_cast<int64_t>(head0) * d;  // first local hidden column
+  const __nv_bfloat16* bgs = static_cast<const __nv_bfloat16*>(W_gs) + c0 * D;  // local rows
+  const __nv_bfloat16* bgl = static_cast<const __nv_bfloat16*>(W_gl) + c0 * D;
+  const __nv_bfloat16* bos = static_cast<const __nv_bfloat16*>(W_os) + c0;      // local columns
+  const __nv_bfloat16* bol = static_cast<const __nv_bfloat16*>(W_ol) + c0;
+  constexpr int BH = BN / 2;
+  CUtensorMap xmap, m_gs, m_gl, zmap, m_os, m_ol;
+  if (!make_rows_map(&xmap, x, D, D, L, BM) || !make_rows_map(&m_gs, bgs, D, D, Dl, BH) ||
+      !make_rows_map(&m_gl, bgl, D, D, Dl, BH) ||
+      !make_rows_map(&zmap, Z, 2 * Dl, 2 * Dl, L, BM) ||
+      !make_rows_map(&m_os, bos, Dl, D, D, BH) || !make_rows_map(&m_ol, bol, Dl, D, D, BH))
+    return VDN_ERR_CUDA;
+  // o_s / o_vda: local head columns with row stride ld_o
+  if (ld_o != Dl) return VDN_ERR_UNSUPPORTED;
+  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
+             current_wait_budget_ns()};
+  const int sms = sm_count_of_current_device();
+  GateArgs g{static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_vda),
+             gamma + c0, eps, static_cast<int>(Dl), d, 1.f / static_cast<float>(d), Z};
+  if (launch_gemm<BSplit::kByN>(ctx, xmap, m_gs, m_gl, L, static_cast<int>(2 * Dl), D,
+                                static_cast<int>(Dl), g, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  if (launch_gemm<BSplit::kByK>(ctx, zmap, m_os, m_ol, L, D, static_cast<int>(2 * Dl),
+                                static_cast<int>(Dl), out, sms) != cudaSuccess)
+    return VDN_ERR_CUDA;
+  return VDN_OK;
+}
+
 }  // namespace
 }  // namespace vdn
 
@@ -693,49 +764,26 @@ vdn_status vdn_hybrid_fuse_shard(int L, int D, int H_local, int d, int head0, co
                                  const void* W_os, const void* W_ol, float* y_partial, void* ws,
                                  size_t ws_bytes, void* stream) {
   NvtxRange nvtx("vdn_hybrid_fuse_shard");
-  const int64_t Dl = static_cast<int64_t>(H_local) * d;
-  if (L < 1 || D < 1 || H_local < 1 || d < 1 || head0 < 0) return VDN_ERR_INVALID_ARG;
-  if (D % d != 0 || static_cast<int64_t>(head0 + H_local) * d > D) return VDN_ERR_INVALID_ARG;
-  if (!x || !o_s || !o_vda || !W_gs || !W_gl || !gamma || !W_os || !W_ol || !y_partial)
-    return VDN_ERR_INVALID_ARG;
-  if (!a16(x) || !a16(o_s) || !a16(o_vda) || !a16(W_gs) || !a16(W_gl) || !a16(W_os) ||
-      !a16(W_ol) || !a16(y_partial) || (reinterpret_cast<uintptr_t>(gamma) & 3u))
-    return VDN_ERR_INVALID_ARG;
-  if (ld_o < Dl || ld_o % 8 || !(eps >= 0.f)) return VDN_ERR_INVALID_ARG;
-  // row-parallel fuse: full-D reduction for the gates, local head columns in
-  // Z, a partial y over the full output width
-  if (d % 128 != 0 || D % 256 != 0 || Dl % 128 != 0) return VDN_ERR_UNSUPPORTED;
-  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
-      ws_bytes < vdn_hybrid_fuse_shard_workspace(L, D, H_local, d))
-    return VDN_ERR_WORKSPACE;
-  __nv_bfloat16* Z = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(ws) + kStatusBytes);
-  const int64_t c0 = static_cast<int64_t>(head0) * d;  // first local hidden column
-  const __nv_bfloat16* bgs = static_cast<const __nv_bfloat16*>(W_gs) + c0 * D;  // local rows
-  const __nv_bfloat16* bgl = static_cast<const __nv_bfloat16*>(W_gl) + c0 * D;
-  const __nv_bfloat16* bos = static_cast<const __nv_bfloat16*>(W_os) + c0;      // local columns
-  const __nv_bfloat16* bol = static_cast<const __nv_bfloat16*>(W_ol) + c0;
-  constexpr int BH = BN / 2;
-  CUtensorMap xmap, m_gs, m_gl, zmap, m_os, m_ol;
-  if (!make_rows_map(&xmap, x, D, D, L, BM) || !make_rows_map(&m_gs, bgs, D, D, Dl, BH) ||
-      !make_rows_map(&m_gl, bgl, D, D, Dl, BH) ||
-      !make_rows_map(&zmap, Z, 2 * Dl, 2 * Dl, L, BM) ||
-      !make_rows_map(&m_os, bos, Dl, D, D, BH) || !make_rows_map(&m_ol, bol, Dl, D, D, BH))
-    return VDN_ERR_CUDA;
-  // o_s / o_vda: local head columns with row stride ld_o
-  if (ld_o != Dl) return VDN_ERR_UNSUPPORTED;
-  Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
-             current_wait_budget_ns()};
-  const int sms = sm_count_of_current_device();
-  GateArgs g{static_cast<const __nv_bfloat16*>(o_s), static_cast<const __nv_bfloat16*>(o_vda),
-             gamma + c0, eps, static_cast<int>(Dl), d, 1.f / static_cast<float>(d), Z};
-  if (launch_gemm<BSplit::kByN>(ctx, xmap, m_gs, m_gl, L, static_cast<int>(2 * Dl), D,
-                                static_cast<int>(Dl), g, sms) != cudaSuccess)
-    return VDN_ERR_CUDA;
-  StoreF32Args so{y_partial};
-  if (launch_gemm<BSplit::kByK>(ctx, zmap, m_os, m_ol, L, D, static_cast<int>(2 * Dl),
-                                static_cast<int>(Dl), so, sms) != cudaSuccess)
-    return VDN_ERR_CUDA;
-  return VDN_OK;
+  return fuse_shard_impl(L, D, H_local, d, head0, x, o_s, o_vda, ld_o, W_gs, W_gl, gamma, eps,
+                         W_os, W_ol, StoreF32Args{y_partial}, y_partial, ws, ws_bytes, stream);
+}
+
+vdn_status vdn_hybrid_fuse_shard_rs(int L, int D, int H_local, int d, int head0, const void* x,
+                                    const void* o_s, const void* o_vda, int64_t ld_o,
+                                    const void* W_gs, const void* W_gl, const float* gamma,
+                                    float eps, const void* W_os, const void* W_ol,
+                                    float* const* y_owners, int G, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  NvtxRange nvtx("vdn_hybrid_fuse_shard_rs");
+  if (y_owners == nullptr || G < 1 || G > 8 || L < 1) return VDN_ERR_INVALID_ARG;
+  RedScatterArgs out{};
+  for (int o = 0; o < G; ++o) {
+    if (y_owners[o] == nullptr || !a16(y_owners[o])) return VDN_ERR_INVALID_ARG;
+    out.owner[o] = y_owners[o];
+  }
+  out.rows = (L + G - 1) / G;
+  return fuse_shard_impl(L, D, H_local, d, head0, x, o_s, o_vda, ld_o, W_gs, W_gl, gamma, eps,
+                         W_os, W_ol, out, y_owners[0], ws, ws_bytes, stream);
 }
 
 // ----------------------------------------------------------------- MXFP8

@@ -28,7 +28,8 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_set_vda_solver", "vdn_hybrid_fuse_shard_workspace", "vdn_hybrid_fuse_shard",
            "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers",
            "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
-           "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8"]
+           "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8",
+           "vdn_hybrid_fuse_shard_rs"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -97,6 +98,11 @@ def lib():
     L.vdn_hybrid_fuse_shard.argtypes = [ctypes.c_int] * 5 + [_P, _P, _P, _I64, _P, _P, _P,
                                                              ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
     L.vdn_hybrid_fuse_shard.restype = ctypes.c_int
+    L.vdn_hybrid_fuse_shard_rs.argtypes = [ctypes.c_int] * 5 + [_P, _P, _P, _I64, _P, _P, _P,
+                                                                ctypes.c_float, _P, _P,
+                                                                ctypes.POINTER(_P), ctypes.c_int,
+                                                                _P, _SZ, _P]
+    L.vdn_hybrid_fuse_shard_rs.restype = ctypes.c_int
     L.vdn_set_vda_solver.argtypes = [ctypes.c_int]
     L.vdn_set_vda_solver.restype = ctypes.c_int
     L.vdn_vda_backward_workspace.argtypes = [S]
@@ -417,6 +423,28 @@ def hybrid_fuse_shard(x, o_s_local, o_vda_local, W_gs, W_gl, gamma, W_os, W_ol, 
                                        ws.numel(), _stream(stream))
     _check(code, "vdn_hybrid_fuse_shard")
     return out, ws
+
+
+def hybrid_fuse_shard_rs(x, o_s_local, o_vda_local, W_gs, W_gl, gamma, W_os, W_ol, d, head0,
+                         owners, eps=1e-6, ws=None, stream=None):
+    """This head shard's contribution to y, added straight into the owners'
+    row blocks (the GEMM fused with the reduce-scatter).  ``owners``: the G
+    fp32 buffers [ceil(L/G), D] (the last may be shorter), zeroed beforehand;
+    device pointers valid on this GPU (local, or peer-mapped)."""
+    _need_cuda(x, o_s_local, o_vda_local, W_gs, W_gl, gamma, W_os, W_ol, ws, *owners)
+    L, D = x.shape
+    H_local = o_s_local.shape[1] // d
+    if ws is None:
+        ws = alloc_workspace(int(lib().vdn_hybrid_fuse_shard_workspace(L, D, H_local, d)),
+                             x.device)
+    ptrs = (_P * len(owners))(*[t.data_ptr() for t in owners])
+    code = lib().vdn_hybrid_fuse_shard_rs(int(L), int(D), int(H_local), int(d), int(head0),
+                                          _ptr(x), _ptr(o_s_local), _ptr(o_vda_local),
+                                          o_s_local.stride(0), _ptr(W_gs), _ptr(W_gl),
+                                          _ptr(gamma), float(eps), _ptr(W_os), _ptr(W_ol), ptrs,
+                                          len(owners), _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "vdn_hybrid_fuse_shard_rs")
+    return ws
 
 
 # ---------------------------------------------------------------- full layer
