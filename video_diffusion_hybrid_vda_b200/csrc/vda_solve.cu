@@ -155,16 +155,25 @@ __global__ void __launch_bounds__(kThreads, 2)
           bad = true;
           piv = 1.f;
         }
-        const float f = (j > c) ? dc[c] * __frcp_rn(piv) : 0.f;  // D[c][j] / D[c][c]
-        const float sq = sqrtf(piv);
-        const float is = __frcp_rn(sq);
+        // rsqrt and products (not the correctly rounded sqrt and reciprocal,
+        // whose longer sequences sit on this serial chain); the pivot column
+        // goes to the other lanes through shared memory in one burst
+        const float is = rsqrtf(piv);                         // 1 / L[c][c]
+        const float f = (j > c) ? dc[c] * (is * is) : 0.f;  // D[c][j] / D[c][c]
+        const float sq = piv * is;                            // L[c][c]
+        float* colc = Pan + (16 * p) * LDP;  // 16 floats; panel rows 16p.. are free
+        if (threadIdx.x == c)
+#pragma unroll
+          for (int r = 0; r < 16; ++r) colc[r] = dc[r];
+        __syncwarp();
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
           if (r > c) {
-            const float v = __shfl_sync(0xffffffffu, dc[r], c);  // D[r][c]
+            const float v = colc[r];  // D[r][c]
             dc[r] = (j == c) ? dc[r] * is : fmaf(-v, f, dc[r]);
           }
         }
+        __syncwarp();  // every lane has read the column before the next pivot's
         if (j == c) dc[c] = sq;
         if (threadIdx.x == c) idg[c] = is;
       }
