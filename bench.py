@@ -346,9 +346,35 @@ def run_vda_backward(args, shape, rank, world):
     if vdn.get_device_status(ws) != 0:
         raise RuntimeError("device status after the timed gradient passes")
     ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
-    del inp, d_o, outs, ws
+
+    # the same pass taking P and the states from a forward run on its workspace
+    o_vda = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
+    vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d, out=o_vda,
+                 ws=ws, stream=stream)
+
+    def step_saved():
+        vdn.vda_backward(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], d_o, T, N, H,
+                         d, dq=outs[0], dk=outs[1], dv=outs[2], dbeta=dbeta, dalpha=dalpha,
+                         ws=ws, stream=stream, reuse_forward=True)
+
+    for _ in range(args.warmup):
+        step_saved()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step_saved()
+    e1.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the gradient passes on a saved forward")
+    ms_saved = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    del inp, d_o, outs, ws, o_vda
     torch.cuda.empty_cache()
-    return ms
+    return ms, ms_saved
 
 
 def run_fuse_mxfp8(args, shape, rank, world):
@@ -405,12 +431,15 @@ def mxfp8_row(work, peaks, ms, dev_rel):
             "max_rel_vs_bf16_fuse": dev_rel, "launches_per_call": 3}
 
 
-def backward_row(work, peaks, ms):
+def backward_row(work, peaks, ms, ms_saved):
     roof_ms = (work["vda_bwd_bytes"] / (peaks["hbm_gbs"] * 1e9) +
                work["vda_bwd_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3
     return {"ms": ms, "bound": "hbm + fp32 alu", "roofline_ms": roof_ms, "frac": roof_ms / ms,
             "hbm_bytes": work["vda_bwd_bytes"], "fp32_alu_flop": work["vda_bwd_alu_flop"],
-            "launches_per_pass": 9}
+            "launches_per_pass": 9,
+            "ms_saved_forward": ms_saved, "launches_saved_forward": 6,
+            "note": "ms: forward recomputed inside; ms_saved_forward: P and states taken "
+                    "from a forward run on the same workspace"}
 
 
 def main():
@@ -468,13 +497,13 @@ def main():
             timeout=__import__("datetime").timedelta(seconds=300))
     peaks, peak_kind = load_peaks()
     if args.part == "vda_backward":
-        ms = run_vda_backward(args, shape, rank, world)
+        ms, ms_saved = run_vda_backward(args, shape, rank, world)
         if rank == 0:
             print(json.dumps({"metric": "VDA gradient pass ms (dq, dk, dv, dbeta, dalpha)",
                               "value": ms, "unit": "ms", "higher_is_better": False,
                               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                               "dtype": "bf16", "data": "synthetic", "config": config,
-                              "vda_backward": backward_row(work, peaks, ms)}))
+                              "vda_backward": backward_row(work, peaks, ms, ms_saved)}))
         if world > 1:
             torch.distributed.destroy_process_group()
         return
@@ -541,7 +570,7 @@ def main():
     }
     if args.part == "all":
         line["vda_backward"] = backward_row(work, peaks,
-                                            run_vda_backward(args, shape, rank, world))
+                                            *run_vda_backward(args, shape, rank, world))
         line["fuse_mxfp8"] = mxfp8_row(work, peaks, *run_fuse_mxfp8(args, shape, rank, world))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(shape)

@@ -159,9 +159,16 @@ VDN_API vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q, co
  * dq, dk, dv: [L, ld_g] bf16, outputs (columns past H*d are not written)
  * dbeta     : [L, H] fp32 output;  dalpha: [T, H] fp32 output
  * ws        : >= vdn_vda_backward_workspace(shape) bytes.
- * The call recomputes the forward's A, B, P, C and states in its workspace
- * (about half of its time at d = 128), so it needs nothing kept from the
- * forward call.  Errors as for vdn_vda_scan.
+ * reuse_forward: 0 -> the call recomputes the forward's A, B, P and states
+ *             in its workspace (about a third of its time at d = 128) and
+ *             needs nothing kept from the forward call.  Non-zero -> ws
+ *             already holds them: the last vdn_vda_scan on this same
+ *             workspace ran on the same q, k, v, beta, alpha with
+ *             states_opt == NULL (a forward workspace is a prefix of a
+ *             gradient-pass workspace, so one allocation of the larger size
+ *             serves both), and prep, solve and scan are skipped.  Stale
+ *             contents give wrong gradients; nothing checks this.
+ * Errors as for vdn_vda_scan.
  * ------------------------------------------------------------------------ */
 VDN_API size_t vdn_vda_backward_workspace(const vdn_shape* shape);
 
@@ -169,7 +176,7 @@ VDN_API vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const
                                     const void* v, int64_t ld, const float* beta,
                                     const float* alpha, const void* d_o, int64_t ld_do, void* dq,
                                     void* dk, void* dv, int64_t ld_g, float* dbeta, float* dalpha,
-                                    void* ws, size_t ws_bytes, void* stream);
+                                    int reuse_forward, void* ws, size_t ws_bytes, void* stream);
 
 /* Pointers into a backward workspace, after vdn_vda_backward on it, to fp32
  * [2, T, H, d, d] arrays: states ([0] = S_fwd, [1] = S_bwd), adjoint

@@ -166,3 +166,20 @@ def test_vda_backward_rejects_bad_arguments(vdn):
     with pytest.raises(vdn.VdnError):
         vdn.vda_backward(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], inp["d_o"],
                          2, 16, 1, 128, ws=vdn.alloc_workspace(1024))
+
+
+@pytest.mark.parametrize("T,N,H,d", [(7, 200, 2, 128), (9, 70, 2, 32)])
+def test_vda_backward_reuses_a_forward_on_its_workspace(vdn, T, N, H, d):
+    """A forward run on the gradient pass's workspace (states kept inside)
+    hands P and the states over: the gradients equal those of the
+    recomputing pass bit for bit."""
+    shape = synth.Shape(T, N, H, d)
+    inp = _inputs(shape, seed=T + N)
+    ref = _run(vdn, shape, inp)[:5]
+    ws = vdn.alloc_workspace(vdn.vda_backward_workspace(T, N, H, d))
+    o, _ = vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
+                        ws=ws)
+    got = _run(vdn, shape, inp, ws=ws, reuse_forward=True)[:5]
+    for g, r in zip(got, ref):
+        assert torch.equal(g, r)
+

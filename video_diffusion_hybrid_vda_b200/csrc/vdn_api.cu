@@ -56,11 +56,11 @@ bool head_dim_padded(int d) { return d == 16 || d == 32; }
 
 bool ld_ok(int64_t ld, int64_t D) { return ld >= D && ld % 8 == 0; }
 
-// VDA workspace: [status 256 B][A][B][P]([X])[states (2x)], each region
+// VDA workspace: [status 256 B][A][B][P][states (2x)]([X]), each region
 // 256-byte aligned, every matrix fp32 [T, H, d, d]; the gradient pass adds
-// the slot X (for G, then E).
+// the slot X (for G, then E) at the end.
 struct VdaLayout {
-  size_t mat_bytes, A, B, P, X, states, total;
+  size_t mat_bytes, A, B, P, states, X, total;
 };
 
 VdaLayout vda_layout(const vdn_shape& s, bool with_x) {
@@ -69,35 +69,37 @@ VdaLayout vda_layout(const vdn_shape& s, bool with_x) {
   l.A = kStatusBytes;
   l.B = l.A + l.mat_bytes;
   l.P = l.B + l.mat_bytes;
-  l.X = l.P + l.mat_bytes;
-  l.states = l.X + (with_x ? l.mat_bytes : 0);
-  l.total = l.states + 2 * l.mat_bytes;
+  l.states = l.P + l.mat_bytes;
+  l.X = l.states + 2 * l.mat_bytes;
+  l.total = l.X + (with_x ? l.mat_bytes : 0);
   return l;
 }
 
 // Workspace of a VDA call.  Head dims 16 and 32 run through a 64-wide padded
-// copy: [status][nact padded activations, bf16 L x H*64][the layout above
-// for d = 64]; the forward pads q' k' v' o' (4), the gradient pass q' k' v'
-// dO' dq' dk' dv' (7).
+// copy: [status][q' k' v' o' bf16 L x H*64][the layout above for d = 64]
+// and, for the gradient pass, [dq' dk' dv'] after it (o' holds dO' there).
+// The forward's workspace is therefore a prefix of the gradient pass's, so
+// one workspace can carry the forward's P and states into the gradient pass.
 struct VdaPlan {
   bool padded;
   vdn_shape inner;  // shape the kernels run on
   size_t act;       // bytes of one padded activation
   size_t inner_off; // where the d = 64 layout (after its status word) starts
   VdaLayout lay;    // layout of the inner shape
+  size_t extra;     // gradient pass: dq' dk' dv'
   size_t total;
 };
 
 VdaPlan vda_plan(const vdn_shape& s, bool backward = false) {
-  const int nact = backward ? 7 : 4;
   VdaPlan p;
   p.padded = head_dim_padded(s.d);
   p.inner = s;
   if (p.padded) p.inner.d = 64;
   p.lay = vda_layout(p.inner, backward);
   p.act = p.padded ? round_up(static_cast<size_t>(s.T) * s.N * s.H * 64 * 2, 256) : 0;
-  p.inner_off = nact * p.act;
-  p.total = p.lay.total + p.inner_off;
+  p.inner_off = 4 * p.act;
+  p.extra = p.inner_off + p.lay.total;
+  p.total = p.extra + (backward ? 3 * p.act : 0);
   return p;
 }
 
@@ -130,7 +132,7 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
                             const void* v, int64_t ld, const float* beta, const float* alpha,
                             const void* d_o, int64_t ld_do, void* dq, void* dk, void* dv,
                             int64_t ld_g, float* dbeta, float* dalpha, float* A, float* B,
-                            float* P, float* X, float* states) {
+                            float* P, float* X, float* states, bool reuse_forward) {
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   const int prep_rows = s.d == 128 ? 32 : 64;
   CUtensorMap kmap_p, vmap_p, qmap_p, domap_p, domap, dqmap, kmap, vmap, dvmap, dkmap;
@@ -148,10 +150,12 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
   float* G = X;
   float* adj = A;
   float* E = X;
-  if (launch_vda_prep(ctx, s, kmap_p, vmap_p, beta, A, B) != cudaSuccess ||
-      launch_vda_solve(ctx, s, A, P) != cudaSuccess ||
-      launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess ||
-      launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
+  if (!reuse_forward &&
+      (launch_vda_prep(ctx, s, kmap_p, vmap_p, beta, A, B) != cudaSuccess ||
+       launch_vda_solve(ctx, s, A, P) != cudaSuccess ||
+       launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess))
+    return VDN_ERR_CUDA;
+  if (launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
       launch_vda_adjoint_scan(ctx, s, P, G, alpha, adj) != cudaSuccess ||
       launch_vda_grad_combine(ctx, s, states, adj, E, dalpha) != cudaSuccess ||
       launch_vda_readout_ex(ctx, s, domap, dqmap, states, true, nullptr) != cudaSuccess ||
@@ -351,8 +355,8 @@ vdn_status vdn_vda_backward_debug_buffers(const vdn_shape* shape, void* ws, floa
 vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k, const void* v,
                             int64_t ld, const float* beta, const float* alpha, const void* d_o,
                             int64_t ld_do, void* dq, void* dk, void* dv, int64_t ld_g,
-                            float* dbeta, float* dalpha, void* ws, size_t ws_bytes,
-                            void* stream) {
+                            float* dbeta, float* dalpha, int reuse_forward, void* ws,
+                            size_t ws_bytes, void* stream) {
   NvtxRange nvtx("vdn_vda_backward");
   if (!shape_ok(shape)) return VDN_ERR_INVALID_ARG;
   const vdn_shape s = *shape;
@@ -381,22 +385,24 @@ vdn_status vdn_vda_backward(const vdn_shape* shape, const void* q, const void* k
              g_budget_ns.load()};
   if (!pl.padded)
     return run_vda_backward(ctx, s, q, k, v, ld, beta, alpha, d_o, ld_do, dq, dk, dv, ld_g,
-                            dbeta, dalpha, A, B, P, X, states);
+                            dbeta, dalpha, A, B, P, X, states, reuse_forward != 0);
 
   // d = 16 or 32: every head zero-padded to 64 columns (exact, see repack.cu)
   const int L = s.T * s.N, H = s.H, d = s.d;
   const int64_t D64 = static_cast<int64_t>(H) * 64;
+  // q' k' v' dO' (the forward's slots; o' takes dO'), then dq' dk' dv'
   uint8_t* pad[7];
-  for (int i = 0; i < 7; ++i) pad[i] = base + kStatusBytes + i * pl.act;
+  for (int i = 0; i < 4; ++i) pad[i] = base + kStatusBytes + i * pl.act;
+  for (int i = 0; i < 3; ++i) pad[4 + i] = base + pl.extra + i * pl.act;
   const void* src[4] = {q, k, v, d_o};
   const int64_t lds[4] = {ld, ld, ld, ld_do};
   cudaStream_t st = ctx.stream;
-  for (int i = 0; i < 4; ++i)
+  for (int i = reuse_forward ? 3 : 0; i < 4; ++i)  // a reused forward left q' k' v' in place
     if (launch_repack_bf16(st, pad[i], D64, src[i], lds[i], 1, L, L, H, 64, d) != cudaSuccess)
       return VDN_ERR_CUDA;
   const vdn_status r = run_vda_backward(ctx, pl.inner, pad[0], pad[1], pad[2], D64, beta, alpha,
                                         pad[3], D64, pad[4], pad[5], pad[6], D64, dbeta, dalpha,
-                                        A, B, P, X, states);
+                                        A, B, P, X, states, reuse_forward != 0);
   if (r != VDN_OK) return r;
   void* dst[3] = {dq, dk, dv};
   for (int i = 0; i < 3; ++i)

@@ -108,7 +108,7 @@ def lib():
     L.vdn_vda_backward_workspace.argtypes = [S]
     L.vdn_vda_backward_workspace.restype = _SZ
     L.vdn_vda_backward.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _P, _I64, _P,
-                                   _P, _P, _SZ, _P]
+                                   _P, ctypes.c_int, _P, _SZ, _P]
     L.vdn_vda_backward.restype = ctypes.c_int
     L.vdn_vda_backward_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 3
     L.vdn_vda_backward_debug_buffers.restype = ctypes.c_int
@@ -244,10 +244,13 @@ def vda_backward_workspace(T, N, H, d):
 
 
 def vda_backward(q, k, v, beta, alpha, d_o, T, N, H, d, dq=None, dk=None, dv=None, dbeta=None,
-                 dalpha=None, ws=None, stream=None):
+                 dalpha=None, ws=None, stream=None, reuse_forward=False):
     """Gradients of o_vda with respect to q, k, v, beta and alpha, given
     d_o = dLoss/do_vda ([T*N, ld] bf16).  Returns (dq, dk, dv, dbeta, dalpha, ws):
-    dq/dk/dv bf16 [T*N, H*d], dbeta fp32 [T*N, H], dalpha fp32 [T, H]."""
+    dq/dk/dv bf16 [T*N, H*d], dbeta fp32 [T*N, H], dalpha fp32 [T, H].
+    reuse_forward: ``ws`` (of vda_backward_workspace size) last served a
+    vda_scan on the same inputs without ``states``; its P and states are
+    used instead of recomputing them."""
     _need_cuda(q, k, v, beta, alpha, d_o, dq, dk, dv, dbeta, dalpha, ws)
     shape = _shape(T, N, H, d)
     dev = q.device
@@ -264,7 +267,8 @@ def vda_backward(q, k, v, beta, alpha, d_o, T, N, H, d, dq=None, dk=None, dv=Non
     code = lib().vdn_vda_backward(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
                                   _ptr(beta), _ptr(alpha), _ptr(d_o), d_o.stride(0), _ptr(dq),
                                   _ptr(dk), _ptr(dv), dq.stride(0), _ptr(dbeta), _ptr(dalpha),
-                                  _ptr(ws), ws.numel(), _stream(stream))
+                                  int(bool(reuse_forward)), _ptr(ws), ws.numel(),
+                                  _stream(stream))
     _check(code, "vdn_vda_backward")
     return dq, dk, dv, dbeta, dalpha, ws
 
