@@ -72,9 +72,10 @@ def work_model(s):
     proj_flop = 4 * 2 * s.L * s.D * s.D                 # gate GEMMs + output GEMMs
     # VDA HBM bytes: prep reads k, v (bf16) and beta; read-out reads q, writes o
     vda_bytes = 2 * s.L * s.D * 2 + s.L * s.H * 4 + 2 * s.L * s.D * 2
-    # FP32 ALU work in FLOP per (frame, head): Cholesky d^3/3, W = L^-1 d^3/3,
-    # P = W^T W and C = B P 2 d^3 each, and both scans a 2 d^3 product each
-    vda_alu_flop = s.T * s.H * (2 * s.d ** 3 // 3 + 4 * s.d ** 3 + 4 * s.d ** 3)
+    # FP32 ALU work in FLOP per (frame, head): the SPD inverse (Cholesky,
+    # W = L^-1 and the triangular product P = W^T W, d^3 / 3 each) and both
+    # scans' (alpha S + B) P, a 2 d^3 product each
+    vda_alu_flop = s.T * s.H * (s.d ** 3 + 4 * s.d ** 3)
     # VDA gradient pass: reads q, k, v, dO (bf16) and beta, writes dq, dk, dv
     # (bf16) and dbeta; FP32 ALU: the forward's solve and scans again, the
     # two adjoint scans (2 d^3 each) and the combine (two d^3 products, 4 d^3)
