@@ -28,13 +28,13 @@ namespace {
 
 constexpr int kThreads = 256;  // 16 row groups x 16 column groups
 
+// Gauss-Jordan: the matrix in registers (rows ty + 16 a, columns tx + 16 b),
+// the published pivot row and column double-buffered in shared memory.
 template <int DH>
 struct SolveCfg {
   static constexpr int RA = DH / 16;   // rows per thread (rows ty + 16 a)
   static constexpr int CB = DH / 16;   // columns per thread (cols tx + 16 b)
-  static constexpr int LD2 = DH + 4;   // row stride of the matrix buffer (float4 rows)
-  static constexpr int MAT = DH * LD2; // floats of the matrix buffer
-  static constexpr int SMEM = MAT * 4 + 4 * DH * 4;
+  static constexpr int SMEM = 4 * DH * 4;
 };
 
 // Load (I + A_sym) into the register tile m (rows ty + 16 a, cols tx + 16 b).
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     vda_solve_gj_kernel(const float* __restrict__ A, float* __restrict__ P, uint32_t* status) {
   using Cfg = SolveCfg<DH>;
   extern __shared__ float sm[];
-  float* rowb = sm + Cfg::MAT;   // 2 x [DH] pivot rows
+  float* rowb = sm;              // 2 x [DH] pivot rows
   float* colb = rowb + 2 * DH;   // 2 x [DH] pivot columns
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
