@@ -17,3 +17,24 @@ def pytest_configure(config):
 def has_gpu():
     import torch
     return torch.cuda.is_available()
+
+
+# Metrics a test reports beside its pass/fail criterion (for example the
+# elementwise relative error of an output), printed at the end of the run.
+_REPORTED = {}
+
+
+@pytest.fixture
+def report_metric():
+    def record(name, value):
+        _REPORTED.setdefault(name, []).append(float(value))
+    return record
+
+
+def pytest_terminal_summary(terminalreporter):
+    if not _REPORTED:
+        return
+    terminalreporter.section("reported metrics (max over the cases that report them)")
+    for name, values in sorted(_REPORTED.items()):
+        terminalreporter.write_line("%s: max %.3e over %d cases" % (name, max(values), len(values)))
+

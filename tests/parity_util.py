@@ -16,6 +16,16 @@ def max_rel(gpu, ref):
     return float(np.abs(gpu - ref).max() / (scale if scale > 0 else 1.0))
 
 
+def elementwise_rel(gpu, ref, floor=1e-3):
+    """Largest elementwise relative error, each element's denominator floored
+    at floor * max|ref| (reported beside the max-relative metric)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    den = np.maximum(np.abs(ref), floor * np.abs(ref).max())
+    den = np.where(den > 0, den, 1.0)
+    return float((np.abs(gpu - ref) / den).max())
+
+
 def per_head_max_rel(gpu, ref, H, d):
     return max(max_rel(gpu[:, h * d:(h + 1) * d], ref[:, h * d:(h + 1) * d]) for h in range(H))
 

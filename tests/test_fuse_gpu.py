@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import oracle
-from tests.parity_util import TOL_BF16, ensure_built, host, max_rel
+from tests.parity_util import TOL_BF16, elementwise_rel, ensure_built, host, max_rel
 from video_diffusion_hybrid_vda_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -50,11 +50,12 @@ def _ref_rows(shape, inp, rows, eps=1e-6):
 
 @pytest.mark.parametrize("T,N,H,d", [(3, 100, 2, 128), (5, 200, 8, 64), (2, 640, 4, 128),
                                      (1, 7, 4, 64)])
-def test_fuse_parity_small(vdn, T, N, H, d):
+def test_fuse_parity_small(vdn, T, N, H, d, report_metric):
     shape, inp = _inputs(T, N, H, d, seed=T + N)
     y = _fuse(vdn, shape, inp)
     ref = _ref_rows(shape, inp, np.arange(shape.L))
     assert max_rel(host(y), ref) <= TOL_BF16
+    report_metric("y_elementwise_rel", elementwise_rel(host(y), ref))
 
 
 def test_fuse_zero_gate_weights(vdn):

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from tests.parity_util import TOL_BF16, ensure_built, host, max_rel, per_head_max_rel
+from tests.parity_util import elementwise_rel, TOL_BF16, ensure_built, host, max_rel, per_head_max_rel
 from video_diffusion_hybrid_vda_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -45,7 +45,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("T,N,H,d", SMALL)
-def test_window_attn_parity_small(vdn, T, N, H, d):
+def test_window_attn_parity_small(vdn, T, N, H, d, report_metric):
     shape = synth.Shape(T, N, H, d)
     inp = synth.make_inputs(shape, seed=T * 100 + N, device="cuda")
     o, lse = _run(vdn, shape, inp)
@@ -53,6 +53,7 @@ def test_window_attn_parity_small(vdn, T, N, H, d):
     o_ref, lse_ref = oracle.window_attn(x["q"], x["k"], x["v"], T, N, H, d)
     assert per_head_max_rel(host(o), o_ref, H, d) <= TOL_BF16
     assert np.abs(host(lse) - lse_ref).max() <= TOL_LSE
+    report_metric("o_s_elementwise_rel", elementwise_rel(host(o), o_ref))
 
 
 @pytest.mark.parametrize("cf,wc,anchors,scale", [
