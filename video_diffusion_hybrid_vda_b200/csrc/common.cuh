@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include <nvtx3/nvToolsExt.h>
 
 #include "../../include/vdn.h"
@@ -36,6 +38,21 @@ struct Launch {
   uint32_t* status;     // device status word
   uint64_t budget_ns;   // bounded-wait budget
 };
+
+// Opt a kernel into `bytes` of dynamic shared memory on the current device,
+// once per device (the attribute is per device; `done` is the kernel's own
+// bit set of devices already done, safe under concurrent callers).
+template <class Kernel>
+cudaError_t set_smem_once(Kernel* kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Budget (ns) of the bounded device waits, set by vdn_set_wait_budget_ns.
 uint64_t current_wait_budget_ns();

@@ -330,13 +330,8 @@ template <BSplit SPLIT, class Args>
 cudaError_t launch_gemm(const Launch& ctx, const CUtensorMap& a, const CUtensorMap& b0,
                         const CUtensorMap& b1, int M, int N, int K, int split_at, const Args& args,
                         int sm_count) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<SPLIT, Args>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(gemm_kernel<SPLIT, Args>, GEMM_SMEM, smem_set)) return e;
   const int ntiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = ntiles < sm_count ? ntiles : sm_count;
   gemm_kernel<SPLIT, Args><<<grid, GEMM_THREADS, GEMM_SMEM, ctx.stream>>>(
@@ -556,13 +551,8 @@ template <class Args>
 cudaError_t launch_gemm_mx(const Launch& ctx, const CUtensorMap& a, const CUtensorMap& b,
                            const uint8_t* a_sf, const uint8_t* b_sf, int M, int N, int K,
                            const Args& args, int sm_count) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_mx_kernel<Args>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, MX_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(gemm_mx_kernel<Args>, MX_SMEM, smem_set)) return e;
   const int ntiles = ((M + MX_BM - 1) / MX_BM) * ((N + MX_BN - 1) / MX_BN);
   const int grid = ntiles < sm_count ? ntiles : sm_count;
   gemm_mx_kernel<Args><<<grid, GEMM_THREADS, MX_SMEM, ctx.stream>>>(

@@ -382,13 +382,8 @@ template <int DH>
 cudaError_t launch_combine_dh(const Launch& ctx, const vdn_shape& s, const float* states,
                               const float* adj, float* E, float* dalpha) {
   using Cfg = CombineCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_grad_combine_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_grad_combine_kernel<DH>, Cfg::SMEM, smem_set)) return e;
   vda_grad_combine_kernel<DH><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       states, adj, E, dalpha, s.T, s.H);
   return cudaGetLastError();
@@ -399,13 +394,8 @@ cudaError_t launch_grad_k_dh(const Launch& ctx, const vdn_shape& s, const CUtens
                              const CUtensorMap& vmap, const CUtensorMap& dkmap, const float* E,
                              const float* adj, const float* beta, float* dbeta) {
   using Cfg = GradKCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_grad_k_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_grad_k_kernel<DH>, Cfg::SMEM, smem_set)) return e;
   vda_grad_k_kernel<DH><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       kmap, vmap, dkmap, E, adj, beta, dbeta, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();

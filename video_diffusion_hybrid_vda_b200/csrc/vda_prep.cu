@@ -268,13 +268,8 @@ template <int DH, bool kGram>
 cudaError_t launch_prep_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const float* beta, float* A, float* B) {
   using C = PrepCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_prep_kernel<DH, kGram>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_prep_kernel<DH, kGram>, C::SMEM, smem_set)) return e;
   const int grid = s.T * s.H;
   vda_prep_kernel<DH, kGram><<<grid, C::THREADS, C::SMEM, ctx.stream>>>(
       kmap, vmap, beta, A, B, s.T, s.N, s.H, ctx.status, ctx.budget_ns);

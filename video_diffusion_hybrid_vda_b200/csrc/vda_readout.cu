@@ -225,13 +225,8 @@ cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUten
                               const CUtensorMap& omap, const float* states,
                               const float* row_scale) {
   using Cfg = ReadoutCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_readout_kernel<DH, kTransS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_readout_kernel<DH, kTransS>, Cfg::SMEM, smem_set)) return e;
   vda_readout_kernel<DH, kTransS><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       qmap, omap, states, row_scale, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();

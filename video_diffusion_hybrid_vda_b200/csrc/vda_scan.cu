@@ -226,13 +226,8 @@ template <int DH, bool kAdjoint>
 cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* X,
                            const float* alpha, float* states) {
   using Cfg = ScanCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_scan_kernel<DH, kAdjoint>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_scan_kernel<DH, kAdjoint>, Cfg::SMEM, smem_set)) return e;
   dim3 grid(DH / kRows, s.H, 2);
   vda_scan_kernel<DH, kAdjoint><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       P, X, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);

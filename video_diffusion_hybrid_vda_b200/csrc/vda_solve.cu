@@ -382,17 +382,10 @@ template <int DH>
 cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* A, float* P,
                             int solver) {
   using Cfg = SolveCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(vda_solve_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         CholCfg<DH>::SMEM);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(vda_solve_gj_kernel<DH>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> chol_set{0};
+  if (cudaError_t e = set_smem_once(vda_solve_kernel<DH>, CholCfg<DH>::SMEM, chol_set)) return e;
+  static std::atomic<uint64_t> gj_set{0};
+  if (cudaError_t e = set_smem_once(vda_solve_gj_kernel<DH>, Cfg::SMEM, gj_set)) return e;
   if (solver == VDN_SOLVER_GAUSS_JORDAN)
     vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
   else

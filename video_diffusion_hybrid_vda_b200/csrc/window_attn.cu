@@ -561,13 +561,8 @@ cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtens
                              const WinSched& sched, float scale, void* o, int64_t ld_o,
                              float* lse) {
   using Cfg = WinCfg<DH>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(window_attn_kernel<DH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(window_attn_kernel<DH>, Cfg::SMEM, smem_set)) return e;
   const int grid = sched.total_tiles * s.H;
   window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       qmap, kmap, vmap, ckmap, cvmap, m_ctx, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
