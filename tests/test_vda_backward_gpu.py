@@ -72,6 +72,7 @@ SMALL = [
     (17, 33, 2, 64),
     (9, 70, 2, 32),     # padded head dims
     (6, 50, 3, 16),
+    (3, 40, 26, 128),   # many heads: the adjoint scan's 64-row blocks
 ]
 
 

@@ -62,6 +62,8 @@ SMALL = [
     (4, 1, 2, 128),
     (3, 4032, 1, 128),  # the full 48x84 frame, several tiles per frame
     (17, 33, 2, 64),
+    (3, 40, 26, 128),   # 156 CTAs of 48-row blocks would not fit 148 SMs: 64-row blocks
+    (3, 20, 40, 64),    # likewise at d = 64 (one 64-row block per state)
 ]
 
 

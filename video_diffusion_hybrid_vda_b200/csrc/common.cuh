@@ -39,6 +39,14 @@ struct Launch {
   uint64_t budget_ns;   // bounded-wait budget
 };
 
+// SMs of the current device (148 on a B200; that figure if the query fails).
+inline int sm_count_of_current_device() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
 // Opt a kernel into `bytes` of dynamic shared memory on the current device,
 // once per device (the attribute is per device; `done` is the kernel's own
 // bit set of devices already done, safe under concurrent callers).

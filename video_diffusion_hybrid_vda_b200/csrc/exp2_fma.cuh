@@ -43,6 +43,14 @@ __device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// max(a, b, c) as one instruction (the three-input form of sm_100); like
+// fmaxf, a NaN operand is ignored when another operand is a number.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // MUFU exponential (hardware ex2.approx).
 __device__ __forceinline__ float exp2_mufu(float x) {
   float y;

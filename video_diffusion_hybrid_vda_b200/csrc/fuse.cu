@@ -562,13 +562,6 @@ cudaError_t launch_gemm_mx(const Launch& ctx, const CUtensorMap& a, const CUtens
 
 bool a16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int sm_count_of_current_device() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
-  return n > 0 ? n : 148;
-}
-
 // The head shard's fuse; Out is the output GEMM's epilogue (an fp32
 // partial, or the reduce-scatter into the owners' buffers).
 template <class Out>

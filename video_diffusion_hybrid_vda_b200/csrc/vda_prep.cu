@@ -11,11 +11,17 @@
 //    rounded product, lo the rounded remainder; their sum carries ~16
 //    mantissa bits) into two more tiles;
 //  * one thread issues tcgen05.mma with both operands MN-major (token rows,
-//    feature columns): D_A += K^T hi + K^T lo, D_B += V^T hi + V^T lo, fp32
-//    accumulation in TMEM;
-//    for d = 64 the A operand is the stacked [K | V] feature block (M = 128)
-//    so one instruction produces both A (rows 0..63) and B (rows 64..127);
-//  * the scaler warps then drain TMEM rows to global fp32 A and B.
+//    feature columns), fp32 accumulation in TMEM.  For d = 128 the K and V
+//    tiles of a stage sit in adjacent 64-column slabs, so [K | V] is one
+//    N = 256 operand: D += hi^T [K | V] + lo^T [K | V], two instructions per
+//    16 tokens, with columns 0..127 of D holding A and 128..255 holding B^T
+//    (the shared-memory operand reads are 24 KB per 16 tokens instead of
+//    32 KB for four N = 128 products).  For d = 64 the stacked [K | V]
+//    feature block is the M = 128 operand against hi and lo, so D holds A
+//    (rows 0..63) and B (rows 64..127);
+//  * the scaler warps then drain TMEM to global fp32 A and B (B^T columns
+//    are stored transposed: per column, a warp writes 32 consecutive floats
+//    of one row of B).
 // The stage is HBM-bound (k and v are read once); the split doubles the
 // tensor-core work, which stays below the HBM time.
 //
@@ -124,6 +130,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
       constexpr uint32_t idesc = idesc_bf16(128, DH, true, true);
+      constexpr uint32_t idesc_kv = idesc_bf16(128, 2 * DH, true, true);
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % C::STAGES;
         if (!mbar_wait(kGram ? &full[s] : &scaled[s], (kb / C::STAGES) & 1, budget_ns)) {
@@ -151,11 +158,9 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
               umma_ss(tmem, kdesc, kdesc, idesc, acc);
             }
           } else if constexpr (DH == 128) {
-            const uint64_t vdesc = sdesc_sw128(vbase + kk * 2048, C::SLAB_BYTES, 1024);
-            umma_ss(tmem, kdesc, hdesc, idesc, acc);
-            umma_ss(tmem, kdesc, ldesc, idesc, 1);
-            umma_ss(tmem + 128, vdesc, hdesc, idesc, acc);
-            umma_ss(tmem + 128, vdesc, ldesc, idesc, 1);
+            // kdesc spans the four slabs K0 K1 V0 V1 (N = 256)
+            umma_ss(tmem, hdesc, kdesc, idesc_kv, acc);
+            umma_ss(tmem, ldesc, kdesc, idesc_kv, 1);
           } else {
             // [K | V] stacked along M: the V slab sits one slab after K.
             umma_ss(tmem, kdesc, hdesc, idesc, acc);
@@ -218,19 +223,28 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       const uint32_t lane_base = tmem + ((quarter * 32) << 16);
       const int64_t mat = (static_cast<int64_t>(t) * H + h) * DH * DH;
       if constexpr (DH == 128) {
+        // columns 0..127: row m of A (gram: unused); 128..255: row m of G
+        // (gram) or column m of B
 #pragma unroll 1
         for (int half = kGram ? 1 : 0; half < 2; ++half) {
-          float* dst = (half == 0 ? A : B) + mat + static_cast<int64_t>(m) * DH;
+          const bool rows = half == 0 || kGram;
+          float* dst = (half == 0 ? A : B) + mat + static_cast<int64_t>(m) * (rows ? DH : 1);
 #pragma unroll 1
           for (int c = 0; c < DH; c += 32) {
             uint32_t r[32];
             tmem_ld32(lane_base + half * 128 + c, r);
             tmem_ld_wait();
+            if (rows) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              *reinterpret_cast<float4*>(dst + c + e) =
-                  make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                              __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+              for (int e = 0; e < 32; e += 4)
+                *reinterpret_cast<float4*>(dst + c + e) =
+                    make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                dst[static_cast<int64_t>(c + e) * DH] = __uint_as_float(r[e]);
+            }
           }
         }
       } else if (!kGram || quarter >= 2) {  // warp-uniform: rows 0..63 are q^T q

@@ -6,17 +6,20 @@
 //   S_bwd_t = (alpha_t S_bwd_{t+1} + B_t) P_t    t = T-1 .. 0, S_bwd_T   = 0
 //
 // with P_t = (I + A_t)^-1 from the solve.  Rows of S evolve independently
-// (row r of S_t needs only row r of S_{t-1}), so each CTA owns 64 rows of
-// one head's state in one direction and runs all T steps; every CTA of the
-// grid is resident at once.  Per step the CTA stages P_t (d x d fp32) and
-// its 64 rows of B_t (one contiguous block) into shared memory with bulk
+// (row r of S_t needs only row r of S_{t-1}), so each CTA owns a block of
+// rows of one head's state in one direction and runs all T steps; every CTA
+// of the grid is resident at once.  The block is 8 x TR rows: TR = 8 (two
+// blocks per state at d = 128), or, when three blocks per state still fit
+// the SMs once, TR = 6 (48-row blocks, the last one 32 rows with the rest
+// masked), which shortens each step by a quarter.  Per step the CTA stages P_t (d x d fp32) and
+// its rows of B_t (one contiguous block) into shared memory with bulk
 // copies, double-buffered so that step t+1's operands land while step t
 // computes (nothing on a step's critical path waits on global memory).
 // Each thread first writes its tile of the bracket alpha S_prev + B_t into
 // the shared rows (row stride d + 4, so four consecutive k of a row are one
-// float4 and the rows of a warp fall in different banks), then computes 8
-// rows x 8 columns of the new state with packed f32x2 FMA: per k it loads 8
-// state and 8 P values for 64 FMA, the ratio at which shared-memory
+// float4 and the rows of a warp fall in different banks), then computes TR
+// rows x 8 columns of the new state with packed f32x2 FMA: per k it loads TR
+// state and 8 P values for 8 TR FMA, a ratio at which shared-memory
 // bandwidth (32 floats per clock per SM) keeps up with the FMA pipes.  The
 // CTA's two halves split the k range of the product (two warps per SM
 // sub-partition keep the packed FMAs issuing); the upper half hands its
@@ -42,33 +45,34 @@
 namespace vdn {
 namespace {
 
-constexpr int kRows = 64;   // rows of S per CTA
-constexpr int kTR = 8;      // rows per thread
+constexpr int kGroups = 8;  // row groups per CTA (TR rows each)
 constexpr int kTC = 8;      // columns per thread
 
-template <int DH>
+template <int DH, int TR>
 struct ScanCfg {
-  static constexpr int HALF = (kRows / kTR) * (DH / kTC);  // threads per k half
-  static constexpr int THREADS = 2 * HALF;                   // 256 (d=128), 128 (d=64)
+  static constexpr int ROWS = kGroups * TR;           // rows of S per CTA
+  static constexpr int BLOCKS = (DH + ROWS - 1) / ROWS;  // row blocks per state
+  static constexpr int HALF = kGroups * (DH / kTC);  // threads per k half
+  static constexpr int THREADS = 2 * HALF;           // 256 (d=128), 128 (d=64)
   static constexpr int P_BYTES = DH * DH * 4;
-  static constexpr int X_BYTES = kRows * DH * 4;  // the CTA's rows of B_t (or G_t)
+  static constexpr int X_BYTES = ROWS * DH * 4;  // the CTA's rows of B_t (or G_t)
   static constexpr int LDS = DH + 4;  // row stride of the state rows in shared memory
-  static constexpr int SMEM = 2 * P_BYTES + 2 * X_BYTES + kRows * LDS * 4 + 64;
+  static constexpr int SMEM = 2 * P_BYTES + 2 * X_BYTES + ROWS * LDS * 4 + 64;
 };
 
-template <int DH, bool kAdjoint>
-__global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
+template <int DH, int TR, bool kAdjoint>
+__global__ void __launch_bounds__(ScanCfg<DH, TR>::THREADS, 1)
     vda_scan_kernel(const float* __restrict__ P, const float* __restrict__ X,
                     const float* __restrict__ alpha, float* __restrict__ states, int T, int H,
                     uint32_t* status, uint64_t budget_ns) {
-  using Cfg = ScanCfg<DH>;
+  using Cfg = ScanCfg<DH, TR>;
   constexpr int CG = DH / kTC;  // column groups
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* Pbuf = reinterpret_cast<float*>(smem_raw);                  // 2 x [DH][DH]
-  float* Xbuf = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // 2 x [kRows][DH]
+  float* Xbuf = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES);  // 2 x [ROWS][DH]
   float* Ss = reinterpret_cast<float*>(smem_raw + 2 * Cfg::P_BYTES + 2 * Cfg::X_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + 2 * Cfg::P_BYTES +
-                                               2 * Cfg::X_BYTES + kRows * Cfg::LDS * 4);
+                                               2 * Cfg::X_BYTES + Cfg::ROWS * Cfg::LDS * 4);
 
   const int rb = blockIdx.x;  // row block
   const int h = blockIdx.y;
@@ -77,8 +81,11 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   const int lt = threadIdx.x % Cfg::HALF;
   const int cg = lt % CG;
   const int rg = lt / CG;
-  const int lrow0 = rg * kTR;                  // first local row of the thread's tile
-  const int row0 = rb * kRows + lrow0;         // first row of S
+  const int lrow0 = rg * TR;                   // first local row of the thread's tile
+  const int row0 = rb * Cfg::ROWS + lrow0;     // first row of S
+  // rows of this block inside the state (the last block may be partial)
+  const int nrows = min(Cfg::ROWS, DH - rb * Cfg::ROWS);
+  const int x_bytes = nrows * DH * 4;
   // the thread's columns: [colA, colA + 4) and [colB, colB + 4)
   const int colA = 4 * cg, colB = DH / 2 + 4 * cg;
   const int64_t mat = static_cast<int64_t>(DH) * DH;
@@ -87,13 +94,13 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   // both operands of the step that visits frame(step), into buffer `buf`
   auto stage = [&](int step, int buf) {
     const int64_t th = static_cast<int64_t>(frame(step)) * H + h;
-    mbar_arrive_expect_tx(&full[buf], Cfg::P_BYTES + Cfg::X_BYTES);
+    mbar_arrive_expect_tx(&full[buf], Cfg::P_BYTES + x_bytes);
     bulk_load(Pbuf + buf * DH * DH, P + th * mat, Cfg::P_BYTES, &full[buf]);
-    bulk_load(Xbuf + buf * kRows * DH, X + th * mat + static_cast<int64_t>(rb) * kRows * DH,
-              Cfg::X_BYTES, &full[buf]);
+    bulk_load(Xbuf + buf * Cfg::ROWS * DH,
+              X + th * mat + static_cast<int64_t>(rb) * Cfg::ROWS * DH, x_bytes, &full[buf]);
   };
 
-  for (int i = threadIdx.x; i < kRows * Cfg::LDS; i += blockDim.x) Ss[i] = 0.f;
+  for (int i = threadIdx.x; i < Cfg::ROWS * Cfg::LDS; i += blockDim.x) Ss[i] = 0.f;
   if (threadIdx.x == 0) {
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
@@ -102,9 +109,9 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   }
   __syncthreads();
 
-  float sprev[kTR][kTC];  // the thread's tile of the previous step's state
+  float sprev[TR][kTC];  // the thread's tile of the previous step's state
 #pragma unroll
-  for (int r = 0; r < kTR; ++r)
+  for (int r = 0; r < TR; ++r)
 #pragma unroll
     for (int c = 0; c < kTC; ++c) sprev[r][c] = 0.f;
 
@@ -133,9 +140,11 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     // step's reads behind the barrier that closed it, and the barrier below
     // publishes U before the multiply
     const bool ok = mbar_wait(&full[b], (step >> 1) & 1, budget_ns);
-    float* Xt = Xbuf + b * kRows * DH;
+    float* Xt = Xbuf + b * Cfg::ROWS * DH;
+    // rows past the state (masked block tail) carry junk that stays in
+    // their own rows and is never stored
 #pragma unroll
-    for (int r = 0; r < kTR; ++r) {
+    for (int r = 0; r < TR; ++r) {
       if (half != 0) break;  // the lower half holds the state
       const float4 xa = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colA);
       const float4 xb = *reinterpret_cast<const float4*>(Xt + (lrow0 + r) * DH + colB);
@@ -153,17 +162,17 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     }
     const float* Pt = Pbuf + b * DH * DH;
     // acc2[r][q]: columns (colA + 2q, +1) for q < 2, (colB + 2(q-2), +1) for q >= 2
-    uint64_t acc2[kTR][kTC / 2];
+    uint64_t acc2[TR][kTC / 2];
 #pragma unroll
-    for (int r = 0; r < kTR; ++r)
+    for (int r = 0; r < TR; ++r)
 #pragma unroll
       for (int q = 0; q < kTC / 2; ++q) acc2[r][q] = 0ull;
     {
 #pragma unroll 1
       for (int k = half * (DH / 2); k < (half + 1) * (DH / 2); k += 4) {
-        float sr[kTR][4];
+        float sr[TR][4];
 #pragma unroll
-        for (int r = 0; r < kTR; ++r) {
+        for (int r = 0; r < TR; ++r) {
           const float4 v = *reinterpret_cast<const float4*>(Ss + (lrow0 + r) * Cfg::LDS + k);
           sr[r][0] = v.x; sr[r][1] = v.y; sr[r][2] = v.z; sr[r][3] = v.w;
         }
@@ -172,7 +181,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
           const ulonglong2 pa = *reinterpret_cast<const ulonglong2*>(Pt + (k + kk) * DH + colA);
           const ulonglong2 pb = *reinterpret_cast<const ulonglong2*>(Pt + (k + kk) * DH + colB);
 #pragma unroll
-          for (int r = 0; r < kTR; ++r) {
+          for (int r = 0; r < TR; ++r) {
             const uint64_t ss = f32x2_pack(sr[r][kk], sr[r][kk]);
             acc2[r][0] = f32x2_fma(ss, pa.x, acc2[r][0]);
             acc2[r][1] = f32x2_fma(ss, pa.y, acc2[r][1]);
@@ -185,7 +194,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     // the upper half's partial sums, through the consumed B buffer
     if (half != 0) {
 #pragma unroll
-      for (int r = 0; r < kTR; ++r) {
+      for (int r = 0; r < TR; ++r) {
         *reinterpret_cast<ulonglong2*>(Xt + (lrow0 + r) * DH + colA) =
             make_ulonglong2(acc2[r][0], acc2[r][1]);
         *reinterpret_cast<ulonglong2*>(Xt + (lrow0 + r) * DH + colB) =
@@ -195,7 +204,7 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
     __syncthreads();  // partials visible; every read of Ss and Pbuf b is done
     if (half == 0) {
 #pragma unroll
-      for (int r = 0; r < kTR; ++r) {
+      for (int r = 0; r < TR; ++r) {
         const ulonglong2 ua = *reinterpret_cast<const ulonglong2*>(Xt + (lrow0 + r) * DH + colA);
         const ulonglong2 ub = *reinterpret_cast<const ulonglong2*>(Xt + (lrow0 + r) * DH + colB);
         const uint64_t v[4] = {f32x2_add(acc2[r][0], ua.x), f32x2_add(acc2[r][1], ua.y),
@@ -205,12 +214,14 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
           sprev[r][2 * q] = f32x2_lo(v[q]);
           sprev[r][2 * q + 1] = f32x2_hi(v[q]);
         }
-        float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
-                     static_cast<int64_t>(row0 + r) * DH;
-        *reinterpret_cast<float4*>(dst + colA) =
-            make_float4(sprev[r][0], sprev[r][1], sprev[r][2], sprev[r][3]);
-        *reinterpret_cast<float4*>(dst + colB) =
-            make_float4(sprev[r][4], sprev[r][5], sprev[r][6], sprev[r][7]);
+        if (lrow0 + r < nrows) {
+          float* dst = out_dir + (static_cast<int64_t>(t) * H + h) * mat +
+                       static_cast<int64_t>(row0 + r) * DH;
+          *reinterpret_cast<float4*>(dst + colA) =
+              make_float4(sprev[r][0], sprev[r][1], sprev[r][2], sprev[r][3]);
+          *reinterpret_cast<float4*>(dst + colB) =
+              make_float4(sprev[r][4], sprev[r][5], sprev[r][6], sprev[r][7]);
+        }
       }
     }
     __syncthreads();  // the partials are read: buffer b may be refilled
@@ -222,16 +233,30 @@ __global__ void __launch_bounds__(ScanCfg<DH>::THREADS, 1)
   }
 }
 
+template <int DH, int TR, bool kAdjoint>
+cudaError_t launch_scan_tr(const Launch& ctx, const vdn_shape& s, const float* P, const float* X,
+                           const float* alpha, float* states) {
+  using Cfg = ScanCfg<DH, TR>;
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(vda_scan_kernel<DH, TR, kAdjoint>, Cfg::SMEM, smem_set))
+    return e;
+  dim3 grid(Cfg::BLOCKS, s.H, 2);
+  vda_scan_kernel<DH, TR, kAdjoint><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      P, X, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+// The finer row blocks (TR = 6 at d = 128, 4 at d = 64) when their grid is
+// resident at once (one CTA per SM: each holds two P_t buffers), else the
+// 64-row blocks.
 template <int DH, bool kAdjoint>
 cudaError_t launch_scan_dh(const Launch& ctx, const vdn_shape& s, const float* P, const float* X,
                            const float* alpha, float* states) {
-  using Cfg = ScanCfg<DH>;
-  static std::atomic<uint64_t> smem_set{0};
-  if (cudaError_t e = set_smem_once(vda_scan_kernel<DH, kAdjoint>, Cfg::SMEM, smem_set)) return e;
-  dim3 grid(DH / kRows, s.H, 2);
-  vda_scan_kernel<DH, kAdjoint><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      P, X, alpha, states, s.T, s.H, ctx.status, ctx.budget_ns);
-  return cudaGetLastError();
+  constexpr int TR_FINE = DH == 128 ? 6 : 4;
+  const int64_t fine_ctas = static_cast<int64_t>(ScanCfg<DH, TR_FINE>::BLOCKS) * s.H * 2;
+  if (fine_ctas <= sm_count_of_current_device())
+    return launch_scan_tr<DH, TR_FINE, kAdjoint>(ctx, s, P, X, alpha, states);
+  return launch_scan_tr<DH, 8, kAdjoint>(ctx, s, P, X, alpha, states);
 }
 
 }  // namespace

@@ -13,7 +13,8 @@
 // start early.
 //
 // Kernel (sm_100a, one CTA per SM):
-//   warp 0      TMA: Q0/Q1 once, then K/V tiles through a 2-stage ring
+//   warp 0      TMA: Q0/Q1 once, then K and V tiles through a 2-stage ring
+//               (K and V slots released separately)
 //   warp 1      tcgen05.mma issue: S_i = Q_i K^T into TMEM, O_i += P_i V with
 //               P_i read from TMEM (the A operand) and V MN-major in smem
 //   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1: one thread
@@ -161,9 +162,14 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   uint8_t* kvbuf = smem + 2 * Cfg::TILE_BYTES;       // stage s: K then V
   uint64_t* bars = reinterpret_cast<uint64_t*>(kvbuf + Cfg::STAGES * 2 * Cfg::TILE_BYTES);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;                      // [STAGES]
-  uint64_t* kv_empty = kv_full + Cfg::STAGES;        // [STAGES]
-  uint64_t* s_full = kv_empty + Cfg::STAGES;         // [2]
+  // K and V of a stage have their own barriers: K is free once both S
+  // products of its tile are done, half a period before V (free after both
+  // PV products), so the next K load starts that much earlier
+  uint64_t* k_full = bars + 1;                       // [STAGES]
+  uint64_t* v_full = k_full + Cfg::STAGES;           // [STAGES]
+  uint64_t* k_empty = v_full + Cfg::STAGES;          // [STAGES]
+  uint64_t* v_empty = k_empty + Cfg::STAGES;         // [STAGES]
+  uint64_t* s_full = v_empty + Cfg::STAGES;          // [2]
   uint64_t* p_half = s_full + 2;                     // [2] P for keys 0..63 stored
   uint64_t* p_ready = p_half + 2;                    // [2] all of P stored
   uint64_t* o_done = p_ready + 2;                    // [2]
@@ -189,8 +195,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < Cfg::STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -233,30 +241,41 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
                       q0 + 128 * i);
       KvCursor cur;
       cur.init(kr);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
+      // K(j) waits for the S products of tile j - STAGES, V(j) for its PV
+      // products; the MMA warp retires them in that order
       for (int j = 0; j < nkv; ++j) {
         const int s = j % Cfg::STAGES;
-        if (j >= Cfg::STAGES &&
-            !mbar_wait(&kv_empty[s], ((j / Cfg::STAGES) & 1) ^ 1, budget_ns)) {
+        const uint32_t par = ((j / Cfg::STAGES) & 1) ^ 1;
+        uint8_t* kb = kvbuf + s * 2 * Cfg::TILE_BYTES;
+        const CUtensorMap* km = cur.ctx ? &ckmap : &kmap;
+        const CUtensorMap* vm = cur.ctx ? &cvmap : &vmap;
+        if (j >= Cfg::STAGES && !mbar_wait(&k_empty[s], par, budget_ns)) {
           record_status(status, kStatusTimeout);
           break;
         }
-        uint8_t* kb = kvbuf + s * 2 * Cfg::TILE_BYTES;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * Cfg::TILE_BYTES);
-        const CUtensorMap* km = cur.ctx ? &ckmap : &kmap;
-        const CUtensorMap* vm = cur.ctx ? &cvmap : &vmap;
-        for (int sl = 0; sl < Cfg::SLABS; ++sl) {
-          tma_load_2d(kb + sl * 16384, km, &kv_full[s], h * DH + 64 * sl, cur.pos);
-          tma_load_2d(kb + Cfg::TILE_BYTES + sl * 16384, vm, &kv_full[s], h * DH + 64 * sl,
-                      cur.pos);
+        mbar_arrive_expect_tx(&k_full[s], Cfg::TILE_BYTES);
+        for (int sl = 0; sl < Cfg::SLABS; ++sl)
+          tma_load_2d(kb + sl * 16384, km, &k_full[s], h * DH + 64 * sl, cur.pos);
+        ++k_issued;
+        if (j >= Cfg::STAGES && !mbar_wait(&v_empty[s], par, budget_ns)) {
+          record_status(status, kStatusTimeout);
+          break;
         }
-        ++issued;
+        mbar_arrive_expect_tx(&v_full[s], Cfg::TILE_BYTES);
+        for (int sl = 0; sl < Cfg::SLABS; ++sl)
+          tma_load_2d(kb + Cfg::TILE_BYTES + sl * 16384, vm, &v_full[s], h * DH + 64 * sl,
+                      cur.pos);
+        ++v_issued;
         cur.next(kr);
       }
       // drain loads still in flight
       mbar_wait(q_full, 0, 200000000ull);
-      for (int j = (issued > Cfg::STAGES ? issued - Cfg::STAGES : 0); j < issued; ++j)
-        if (!mbar_wait(&kv_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull))
+      for (int j = (k_issued > Cfg::STAGES ? k_issued - Cfg::STAGES : 0); j < k_issued; ++j)
+        if (!mbar_wait(&k_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull))
+          record_status(status, kStatusTimeout);
+      for (int j = (v_issued > Cfg::STAGES ? v_issued - Cfg::STAGES : 0); j < v_issued; ++j)
+        if (!mbar_wait(&v_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull))
           record_status(status, kStatusTimeout);
     }
   } else if (warp == 1) {
@@ -284,14 +303,16 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
           umma_ts(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8,
                   sdesc_sw128(vb + kk * 2048, 16384, 1024), idesc_o, (j > 0 || kk > 0));
       };
-      if (ok && (ok = mbar_wait(&kv_full[0], 0, budget_ns))) {
+      if (ok && (ok = mbar_wait(&k_full[0], 0, budget_ns))) {
         tc_fence_after();
         issue_s(0, 0);
         issue_s(1, 0);
+        umma_commit(&k_empty[0]);
       }
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j % Cfg::STAGES;
         const bool more = j + 1 < nkv;
+        if (!(ok = mbar_wait(&v_full[s], (j / Cfg::STAGES) & 1, budget_ns))) break;
         if (!(ok = mbar_wait(&p_half[0], j & 1, budget_ns))) break;
         tc_fence_after();
         issue_o(0, j, 0, 4);
@@ -301,7 +322,7 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         umma_commit(&o_done[0]);
         if (more) {
           const int sn = (j + 1) % Cfg::STAGES;
-          if (!(ok = mbar_wait(&kv_full[sn], ((j + 1) / Cfg::STAGES) & 1, budget_ns))) break;
+          if (!(ok = mbar_wait(&k_full[sn], ((j + 1) / Cfg::STAGES) & 1, budget_ns))) break;
           tc_fence_after();
           issue_s(0, j + 1);
         }
@@ -312,8 +333,11 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         tc_fence_after();
         issue_o(1, j, 4, 8);
         umma_commit(&o_done[1]);
-        umma_commit(&kv_empty[s]);
-        if (more) issue_s(1, j + 1);
+        umma_commit(&v_empty[s]);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit(&k_empty[(j + 1) % Cfg::STAGES]);
+        }
       }
       if (!ok) record_status(status, kStatusTimeout);
       umma_commit(mma_done);
@@ -360,11 +384,17 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         for (int c = 0; c < 64; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
+      // row max over eight running maxima, two scores per three-input max
+      auto sv = [&](int c) { return __uint_as_float(sr[c]); };
       float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+      for (int a = 0; a < 8; ++a) mx8[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      for (int c = 24; c < 56; c += 16)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], sv(56 + a));
       tmem_ld_wait();
       reg_fence(s2);
       reg_fence(s3);
@@ -374,12 +404,12 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
 #pragma unroll
-      for (int c = 64; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      for (int c = 64; c < 128; c += 16)
 #pragma unroll
-      for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int c = 0; c < w; ++c) mx8[c] = fmaxf(mx8[c], mx8[c + w]);
-      const float mt = mx8[0] * scale_log2;
+        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
+      const float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7])) *
+                       scale_log2;
       // Lazy rescale: only when some row's max grew by more than 2^8.  The
       // decision is taken per warp (the O accesses are warp-collective); rows
       // of a rescaling warp move to max(m_used, mt), a factor of 1 for rows
