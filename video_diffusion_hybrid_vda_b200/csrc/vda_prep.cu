@@ -6,10 +6,12 @@
 // Design (sm_100a):
 //  * one CTA per (t, h); the token dimension is the GEMM reduction;
 //  * TMA streams [BK tokens x d] tiles of k and v into 128B-swizzled shared
-//    memory through a 3-D frame view, so rows past the frame read as zero;
+//    memory through a 3-D frame view, so rows past the frame read as zero,
+//    over a ring of 4 stages (6 in gram mode);
 //  * four "scaler" warps write beta_i * k_i as a bf16 pair hi + lo (hi the
 //    rounded product, lo the rounded remainder; their sum carries ~16
-//    mantissa bits) into two more tiles;
+//    mantissa bits) into a ring of their own (2 stages), so the k/v ring
+//    keeps more of its bytes in flight from HBM;
 //  * one thread issues tcgen05.mma with both operands MN-major (token rows,
 //    feature columns), fp32 accumulation in TMEM.  For d = 128 the K and V
 //    tiles of a stage sit in adjacent 64-column slabs, so [K | V] is one
@@ -34,34 +36,39 @@
 namespace vdn {
 namespace {
 
-template <int DH>
+template <int DH, bool kGram>
 struct PrepCfg {
   static constexpr int BK = DH == 128 ? 32 : 64;  // tokens per pipeline stage
   static constexpr int SLABS = DH / 64;           // 64-column slabs per tile
   static constexpr int SLAB_BYTES = BK * 128;
   static constexpr int TILE_BYTES = SLABS * SLAB_BYTES;
-  static constexpr int STAGE_BYTES = 4 * TILE_BYTES;  // K, V, (beta*K)_hi, (beta*K)_lo
-  static constexpr int STAGES = 3;
+  static constexpr int KV_BYTES = 2 * TILE_BYTES;  // K then V (adjacent slabs)
+  static constexpr int HL_BYTES = 2 * TILE_BYTES;  // (beta*K)_hi then (beta*K)_lo
+  static constexpr int KV_STAGES = kGram ? 6 : 4;
+  static constexpr int HL_STAGES = kGram ? 0 : 2;
   static constexpr int TMEM_COLS = DH == 128 ? 256 : 64;
   static constexpr int THREADS = 192;  // warp0 TMA, warp1 MMA, warps2-5 scale+epilogue
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+  static constexpr int SMEM = 1024 + KV_STAGES * KV_BYTES + HL_STAGES * HL_BYTES + 256;
   static constexpr int CHUNKS_PER_THREAD = TILE_BYTES / 16 / 128;
 };
 
 template <int DH, bool kGram>
-__global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
+__global__ void __launch_bounds__(PrepCfg<DH, kGram>::THREADS, 1)
     vda_prep_kernel(const __grid_constant__ CUtensorMap kmap,
                     const __grid_constant__ CUtensorMap vmap, const float* __restrict__ beta,
                     float* __restrict__ A, float* __restrict__ B, int T, int N, int H,
                     uint32_t* status, uint64_t budget_ns) {
-  using C = PrepCfg<DH>;
+  using C = PrepCfg<DH, kGram>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* scaled = full + C::STAGES;
-  uint64_t* empty = scaled + C::STAGES;
-  uint64_t* accum_full = empty + C::STAGES;
+  uint8_t* kv_ring = smem;
+  uint8_t* hl_ring = smem + C::KV_STAGES * C::KV_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(hl_ring + C::HL_STAGES * C::HL_BYTES);
+  uint64_t* empty = full + C::KV_STAGES;    // [KV_STAGES]
+  uint64_t* scaled = empty + C::KV_STAGES;  // [HL_STAGES] hi/lo written
+  uint64_t* hl_free = scaled + 2;           // [HL_STAGES] hi/lo consumed
+  uint64_t* accum_full = hl_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_full + 1);
 
   const int th = blockIdx.x;  // = t * H + h
@@ -71,10 +78,13 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
   const uint32_t warp = warp_id();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KV_STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&scaled[s], 128);
       mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < C::HL_STAGES; ++s) {
+      mbar_init(&scaled[s], 128);
+      mbar_init(&hl_free[s], 1);
     }
     mbar_init(accum_full, 1);
     fence_mbar_init();
@@ -90,10 +100,10 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto stage_k = [&](int s) { return smem + s * C::STAGE_BYTES; };
-  auto stage_v = [&](int s) { return smem + s * C::STAGE_BYTES + C::TILE_BYTES; };
-  auto stage_hi = [&](int s) { return smem + s * C::STAGE_BYTES + 2 * C::TILE_BYTES; };
-  auto stage_lo = [&](int s) { return smem + s * C::STAGE_BYTES + 3 * C::TILE_BYTES; };
+  auto stage_k = [&](int s) { return kv_ring + s * C::KV_BYTES; };
+  auto stage_v = [&](int s) { return kv_ring + s * C::KV_BYTES + C::TILE_BYTES; };
+  auto stage_hi = [&](int s) { return hl_ring + s * C::HL_BYTES; };
+  auto stage_lo = [&](int s) { return hl_ring + s * C::HL_BYTES + C::TILE_BYTES; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -101,9 +111,9 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       int issued = 0;
       bool ok = true;
       for (int kb = 0; kb < nk && ok; ++kb) {
-        const int s = kb % C::STAGES;
-        if (kb >= C::STAGES) {
-          if (!mbar_wait(&empty[s], ((kb / C::STAGES) & 1) ^ 1, budget_ns)) {
+        const int s = kb % C::KV_STAGES;
+        if (kb >= C::KV_STAGES) {
+          if (!mbar_wait(&empty[s], ((kb / C::KV_STAGES) & 1) ^ 1, budget_ns)) {
             record_status(status, kStatusTimeout);
             ok = false;
             break;
@@ -119,9 +129,9 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
         ++issued;
       }
       // Drain: the last loads of every stage must have landed before exit.
-      for (int kb = (issued > C::STAGES ? issued - C::STAGES : 0); kb < issued; ++kb) {
-        const int s = kb % C::STAGES;
-        if (!mbar_wait(&full[s], (kb / C::STAGES) & 1, 200000000ull)) {
+      for (int kb = (issued > C::KV_STAGES ? issued - C::KV_STAGES : 0); kb < issued; ++kb) {
+        const int s = kb % C::KV_STAGES;
+        if (!mbar_wait(&full[s], (kb / C::KV_STAGES) & 1, 200000000ull)) {
           record_status(status, kStatusTimeout);
         }
       }
@@ -132,16 +142,20 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16(128, DH, true, true);
       constexpr uint32_t idesc_kv = idesc_bf16(128, 2 * DH, true, true);
       for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % C::STAGES;
-        if (!mbar_wait(kGram ? &full[s] : &scaled[s], (kb / C::STAGES) & 1, budget_ns)) {
+        const int s = kb % C::KV_STAGES;
+        const int hs = kGram ? 0 : kb % C::HL_STAGES;
+        // the k/v stage has landed, and (scaled) its hi/lo tiles are written
+        if (!mbar_wait(&full[s], (kb / C::KV_STAGES) & 1, budget_ns) ||
+            (!kGram && !mbar_wait(&scaled[hs], (kb / (kGram ? 1 : C::HL_STAGES)) & 1,
+                                  budget_ns))) {
           record_status(status, kStatusTimeout);
           break;
         }
         tc_fence_after();
         const uint32_t kbase = smem_u32(stage_k(s));
         const uint32_t vbase = smem_u32(stage_v(s));
-        const uint32_t hbase = smem_u32(stage_hi(s));
-        const uint32_t lbase = smem_u32(stage_lo(s));
+        const uint32_t hbase = smem_u32(stage_hi(hs));
+        const uint32_t lbase = smem_u32(stage_lo(hs));
 #pragma unroll
         for (int kk = 0; kk < C::BK / 16; ++kk) {
           const uint32_t acc = (kb | kk) != 0;
@@ -168,6 +182,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
           }
         }
         umma_commit(&empty[s]);
+        if constexpr (!kGram) umma_commit(&hl_free[hs]);
       }
       umma_commit(accum_full);
     }
@@ -176,7 +191,8 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
     const int tid = threadIdx.x - 64;  // 0..127
     bool ok = true;
     for (int kb = 0; kb < (kGram ? 0 : nk); ++kb) {
-      const int s = kb % C::STAGES;
+      const int s = kb % C::KV_STAGES;
+      const int hs = kb % (kGram ? 1 : C::HL_STAGES);
       // beta for the rows this thread touches in this stage
       float bv[C::CHUNKS_PER_THREAD];
 #pragma unroll
@@ -186,14 +202,19 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
         const int i = kb * C::BK + row;
         bv[j] = i < N ? __ldg(beta + (static_cast<int64_t>(t) * N + i) * H + h) : 0.f;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (kb / C::STAGES) & 1, budget_ns))) {
+      // the hi/lo stage must have been consumed by the MMAs of kb - HL_STAGES
+      const bool got = mbar_wait(&full[s], (kb / C::KV_STAGES) & 1, budget_ns) &&
+                       (kb < C::HL_STAGES ||
+                        mbar_wait(&hl_free[hs], ((kb / (kGram ? 1 : C::HL_STAGES)) & 1) ^ 1,
+                                  budget_ns));
+      if (!__all_sync(0xffffffffu, got)) {
         record_status(status, kStatusTimeout);
         ok = false;
         break;
       }
       const uint8_t* ks = stage_k(s);
-      uint8_t* his = stage_hi(s);
-      uint8_t* los = stage_lo(s);
+      uint8_t* his = stage_hi(hs);
+      uint8_t* los = stage_lo(hs);
 #pragma unroll
       for (int j = 0; j < C::CHUNKS_PER_THREAD; ++j) {
         const int off = (tid + 128 * j) * 16;
@@ -212,7 +233,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
         *reinterpret_cast<uint4*>(los + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&scaled[s]);
+      mbar_arrive(&scaled[hs]);
     }
     // ------------------------------------------------------------ epilogue
     // warp-uniform: the TMEM loads below are warp-collective
@@ -281,7 +302,7 @@ __global__ void __launch_bounds__(PrepCfg<DH>::THREADS, 1)
 template <int DH, bool kGram>
 cudaError_t launch_prep_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, const float* beta, float* A, float* B) {
-  using C = PrepCfg<DH>;
+  using C = PrepCfg<DH, kGram>;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_once(vda_prep_kernel<DH, kGram>, C::SMEM, smem_set)) return e;
   const int grid = s.T * s.H;

@@ -75,8 +75,7 @@ struct CholCfg {
   static constexpr int LDL = DH + 4;   // row stride of the matrix (float4 rows)
   static constexpr int LDP = 20;       // row stride of the 16-wide panel buffer
   static constexpr int LDT = DH + 4;   // row stride of the 16-row T buffer (aliases the panel)
-  // panel rows, plus 16 rows of padding below the last diagonal block
-  static constexpr int PANEL = ((DH + 16) * LDP > 16 * LDT) ? (DH + 16) * LDP : 16 * LDT;
+  static constexpr int PANEL = (DH * LDP > 16 * LDT) ? DH * LDP : 16 * LDT;
   static constexpr int SMEM = (DH * LDL + PANEL + 16) * 4;
 };
 
@@ -144,42 +143,45 @@ __global__ void __launch_bounds__(kThreads, 2)
   for (int p = 0; p < NB; ++p) {
     float* Dg = Ls + (16 * p) * LDL + 16 * p;  // diagonal block (p, p)
     if (threadIdx.x < 32) {
-      // Right-looking factorization of the diagonal block, one pivot per
-      // pass of a short runtime loop (an unrolled 16-pivot sequence is about
-      // a thousand instructions, fetched anew for every block).  Lane j
-      // (mod 16) holds column j of the trailing Schur complement shifted up
-      // to the pivot row: dc[r] = D[c + r][j] at pivot c, so every register
-      // index is a constant.  Lane c writes column c of L (rows c.., into
-      // the panel rows 16p.., which are free; rows past the block land in
-      // the panel buffer's padding) and the other lanes read it back.
+      // lane j (mod 16) holds column j of the diagonal block
       const int j = threadIdx.x & 15;
-      float* Lp = Pan + (16 * p) * LDP;
       float dc[16];
 #pragma unroll
       for (int r = 0; r < 16; ++r) dc[r] = Dg[r * LDL + j];
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 16; ++c) {
-        float piv = __shfl_sync(0xffffffffu, dc[0], c);  // D[c][c]
+        float piv = __shfl_sync(0xffffffffu, dc[c], c);
         if (!(piv > 0.f)) {  // also catches NaN
           bad = true;
           piv = 1.f;
         }
         // rsqrt and products (not the correctly rounded sqrt and reciprocal,
-        // whose longer sequences sit on this serial chain)
-        const float is = rsqrtf(piv);  // 1 / L[c][c]
-        float* lc = Lp + c * LDP + c;  // L[c + r][c] at lc[r * LDP]
-        if (threadIdx.x == c) {
+        // whose longer sequences sit on this serial chain); the pivot column
+        // goes to the other lanes through shared memory in one burst
+        const float is = rsqrtf(piv);                         // 1 / L[c][c]
+        const float f = (j > c) ? dc[c] * (is * is) : 0.f;  // D[c][j] / D[c][c]
+        const float sq = piv * is;                            // L[c][c]
+        float* colc = Pan + (16 * p) * LDP;  // 16 floats; panel rows 16p.. are free
+        if (threadIdx.x == c)
 #pragma unroll
-          for (int r = 0; r < 16; ++r) lc[r * LDP] = dc[r] * is;
-          idg[c] = is;
-        }
+          for (int r = 0; r < 16; ++r) colc[r] = dc[r];
         __syncwarp();
-        // D[c + r][j] -= L[c + r][c] L[j][c], shifted up by one row
-        const float f = dc[0] * is;  // L[j][c] (meaningful for j > c)
 #pragma unroll
-        for (int r = 1; r < 16; ++r) dc[r - 1] = fmaf(-lc[r * LDP], f, dc[r]);
-        dc[15] = 0.f;
+        for (int r = 0; r < 16; ++r) {
+          if (r > c) {
+            const float v = colc[r];  // D[r][c]
+            dc[r] = (j == c) ? dc[r] * is : fmaf(-v, f, dc[r]);
+          }
+        }
+        __syncwarp();  // every lane has read the column before the next pivot's
+        if (j == c) dc[c] = sq;
+        if (threadIdx.x == c) idg[c] = is;
       }
+      // L_pp (zero above the diagonal) into the panel rows 16p.. (free now)
+      float* Lp = Pan + (16 * p) * LDP;
+      if (threadIdx.x < 16)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Lp[r * LDP + j] = r < j ? 0.f : dc[r];
       __syncwarp();
       // column j of W_pp by forward substitution (rows above j come out 0)
       float w[16];
