@@ -202,3 +202,22 @@ def test_window_attn_rescale_in_one_row_of_a_warp(vdn):
                                         ctx_k=host(ck), ctx_v=host(cv))
     assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16
     assert np.abs(host(lse) - lse_ref).max() <= TOL_LSE
+
+
+def test_window_attn_rescale_on_second_half_keys(vdn):
+    """Keys 64..127 of a later tile carry a jump of the running max far above
+    2^8 (one row at a time, in a full and in a ragged context tile): the
+    rescale is decided only after the whole row of the tile is read."""
+    shape = synth.Shape(6, 64, 1, 128)
+    inp = synth.make_inputs(shape, seed=13, device="cuda")
+    ck, cv = _ctx(250, shape.D, seed=14)
+    ck = (ck.float() * 0.05).to(torch.bfloat16)
+    ck[100] = inp["q"][5]          # column 100 of the first context tile
+    ck[200] = inp["q"][50] * 2     # column 72 of the second (ragged, 122 keys)
+    ck[250 - 1] = inp["q"][7] * 3  # the last key of the ragged tile
+    o, lse = _run(vdn, shape, inp, ctx_k=ck, ctx_v=cv)
+    x = {k: host(v) for k, v in inp.items() if k in ("q", "k", "v")}
+    o_ref, lse_ref = oracle.window_attn(x["q"], x["k"], x["v"], *shape_args(shape),
+                                        ctx_k=host(ck), ctx_v=host(cv))
+    assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16
+    assert np.abs(host(lse) - lse_ref).max() <= TOL_LSE
