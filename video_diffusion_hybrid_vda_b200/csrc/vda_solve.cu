@@ -79,15 +79,20 @@ struct CholCfg {
   static constexpr int SMEM = (DH * LDL + PANEL + 16) * 4;
 };
 
-// 16-term dot product of two 16-float rows in shared memory (16-byte aligned)
-__device__ __forceinline__ float dot16(const float* x, const float* y) {
+// A 16-float row of shared memory (16-byte aligned) into registers, and
+// its dot product with another such row (packed f32x2, pairs summed last).
+__device__ __forceinline__ void load_row16(const float* x, ulonglong2 (&r)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) r[q] = *reinterpret_cast<const ulonglong2*>(x + 4 * q);
+}
+
+__device__ __forceinline__ float dot16_reg(const ulonglong2 (&a)[4], const float* y) {
   uint64_t acc = 0ull;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(x + 4 * q);
     const ulonglong2 b = *reinterpret_cast<const ulonglong2*>(y + 4 * q);
-    acc = f32x2_fma(a.x, b.x, acc);
-    acc = f32x2_fma(a.y, b.y, acc);
+    acc = f32x2_fma(a[q].x, b.x, acc);
+    acc = f32x2_fma(a[q].y, b.y, acc);
   }
   return f32x2_lo(acc) + f32x2_hi(acc);
 }
@@ -200,19 +205,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     if (p + 1 == NB) break;
 
-    // L_ip = A_ip W_pp^T: row ty of A_ip against row tx of W_pp
+    // L_ip = A_ip W_pp^T: row ty of A_ip against row tx of W_pp (that row
+    // held in registers across the block rows i: half the shared loads)
+    {
+      ulonglong2 wr[4];
+      load_row16(Dg + tx * LDL, wr);
 #pragma unroll 1
-    for (int i = p + 1; i < NB; ++i)
-      Pan[(16 * i + ty) * LDP + tx] = dot16(Ls + (16 * i + ty) * LDL + 16 * p, Dg + tx * LDL);
+      for (int i = p + 1; i < NB; ++i)
+        Pan[(16 * i + ty) * LDP + tx] = dot16_reg(wr, Ls + (16 * i + ty) * LDL + 16 * p);
+    }
     __syncthreads();
 
-    // trailing update of the lower blocks right of panel p; L_ip into place
+    // trailing update of the lower blocks right of panel p (row ty of L_ap
+    // in registers across the block columns b); L_ip into place
 #pragma unroll 1
     for (int a = p + 1; a < NB; ++a) {
-      const float* la = Pan + (16 * a + ty) * LDP;
+      ulonglong2 la[4];
+      load_row16(Pan + (16 * a + ty) * LDP, la);
 #pragma unroll 1
       for (int b = p + 1; b <= a; ++b)
-        Ls[(16 * a + ty) * LDL + 16 * b + tx] -= dot16(la, Pan + (16 * b + tx) * LDP);
+        Ls[(16 * a + ty) * LDL + 16 * b + tx] -= dot16_reg(la, Pan + (16 * b + tx) * LDP);
       Ls[(16 * a + ty) * LDL + 16 * p + tx] = Pan[(16 * a + ty) * LDP + tx];
     }
     __syncthreads();

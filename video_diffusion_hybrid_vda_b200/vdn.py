@@ -540,7 +540,10 @@ class HybridLayer:
         ``outs`` a list of host tensors [T*N, D] bf16 that receive y.  Copies
         run on ``copy_stream`` into two device staging sets, so the input of
         video i+1 and the result of video i-1 move while video i computes.
-        Returns after enqueueing; synchronise the streams to read ``outs``.
+        q, k, v are copied first: the window Softmax, which needs only them,
+        starts before beta, alpha and x have landed (this shortens the
+        pipeline's fill).  Returns after enqueueing; synchronise the streams
+        to read ``outs``.
         """
         if len(batches) != len(outs):
             raise ValueError("one output per batch")
@@ -556,6 +559,7 @@ class HybridLayer:
             self._ys = [torch.empty((self.L, self.D), dtype=torch.bfloat16, device=dev)
                         for _ in range(2)]
         stages, ys = self._stages, self._ys
+        loaded_qkv = [torch.cuda.Event() for _ in batches]
         loaded = [torch.cuda.Event() for _ in batches]
         computed = [torch.cuda.Event() for _ in batches]
         T, N, H, d = self.T, self.N, self.H, self.d
@@ -565,8 +569,10 @@ class HybridLayer:
             with torch.cuda.stream(copy_stream):
                 if i >= 2:
                     copy_stream.wait_event(computed[i - 2])   # stage i % 2 is free
-                for dst, src in zip(stages[i % 2], batches[i]):
+                for n, (dst, src) in enumerate(zip(stages[i % 2], batches[i])):
                     dst.copy_(src, non_blocking=True)
+                    if n == 2:
+                        loaded_qkv[i].record(copy_stream)
                 loaded[i].record(copy_stream)
 
         copy_stream.wait_stream(stream)  # copies start after work already on `stream`
@@ -574,13 +580,14 @@ class HybridLayer:
         for i in range(len(batches)):
             if i + 1 < len(batches):
                 load(i + 1)
-            stream.wait_event(loaded[i])
+            stream.wait_event(loaded_qkv[i])
             if i >= 2:
                 stream.wait_event(self._read[i - 2])           # y buffer i % 2 is free
             q, k, v, beta, alpha, x = stages[i % 2]
             y = ys[i % 2]
             window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win,
                         stream=stream)
+            stream.wait_event(loaded[i])                        # beta, alpha, x
             vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
                      stream=stream)
             self._fuse(x, y, stream)
