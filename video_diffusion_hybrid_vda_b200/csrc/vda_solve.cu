@@ -73,10 +73,11 @@ template <int DH>
 struct CholCfg {
   static constexpr int NB = DH / 16;
   static constexpr int LDL = DH + 4;   // row stride of the matrix (float4 rows)
-  static constexpr int LDP = 20;       // row stride of the 16-wide panel buffer
-  static constexpr int LDT = DH + 4;   // row stride of the 16-row T buffer (aliases the panel)
-  static constexpr int PANEL = (DH * LDP > 16 * LDT) ? DH * LDP : 16 * LDT;
-  static constexpr int SMEM = (DH * LDL + PANEL + 16) * 4;
+  static constexpr int LDP = 20;       // row stride of the 16-wide panel buffer, of the
+                                       // transposed T blocks (aliasing it) and of WTd
+  static constexpr int PANEL = DH * LDP;
+  static constexpr int WTD = NB * 16 * LDP;  // transposed diagonal blocks W_pp^T
+  static constexpr int SMEM = (DH * LDL + PANEL + 16 + WTD) * 4;
 };
 
 // A 16-float row of shared memory (16-byte aligned) into registers, and
@@ -104,11 +105,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   constexpr int NB = Cfg::NB;
   constexpr int LDL = Cfg::LDL;
   constexpr int LDP = Cfg::LDP;
-  constexpr int LDT = Cfg::LDT;
   extern __shared__ __align__(16) float sm[];
   float* Ls = sm;                   // [DH][LDL]: the matrix, then L / W blocks
-  float* Pan = Ls + DH * LDL;       // [DH][LDP] panel L_ip; in step 2 [16][LDT] T rows
+  float* Pan = Ls + DH * LDL;       // [DH][LDP] panel L_ip; in step 2 the T_ij^T rows
   float* idg = Pan + Cfg::PANEL;    // [16] 1 / L_pp[r][r]
+  float* WTd = idg + 16;            // [NB][16][LDP] W_pp^T
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
   const int64_t mat = static_cast<int64_t>(blockIdx.x) * DH * DH;
@@ -198,9 +199,16 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int k = 0; k < r; ++k) acc = fmaf(-lr[k], w[k], acc);
         w[r] = acc * idg[r];
       }
-      if (threadIdx.x < 16)
+      if (threadIdx.x < 16) {
 #pragma unroll
         for (int r = 0; r < 16; ++r) Dg[r * LDL + j] = w[r];
+        // row j of W_pp^T, for the products of step 2
+        float* wt = WTd + (16 * p + j) * LDP;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<float4*>(wt + 4 * q) =
+              make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      }
     }
     __syncthreads();
     if (p + 1 == NB) break;
@@ -231,42 +239,47 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   // ---------------------------------------------------------------- 2. W = L^-1
-  // block row 0 holds W_00 already; the diagonal blocks hold W_ii
+  // Block row by block row: T_ij = sum_{k=j}^{i-1} L_ik W_kj (j < i), then
+  // W_ij = -W_ii T_ij.  Every product pairs two contiguous 16-float rows:
+  // W_kj is read through its transpose, kept in the strictly upper block
+  // (j, k) of the matrix buffer for k > j (nothing else reads those blocks)
+  // and in WTd for k = j, and T through its transpose in the panel buffer.
+  // Block row 0 holds W_00 already; the diagonal blocks hold W_ii.
+  {
+    constexpr int NT = NB - 1;  // T blocks of the last block row
 #pragma unroll 1
-  for (int i = 1; i < NB; ++i) {
-    const float* li = Ls + (16 * i + ty) * LDL;  // row ty of block row i
-#pragma unroll 1
-    for (int j = 0; j < i; ++j) {
-      float t = 0.f;
-#pragma unroll 1
-      for (int k = j; k < i; ++k) {
-        const float* wkj = Ls + (16 * k) * LDL + 16 * j + tx;  // column tx of W_kj
-        float lr[16];
+    for (int i = 1; i < NB; ++i) {
+      const float* li = Ls + (16 * i + ty) * LDL;  // row ty of block row i
+      float t[NT];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 v = *reinterpret_cast<const float4*>(li + 16 * k + 4 * q);
-          lr[4 * q] = v.x; lr[4 * q + 1] = v.y; lr[4 * q + 2] = v.z; lr[4 * q + 3] = v.w;
+      for (int j = 0; j < NT; ++j) t[j] = 0.f;
+#pragma unroll 1
+      for (int k = 0; k < i; ++k) {
+        ulonglong2 lr[4];
+        load_row16(li + 16 * k, lr);  // row ty of L_ik, for every j <= k
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (j <= k) {
+            const float* wt = j == k ? WTd + (16 * j + tx) * LDP
+                                     : Ls + (16 * j + tx) * LDL + 16 * k;  // row tx of W_kj^T
+            t[j] += dot16_reg(lr, wt);
+          }
         }
-#pragma unroll
-        for (int n = 0; n < 16; ++n) t = fmaf(lr[n], wkj[n * LDL], t);
       }
-      Pan[ty * LDT + 16 * j + tx] = t;  // T_ij
-    }
-    __syncthreads();  // T complete; every read of L_i* is done
-    float wi[16];     // row ty of W_ii
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float4 v = *reinterpret_cast<const float4*>(li + 16 * i + 4 * q);
-      wi[4 * q] = v.x; wi[4 * q + 1] = v.y; wi[4 * q + 2] = v.z; wi[4 * q + 3] = v.w;
-    }
+      for (int j = 0; j < NT; ++j)
+        if (j < i) Pan[(16 * j + tx) * LDP + ty] = t[j];  // T_ij^T
+      __syncthreads();  // T complete; every read of L_i* is done
+      ulonglong2 wi[4];
+      load_row16(li + 16 * i, wi);  // row ty of W_ii
 #pragma unroll 1
-    for (int j = 0; j < i; ++j) {
-      float acc = 0.f;
-#pragma unroll
-      for (int n = 0; n < 16; ++n) acc = fmaf(wi[n], Pan[n * LDT + 16 * j + tx], acc);
-      Ls[(16 * i + ty) * LDL + 16 * j + tx] = -acc;
+      for (int j = 0; j < i; ++j) {
+        const float w = -dot16_reg(wi, Pan + (16 * j + tx) * LDP);  // W_ij[ty][tx]
+        Ls[(16 * i + ty) * LDL + 16 * j + tx] = w;
+        Ls[(16 * j + tx) * LDL + 16 * i + ty] = w;  // W_ij^T into block (j, i)
+      }
+      __syncthreads();  // W_i* complete; T free again
     }
-    __syncthreads();  // W_i* complete; T free again
   }
 
   // ---------------------------------------------------------------- 3. P = W^T W
