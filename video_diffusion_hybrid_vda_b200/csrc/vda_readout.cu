@@ -167,6 +167,11 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
     const bool leader = threadIdx.x == 64;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
+      const int tok = j * 128 + row;
+      // the row's scale is fetched before the wait, off the tile's path
+      const float rs = row_scale == nullptr ? 1.f
+                       : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
+                                 : 0.f;
       if (leader) bulk_wait_read<Cfg::OUT_BUFS - 1>();  // staging buffer b is free again
       const bool ok = mbar_wait(&tfull[b], (j >> 1) & 1, budget_ns);
       // collective decision (also the barrier that publishes "buffer free"),
@@ -176,10 +181,6 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int tok = j * 128 + row;
-      const float rs = row_scale == nullptr ? 1.f
-                       : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
-                                 : 0.f;
       uint8_t* ob = obuf + b * Cfg::QTILE_BYTES;
       const uint32_t taddr = tmem + b * DH + ((quarter * 32) << 16);
 #pragma unroll
