@@ -165,13 +165,19 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane_id();
     const bool leader = threadIdx.x == 64;
+    // the row's scale for tile j (1 without row_scale), fetched one tile
+    // ahead so its load latency is off the tile's path
+    auto scale_of = [&](int j) {
+      const int tok = j * 128 + row;
+      return row_scale == nullptr ? 1.f
+             : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
+                       : 0.f;
+    };
+    float rs_next = ntiles > 0 ? scale_of(0) : 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
-      const int tok = j * 128 + row;
-      // the row's scale is fetched before the wait, off the tile's path
-      const float rs = row_scale == nullptr ? 1.f
-                       : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
-                                 : 0.f;
+      const float rs = rs_next;
+      if (j + 1 < ntiles) rs_next = scale_of(j + 1);
       if (leader) bulk_wait_read<Cfg::OUT_BUFS - 1>();  // staging buffer b is free again
       const bool ok = mbar_wait(&tfull[b], (j >> 1) & 1, budget_ns);
       // collective decision (also the barrier that publishes "buffer free"),
