@@ -103,9 +103,10 @@ def clocks_start():
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     dev = os.environ.get("LOCAL_RANK", "0")
     try:
-        p = subprocess.Popen(["nvidia-smi", f"--id={dev}", f"--query-gpu={q}",
-                              "--format=csv,noheader,nounits", "-lms", "200"],
-                             stdout=open(path, "w"), stderr=subprocess.DEVNULL)
+        with open(path, "w") as out:  # the sampler keeps its own descriptor
+            p = subprocess.Popen(["nvidia-smi", f"--id={dev}", f"--query-gpu={q}",
+                                  "--format=csv,noheader,nounits", "-lms", "200"],
+                                 stdout=out, stderr=subprocess.DEVNULL)
     except OSError:
         p = None
     return p, path

@@ -20,7 +20,10 @@ import numpy as np
 
 
 def sigmoid(z):
-    return 1.0 / (1.0 + np.exp(-z))
+    # exp(-z) overflows to inf for z below about -709; 1 / (1 + inf) = 0 is
+    # then the exact float64 result, so the overflow is not reported
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
 
 
 def rmsnorm_heads(o, H, d, gamma, eps):

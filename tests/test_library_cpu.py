@@ -20,14 +20,19 @@ def L():
     return vdn
 
 
+def _header():
+    with open(os.path.join(ROOT, "include", "vdn.h"), encoding="utf-8") as f:
+        return f.read()
+
+
 def _declared():
-    src = open(os.path.join(ROOT, "include", "vdn.h")).read()
+    src = _header()
     return sorted(set(re.findall(r"^VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(", src, re.M)))
 
 
 def _declared_param_counts():
     """Number of parameters of every VDN_API function in include/vdn.h."""
-    src = open(os.path.join(ROOT, "include", "vdn.h")).read()
+    src = _header()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     out = {}
     for m in re.finditer(r"VDN_API\s+[\w\s\*]+?\b(vdn_\w+)\s*\(([^)]*)\)", src):

@@ -313,10 +313,11 @@ def test_mask_density_near_pages_figures():
     import os
     path = os.path.join(os.path.dirname(__file__), "golden", "mask_density.txt")
     pages = {}
-    for line in open(path):
-        if line.strip() and not line.startswith("#"):
-            T, pct = line.split()[:2]
-            pages[int(T)] = float(pct)
+    with open(path, encoding="utf-8") as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                T, pct = line.split()[:2]
+                pages[int(T)] = float(pct)
     for T, pct in pages.items():
         ours = 100.0 * oracle.mask_pair_count(T) / (T * T)
         assert abs(ours - pct) < 2.5, (T, ours, pct)
