@@ -272,6 +272,26 @@ VDN_API vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, co
                                        float scale, void* o, int64_t ld_o, float* lse_opt,
                                        void* ws, size_t ws_bytes, void* stream);
 
+/* The window Softmax's work plan, as the kernel launch uses it (host only:
+ * no CUDA call, no device memory).  Consecutive query frames with the same
+ * visible key frames (the mask of vdn_window_attn) form a segment; segments
+ * are listed heaviest first (most visible keys), the order their CTAs are
+ * launched in.  Per segment, 12 ints into segs[12*g ..]:
+ *   q0, q1        query token rows [q0, q1) (whole frames);
+ *   tile_base     index of its first 256-row CTA tile in launch order;
+ *   ntiles        its 256-row CTA tiles, ceil((q1 - q0) / 256);
+ *   nint          key intervals (1..3: the window, frame 0, frame T-1);
+ *   nkv           128-key tiles over those intervals (each rounded up);
+ *   k0, k1 x 3    key token intervals [k0, k1), unused ones 0.
+ * *nseg receives the number of segments.  Returns VDN_ERR_INVALID_ARG for
+ * a bad argument or when max_segs < *nseg (nothing written to segs then),
+ * VDN_ERR_UNSUPPORTED when the plan does not fit the kernel's fixed table
+ * (more than 256 segments or 3 intervals), which vdn_window_attn reports
+ * the same way. */
+VDN_API vdn_status vdn_window_attn_schedule(const vdn_shape* shape, int chunk_frames,
+                                            int window_chunks, unsigned anchors, int* segs,
+                                            int max_segs, int* nseg);
+
 /* ------------------------------------------------------------------------
  * Branch calibration and output projections (10100.com article, 方法概述
  * item 3; hotpaper.ai summary, 기술적 접근법).

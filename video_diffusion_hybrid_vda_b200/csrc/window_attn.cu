@@ -701,6 +701,37 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
   return e == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
 }
 
+vdn_status vdn_window_attn_schedule(const vdn_shape* shape, int chunk_frames, int window_chunks,
+                                   unsigned anchors, int* segs, int max_segs, int* nseg) {
+  if (shape == nullptr || shape->T < 1 || shape->N < 1 || nseg == nullptr)
+    return VDN_ERR_INVALID_ARG;
+  if (chunk_frames < 1 || window_chunks < 0 || anchors > 3u || max_segs < 0 ||
+      (max_segs > 0 && segs == nullptr))
+    return VDN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(shape->T) * shape->N >= (int64_t(1) << 31) - 512)
+    return VDN_ERR_INVALID_ARG;
+  thread_local WinSched sched;
+  if (!build_schedule(*shape, chunk_frames, window_chunks, anchors, &sched))
+    return VDN_ERR_UNSUPPORTED;
+  *nseg = sched.nseg;
+  if (sched.nseg > max_segs) return VDN_ERR_INVALID_ARG;
+  for (int g = 0; g < sched.nseg; ++g) {
+    const WinSeg& w = sched.seg[g];
+    int* o = segs + 12 * g;
+    o[0] = w.q0;
+    o[1] = w.q1;
+    o[2] = w.tile_base;
+    o[3] = w.ntiles;
+    o[4] = w.nint;
+    o[5] = w.nkv;
+    for (int v = 0; v < 3; ++v) {
+      o[6 + 2 * v] = v < w.nint ? w.k0[v] : 0;
+      o[7 + 2 * v] = v < w.nint ? w.k1[v] : 0;
+    }
+  }
+  return VDN_OK;
+}
+
 vdn_status vdn_window_attn(const vdn_shape* shape, const void* q, const void* k, const void* v,
                            int64_t ld, int chunk_frames, int window_chunks, unsigned anchors,
                            float scale, void* o, int64_t ld_o, float* lse_opt, void* ws,

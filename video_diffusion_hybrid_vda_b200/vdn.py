@@ -29,7 +29,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers",
            "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
            "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8",
-           "vdn_hybrid_fuse_shard_rs"]
+           "vdn_hybrid_fuse_shard_rs", "vdn_window_attn_schedule"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -78,6 +78,10 @@ def lib():
                                       ctypes.c_int, ctypes.c_int, ctypes.c_uint, ctypes.c_float,
                                       _P, _I64, _P, _P, _SZ, _P]
     L.vdn_window_attn_ctx.restype = ctypes.c_int
+    L.vdn_window_attn_schedule.argtypes = [S, ctypes.c_int, ctypes.c_int, ctypes.c_uint,
+                                           ctypes.POINTER(ctypes.c_int), ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int)]
+    L.vdn_window_attn_schedule.restype = ctypes.c_int
     L.vdn_hybrid_fuse_workspace.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.vdn_hybrid_fuse_workspace.restype = _SZ
     L.vdn_hybrid_fuse.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P,
@@ -350,6 +354,32 @@ def hybrid_fuse_mxfp8(x, o_s, o_vda, wg, gamma, wo, H, eps=1e-6, out=None, ws=No
 
 
 # ---------------------------------------------------------------- window Softmax
+
+SCHEDULE_FIELDS = ("q0", "q1", "tile_base", "ntiles", "nint", "nkv")
+
+
+def window_attn_schedule(T, N, chunk_frames=5, window_chunks=1, anchors=3):
+    """The window Softmax's work plan (host only): a list of segments in
+    launch order, each a dict with q0, q1, tile_base, ntiles, nint, nkv and
+    'keys', the list of its key intervals (k0, k1)."""
+    L = lib()
+    shape = Shape(T, N, 1, 128)
+    n = ctypes.c_int(0)
+    code = L.vdn_window_attn_schedule(ctypes.byref(shape), chunk_frames, window_chunks, anchors,
+                                      None, 0, ctypes.byref(n))
+    if code not in (VDN_OK, 1) or (code == 1 and n.value == 0):
+        _check(code, "vdn_window_attn_schedule")
+    buf = (ctypes.c_int * (12 * max(n.value, 1)))()
+    _check(L.vdn_window_attn_schedule(ctypes.byref(shape), chunk_frames, window_chunks, anchors,
+                                      buf, n.value, ctypes.byref(n)), "vdn_window_attn_schedule")
+    segs = []
+    for g in range(n.value):
+        row = buf[12 * g: 12 * g + 12]
+        seg = dict(zip(SCHEDULE_FIELDS, row[:6]))
+        seg["keys"] = [(row[6 + 2 * v], row[7 + 2 * v]) for v in range(seg["nint"])]
+        segs.append(seg)
+    return segs
+
 
 def window_attn_workspace(T, N, H, d):
     return int(lib().vdn_window_attn_workspace(ctypes.byref(_shape(T, N, H, d))))
