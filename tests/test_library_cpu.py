@@ -120,3 +120,79 @@ def test_window_and_fuse_reject_bad_arguments_on_host(L):
     r = lib.vdn_hybrid_fuse(16, 128, 1, None, P(16), P(16), P(16), P(16), P(16), 1e-6, P(16),
                             P(16), P(16), P(256), 1 << 30, None)
     assert r in (1, 2)
+
+
+def test_gradient_and_mxfp8_entry_points_reject_bad_arguments_on_host(L):
+    """Every refusal below happens before any CUDA call (no GPU here): the
+    pointers are aligned or misaligned fake addresses that are never read."""
+    lib = L.lib()
+    P = ctypes.c_void_p
+    FP = ctypes.c_void_p
+    A = 4096  # a 16-byte (and 256-byte) aligned stand-in address
+
+    def bwd(shape, q=A, ld=128, ld_g=128, dbeta=A, ws=A, ws_bytes=1 << 40):
+        return lib.vdn_vda_backward(ctypes.byref(shape) if shape is not None else None,
+                                    P(q), P(A), P(A), ld, FP(A), FP(A), P(A), 128, P(A), P(A),
+                                    P(A), ld_g, FP(dbeta), FP(A), 0, P(ws), ws_bytes, None)
+
+    ok = L.Shape(4, 8, 1, 128)
+    assert bwd(None) == 1
+    assert bwd(L.Shape(4, 8, 1, 96)) == 2                  # head dim
+    assert bwd(ok, q=0) == 1                               # null
+    assert bwd(ok, q=A + 8) == 1                           # misaligned activation
+    assert bwd(ok, dbeta=A + 2) == 1                       # misaligned fp32 output
+    assert bwd(ok, ld=100) == 1
+    assert bwd(ok, ld_g=120) == 1
+    assert bwd(ok, ws=0) == 3
+    assert bwd(ok, ws_bytes=1024) == 3
+
+    q = lib.vdn_mxfp8_quantize
+    assert q(None, 4, 128, 128, P(A), P(A), None) == 1
+    assert q(P(A), 4, 96, 96, P(A), P(A), None) == 1       # cols not a multiple of 128
+    assert q(P(A), 0, 128, 128, P(A), P(A), None) == 1
+    assert q(P(A + 4), 4, 128, 128, P(A), P(A), None) == 1
+
+    g = lib.vdn_gemm_mxfp8
+    assert g(0, 32, 128, P(A), P(A), P(A), P(A), P(A), 0, P(A), 256, None) == 1
+    assert g(128, 32, 96, P(A), P(A), P(A), P(A), P(A), 0, P(A), 256, None) == 2   # K % 128
+    assert g(128, 40, 128, P(A), P(A), P(A), P(A), P(A), 0, P(A), 256, None) == 2  # N % 32
+    assert g(128, 32, 128, P(A + 8), P(A), P(A), P(A), P(A), 0, P(A), 256, None) == 1
+    assert g(128, 32, 128, P(A), P(A), P(A), P(A), P(A), 0, None, 256, None) == 3
+
+    f = lib.vdn_hybrid_fuse_mxfp8
+    args = [P(A)] * 5
+    assert f(16, 3072, 25, *args, FP(A), 1e-6, P(A), P(A), P(A), P(A), 1 << 40, None) == 1
+    assert f(16, 3072, 24, None, *args[1:], FP(A), 1e-6, P(A), P(A), P(A), P(A), 1 << 40,
+             None) == 1
+    assert f(16, 3000, 24, *args, FP(A), 1e-6, P(A), P(A), P(A), P(A), 1 << 40, None) == 2
+    assert f(16, 3072, 24, *args, FP(A), 1e-6, P(A), P(A), P(A), None, 1 << 40, None) == 3
+
+    rs = lib.vdn_hybrid_fuse_shard_rs
+    owners = (ctypes.c_void_p * 9)(*([A] * 9))
+    common = [P(A), P(A), P(A), 128, P(A), P(A), FP(A), 1e-6, P(A), P(A)]
+    assert rs(16, 128, 1, 128, 0, *common, None, 2, P(A), 1 << 40, None) == 1
+    assert rs(16, 128, 1, 128, 0, *common, owners, 9, P(A), 1 << 40, None) == 1  # G > 8
+    assert rs(16, 128, 1, 128, 0, *common, owners, 0, P(A), 1 << 40, None) == 1
+    bad = (ctypes.c_void_p * 2)(A, A + 4)
+    assert rs(16, 128, 1, 128, 0, *common, bad, 2, P(A), 1 << 40, None) == 1
+
+
+def test_window_context_entry_rejects_bad_arguments_on_host(L):
+    lib = L.lib()
+    P = ctypes.c_void_p
+    A = 4096
+    s = L.Shape(10, 16, 1, 128)
+
+    def ctx(m_ctx=4, ck=A, ld_ctx=128, cf=5, wc=1, anchors=3, ws=A):
+        return lib.vdn_window_attn_ctx(ctypes.byref(s), P(A), P(A), P(A), 128, P(ck), P(A),
+                                       ld_ctx, m_ctx, cf, wc, anchors, 0.0, P(A), 128, None,
+                                       P(ws), 1 << 30, None)
+
+    assert ctx(m_ctx=-1) == 1
+    assert ctx(ck=0) == 1                                   # context keys missing
+    assert ctx(ck=A + 8) == 1
+    assert ctx(ld_ctx=100) == 1
+    assert ctx(cf=0) == 1
+    assert ctx(wc=-1) == 1
+    assert ctx(anchors=4) == 1
+    assert ctx(ws=0) == 3
