@@ -1,5 +1,12 @@
 """Build libvdn.so in-tree from csrc/*.cu for sm_100a (nvcc cross-compiles
-without a GPU).  Usage: ``python -m video_diffusion_hybrid_vda_b200.build``."""
+without a GPU).  Usage: ``python -m video_diffusion_hybrid_vda_b200.build``
+(``--force`` rebuilds, ``-v`` prints ptxas register and spill counts).
+
+Build-time switches of the kernels are passed as preprocessor definitions
+in ``VDN_NVCC_DEFINES`` (comma-separated ``NAME=VALUE``), e.g.
+``VDN_NVCC_DEFINES=VDN_EXP2_FMA_PAIRS=4`` for the window Softmax's
+FMA-pipe share of the exponentials; a build with definitions should be
+forced, since the up-to-date check looks at file times only."""
 
 import glob
 import os
@@ -37,13 +44,25 @@ def up_to_date():
     return all(os.path.getmtime(p) <= t for p in sources() + headers() + [__file__])
 
 
+def defines():
+    """-D flags from VDN_NVCC_DEFINES (comma-separated NAME=VALUE)."""
+    spec = os.environ.get("VDN_NVCC_DEFINES", "").strip()
+    out = []
+    for item in filter(None, (x.strip() for x in spec.split(","))):
+        name = item.split("=", 1)[0]
+        if not name.isidentifier():
+            raise ValueError(f"VDN_NVCC_DEFINES: bad definition {item!r}")
+        out.append("-D" + item)
+    return out
+
+
 def build(force=False, verbose=False, jobs=None):
     """Compile every csrc/*.cu to an object and link libvdn.so."""
     if not force and up_to_date():
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    inc = ["-I", os.path.join(os.path.dirname(HERE), "include")]
+    inc = ["-I", os.path.join(os.path.dirname(HERE), "include"), *defines()]
     procs, objs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
