@@ -102,3 +102,32 @@ def test_gemm_mx_is_the_product_of_dequantized_operands():
             assert abs(c[i, j] - sum(A[i, k] * B[j, k] for k in range(64))) < 1e-12
     # and close to the unquantized product (E4M3 keeps ~2 significant digits)
     assert np.abs(c - a @ b.T).max() < 0.1 * np.abs(a @ b.T).max()
+
+
+def test_fuse_is_exact_on_operands_the_format_holds():
+    """Special case that reduces to the plain fuse: with zero gate weights
+    (gates exactly 1/2), o_vda = 0 (RMSNorm gives 0) and small integers in o_s
+    and W_os (every 32-element block then holds only values E4M3 represents
+    under its shared scale), every quantization step is exact, so the MXFP8
+    fuse equals 0.5 * o_s W_os^T and the float64 fuse exactly."""
+    from oracle import fuse as ofuse
+    rng = np.random.default_rng(3)
+    L, D, H = 64, 128, 2
+    x = rng.standard_normal((L, D))
+    o_s = rng.integers(-8, 9, (L, D)).astype(np.float64)
+    o_vda = np.zeros((L, D))
+    W_gs = np.zeros((D, D))
+    W_gl = np.zeros((D, D))
+    W_os = rng.integers(-8, 9, (D, D)).astype(np.float64)
+    W_ol = rng.integers(-8, 9, (D, D)).astype(np.float64)
+    gamma = np.ones(D)
+    y_mx = mxfp8.hybrid_fuse_mxfp8(x, o_s, o_vda, W_gs, W_gl, gamma, 1e-6, W_os, W_ol, H)
+    y = ofuse.hybrid_fuse(x, o_s, o_vda, W_gs, W_gl, gamma, 1e-6, W_os, W_ol, H)
+    np.testing.assert_array_equal(y_mx, 0.5 * o_s @ W_os.T)
+    np.testing.assert_array_equal(y_mx, y)
+    # one value off the format's grid in o_s moves the result: the check
+    # above is not vacuous
+    o_s2 = o_s.copy()
+    o_s2[0, 0] = 7.3
+    y2 = mxfp8.hybrid_fuse_mxfp8(x, o_s2, o_vda, W_gs, W_gl, gamma, 1e-6, W_os, W_ol, H)
+    assert not np.array_equal(y2[0], 0.5 * o_s2[0] @ W_os.T)
