@@ -29,8 +29,8 @@ pages' description of the method:
 * ``mxfp8``        -- MXFP8 quantization (E4M3 elements, UE8M0 block scales)
                       and the fuse with MXFP8 projections.
 
-The readings taken where the pages are silent are listed in CONVENTIONS.md
-beside this file.  Parity status of every function is pinned by the
+The readings taken where the pages are silent are stated in each module's
+docstring.  Parity status of every function is pinned by the
 ``-m "not gpu"`` tests in ``tests/test_oracle_pins.py``; none is unpinned.
 """
 

@@ -7,7 +7,7 @@ has its own output projection and the two projections are added.  The
 Korean summary on hotpaper.ai (기술적 접근법) repeats that RMS normalisation
 and learnable gates calibrate the two paths.
 
-Readings (also in CONVENTIONS.md):
+Readings of the pages taken here:
 * gates are elementwise over the hidden size D, computed from the block
   input x ("content-dependent"), without bias: g = sigmoid(x W^T);
 * a gate multiplies its branch output before that branch's projection;

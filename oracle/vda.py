@@ -19,7 +19,7 @@ Layout (frame-major, matching the CUDA library): a token row r = t*N + i;
 q, k, v are [L, D] with head h in columns [h*d, (h+1)*d); beta is [L, H];
 alpha is [T, H]; states are [T, H, d, d] with S[..., v_dim, k_dim].
 
-Readings of the pages (also in CONVENTIONS.md):
+Readings of the pages taken here:
 * both scans include frame t's own write; the read-out sums the two
   directions' states: o_t = (S_fwd_t + S_bwd_t) q  (``combine="sum"``);
   ``combine="fwd_incl_bwd_excl"`` is kept for study only;

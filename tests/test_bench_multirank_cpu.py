@@ -54,3 +54,14 @@ def test_weak_scaling_value():
     assert bench.weak_scaling_value(1, 411264, 1000.0) == pytest.approx(411264.0)
     assert bench.weak_scaling_value(8, 411264, 500.0) == pytest.approx(8 * 411264 * 2.0)
     assert bench.max_over_ranks([1.0, 2.0], torch.device("cpu"), 1) == [1.0, 2.0]
+
+
+def test_bench_work_model_pair_count_matches_oracle():
+    """The bench's own frame-pair count (its work model for the roofline)
+    equals the oracle's mask for the layer shapes and the mask variants."""
+    import bench
+    import oracle
+    for T in (1, 2, 3, 10, 17, 42, 72, 102):
+        for cf, wc, anchors in ((5, 1, 3), (5, 0, 0), (3, 2, 1), (5, 1, 2)):
+            assert bench.mask_pair_count(T, cf, wc, anchors) == \
+                oracle.mask_pair_count(T, chunk_frames=cf, window_chunks=wc, anchors=anchors)

@@ -131,3 +131,38 @@ def test_fuse_is_exact_on_operands_the_format_holds():
     o_s2[0, 0] = 7.3
     y2 = mxfp8.hybrid_fuse_mxfp8(x, o_s2, o_vda, W_gs, W_gl, gamma, 1e-6, W_os, W_ol, H)
     assert not np.array_equal(y2[0], 0.5 * o_s2[0] @ W_os.T)
+
+
+def test_fuse_quantizes_the_gated_branch_inputs():
+    """Hand-worked case where the gated Softmax output g_s * o_s lies off the
+    E4M3 grid, so the MXFP8 fuse must round Z = [g_s o_s | g_l n] before the
+    output GEMM.  Zero gate weights give g = 1/2 exactly, o_vda = 0 gives
+    n = 0, W_os = I (every 32-block holds one 1: scale 2^-8, code 256, exact),
+    so y = quantized(Z)[:, :D] and the rounding can be read off by hand.
+
+    Per 32-element block of a row of Z (OCP MX: e = floor(log2 amax) - 8,
+    elements v / 2^e rounded to nearest E4M3, ties to the even code):
+      block 0: only 1.15 (o_s = 2.3): e = -8, 1.15 * 256 = 294.4, E4M3
+               neighbours 288 and 320 (step 32 in [256, 512)) -> 288 -> 1.125;
+      block 1: only 1.28125 (o_s = 2.5625): 328 -> 320 -> 1.25;
+      block 2: 3.0 (o_s = 6) and 1.15: e = floor(log2 3) - 8 = -7, 3 * 128 =
+               384 exact; 1.15 * 128 = 147.2, neighbours 144 and 160 (step 16
+               in [128, 256)) -> 144 -> 1.125;
+      block 3: 1.0625 (o_s = 2.125): 272 lies halfway between 256 (code 0x78,
+               even) and 288 (0x79) -> ties to even -> 256 -> 1.0.
+    Skipping the quantization of Z would give 1.15, 1.28125, 1.15, 1.0625.
+    """
+    L, D, H = 4, 128, 2
+    o_s = np.zeros((L, D))
+    o_s[0, 3] = 2.3
+    o_s[0, 40] = 2.5625
+    o_s[0, 64], o_s[0, 70] = 6.0, 2.3
+    o_s[0, 100] = 2.125
+    x = np.random.default_rng(4).standard_normal((L, D))
+    zeros = np.zeros((D, D))
+    y = mxfp8.hybrid_fuse_mxfp8(x, o_s, np.zeros((L, D)), zeros, zeros, np.ones(D), 1e-6,
+                                np.eye(D), zeros, H)
+    expect = np.zeros((L, D))
+    expect[0, 3], expect[0, 40], expect[0, 64], expect[0, 70], expect[0, 100] = (
+        1.125, 1.25, 3.0, 1.125, 1.0)
+    np.testing.assert_array_equal(y, expect)

@@ -136,6 +136,43 @@ def test_transition_is_non_expansive(T, N, H, d):
             assert sv.min() < x["alpha"][t, h]
 
 
+@pytest.mark.parametrize("T,N,H,d", [(10, 16, 1, 16), (6, 40, 3, 8)])
+def test_transition_is_what_the_scan_applies(T, N, H, d):
+    """M_t is the map the scans apply to the inherited state (方法概述 item 2:
+    the decayed old state is carried through (I + A_t)^-1).
+
+    Two pins that tie transition_matrix to the recurrence, not only to its
+    norm bound: (1) every forward and backward state obeys
+    S_t = S_prev M_t + S_t^(0), where S_t^(0) is the frame's state from a zero
+    inherited state; (2) two scans of one frame from different inherited
+    states differ by exactly their difference times M_t.  Dropping alpha_t,
+    inverting I + A_t the wrong way, or transposing M_t fails one of them
+    (alpha_t < 1 and A_t is not a multiple of I in these inputs).
+    """
+    s = synth.Shape(T, N, H, d)
+    x = {kk: vv.numpy().astype(np.float64)
+         for kk, vv in synth.make_inputs(s, torch.float32, seed=11).items()}
+    A, B = oracle.vda_prep(x["k"], x["v"], x["beta"], T, N, H, d)
+    S_fwd, S_bwd = oracle.vda_scan(A, B, x["alpha"])
+    zero = np.zeros((d, d))
+    rng = np.random.default_rng(5)
+    for h in range(H):
+        for t in range(T):
+            M = oracle.transition_matrix(x["alpha"][t, h], A[t, h])
+            S0 = oracle.vda_frame_state(zero, A[t, h], B[t, h])
+            prev_f = S_fwd[t - 1, h] if t > 0 else zero
+            prev_b = S_bwd[t + 1, h] if t + 1 < T else zero
+            np.testing.assert_allclose(S_fwd[t, h], prev_f @ M + S0, atol=1e-12)
+            np.testing.assert_allclose(S_bwd[t, h], prev_b @ M + S0, atol=1e-12)
+            # a non-symmetric perturbation of the inherited state, so that
+            # M and M^T act differently on it
+            X, Y = rng.standard_normal((d, d)), rng.standard_normal((d, d))
+            a = x["alpha"][t, h]
+            dS = (oracle.vda_frame_state(a * X, A[t, h], B[t, h])
+                  - oracle.vda_frame_state(a * Y, A[t, h], B[t, h]))
+            np.testing.assert_allclose(dS, (X - Y) @ M, atol=1e-12)
+
+
 # ------------------------------------------------------ one token per frame
 
 def _per_token_delta_rule(q, k, v, beta, alpha, T, H, d):
