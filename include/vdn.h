@@ -113,23 +113,27 @@ VDN_API vdn_status vdn_vda_debug_buffers(const vdn_shape* shape, void* ws, float
  * entry point exists for callers that cannot allocate device memory (for
  * example a plugin inside a host framework that owns every device
  * allocation, or a loop with a fixed memory budget where cudaMalloc is not
- * allowed).  It computes exactly what vdn_vda_scan computes, with the same
- * arguments minus ws/ws_bytes, and allocates nothing: its scratch is a
- * fixed 64 MiB array of this library's own device memory, present on every
- * GPU that loads the library until the process exits.
- *  - Limit: 256 + 5 * T*H*d*d*4 bytes must fit in 64 MiB (e.g. T*H <= 204
- *    at d = 128, <= 819 at d = 64); larger shapes return VDN_ERR_WORKSPACE
- *    before anything is enqueued.
+ * allowed).  It runs vdn_vda_scan's own validation and launch sequence, with
+ * the same arguments minus ws/ws_bytes, on a fixed 64 MiB array of this
+ * library's own device memory instead of a workspace; that array is present
+ * on every GPU that loads the library until the process exits.  Every head
+ * dim vdn_vda_scan takes (16, 32, 64, 128) is served; 16 and 32 run on
+ * padded copies in the array, as they do in a workspace.
+ *  - Limit: vdn_vda_scan_workspace(shape) must be <= 64 MiB (at d = 64 or
+ *    128 that is 256 + 5 * T*H*d*d*4 bytes, e.g. T*H <= 204 at d = 128,
+ *    <= 819 at d = 64); larger shapes return VDN_ERR_WORKSPACE before
+ *    anything is enqueued.
  *  - The first call on a device looks up the array's device address (once
- *    per device, with that device current); make that first call before any
- *    stream capture.
+ *    per device, with that device current) and caches it; make that first
+ *    call before any stream capture.  The cached address is not valid
+ *    across cudaDeviceReset of that device.
  *  - Every call shares the one array: calls that overlap on the GPU (other
  *    streams, other host threads) race and corrupt each other's results.
  *    The array keeps the last call's contents; each call clears the status
  *    word it uses and overwrites everything else it reads.
- *  - dev_status_opt: NULL, or device memory that receives, as the call's
- *    last operation on `stream`, this call's device status bits
- *    (0 = ok, bit 0 = numeric failure, bit 1 = a wait ran out of time).
+ *  - dev_status_opt: NULL, or 4-byte aligned device memory that receives,
+ *    as the call's last operation on `stream`, this call's device status
+ *    bits (0 = ok, bit 0 = numeric failure, bit 1 = a wait ran out of time).
  * No cudaMalloc, cudaFree or allocating library routine is called. */
 VDN_API vdn_status vdn_vda_scan_static(const vdn_shape* shape, const void* q, const void* k,
                                        const void* v, int64_t ld, const float* beta,

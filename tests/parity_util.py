@@ -9,6 +9,14 @@ TOL_BF16 = 2e-2
 TOL_STATE = 1e-3
 
 
+# Bound on the elementwise relative error (each element's denominator floored
+# at 1e-3 max|ref|).  The max-relative tolerances above allow up to 20 at the
+# floor; the kernels measure at most 1.6 (o_vda), 1.5 (o_s) and 1.35 (y), an
+# absolute error of ~1.5e-3 max|ref| on elements just above the floor.  This
+# bound keeps 2.5x headroom over that, so a doubling of the error fails.
+TOL_ELEMENTWISE = 4.0
+
+
 def max_rel(gpu, ref):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

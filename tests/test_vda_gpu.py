@@ -12,7 +12,7 @@ import pytest
 import torch
 
 import oracle
-from tests.parity_util import (TOL_BF16, TOL_STATE, elementwise_rel, ensure_built, host, max_rel,
+from tests.parity_util import (TOL_BF16, TOL_STATE, elementwise_rel, TOL_ELEMENTWISE, ensure_built, host, max_rel,
                                per_head_max_rel)
 from video_diffusion_hybrid_vda_b200 import synth
 
@@ -91,7 +91,9 @@ def test_vda_parity_small(vdn, T, N, H, d, report_metric):
             assert max_rel(st[1, t, h], S_bwd[t, h]) <= TOL_STATE, ("bwd", t, h)
     o_ref = oracle.vda_readout(x["q"], S_fwd, S_bwd, T, N, H, d)
     assert per_head_max_rel(host(o), o_ref, H, d) <= TOL_BF16
-    report_metric("o_vda_elementwise_rel", elementwise_rel(host(o), o_ref))
+    err_el = elementwise_rel(host(o), o_ref)
+    report_metric("o_vda_elementwise_rel", err_el)
+    assert err_el <= TOL_ELEMENTWISE
 
 
 def test_vda_strided_rows(vdn):
@@ -154,7 +156,8 @@ def test_vda_parity_full_layer_all_heads(vdn, T):
 
 @pytest.mark.parametrize("shape", synth.sweep_shapes(), ids=lambda s: f"T{s.T}N{s.N}d{s.d}H{s.H}")
 def test_vda_parity_scan_sweep_sampled(vdn, shape):
-    _sampled_parity(vdn, shape, heads=[shape.H - 1], n_rows=16, seed=1)
+    # first, middle and last head: all frames' states and 48 sampled rows each
+    _sampled_parity(vdn, shape, heads=[0, shape.H // 2, shape.H - 1], n_rows=48, seed=1)
 
 
 def test_vda_timeout_path_reports_and_recovers(vdn):
@@ -209,3 +212,36 @@ def test_vda_gauss_jordan_solver(vdn, T, N, H, d):
 def test_vda_solver_rejects_unknown(vdn):
     with pytest.raises(vdn.VdnError):
         vdn.set_vda_solver(7)
+
+
+@pytest.mark.parametrize("solver", [0, 1])
+@pytest.mark.parametrize("fault", ["nan", "indefinite"])
+def test_vda_numeric_failure_reports_and_recovers(vdn, solver, fault):
+    """Failures made on the host, none of which faults the GPU: a NaN in beta
+    makes A_t NaN, and a beta of -50 on every token of one frame makes
+    I + A_t indefinite (1 - 50 lambda_max < 0).  Either way some pivot of the
+    solve is NaN or non-positive (Sylvester: an SPD-less symmetric matrix has
+    a non-positive leading pivot, for Cholesky and for Gauss-Jordan without
+    pivoting alike), the status word reads VDN_ERR_NUMERIC, and the next call
+    on the same workspace after a reset is correct."""
+    shape = synth.Shape(4, 40, 2, 64)
+    inp = _inputs(shape, seed=21)
+    bad = inp["beta"].clone()
+    if fault == "nan":
+        bad[45, 1] = float("nan")
+    else:
+        bad[2 * shape.N:3 * shape.N, 0] = -50.0
+    try:
+        vdn.set_vda_solver(solver)
+        o, ws = vdn.vda_scan(inp["q"], inp["k"], inp["v"], bad, inp["alpha"],
+                             *shape_args(shape))
+        assert vdn.get_device_status(ws) == 5          # VDN_ERR_NUMERIC
+        vdn.reset_device_status(ws)
+        o, ws = vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"],
+                             *shape_args(shape), ws=ws)
+        assert vdn.get_device_status(ws) == 0
+    finally:
+        vdn.set_vda_solver(vdn.SOLVER_CHOLESKY)
+    x = {k: host(v) for k, v in inp.items()}
+    o_ref, _, _ = oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], *shape_args(shape))
+    assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16

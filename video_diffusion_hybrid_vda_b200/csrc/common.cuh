@@ -68,6 +68,13 @@ uint64_t current_wait_budget_ns();
 // Solver of the VDA closed form, set by vdn_set_vda_solver.
 int current_vda_solver();
 
+// vdn_vda_scan's validation and launch sequence on the workspace `ws`; with
+// clear_status the workspace's status word is zeroed on the stream first.
+vdn_status vda_scan_checked(const vdn_shape* shape, const void* q, const void* k, const void* v,
+                            int64_t ld, const float* beta, const float* alpha, void* o_vda,
+                            int64_t ld_o, float* states_opt, void* ws, size_t ws_bytes,
+                            void* stream, bool clear_status);
+
 // ---- tensor maps (built on the host with the driver's encoder) ----------
 
 // 3-D bf16 view of a frame-major [T*N, ld] activation: dims {cols, N, T}.

@@ -284,6 +284,20 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
                         int64_t ld_o, float* states_opt, void* ws, size_t ws_bytes,
                         void* stream) {
   NvtxRange nvtx("vdn_vda_scan");
+  return vdn::vda_scan_checked(shape, q, k, v, ld, beta, alpha, o_vda, ld_o, states_opt, ws,
+                               ws_bytes, stream, false);
+}
+
+}  // extern "C"
+
+// Validation and launch sequence of vdn_vda_scan, shared with the
+// allocation-free entry point (which passes its fixed scratch array as the
+// workspace and asks for the status word to be cleared first).
+vdn_status vdn::vda_scan_checked(const vdn_shape* shape, const void* q, const void* k,
+                                 const void* v, int64_t ld, const float* beta,
+                                 const float* alpha, void* o_vda, int64_t ld_o,
+                                 float* states_opt, void* ws, size_t ws_bytes, void* stream,
+                                 bool clear_status) {
   if (!shape_ok(shape)) return VDN_ERR_INVALID_ARG;
   const vdn_shape s = *shape;
   if (!head_dim_supported(s.d)) return VDN_ERR_UNSUPPORTED;
@@ -306,6 +320,8 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
   float* states_ws = reinterpret_cast<float*>(inner + pl.lay.states);
   Launch ctx{static_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(ws),
              g_budget_ns.load()};
+  if (clear_status && cudaMemsetAsync(ws, 0, sizeof(uint32_t), ctx.stream) != cudaSuccess)
+    return VDN_ERR_CUDA;
   if (!pl.padded)
     return run_vda(ctx, s, q, k, v, ld, beta, alpha, o_vda, ld_o, A, B, P,
                    states_opt ? states_opt : states_ws);
@@ -333,6 +349,8 @@ vdn_status vdn_vda_scan(const vdn_shape* shape, const void* q, const void* k, co
     return VDN_ERR_CUDA;
   return VDN_OK;
 }
+
+extern "C" {
 
 // ----------------------------------------------------------------- VDA gradients
 

@@ -228,6 +228,26 @@ def vda_scan(q, k, v, beta, alpha, T, N, H, d, out=None, states=None, ws=None, s
     return out, ws
 
 
+def vda_scan_static(q, k, v, beta, alpha, T, N, H, d, out=None, states=None, status=None,
+                    stream=None):
+    """vda_scan without a workspace (vdn_vda_scan_static): the library's fixed
+    device scratch array serves instead, for callers that cannot allocate.
+    Returns (o_vda, status) where ``status`` (int32 [1] on the device, or the
+    tensor given) receives the call's device status bits.  Calls that overlap
+    on the GPU share the array and race."""
+    _need_cuda(q, k, v, beta, alpha, out, states, status)
+    shape = _shape(T, N, H, d)
+    if out is None:
+        out = torch.empty((T * N, H * d), dtype=torch.bfloat16, device=q.device)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    code = lib().vdn_vda_scan_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), q.stride(0),
+                                     _ptr(beta), _ptr(alpha), _ptr(out), out.stride(0),
+                                     _ptr(states), _ptr(status), _stream(stream))
+    _check(code, "vdn_vda_scan_static")
+    return out, status
+
+
 def vda_debug_buffers(ws, T, N, H, d):
     """(A, B, P) views into a VDA workspace, each fp32 [T, H, d, d]."""
     ptrs = [ctypes.c_void_p() for _ in range(3)]
