@@ -41,6 +41,19 @@ namespace {
 
 constexpr int kMaxSegs = 256;
 
+// P is stored in four 32-key chunks; the PV product of the first this-many
+// chunks is issued as soon as they are stored, the rest once the row is done.
+#ifndef VDN_P_EARLY_CHUNKS
+#define VDN_P_EARLY_CHUNKS 2
+#endif
+static_assert(VDN_P_EARLY_CHUNKS >= 1 && VDN_P_EARLY_CHUNKS <= 3, "1..3 of the 4 chunks");
+
+// Head dim 128 runs on the CTA-pair kernel (2-SM MMAs) unless this is 0,
+// which selects the one-CTA kernel (kept for head dim 64 and comparisons).
+#ifndef VDN_WINDOW_PAIR
+#define VDN_WINDOW_PAIR 1
+#endif
+
 // Of every 16 score pairs in a 32-column chunk, this many take the FMA-pipe
 // exponential and the rest the MUFU (measured on B200: see profiles/).
 #ifndef VDN_EXP2_FMA_PAIRS
@@ -54,6 +67,8 @@ struct WinSeg {
   int q0, q1;      // query token rows [q0, q1)
   int tile_base;   // first CTA tile index of this segment (launch order)
   int ntiles;      // 256-row CTA tiles
+  int pair_base;   // first CTA-pair index of this segment (pair kernel)
+  int npairs;      // 512-row CTA pairs
   int nint;        // key intervals (1..3)
   int k0[3], k1[3];
   int nkv;         // 128-key tiles over all intervals
@@ -62,6 +77,7 @@ struct WinSeg {
 struct WinSched {
   int nseg;
   int total_tiles;
+  int total_pairs;
   WinSeg seg[kMaxSegs];
 };
 
@@ -143,6 +159,178 @@ struct KvCursor {
   }
   __device__ int valid() const { return min(128, end - pos); }
 };
+
+// One softmax warpgroup (tile i of the CTA's two 128-row query tiles): one
+// thread per query row.  For every key tile it waits for S_i, takes the row
+// max, rescales O_i in TMEM when the max grew by more than 2^8 (warp-uniform
+// decision), writes P = 2^(s - m) over S as bf16 in two halves (reporting
+// each half through arrive_half / arrive_ready), and at the end normalises
+// O_i by the row sum and stores the row (and its log-sum-exp).
+template <int DH, class ArriveHalf, class ArriveReady>
+__device__ __forceinline__ void softmax_warpgroup(
+    int i, uint32_t tmem, uint64_t* s_full, uint64_t* o_done, ArriveHalf arrive_half,
+    ArriveReady arrive_ready, const KvRange& kr, int nkv, float scale_log2, int q0, int q_end,
+    int h, int L, __nv_bfloat16* __restrict__ out, int64_t ld_o, float* __restrict__ lse,
+    uint32_t* status, uint64_t budget_ns) {
+  const uint32_t quarter = warp_id() & 3;
+  const int row = quarter * 32 + lane_id();
+  const uint32_t lane_off = (quarter * 32) << 16;
+  const uint32_t s_addr = tmem + 128 * i + lane_off;
+  const uint32_t o_addr = tmem + 256 + 128 * i + lane_off;
+  float m_used = -INFINITY;  // running max, log2 domain (scaled)
+  float l = 0.f;
+  KvCursor cur;
+  cur.init(kr);
+  bool ok = true;
+  for (int j = 0; j < nkv; ++j) {
+    const int valid = cur.valid();
+    cur.next(kr);
+    // warp-uniform decision: tcgen05.ld/st below are warp-collective
+    if (!__all_sync(0xffffffffu, mbar_wait(&s_full[i], j & 1, budget_ns))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    uint32_t sr[128];
+    uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+    uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+    uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+    uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+    // first half of the row, then start loading the second half while the
+    // first half's max is taken
+    tmem_ld32(s_addr, s0);
+    tmem_ld32(s_addr + 32, s1);
+    tmem_ld_wait();
+    reg_fence(s0);
+    reg_fence(s1);
+    tmem_ld32(s_addr + 64, s2);
+    tmem_ld32(s_addr + 96, s3);
+    if (valid < 64) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c)
+        if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+    }
+    // row max over eight running maxima, two scores per three-input max
+    auto sv = [&](int c) { return __uint_as_float(sr[c]); };
+    float mx8[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mx8[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
+#pragma unroll
+    for (int c = 24; c < 56; c += 16)
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
+#pragma unroll
+    for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], sv(56 + a));
+    tmem_ld_wait();
+    reg_fence(s2);
+    reg_fence(s3);
+    if (valid < 128) {
+#pragma unroll
+      for (int c = 64; c < 128; ++c)
+        if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+    }
+#pragma unroll
+    for (int c = 64; c < 128; c += 16)
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
+    const float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                           fmaxf(mx8[6], mx8[7])) *
+                     scale_log2;
+    // Lazy rescale: only when some row's max grew by more than 2^8.  The
+    // decision is taken per warp (the O accesses are warp-collective); rows
+    // of a rescaling warp move to max(m_used, mt), a factor of 1 for rows
+    // whose max did not grow.
+    if (__any_sync(0xffffffffu, mt > m_used + 8.f)) {
+      const float m_new = fmaxf(m_used, mt);
+      const float factor = exp2_mufu(m_used - m_new);  // 0 on the first tile
+      l *= factor;
+      if (j > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done[i], (j - 1) & 1, budget_ns))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(o_addr + c, o);
+          tmem_ld_wait();
+          reg_fence(o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+          tmem_st32(o_addr + c, o);
+        }
+      }
+      m_used = m_new;
+    }
+    // p = 2^(s * scale_log2 - m) with the argument by packed f32x2 FMA and
+    // four packed partial sums; one pair in four takes the FMA-pipe
+    // exponential, the rest the MUFU.  P goes back over S as bf16 in two
+    // halves, so the PV product can start on keys 0..63.
+    const uint64_t cc = f32x2_pack(scale_log2, scale_log2);
+    const uint64_t nm = f32x2_pack(-m_used, -m_used);
+    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const uint64_t xs = f32x2_fma(
+            (static_cast<uint64_t>(sr[32 * q + 2 * e + 1]) << 32) | sr[32 * q + 2 * e], cc, nm);
+        uint64_t pp;
+        if (VDN_EXP2_FMA_PAIRS > 0 &&
+            (e % (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1))) ==
+                (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1)) - 1) {
+          pp = exp2_fma_x2(xs);
+        } else {
+          pp = f32x2_pack(exp2_mufu(f32x2_lo(xs)), exp2_mufu(f32x2_hi(xs)));
+        }
+        acc2[e & 3] = f32x2_add(acc2[e & 3], pp);
+        pk[e] = pack_bf16x2(f32x2_lo(pp), f32x2_hi(pp));
+      }
+      tmem_st16(s_addr + 16 * q, pk);
+      if (q == VDN_P_EARLY_CHUNKS - 1) {
+        tmem_st_wait();
+        tc_fence_before();
+        arrive_half();
+      }
+    }
+    acc2[0] = f32x2_add(f32x2_add(acc2[0], acc2[1]), f32x2_add(acc2[2], acc2[3]));
+    l += f32x2_lo(acc2[0]) + f32x2_hi(acc2[0]);
+    tmem_st_wait();
+    tc_fence_before();
+    arrive_ready();
+  }
+  // ------------------------------------------------------------ epilogue
+  if (__all_sync(0xffffffffu, ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns))) {
+    tc_fence_after();
+    const int r = q0 + 128 * i + row;
+    const bool live = r < q_end;
+    const float inv = 1.f / l;
+    __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * DH;
+#pragma unroll 1
+    for (int c = 0; c < DH; c += 32) {
+      uint32_t o[32];
+      tmem_ld32(o_addr + c, o);
+      tmem_ld_wait();
+      if (live) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 u;
+          u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
+          u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+          u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+          u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + c + e) = u;
+        }
+      }
+    }
+    if (live && lse != nullptr)
+      lse[static_cast<int64_t>(h) * L + r] = (m_used + log2f(l)) * 0.69314718055994531f;
+  } else {
+    record_status(status, kStatusTimeout);
+  }
+}
 
 template <int DH>
 __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
@@ -315,10 +503,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         if (!(ok = mbar_wait(&v_full[s], (j / Cfg::STAGES) & 1, budget_ns))) break;
         if (!(ok = mbar_wait(&p_half[0], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(0, j, 0, 4);
+        issue_o(0, j, 0, 2 * VDN_P_EARLY_CHUNKS);
         if (!(ok = mbar_wait(&p_ready[0], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(0, j, 4, 8);
+        issue_o(0, j, 2 * VDN_P_EARLY_CHUNKS, 8);
         umma_commit(&o_done[0]);
         if (more) {
           const int sn = (j + 1) % Cfg::STAGES;
@@ -328,10 +516,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
         }
         if (!(ok = mbar_wait(&p_half[1], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(1, j, 0, 4);
+        issue_o(1, j, 0, 2 * VDN_P_EARLY_CHUNKS);
         if (!(ok = mbar_wait(&p_ready[1], j & 1, budget_ns))) break;
         tc_fence_after();
-        issue_o(1, j, 4, 8);
+        issue_o(1, j, 2 * VDN_P_EARLY_CHUNKS, 8);
         umma_commit(&o_done[1]);
         umma_commit(&v_empty[s]);
         if (more) {
@@ -346,164 +534,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     // ================================================================ softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
     const int i = (warp - 4) >> 2;  // query tile of this warpgroup
-    const uint32_t quarter = warp & 3;
-    const int row = quarter * 32 + lane_id();
-    const uint32_t lane_off = (quarter * 32) << 16;
-    const uint32_t s_addr = tmem + 128 * i + lane_off;
-    const uint32_t o_addr = tmem + 256 + 128 * i + lane_off;
-    float m_used = -INFINITY;  // running max, log2 domain (scaled)
-    float l = 0.f;
-    KvCursor cur;
-    cur.init(kr);
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      const int valid = cur.valid();
-      cur.next(kr);
-      // warp-uniform decision: tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[i], j & 1, budget_ns))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sr[128];
-      uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-      uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-      uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-      uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-      // first half of the row, then start loading the second half while the
-      // first half's max is taken
-      tmem_ld32(s_addr, s0);
-      tmem_ld32(s_addr + 32, s1);
-      tmem_ld_wait();
-      reg_fence(s0);
-      reg_fence(s1);
-      tmem_ld32(s_addr + 64, s2);
-      tmem_ld32(s_addr + 96, s3);
-      if (valid < 64) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row max over eight running maxima, two scores per three-input max
-      auto sv = [&](int c) { return __uint_as_float(sr[c]); };
-      float mx8[8];
-#pragma unroll
-      for (int a = 0; a < 8; ++a) mx8[a] = fmax3(sv(a), sv(a + 8), sv(a + 16));
-#pragma unroll
-      for (int c = 24; c < 56; c += 16)
-#pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
-#pragma unroll
-      for (int a = 0; a < 8; ++a) mx8[a] = fmaxf(mx8[a], sv(56 + a));
-      tmem_ld_wait();
-      reg_fence(s2);
-      reg_fence(s3);
-      if (valid < 128) {
-#pragma unroll
-        for (int c = 64; c < 128; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-      }
-#pragma unroll
-      for (int c = 64; c < 128; c += 16)
-#pragma unroll
-        for (int a = 0; a < 8; ++a) mx8[a] = fmax3(mx8[a], sv(c + a), sv(c + 8 + a));
-      const float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                             fmaxf(mx8[6], mx8[7])) *
-                       scale_log2;
-      // Lazy rescale: only when some row's max grew by more than 2^8.  The
-      // decision is taken per warp (the O accesses are warp-collective); rows
-      // of a rescaling warp move to max(m_used, mt), a factor of 1 for rows
-      // whose max did not grow.
-      if (__any_sync(0xffffffffu, mt > m_used + 8.f)) {
-        const float m_new = fmaxf(m_used, mt);
-        const float factor = exp2_mufu(m_used - m_new);  // 0 on the first tile
-        l *= factor;
-        if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&o_done[i], (j - 1) & 1, budget_ns))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c = 0; c < DH; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(o_addr + c, o);
-            tmem_ld_wait();
-            reg_fence(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(o_addr + c, o);
-          }
-        }
-        m_used = m_new;
-      }
-      // p = 2^(s * scale_log2 - m) with the argument by packed f32x2 FMA and
-      // four packed partial sums; one pair in four takes the FMA-pipe
-      // exponential, the rest the MUFU.  P goes back over S as bf16 in two
-      // halves, so the PV product can start on keys 0..63.
-      const uint64_t cc = f32x2_pack(scale_log2, scale_log2);
-      const uint64_t nm = f32x2_pack(-m_used, -m_used);
-      uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint64_t xs = f32x2_fma(
-              (static_cast<uint64_t>(sr[32 * q + 2 * e + 1]) << 32) | sr[32 * q + 2 * e], cc, nm);
-          uint64_t pp;
-          if (VDN_EXP2_FMA_PAIRS > 0 &&
-              (e % (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1))) ==
-                  (16 / (VDN_EXP2_FMA_PAIRS > 0 ? VDN_EXP2_FMA_PAIRS : 1)) - 1) {
-            pp = exp2_fma_x2(xs);
-          } else {
-            pp = f32x2_pack(exp2_mufu(f32x2_lo(xs)), exp2_mufu(f32x2_hi(xs)));
-          }
-          acc2[e & 3] = f32x2_add(acc2[e & 3], pp);
-          pk[e] = pack_bf16x2(f32x2_lo(pp), f32x2_hi(pp));
-        }
-        tmem_st16(s_addr + 16 * q, pk);
-        if (q == 1) {
-          tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_half[i]);
-        }
-      }
-      acc2[0] = f32x2_add(f32x2_add(acc2[0], acc2[1]), f32x2_add(acc2[2], acc2[3]));
-      l += f32x2_lo(acc2[0]) + f32x2_hi(acc2[0]);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_ready[i]);
-    }
-    // ------------------------------------------------------------ epilogue
-    if (__all_sync(0xffffffffu, ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns))) {
-      tc_fence_after();
-      const int r = q0 + 128 * i + row;
-      const bool live = r < q_end;
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * DH;
-#pragma unroll 1
-      for (int c = 0; c < DH; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(o_addr + c, o);
-        tmem_ld_wait();
-        if (live) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint4 u;
-            u.x = pack_bf16x2(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv);
-            u.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-            u.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
-            u.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
-            *reinterpret_cast<uint4*>(dst + c + e) = u;
-          }
-        }
-      }
-      if (live && lse != nullptr)
-        lse[static_cast<int64_t>(h) * L + r] = (m_used + log2f(l)) * 0.69314718055994531f;
-    } else {
-      record_status(status, kStatusTimeout);
-    }
+    softmax_warpgroup<DH>(
+        i, tmem, s_full, o_done, [&] { mbar_arrive(&p_half[i]); },
+        [&] { mbar_arrive(&p_ready[i]); }, kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse,
+        status, budget_ns);
   }
 
   tc_fence_before();
@@ -512,6 +546,272 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     tc_fence_after();
     mbar_wait(mma_done, 0, 200000000ull);
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- CTA-pair kernel
+//
+// Head dim 128 on the 2-SM MMA.  A cluster of two CTAs takes 512 query rows
+// of one segment and head (256 each: two 128-row tiles per CTA, as above).
+// S_i = Q_i K^T and O_i += P_i V are issued by the even CTA (the leader) as
+// cta_group::2 MMAs of M = 256: rows 0..127 are the leader's tile i, rows
+// 128..255 the odd CTA's, and each CTA receives its own rows in its own TMEM
+// (the same S0 S1 O0 O1 columns as the one-CTA kernel).  B is split between
+// the pair by N: per key tile the leader holds keys 0..63 and the odd CTA keys
+// 64..127 (all head dims) for S, and for PV the leader holds V columns 0..63
+// and the odd CTA columns 64..127 (all 128 keys).  Each CTA therefore loads
+// 32 KB per key tile instead of 64 KB, and each MMA reads its A rows and half
+// of B from each SM's shared memory: 6 KB per K = 16 step of S instead of
+// 8 KB, 2 KB per step of PV instead of 4 KB.
+//
+// Synchronisation: every TMA load of both CTAs completes on the leader's
+// full barriers (cta_group::2 loads, no multicast); the leader's MMA commits
+// arrive on both CTAs' barriers (S ready, O done, stage free, all done); the
+// softmax warps of both CTAs report P to the leader's barriers, one arrival
+// per warp.  Both CTAs initialise all barriers and meet at a cluster barrier
+// before the first load, and again before TMEM is released and they exit, so
+// neither leaves while the other may still touch its barriers or memory.
+template <int DH>
+struct WinPairCfg {
+  static_assert(DH == 128, "the pair kernel serves head dim 128");
+  static constexpr int SLABS = DH / 64;                 // 64-column slabs of a row
+  static constexpr int Q_TILE = SLABS * 128 * 128;      // 128 query rows x DH bf16
+  static constexpr int K_HALF = SLABS * 64 * 128;       // 64 keys x DH bf16
+  static constexpr int V_HALF = 128 * 128;              // 128 keys x 64 columns bf16
+  static constexpr int STAGE = K_HALF + V_HALF;
+  static constexpr int STAGES = 4;
+  static constexpr int THREADS = 384;
+  static constexpr int SMEM = 1024 + 2 * Q_TILE + STAGES * STAGE + 512;
+};
+
+template <int DH>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WinPairCfg<DH>::THREADS, 1)
+    window_attn_pair_kernel(const __grid_constant__ CUtensorMap qmap,
+                            const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap vmap,
+                            const __grid_constant__ CUtensorMap ckmap,
+                            const __grid_constant__ CUtensorMap cvmap, int m_ctx,
+                            const __grid_constant__ WinSched sched, int H, int L,
+                            float scale_log2, __nv_bfloat16* __restrict__ out, int64_t ld_o,
+                            float* __restrict__ lse, uint32_t* status, uint64_t budget_ns) {
+  using Cfg = WinPairCfg<DH>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* qbuf = smem;                              // Q0, Q1 of this CTA
+  uint8_t* kvbuf = smem + 2 * Cfg::Q_TILE;           // stage s: K half, then V half
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kvbuf + Cfg::STAGES * Cfg::STAGE);
+  uint64_t* q_full = bars;                           // leader: Q of both CTAs
+  uint64_t* k_full = bars + 1;                       // leader: [STAGES] both K halves
+  uint64_t* v_full = k_full + Cfg::STAGES;           // leader: [STAGES] both V halves
+  uint64_t* k_empty = v_full + Cfg::STAGES;          // both: [STAGES]
+  uint64_t* v_empty = k_empty + Cfg::STAGES;         // both: [STAGES]
+  uint64_t* s_full = v_empty + Cfg::STAGES;          // both: [2]
+  uint64_t* p_half = s_full + 2;                     // leader: [2], 8 warps
+  uint64_t* p_ready = p_half + 2;                    // leader: [2], 8 warps
+  uint64_t* o_done = p_ready + 2;                    // both: [2]
+  uint64_t* mma_done = o_done + 2;                   // both
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const uint32_t rank = cluster_ctarank();           // 0: leader, 1: its partner
+  const int pair_lin = blockIdx.x >> 1;
+  const int h = pair_lin / sched.total_pairs;
+  const int pair = pair_lin % sched.total_pairs;
+  int si = 0;
+  while (si + 1 < sched.nseg && pair >= sched.seg[si + 1].pair_base) ++si;
+  const WinSeg& seg = sched.seg[si];
+  // rows past the segment (the odd CTA of a segment's last pair may have
+  // none) are computed but never stored
+  const int q0 = seg.q0 + (pair - seg.pair_base) * 512 + static_cast<int>(rank) * 256;
+  const int q_end = seg.q1;
+  const int nkv = seg.nkv + (m_ctx + 127) / 128;
+  KvRange kr;
+  kr.load(seg, m_ctx);
+  const uint32_t warp = warp_id();
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_half[i], 8);
+      mbar_init(&p_ready[i], 8);
+      mbar_init(&o_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&qmap);
+    tma_prefetch_desc(&kmap);
+    tma_prefetch_desc(&vmap);
+    if (m_ctx > 0) {
+      tma_prefetch_desc(&ckmap);
+      tma_prefetch_desc(&cvmap);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any load or remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;\n" ::: "memory");
+  }
+  if (warp == 0) {
+    // ================================================================ TMA (both CTAs)
+    if (elect_one()) {
+      const uint32_t lq_full = mapa_shared(smem_u32(q_full), 0);
+      if (rank == 0) mbar_arrive_expect_tx(q_full, 4 * Cfg::Q_TILE);
+      for (int i = 0; i < 2; ++i)
+        for (int sl = 0; sl < Cfg::SLABS; ++sl)
+          tma_load_2d_pair(qbuf + i * Cfg::Q_TILE + sl * 16384, &qmap, lq_full,
+                           h * DH + 64 * sl, q0 + 128 * i);
+      KvCursor cur;
+      cur.init(kr);
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % Cfg::STAGES;
+        const uint32_t par = ((j / Cfg::STAGES) & 1) ^ 1;
+        uint8_t* kb = kvbuf + s * Cfg::STAGE;
+        const CUtensorMap* km = cur.ctx ? &ckmap : &kmap;
+        const CUtensorMap* vm = cur.ctx ? &cvmap : &vmap;
+        if (j >= Cfg::STAGES && !mbar_wait(&k_empty[s], par, budget_ns)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        // this CTA's 64 keys of the tile, every head-dim slab
+        if (rank == 0) mbar_arrive_expect_tx(&k_full[s], 2 * Cfg::K_HALF);
+        for (int sl = 0; sl < Cfg::SLABS; ++sl)
+          tma_load_2d_pair(kb + sl * 8192, km, mapa_shared(smem_u32(&k_full[s]), 0),
+                           h * DH + 64 * sl, cur.pos + 64 * static_cast<int>(rank));
+        if (j >= Cfg::STAGES && !mbar_wait(&v_empty[s], par, budget_ns)) {
+          record_status(status, kStatusTimeout);
+          break;
+        }
+        // all 128 keys of the tile, this CTA's 64 value columns
+        if (rank == 0) mbar_arrive_expect_tx(&v_full[s], 2 * Cfg::V_HALF);
+        tma_load_2d_pair(kb + Cfg::K_HALF, vm, mapa_shared(smem_u32(&v_full[s]), 0),
+                         h * DH + 64 * static_cast<int>(rank), cur.pos);
+        ++issued;
+        cur.next(kr);
+      }
+      // the leader's full barriers count both CTAs' bytes: wait for the last
+      // phases so that no load is in flight when the pair exits
+      if (rank == 0) {
+        mbar_wait(q_full, 0, 200000000ull);
+        for (int j = (issued > Cfg::STAGES ? issued - Cfg::STAGES : 0); j < issued; ++j) {
+          if (!mbar_wait(&k_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull) ||
+              !mbar_wait(&v_full[j % Cfg::STAGES], (j / Cfg::STAGES) & 1, 200000000ull))
+            record_status(status, kStatusTimeout);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA (leader)
+    if (rank == 0 && elect_one()) {
+      constexpr uint32_t idesc_s = idesc_bf16(256, 128, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16(256, DH, false, true);
+      constexpr uint16_t kBoth = 3;
+      const uint32_t qb = smem_u32(qbuf);
+      bool ok = mbar_wait(q_full, 0, budget_ns);
+      auto issue_s = [&](int i, int j) {
+        const uint32_t kb = smem_u32(kvbuf + (j % Cfg::STAGES) * Cfg::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          const uint32_t qoff = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t koff = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_ss_pair(tmem + 128 * i, sdesc_sw128(qb + i * Cfg::Q_TILE + qoff, 16, 1024),
+                       sdesc_sw128(kb + koff, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit_pair(&s_full[i], kBoth);
+      };
+      // O_i += P_i V for keys [16 k0, 16 k1) of the tile
+      auto issue_o = [&](int i, int j, int k0, int k1) {
+        const uint32_t vb = smem_u32(kvbuf + (j % Cfg::STAGES) * Cfg::STAGE + Cfg::K_HALF);
+        for (int kk = k0; kk < k1; ++kk)
+          umma_ts_pair(tmem + 256 + 128 * i, tmem + 128 * i + kk * 8,
+                       sdesc_sw128(vb + kk * 2048, 16384, 1024), idesc_o, (j > 0 || kk > 0));
+      };
+      if (ok && (ok = mbar_wait(&k_full[0], 0, budget_ns))) {
+        tc_fence_after();
+        issue_s(0, 0);
+        issue_s(1, 0);
+        umma_commit_pair(&k_empty[0], kBoth);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % Cfg::STAGES;
+        const bool more = j + 1 < nkv;
+        if (!(ok = mbar_wait(&v_full[s], (j / Cfg::STAGES) & 1, budget_ns))) break;
+        if (!(ok = mbar_wait(&p_half[0], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(0, j, 0, 2 * VDN_P_EARLY_CHUNKS);
+        if (!(ok = mbar_wait(&p_ready[0], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(0, j, 2 * VDN_P_EARLY_CHUNKS, 8);
+        umma_commit_pair(&o_done[0], kBoth);
+        if (more) {
+          const int sn = (j + 1) % Cfg::STAGES;
+          if (!(ok = mbar_wait(&k_full[sn], ((j + 1) / Cfg::STAGES) & 1, budget_ns))) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
+        }
+        if (!(ok = mbar_wait(&p_half[1], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(1, j, 0, 2 * VDN_P_EARLY_CHUNKS);
+        if (!(ok = mbar_wait(&p_ready[1], j & 1, budget_ns))) break;
+        tc_fence_after();
+        issue_o(1, j, 2 * VDN_P_EARLY_CHUNKS, 8);
+        umma_commit_pair(&o_done[1], kBoth);
+        umma_commit_pair(&v_empty[s], kBoth);
+        if (more) {
+          issue_s(1, j + 1);
+          umma_commit_pair(&k_empty[(j + 1) % Cfg::STAGES], kBoth);
+        }
+      }
+      if (!ok) record_status(status, kStatusTimeout);
+      umma_commit_pair(mma_done, kBoth);
+    }
+  } else if (warp >= 4) {
+    // ================================================================ softmax (both CTAs)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
+    const int i = (warp - 4) >> 2;  // query tile of this warpgroup
+    const uint32_t lp_half = mapa_shared(smem_u32(&p_half[i]), 0);
+    const uint32_t lp_ready = mapa_shared(smem_u32(&p_ready[i]), 0);
+    // one arrival per warp on the leader's barrier, after every lane's TMEM
+    // stores have completed (tcgen05.wait::st and the fence precede it)
+    softmax_warpgroup<DH>(
+        i, tmem, s_full, o_done,
+        [&] {
+          __syncwarp();
+          if (lane_id() == 0) mbar_arrive_cluster(lp_half);
+        },
+        [&] {
+          __syncwarp();
+          if (lane_id() == 0) mbar_arrive_cluster(lp_ready);
+        },
+        kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse, status, budget_ns);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // the leader's MMAs read this CTA's shared memory and write its TMEM
+    tc_fence_after();
+    mbar_wait(mma_done, 0, 200000000ull);
+  }
+  cluster_sync();  // neither CTA leaves while the other may still reach it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -564,7 +864,7 @@ bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSch
   std::stable_sort(raw.begin(), raw.end(), [](const Raw& a, const Raw& b) { return a.work > b.work; });
   memset(out, 0, sizeof(*out));
   out->nseg = static_cast<int>(raw.size());
-  int base = 0;
+  int base = 0, pbase = 0;
   for (size_t k = 0; k < raw.size(); ++k) {
     WinSeg& g = out->seg[k];
     g.q0 = raw[k].f0 * s.N;
@@ -572,6 +872,9 @@ bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSch
     g.ntiles = (g.q1 - g.q0 + 255) / 256;
     g.tile_base = base;
     base += g.ntiles;
+    g.npairs = (g.ntiles + 1) / 2;
+    g.pair_base = pbase;
+    pbase += g.npairs;
     g.nint = static_cast<int>(raw[k].runs.size());
     g.nkv = 0;
     for (int v = 0; v < g.nint; ++v) {
@@ -581,6 +884,7 @@ bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSch
     }
   }
   out->total_tiles = base;
+  out->total_pairs = pbase;
   return true;
 }
 
@@ -597,6 +901,24 @@ cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtens
   window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
       qmap, kmap, vmap, ckmap, cvmap, m_ctx, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
       static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+// Head dim 128 on the CTA-pair kernel.  kmap_half / ckmap_half read 64-key
+// boxes (each CTA of a pair loads half of a 128-key tile).
+cudaError_t launch_window_pair(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                               const CUtensorMap& kmap_half, const CUtensorMap& vmap,
+                               const CUtensorMap& ckmap_half, const CUtensorMap& cvmap,
+                               int m_ctx, const WinSched& sched, float scale, void* o,
+                               int64_t ld_o, float* lse) {
+  using Cfg = WinPairCfg<128>;
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(window_attn_pair_kernel<128>, Cfg::SMEM, smem_set)) return e;
+  const int grid = 2 * sched.total_pairs * s.H;  // a multiple of the cluster size
+  window_attn_pair_kernel<128><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, kmap_half, vmap, ckmap_half, cvmap, m_ctx, sched, s.H, s.T * s.N,
+      scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status,
+      ctx.budget_ns);
   return cudaGetLastError();
 }
 
@@ -677,7 +999,8 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
   }
   thread_local WinSched sched;  // ~12 KB; copied into the launch's parameters
   if (!build_schedule(s, chunk_frames, window_chunks, anchors, &sched)) return VDN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(sched.total_tiles) * s.H >= (int64_t(1) << 31))
+  if (static_cast<int64_t>(sched.total_tiles) * s.H >= (int64_t(1) << 31) ||
+      2 * static_cast<int64_t>(sched.total_pairs) * s.H >= (int64_t(1) << 31))
     return VDN_ERR_UNSUPPORTED;
   const int64_t L = static_cast<int64_t>(s.T) * s.N;
   CUtensorMap qmap, kmap, vmap, ckmap, cvmap;
@@ -694,6 +1017,19 @@ vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, const void
   }
   Launch ctx{static_cast<cudaStream_t>(stream), static_cast<uint32_t*>(ws),
              current_wait_budget_ns()};
+  if (VDN_WINDOW_PAIR && s.d == 128) {
+    CUtensorMap kmap_half, ckmap_half;
+    if (!make_rows_map(&kmap_half, k, D, ld, L, 64)) return VDN_ERR_CUDA;
+    if (m_ctx > 0) {
+      if (!make_rows_map(&ckmap_half, ctx_k, D, ld_ctx, m_ctx, 64)) return VDN_ERR_CUDA;
+    } else {
+      ckmap_half = kmap_half;  // unused
+    }
+    return launch_window_pair(ctx, s, qmap, kmap_half, vmap, ckmap_half, cvmap, m_ctx, sched, sc,
+                              o, ld_o, lse_opt) == cudaSuccess
+               ? VDN_OK
+               : VDN_ERR_CUDA;
+  }
   cudaError_t e = s.d == 128 ? launch_window_dh<128>(ctx, s, qmap, kmap, vmap, ckmap, cvmap, m_ctx,
                                                      sched, sc, o, ld_o, lse_opt)
                              : launch_window_dh<64>(ctx, s, qmap, kmap, vmap, ckmap, cvmap, m_ctx,
