@@ -8,7 +8,8 @@ timed region starts; each activation (2.5 GB) is larger than L2, so no L2
 flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload layer102|layer42|small] [--part all|layer|vda_backward]
+                    [--workload layer102|layer42|small]
+                    [--part all|layer|vda_backward|fuse_mxfp8|scan_sweep]
 
 The line also carries two rows timed on their own, not part of the step:
 ``vda_backward``, the VDA gradient pass (dq, dk, dv, dbeta, dalpha from
@@ -16,7 +17,9 @@ dL/do_vda, forward recomputed inside), and ``fuse_mxfp8``, the fuse with
 both projection GEMMs in MXFP8 (x quantized inside the timed call, weights
 quantized beforehand), against the FP8 peak and beside the bf16 fuse's
 output.  ``--part vda_backward`` / ``--part fuse_mxfp8`` time only that
-row (for launch lists and captures).
+row (for launch lists and captures).  ``--part scan_sweep`` times the VDA
+branch alone at every point of the scan-only sweep (T 42/72/102 x N
+1008/4032 x d 64/128 x H 24/48), each against its roofline.
 
 With N > 1 (torchrun) every rank runs its own video (independent problems,
 no collective on the data path): weak scaling, time = max over ranks.
@@ -424,6 +427,56 @@ def run_fuse_mxfp8(args, shape, rank, world):
     return ms, dev_rel
 
 
+def run_scan_sweep(args, rank, world, peaks):
+    """The VDA branch alone (prep, solve, both scans, read-out: one
+    vdn_vda_scan call) at every point of the scan-only sweep, each timed with
+    CUDA events over `steps` calls after `warmup`; one row per point with its
+    roofline (HBM bytes at the measured copy bandwidth plus FP32 work at the
+    FP32 peak, the same terms as the layer's VDA row)."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for shape in synth.sweep_shapes():
+        T, N, H, d = shape.T, shape.N, shape.H, shape.d
+        inp = synth.make_inputs(shape, seed=rank, device=dev)
+        out = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
+        ws = vdn.alloc_workspace(vdn.vda_scan_workspace(T, N, H, d), dev)
+
+        def call():
+            vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
+                         out=out, ws=ws, stream=stream)
+
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for a, b in evs:
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if vdn.get_device_status(ws) != 0:
+            raise RuntimeError("device status after the sweep point %s" % (shape,))
+        ms = max_over_ranks([statistics.median(a.elapsed_time(b) for a, b in evs)], dev,
+                            world)[0]
+        w = work_model(shape)
+        roof_ms = (w["vda_bytes"] / (peaks["hbm_gbs"] * 1e9) +
+                   w["vda_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3
+        rows.append({"T": T, "N": N, "d": d, "H": H, "ms": ms,
+                     "tokens_per_s": shape.L / (ms / 1e3), "roofline_ms": roof_ms,
+                     "frac": roof_ms / ms, "hbm_bytes": w["vda_bytes"],
+                     "fp32_alu_flop": w["vda_alu_flop"]})
+        del inp, out, ws
+        torch.cuda.empty_cache()
+    return rows
+
+
 def mxfp8_row(work, peaks, ms, dev_rel):
     peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     tf = work["proj_flop"] / (ms / 1e3) / 1e12
@@ -455,7 +508,7 @@ def main():
     ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
                     help="solver of (I + A)^-1 in the VDA branch")
     ap.add_argument("--part", default="all",
-                    choices=["all", "layer", "vda_backward", "fuse_mxfp8"],
+                    choices=["all", "layer", "vda_backward", "fuse_mxfp8", "scan_sweep"],
                     help="what to time: the layer step and the two side rows (all), or one "
                          "of them")
     args = ap.parse_args()
@@ -506,6 +559,22 @@ def main():
                               "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                               "dtype": "bf16", "data": "synthetic", "config": config,
                               "vda_backward": backward_row(work, peaks, ms, ms_saved)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
+    if args.part == "scan_sweep":
+        rows = run_scan_sweep(args, rank, world, peaks)
+        if rank == 0:
+            print(json.dumps({"metric": "VDA branch ms and tokens/s over the scan-only sweep "
+                                        "(prep, solve, both scans, read-out)",
+                              "value": statistics.median(r["frac"] for r in rows),
+                              "unit": "median fraction of roofline", "higher_is_better": True,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "dtype": "bf16 inputs, fp32 state", "data": "synthetic",
+                              "config": {"workload": "vda_scan_sweep T{42,72,102} x "
+                                                     "N{1008,4032} x d{64,128} x H{24,48}",
+                                         "timing": "median of steps, CUDA events"},
+                              "rows": rows}))
         if world > 1:
             torch.distributed.destroy_process_group()
         return
