@@ -23,6 +23,9 @@ branch alone at every point of the scan-only sweep (T 42/72/102 x N
 
 With N > 1 (torchrun) every rank runs its own video (independent problems,
 no collective on the data path): weak scaling, time = max over ranks.
+``--parallel seq`` instead splits one video over the ranks by token rows,
+with the attention branches run head-parallel between two all-to-alls
+(strong scaling; on one GPU a one-rank group).
 ``--impl reference`` times the float64 CPU oracle instead, on a bounded
 sample of the same workload, extrapolated by work.
 """
@@ -153,6 +156,15 @@ def max_over_ranks(values, device, world):
     t = torch.tensor(values, dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return t.tolist()
+
+
+def free_port():
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    return port
 
 
 def weak_scaling_value(world, tokens_per_rank, ms_per_step):
@@ -310,6 +322,47 @@ def run_gpu(args, shape, rank, world):
     return dict(ms=ms, win_ms=t[2] / args.steps, vda_ms=t[3] / args.steps,
                 fuse_ms=t[4] / args.steps, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
                 clocks=clocks, launches=layer.kernels_per_forward * args.steps)
+
+
+def run_seq_sharded(args, shape, rank, world):
+    """One video split over the ranks (SeqShardedLayer): each rank holds a
+    block of token rows; all-to-alls move its heads' rows in and the branch
+    outputs back; time of `steps` layer passes, max over ranks."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=0, device=dev, with_fuse=True)
+    layer = vdn.SeqShardedLayer(shape.T, shape.N, shape.H, shape.d, inp["W_gs"], inp["W_gl"],
+                                inp["W_os"], inp["W_ol"], inp["gamma"], device=dev)
+    r = layer.rows
+    mine = [inp[n][r].contiguous() for n in ("q", "k", "v", "beta")] + \
+        [inp["alpha"], inp["x"][r].contiguous()]
+    del inp
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        layer.forward(*mine)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = clocks_start()
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        layer.forward(*mine)
+    end.record(stream)
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = clocks_stop(clk)
+    if max(get_status(w) for w in layer.workspaces) != 0:
+        raise RuntimeError("device status after the sharded steps")
+    ms = max_over_ranks([start.elapsed_time(end)], dev, world)[0]
+    return ms / args.steps, clocks
+
+
+def get_status(ws):
+    from video_diffusion_hybrid_vda_b200 import vdn
+    return vdn.get_device_status(ws)
 
 
 def run_vda_backward(args, shape, rank, world):
@@ -507,6 +560,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
                     help="solver of (I + A)^-1 in the VDA branch")
+    ap.add_argument("--parallel", default="videos", choices=["videos", "seq"],
+                    help="with several GPUs: every rank runs its own video (videos, weak "
+                         "scaling), or one video is split over the ranks by token rows with "
+                         "head-parallel attention in between (seq, strong scaling)")
     ap.add_argument("--part", default="all",
                     choices=["all", "layer", "vda_backward", "fuse_mxfp8", "scan_sweep"],
                     help="what to time: the layer step and the two side rows (all), or one "
@@ -551,6 +608,23 @@ def main():
             "nccl", device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
             timeout=__import__("datetime").timedelta(seconds=300))
     peaks, peak_kind = load_peaks()
+    if args.parallel == "seq":
+        if world == 1:
+            torch.distributed.init_process_group(
+                "nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:%d" % free_port(),
+                device_id=torch.device("cuda", 0))
+        ms, clocks = run_seq_sharded(args, shape, rank, world)
+        if rank == 0:
+            config.update({"global_batch": 1, "parallelism": f"sequence x{world}, "
+                           "head-parallel attention (all-to-all)"})
+            print(json.dumps({
+                "metric": METRIC, "value": shape.L / (ms / 1e3), "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config,
+                "gpu_launches": 7 * args.steps, "clocks": clocks}))
+        torch.distributed.destroy_process_group()
+        return
     if args.part == "vda_backward":
         ms, ms_saved = run_vda_backward(args, shape, rank, world)
         if rank == 0:

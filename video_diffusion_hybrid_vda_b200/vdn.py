@@ -7,6 +7,7 @@ device memory and the stream.  If the library is missing, every call raises
 """
 
 import ctypes
+import functools
 import os
 
 import torch
@@ -656,19 +657,25 @@ class HybridLayer:
 
 
 class HeadShardedLayer:
-    """One video's hybrid layer split by heads over a process group.
+    """One video's hybrid layer split by heads over a process group, for a
+    caller that holds the full activations on every rank.
 
     Rank r of G owns heads [r H/G, (r+1) H/G).  The window Softmax and VDA
     branches are per head, so each rank runs them on its own head columns
     (views into the full [T*N, D] activations) with no communication; the
     fuse is row-parallel: each rank forms its hidden columns of the gated
     branch inputs and an fp32 partial of y over the full width
-    (vdn_hybrid_fuse_shard), and the partials are summed across ranks with
-    one all-reduce.  ``ops`` replaces the four compute calls (tests only).
+    (vdn_hybrid_fuse_shard).  One reduce-scatter sums the partials and leaves
+    rank r the rows [r R, (r+1) R) of y, R = ceil(T*N / G) (the fp32 sum adds
+    no bf16 rounding; each rank receives 1/G of the sum instead of all of
+    it).  ``output="rows"`` returns that row block in bf16, ``output="full"``
+    also all-gathers the bf16 blocks into the whole y on every rank.
+    ``ops`` replaces the compute calls (tests only).
     """
 
     def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, group=None,
-                 device=None, ops=None, act_dtype=torch.bfloat16, acc_dtype=torch.float32):
+                 device=None, ops=None, act_dtype=torch.bfloat16, acc_dtype=torch.float32,
+                 output="full"):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -676,25 +683,44 @@ class HeadShardedLayer:
         self.world = dist.get_world_size(group)
         if H % self.world:
             raise ValueError("heads must divide evenly over the ranks")
+        if output not in ("rows", "full"):
+            raise ValueError("output: 'rows' or 'full'")
+        self.output = output
         self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
         self.L, self.D = self.T * self.N, self.H * self.d
         self.Hl = self.H // self.world
         self.head0 = self.rank * self.Hl
         self.cols = slice(self.head0 * self.d, (self.head0 + self.Hl) * self.d)
+        self.R = -(-self.L // self.world)           # rows of y each rank receives
+        self.rows = slice(min(self.rank * self.R, self.L), min((self.rank + 1) * self.R, self.L))
         self.device = torch.device(device) if device is not None else torch.device("cuda")
         dev = self.device
         self.W = [w.to(dev, act_dtype).contiguous() for w in (W_gs, W_gl, W_os, W_ol)]
         self.gamma = gamma.to(dev, acc_dtype).contiguous()
         self.eps = float(eps)
-        self.ops = ops or {"window_attn": window_attn, "vda_scan": vda_scan,
-                           "fuse_shard": hybrid_fuse_shard}
         Dl = self.Hl * self.d
+        if ops is None:
+            Hl, d = self.Hl, self.d
+            ws_win = alloc_workspace(window_attn_workspace(T, N, Hl, d), dev)
+            ws_vda = alloc_workspace(vda_scan_workspace(T, N, Hl, d), dev)
+            ws_fuse = alloc_workspace(
+                int(lib().vdn_hybrid_fuse_shard_workspace(self.L, self.D, Hl, d)), dev)
+            ops = {"window_attn": functools.partial(window_attn, ws=ws_win),
+                   "vda_scan": functools.partial(vda_scan, ws=ws_vda),
+                   "fuse_shard": functools.partial(hybrid_fuse_shard, ws=ws_fuse)}
+            self.workspaces = (ws_win, ws_vda, ws_fuse)
+        self.ops = ops
         self.o_s = torch.empty((self.L, Dl), dtype=act_dtype, device=dev)
         self.o_vda = torch.empty((self.L, Dl), dtype=act_dtype, device=dev)
-        self.y_partial = torch.empty((self.L, self.D), dtype=acc_dtype, device=dev)
-        self.y = torch.empty((self.L, self.D), dtype=act_dtype, device=dev)
+        # G*R rows so that every rank's block has R rows; rows past L stay zero
+        self.y_partial = torch.zeros((self.world * self.R, self.D), dtype=acc_dtype, device=dev)
+        self.y_rows32 = torch.empty((self.R, self.D), dtype=acc_dtype, device=dev)
+        self.y_rows = torch.empty((self.R, self.D), dtype=act_dtype, device=dev)
+        self.y = (torch.empty((self.world * self.R, self.D), dtype=act_dtype, device=dev)
+                  if output == "full" else None)
 
     def forward(self, q, k, v, beta, alpha, x):
+        """y (full, [T*N, D]) or this rank's rows of y ([rows, D], rows = self.rows)."""
         c, Hl, d = self.cols, self.Hl, self.d
         h0, h1 = self.head0, self.head0 + self.Hl
         ql, kl, vl = q[:, c], k[:, c], v[:, c]             # views, row stride D
@@ -703,7 +729,96 @@ class HeadShardedLayer:
         self.ops["window_attn"](ql, kl, vl, self.T, self.N, Hl, d, out=self.o_s)
         self.ops["vda_scan"](ql, kl, vl, beta_l, alpha_l, self.T, self.N, Hl, d, out=self.o_vda)
         self.ops["fuse_shard"](x, self.o_s, self.o_vda, *self.W[:2], self.gamma, *self.W[2:], d,
-                               h0, eps=self.eps, out=self.y_partial)
-        self.dist.all_reduce(self.y_partial, group=self.group)
-        self.y.copy_(self.y_partial)
+                               h0, eps=self.eps, out=self.y_partial[:self.L])
+        self.dist.reduce_scatter_tensor(self.y_rows32, self.y_partial, group=self.group)
+        self.y_rows.copy_(self.y_rows32)                    # fp32 sum -> bf16
+        if self.output == "rows":
+            return self.y_rows[:self.rows.stop - self.rows.start]
+        self.dist.all_gather_into_tensor(self.y, self.y_rows, group=self.group)
+        return self.y[:self.L]
+
+
+class SeqShardedLayer:
+    """One video's hybrid layer for a caller whose activations are split by
+    token rows over a process group (sequence parallelism), with the
+    attention run head-parallel in between (all-to-all, Ulysses style).
+
+    Rank r of G holds token rows [r R, (r+1) R) of q, k, v, x and beta,
+    R = T*N / G, and the whole alpha.  One all-to-all per tensor gives every
+    rank all T*N rows of its H/G heads; the window Softmax and VDA run there
+    (both need every token of a head and nothing of the other heads); an
+    all-to-all per branch output brings the rows back; the fuse then runs on
+    the rank's own rows with the full weights (gates, RMSNorm and both
+    projections are per token), so no reduction is needed.  Bytes each rank
+    sends per layer: (G-1)/G of 5 activations' row blocks (q, k, v out, o_s,
+    o_vda back) plus beta.  The column blocks are packed into and out of the
+    contiguous all-to-all buffers with copies.  ``ops`` replaces the compute
+    calls (tests only).
+    """
+
+    def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, group=None,
+                 device=None, ops=None, act_dtype=torch.bfloat16, acc_dtype=torch.float32):
+        import torch.distributed as dist
+        self.dist = dist
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = G = dist.get_world_size(group)
+        self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
+        self.L, self.D = self.T * self.N, self.H * self.d
+        if self.H % G or self.L % G:
+            raise ValueError("heads and token rows must divide evenly over the ranks")
+        self.R, self.Hl = self.L // G, self.H // G
+        self.C = self.Hl * self.d
+        self.head0 = self.rank * self.Hl
+        self.rows = slice(self.rank * self.R, (self.rank + 1) * self.R)
+        self.device = torch.device(device) if device is not None else torch.device("cuda")
+        dev = self.device
+        self.W = [w.to(dev, act_dtype).contiguous() for w in (W_gs, W_gl, W_os, W_ol)]
+        self.gamma = gamma.to(dev, acc_dtype).contiguous()
+        self.eps = float(eps)
+        L, R, C, D = self.L, self.R, self.C, self.D
+        if ops is None:
+            Hl, d = self.Hl, self.d
+            ws_win = alloc_workspace(window_attn_workspace(T, N, Hl, d), dev)
+            ws_vda = alloc_workspace(vda_scan_workspace(T, N, Hl, d), dev)
+            ws_fuse = alloc_workspace(hybrid_fuse_workspace(R, D, self.H), dev)
+            ops = {"window_attn": functools.partial(window_attn, ws=ws_win),
+                   "vda_scan": functools.partial(vda_scan, ws=ws_vda),
+                   "fuse": functools.partial(hybrid_fuse, ws=ws_fuse)}
+            self.workspaces = (ws_win, ws_vda, ws_fuse)
+        self.ops = ops
+        mk = lambda *shape, dt=act_dtype: torch.empty(shape, dtype=dt, device=dev)
+        self.send = [mk(G, R, C) for _ in range(3)]          # q, k, v column blocks
+        self.heads = [mk(L, C) for _ in range(3)]            # all rows of this rank's heads
+        self.beta_send, self.beta_l = mk(G, R, self.Hl, dt=acc_dtype), mk(L, self.Hl, dt=acc_dtype)
+        self.o_s, self.o_vda = mk(L, C), mk(L, C)             # branch outputs, this rank's heads
+        self.back = [mk(G, R, C) for _ in range(2)]          # their column blocks of my rows
+        self.o_s_rows, self.o_vda_rows = mk(R, D), mk(R, D)
+        self.y = mk(R, D)
+
+    def _to_heads(self, src, send, recv, width):
+        """[R, G*width] row block -> [G*R, width]: all rows of this rank's columns."""
+        G, R = self.world, self.R
+        send.copy_(src.reshape(R, G, width).transpose(0, 1))
+        self.dist.all_to_all_single(recv.view(G, R, width), send, group=self.group)
+
+    def forward(self, q, k, v, beta, alpha, x):
+        """This rank's rows of y ([R, D]) from its rows of q, k, v, x ([R, D]),
+        beta ([R, H]) and the whole alpha ([T, H])."""
+        G, R, C, Hl, d = self.world, self.R, self.C, self.Hl, self.d
+        for src, send, recv in zip((q, k, v), self.send, self.heads):
+            self._to_heads(src, send, recv, C)
+        self._to_heads(beta, self.beta_send, self.beta_l, Hl)
+        alpha_l = alpha[:, self.head0:self.head0 + Hl].contiguous()
+        ql, kl, vl = self.heads
+        self.ops["window_attn"](ql, kl, vl, self.T, self.N, Hl, d, out=self.o_s)
+        self.ops["vda_scan"](ql, kl, vl, self.beta_l, alpha_l, self.T, self.N, Hl, d,
+                             out=self.o_vda)
+        for o, back, rows in zip((self.o_s, self.o_vda), self.back,
+                                 (self.o_s_rows, self.o_vda_rows)):
+            # chunk g of o holds rank g's rows: it goes back to rank g
+            self.dist.all_to_all_single(back, o.view(G, R, C), group=self.group)
+            rows.view(R, G, C).copy_(back.transpose(0, 1))
+        self.ops["fuse"](x, self.o_s_rows, self.o_vda_rows, self.W[0], self.W[1], self.gamma,
+                         self.W[2], self.W[3], self.H, eps=self.eps, out=self.y)
         return self.y
