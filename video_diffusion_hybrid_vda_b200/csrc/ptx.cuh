@@ -409,6 +409,42 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
                : "memory");
 }
 
+// Arrive on a barrier of another CTA of the cluster, releasing at cluster
+// scope everything this thread has written or observed (through an acquire)
+// before, for a consumer in that CTA that reads this CTA's shared memory.
+__device__ __forceinline__ void mbar_arrive_release_cluster(uint32_t bar_cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   bar_cluster_addr)
+               : "memory");
+}
+
+// mbar_wait that acquires at cluster scope: the pairing side of
+// mbar_arrive_release_cluster, for a thread that then lets the tensor core
+// read the other CTA's shared memory.
+__device__ __forceinline__ bool mbar_test_acquire_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_acquire_cluster(uint64_t* bar, uint32_t parity,
+                                                          uint64_t budget_ns) {
+  if (mbar_test_acquire_cluster(bar, parity)) return true;
+  if (budget_ns == 0) return false;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (true) {
+    if (mbar_test_acquire_cluster(bar, parity)) return true;
+    if ((++n & 63u) == 0 && globaltimer_ns() - t0 > budget_ns) return false;
+  }
+}
+
 // Every thread of every CTA of the cluster arrives and waits.
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");

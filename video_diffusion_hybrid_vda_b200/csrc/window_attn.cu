@@ -166,12 +166,18 @@ struct KvCursor {
 // decision), writes P = 2^(s - m) over S as bf16 in two halves (reporting
 // each half through arrive_half / arrive_ready), and at the end normalises
 // O_i by the row sum and stores the row (and its log-sum-exp).
-template <int DH, class ArriveHalf, class ArriveReady>
+//
+// P_SMEM: P goes to this warpgroup's tile `pbuf` in shared memory (bf16,
+// K-major, 128-byte swizzle, two 64-key slabs) instead of back over S in
+// TMEM, so S_i is free once it has been loaded (reported through s_free)
+// and the next S_i product overlaps this tile's exponentials; before writing
+// P the warpgroup waits for the previous tile's PV product (it reads pbuf).
+template <int DH, bool P_SMEM, class ArriveHalf, class ArriveReady, class SFree>
 __device__ __forceinline__ void softmax_warpgroup(
     int i, uint32_t tmem, uint64_t* s_full, uint64_t* o_done, ArriveHalf arrive_half,
-    ArriveReady arrive_ready, const KvRange& kr, int nkv, float scale_log2, int q0, int q_end,
-    int h, int L, __nv_bfloat16* __restrict__ out, int64_t ld_o, float* __restrict__ lse,
-    uint32_t* status, uint64_t budget_ns) {
+    ArriveReady arrive_ready, SFree s_free, uint8_t* pbuf, const KvRange& kr, int nkv,
+    float scale_log2, int q0, int q_end, int h, int L, __nv_bfloat16* __restrict__ out,
+    int64_t ld_o, float* __restrict__ lse, uint32_t* status, uint64_t budget_ns) {
   const uint32_t quarter = warp_id() & 3;
   const int row = quarter * 32 + lane_id();
   const uint32_t lane_off = (quarter * 32) << 16;
@@ -224,6 +230,10 @@ __device__ __forceinline__ void softmax_warpgroup(
     tmem_ld_wait();
     reg_fence(s2);
     reg_fence(s3);
+    if constexpr (P_SMEM) {
+      tc_fence_before();
+      s_free();  // all of S_i is in registers: the next S_i may overwrite it
+    }
     if (valid < 128) {
 #pragma unroll
       for (int c = 64; c < 128; ++c)
@@ -270,6 +280,11 @@ __device__ __forceinline__ void softmax_warpgroup(
     const uint64_t cc = f32x2_pack(scale_log2, scale_log2);
     const uint64_t nm = f32x2_pack(-m_used, -m_used);
     uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+    // P_SMEM: the row's 128 probabilities stay in registers (64 packed
+    // words, reusing the scores' registers as they die) until the previous
+    // tile's PV product has read pbuf, which is waited for only after the
+    // exponentials
+    uint32_t pall[P_SMEM ? 64 : 1];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       uint32_t pk[16];
@@ -288,17 +303,43 @@ __device__ __forceinline__ void softmax_warpgroup(
         acc2[e & 3] = f32x2_add(acc2[e & 3], pp);
         pk[e] = pack_bf16x2(f32x2_lo(pp), f32x2_hi(pp));
       }
-      tmem_st16(s_addr + 16 * q, pk);
-      if (q == VDN_P_EARLY_CHUNKS - 1) {
-        tmem_st_wait();
-        tc_fence_before();
-        arrive_half();
+      if constexpr (P_SMEM) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pall[16 * q + e] = pk[e];
+      } else {
+        tmem_st16(s_addr + 16 * q, pk);
+        if (q == VDN_P_EARLY_CHUNKS - 1) {
+          tmem_st_wait();
+          tc_fence_before();
+          arrive_half();
+        }
       }
     }
     acc2[0] = f32x2_add(f32x2_add(acc2[0], acc2[1]), f32x2_add(acc2[2], acc2[3]));
     l += f32x2_lo(acc2[0]) + f32x2_hi(acc2[0]);
-    tmem_st_wait();
-    tc_fence_before();
+    if constexpr (P_SMEM) {
+      // pbuf is read by the previous tile's PV product
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done[i], (j - 1) & 1, budget_ns))) {
+        ok = false;
+        break;
+      }
+      // keys 32q .. 32q+31 of this row: four 16-byte chunks of slab q / 2
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint8_t* slab = pbuf + (q >> 1) * 16384 + row * 128;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t c = 4 * (q & 1) + m;
+          *reinterpret_cast<uint4*>(slab + ((c ^ (row & 7)) << 4)) =
+              make_uint4(pall[16 * q + 4 * m], pall[16 * q + 4 * m + 1],
+                         pall[16 * q + 4 * m + 2], pall[16 * q + 4 * m + 3]);
+        }
+      }
+      fence_proxy_async_smem();  // the tensor core reads pbuf through the async proxy
+    } else {
+      tmem_st_wait();
+      tc_fence_before();
+    }
     arrive_ready();
   }
   // ------------------------------------------------------------ epilogue
@@ -534,10 +575,10 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     // ================================================================ softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
     const int i = (warp - 4) >> 2;  // query tile of this warpgroup
-    softmax_warpgroup<DH>(
+    softmax_warpgroup<DH, false>(
         i, tmem, s_full, o_done, [&] { mbar_arrive(&p_half[i]); },
-        [&] { mbar_arrive(&p_ready[i]); }, kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse,
-        status, budget_ns);
+        [&] { mbar_arrive(&p_ready[i]); }, [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, L,
+        out, ld_o, lse, status, budget_ns);
   }
 
   tc_fence_before();
@@ -788,7 +829,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WinPairCfg<DH>::THRE
     const uint32_t lp_ready = mapa_shared(smem_u32(&p_ready[i]), 0);
     // one arrival per warp on the leader's barrier, after every lane's TMEM
     // stores have completed (tcgen05.wait::st and the fence precede it)
-    softmax_warpgroup<DH>(
+    softmax_warpgroup<DH, false>(
         i, tmem, s_full, o_done,
         [&] {
           __syncwarp();
@@ -798,7 +839,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WinPairCfg<DH>::THRE
           __syncwarp();
           if (lane_id() == 0) mbar_arrive_cluster(lp_ready);
         },
-        kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse, status, budget_ns);
+        [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse, status,
+        budget_ns);
   }
 
   tc_fence_before();
