@@ -121,3 +121,82 @@ def hybrid_fuse_mxfp8(x, o_s, o_vda, W_gs, W_gl, gamma, eps, W_os, W_ol, H):
     zq = mx_quantize(Z)
     woq = mx_quantize(np.concatenate([W_os, W_ol], axis=1))
     return gemm_mx(*zq, *woq)
+
+
+# ---------------------------------------------------------------- window Softmax
+
+def mx_quantize_columns(x):
+    """MX quantization along the rows of x [R, C] (R a multiple of 32): blocks
+    of 32 consecutive rows of each column, as for the value operand of the PV
+    product (its contraction runs over key tokens).  Returns the dequantized
+    values [R, C]."""
+    codes, scales = mx_quantize(np.asarray(x, dtype=np.float64).T)
+    return mx_dequantize(codes, scales).T
+
+
+def window_attn_mxfp8_rows(q, k, v, T, N, H, d, rows, chunk_frames=5, window_chunks=1,
+                           anchors=3, scale=None, heads=None):
+    """Window-and-anchor Softmax with both products on MXFP8 operands, for the
+    given query token rows.  Returns (o [len(rows), H*d], lse [H, len(rows)]).
+
+    Every operand is quantized in blocks of 32 along the contraction of its
+    product (OCP MX, as ``mx_quantize``):
+      * q and k per token and head along d (the S = q k^T contraction);
+      * v per column along the key tokens, in blocks of 32 consecutive token
+        rows counted from row 0 (the P V contraction);
+      * the probabilities per query row along the keys, in blocks of 32
+        consecutive keys of each visible key interval.
+    With s = q^ . k^ * scale, s2 = s log2(e) and m = ceil(max over the row's
+    visible keys of s2) (an integer, so the block quantization of P does not
+    depend on which upper bound of the row maximum is subtracted):
+      P = 2^(s2 - m),  l = sum P,  o = sum_keys P^ v^ / l,
+      lse = (m + log2 l) ln 2.
+    The row sum l is taken over the unquantized P.  The visible key
+    intervals (whole frames) start and end on multiples of 32, i.e. N is a
+    multiple of 32.
+    """
+    if N % 32 or d % 32:
+        raise ValueError("tokens per frame and head dim must be multiples of 32")
+    from .window_attn import visible_key_frames
+    scale = 1.0 / np.sqrt(d) if scale is None or scale <= 0 else float(scale)
+    rows = np.asarray(rows, dtype=np.int64)
+    heads = range(H) if heads is None else heads
+    out = np.zeros((len(rows), H * d))
+    lse = np.zeros((H, len(rows)))
+    frames = rows // N
+    log2e = 1.0 / np.log(2.0)
+    for h in heads:
+        c = slice(h * d, (h + 1) * d)
+        kq_cache, vq_cache = {}, {}
+
+        def quantized_frames(tk):
+            # a frame's keys and values: 32-aligned row blocks of the tensor
+            if tk not in kq_cache:
+                r = slice(tk * N, (tk + 1) * N)
+                kq_cache[tk] = mx_dequantize(*mx_quantize(np.asarray(k[r, c], dtype=np.float64)))
+                vq_cache[tk] = mx_quantize_columns(np.asarray(v[r, c], dtype=np.float64))
+            return kq_cache[tk], vq_cache[tk]
+
+        for tq in np.unique(frames):
+            sel = np.nonzero(frames == tq)[0]
+            kf = visible_key_frames(int(tq), T, chunk_frames, window_chunks, anchors)
+            Kq = np.vstack([quantized_frames(tk)[0] for tk in kf])
+            Vq = np.vstack([quantized_frames(tk)[1] for tk in kf])
+            Qq = mx_dequantize(*mx_quantize(np.asarray(q[rows[sel], c], dtype=np.float64)))
+            s2 = (Qq @ Kq.T) * scale * log2e
+            m = np.ceil(s2.max(axis=1, keepdims=True))
+            P = np.exp2(s2 - m)
+            l = P.sum(axis=1, keepdims=True)
+            # blocks of 32 keys: the keys are whole frames of N (a multiple of
+            # 32) tokens, so consecutive 32-key groups of the row are the blocks
+            Pq = mx_dequantize(*mx_quantize(P))
+            out[sel, c] = (Pq @ Vq) / l
+            lse[h, sel] = (m[:, 0] + np.log2(l[:, 0])) / log2e
+    return out, lse
+
+
+def window_attn_mxfp8(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3,
+                      scale=None):
+    """window_attn_mxfp8_rows for every token row."""
+    return window_attn_mxfp8_rows(q, k, v, T, N, H, d, np.arange(T * N), chunk_frames,
+                                  window_chunks, anchors, scale)

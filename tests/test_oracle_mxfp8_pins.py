@@ -5,6 +5,7 @@ known maxima, the quantization error bound, and the tile layout of the
 scale bytes on hand-computed offsets."""
 
 import numpy as np
+import pytest
 import torch
 
 from oracle import mxfp8
@@ -166,3 +167,83 @@ def test_fuse_quantizes_the_gated_branch_inputs():
     expect[0, 3], expect[0, 40], expect[0, 64], expect[0, 70], expect[0, 100] = (
         1.125, 1.25, 3.0, 1.125, 1.0)
     np.testing.assert_array_equal(y, expect)
+
+
+# ---------------------------------------------------------------- window Softmax
+
+def _dense_mxfp8_window(q, k, v, T, N, d, scale):
+    """One head of the MXFP8 window Softmax written densely, independently of
+    the oracle's interval loop: an explicit [L, L] frame mask, operands
+    quantized as whole tensors (q, k along d per row; v along the token rows
+    per column), and P quantized in blocks of 32 over each full row of L keys
+    (masked keys are 0 there; the visible intervals are 32-aligned, so no block
+    mixes visible and masked keys)."""
+    import oracle
+    L = T * N
+    vis = np.array([[oracle.frame_visible(r // N, c // N, T) for c in range(L)]
+                    for r in range(L)])
+    qq = mxfp8.mx_dequantize(*mxfp8.mx_quantize(q))
+    kq = mxfp8.mx_dequantize(*mxfp8.mx_quantize(k))
+    vc, vs = mxfp8.mx_quantize(v.T)
+    vq = mxfp8.mx_dequantize(vc, vs).T
+    s2 = np.where(vis, (qq @ kq.T) * scale / np.log(2.0), -np.inf)
+    m = np.ceil(s2.max(axis=1, keepdims=True))
+    P = np.where(vis, np.exp2(s2 - m), 0.0)
+    Pq = mxfp8.mx_dequantize(*mxfp8.mx_quantize(P))
+    l = P.sum(axis=1, keepdims=True)
+    return (Pq @ vq) / l, (m[:, 0] + np.log2(l[:, 0])) * np.log(2.0)
+
+
+@pytest.mark.parametrize("T,N,d", [(17, 32, 64), (12, 64, 32), (6, 32, 32)])
+def test_window_mxfp8_equals_dense_brute_force(T, N, d):
+    rng = np.random.default_rng(T * 7 + N)
+    H = 2
+    L = T * N
+    q, k, v = (rng.standard_normal((L, H * d)) for _ in range(3))
+    o, lse = mxfp8.window_attn_mxfp8(q, k, v, T, N, H, d)
+    for h in range(H):
+        c = slice(h * d, (h + 1) * d)
+        o_ref, lse_ref = _dense_mxfp8_window(q[:, c], k[:, c], v[:, c], T, N, d,
+                                             1.0 / np.sqrt(d))
+        np.testing.assert_allclose(o[:, c], o_ref, rtol=1e-11, atol=1e-11)
+        np.testing.assert_allclose(lse[h], lse_ref, rtol=1e-11, atol=1e-11)
+
+
+def test_window_mxfp8_uniform_scores_give_the_window_mean():
+    """Special case that reduces to the float64 window Softmax exactly: k = 0
+    gives equal scores, so P = 1 everywhere (exact in E4M3 under its block
+    scale) and the output is the mean of the visible values; small integers
+    in v are exact under any block scale of their block (|v| <= 8), so the
+    MXFP8 result equals the unquantized one."""
+    import oracle
+    rng = np.random.default_rng(11)
+    T, N, H, d = 17, 32, 2, 32
+    L = T * N
+    q = rng.standard_normal((L, H * d))
+    k = np.zeros((L, H * d))
+    v = rng.integers(-8, 9, (L, H * d)).astype(np.float64)
+    o, lse = mxfp8.window_attn_mxfp8(q, k, v, T, N, H, d)
+    o_ref, lse_ref = oracle.window_attn(q, k, v, T, N, H, d)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_window_mxfp8_near_the_exact_softmax_on_layer_like_inputs():
+    """What the format costs: on inputs drawn like the layer's (q, v ~ N(0, 1),
+    keys L2-normalised per token and head) the MXFP8 window Softmax stays
+    within a few per cent (max over the output, relative to max |o|) of the
+    float64 one (measured 5.4 % max, 3.9 % RMS: the probabilities of these
+    nearly flat rows sit in one binade, where E4M3 steps are 1/8, and the
+    output is an average of ~1000 values, small against max |v|)."""
+    import oracle
+    rng = np.random.default_rng(12)
+    T, N, H, d = 17, 64, 2, 128
+    L = T * N
+    q, v = rng.standard_normal((L, H * d)), rng.standard_normal((L, H * d))
+    k = rng.standard_normal((L, H, d))
+    k = (k / np.linalg.norm(k, axis=2, keepdims=True)).reshape(L, H * d)
+    rows = np.arange(0, L, 7)
+    o, _ = mxfp8.window_attn_mxfp8_rows(q, k, v, T, N, H, d, rows)
+    o_ref, _ = oracle.window_attn_rows(q, k, v, T, N, H, d, rows)
+    err = np.abs(o - o_ref).max() / np.abs(o_ref).max()
+    assert 1e-3 < err < 0.1
