@@ -276,6 +276,37 @@ VDN_API vdn_status vdn_window_attn_ctx(const vdn_shape* shape, const void* q, co
                                        float scale, void* o, int64_t ld_o, float* lse_opt,
                                        void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Window-and-anchor Softmax with MXFP8 products (10100.com article: the
+ * window Softmax of 方法概述 item 1, run under the MXFP8 inference of
+ * 实验结果 / 效率阶梯; the pages name the format only, the OCP Microscaling
+ * definition is taken: E4M3 elements, one UE8M0 power-of-two scale per 32
+ * elements along each product's contraction).
+ *
+ * Same mask and arguments as vdn_window_attn, and the same bf16 output; the
+ * call quantizes into the workspace, then runs the attention:
+ *   q, k : blocks of 32 along the head dim, per token and head;
+ *   v    : blocks of 32 consecutive token rows (from row 0), per column;
+ *   P    : blocks of 32 consecutive keys of a row, with P = 2^(s log2 e - m)
+ *          for an integer row maximum m; the row sum adds the unquantized P,
+ *          the output is sum(P^ v^) / sum(P).
+ * lse_opt: NULL or fp32 [H, L], the natural log of the row sum of exp(s).
+ * Supported: head dim 128 and N (tokens per frame) a multiple of 32, so
+ * every visible key interval starts on a value block (else
+ * VDN_ERR_UNSUPPORTED); no context keys.
+ * ws: >= vdn_window_attn_mxfp8_workspace(shape) bytes, 256-byte aligned:
+ *   status word, the E4M3 codes of q, k, v (3 x L x H*d bytes) and their
+ *   scale bytes (2 x L x H*d/32 + ceil(L/32) x H*d).
+ * Errors as for vdn_window_attn.
+ * ------------------------------------------------------------------------ */
+VDN_API size_t vdn_window_attn_mxfp8_workspace(const vdn_shape* shape);
+
+VDN_API vdn_status vdn_window_attn_mxfp8(const vdn_shape* shape, const void* q, const void* k,
+                                         const void* v, int64_t ld, int chunk_frames,
+                                         int window_chunks, unsigned anchors, float scale,
+                                         void* o, int64_t ld_o, float* lse_opt, void* ws,
+                                         size_t ws_bytes, void* stream);
+
 /* The window Softmax's work plan, as the kernel launch uses it (host only:
  * no CUDA call, no device memory).  Consecutive query frames with the same
  * visible key frames (the mask of vdn_window_attn) form a segment; segments

@@ -34,12 +34,12 @@
 #include "exp2_fma.cuh"
 #include "ptx.cuh"
 #include "repack.cuh"
+#include "window_sched.cuh"
 
 namespace vdn {
 
 namespace {
 
-constexpr int kMaxSegs = 256;
 
 // P is stored in four 32-key chunks; the PV product of the first this-many
 // chunks is issued as soon as they are stored, the rest once the row is done.
@@ -63,24 +63,6 @@ static_assert(VDN_EXP2_FMA_PAIRS == 0 || VDN_EXP2_FMA_PAIRS == 2 || VDN_EXP2_FMA
                   VDN_EXP2_FMA_PAIRS == 8,
               "VDN_EXP2_FMA_PAIRS must divide 16 pairs evenly");
 
-struct WinSeg {
-  int q0, q1;      // query token rows [q0, q1)
-  int tile_base;   // first CTA tile index of this segment (launch order)
-  int ntiles;      // 256-row CTA tiles
-  int pair_base;   // first CTA-pair index of this segment (pair kernel)
-  int npairs;      // 512-row CTA pairs
-  int nint;        // key intervals (1..3)
-  int k0[3], k1[3];
-  int nkv;         // 128-key tiles over all intervals
-};
-
-struct WinSched {
-  int nseg;
-  int total_tiles;
-  int total_pairs;
-  WinSeg seg[kMaxSegs];
-};
-
 template <int DH>
 struct WinCfg {
   static constexpr int SLABS = DH / 64;
@@ -88,76 +70,6 @@ struct WinCfg {
   static constexpr int STAGES = 2;
   static constexpr int THREADS = 384;
   static constexpr int SMEM = 1024 + 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 512;
-};
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-// Compiler-level fence: uses of r cannot be scheduled before this point
-// (placed right after tcgen05.wait::ld, which makes the loaded values valid).
-__device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
-                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31]));
-}
-
-// The key intervals of one segment, held in registers, and a cursor over
-// its 128-key tiles (start row, number of valid keys).
-struct KvRange {
-  int nint, a0, a1, a2, b0, b1, b2;
-  int mctx;  // context (text/audio) keys, visible to every query, after the video keys
-  __device__ void load(const WinSeg& s, int m_ctx) {
-    mctx = m_ctx;
-    nint = s.nint;
-    a0 = s.k0[0];
-    a1 = s.k0[1];
-    a2 = s.k0[2];
-    b0 = s.k1[0];
-    b1 = s.k1[1];
-    b2 = s.k1[2];
-  }
-  __device__ int start(int iv) const { return iv == 0 ? a0 : (iv == 1 ? a1 : a2); }
-  __device__ int end(int iv) const { return iv == 0 ? b0 : (iv == 1 ? b1 : b2); }
-};
-
-struct KvCursor {
-  int iv, pos, end;
-  bool ctx;  // true once the cursor walks the context keys
-  __device__ void init(const KvRange& r) {
-    iv = 0;
-    pos = r.a0;
-    end = r.b0;
-    ctx = false;
-  }
-  __device__ void next(const KvRange& r) {
-    pos += 128;
-    if (pos >= end && !ctx) {
-      if (iv + 1 < r.nint) {
-        ++iv;
-        pos = r.start(iv);
-        end = r.end(iv);
-      } else if (r.mctx > 0) {
-        ctx = true;
-        pos = 0;
-        end = r.mctx;
-      }
-    }
-  }
-  __device__ int valid() const { return min(128, end - pos); }
 };
 
 // One softmax warpgroup (tile i of the CTA's two 128-row query tiles): one
@@ -881,6 +793,44 @@ std::vector<std::pair<int, int>> key_runs(int tq, int T, int cf, int wc, unsigne
   return runs;
 }
 
+template <int DH>
+cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                             const CUtensorMap& kmap, const CUtensorMap& vmap,
+                             const CUtensorMap& ckmap, const CUtensorMap& cvmap, int m_ctx,
+                             const WinSched& sched, float scale, void* o, int64_t ld_o,
+                             float* lse) {
+  using Cfg = WinCfg<DH>;
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(window_attn_kernel<DH>, Cfg::SMEM, smem_set)) return e;
+  const int grid = sched.total_tiles * s.H;
+  window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, kmap, vmap, ckmap, cvmap, m_ctx, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
+      static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status, ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+// Head dim 128 on the CTA-pair kernel.  kmap_half / ckmap_half read 64-key
+// boxes (each CTA of a pair loads half of a 128-key tile).
+cudaError_t launch_window_pair(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
+                               const CUtensorMap& kmap_half, const CUtensorMap& vmap,
+                               const CUtensorMap& ckmap_half, const CUtensorMap& cvmap,
+                               int m_ctx, const WinSched& sched, float scale, void* o,
+                               int64_t ld_o, float* lse) {
+  using Cfg = WinPairCfg<128>;
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = set_smem_once(window_attn_pair_kernel<128>, Cfg::SMEM, smem_set)) return e;
+  const int grid = 2 * sched.total_pairs * s.H;  // a multiple of the cluster size
+  window_attn_pair_kernel<128><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, kmap_half, vmap, ckmap_half, cvmap, m_ctx, sched, s.H, s.T * s.N,
+      scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status,
+      ctx.budget_ns);
+  return cudaGetLastError();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
 bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSched* out) {
   struct Raw {
     int f0, f1;
@@ -930,43 +880,6 @@ bool build_schedule(const vdn_shape& s, int cf, int wc, unsigned anchors, WinSch
   return true;
 }
 
-template <int DH>
-cudaError_t launch_window_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
-                             const CUtensorMap& kmap, const CUtensorMap& vmap,
-                             const CUtensorMap& ckmap, const CUtensorMap& cvmap, int m_ctx,
-                             const WinSched& sched, float scale, void* o, int64_t ld_o,
-                             float* lse) {
-  using Cfg = WinCfg<DH>;
-  static std::atomic<uint64_t> smem_set{0};
-  if (cudaError_t e = set_smem_once(window_attn_kernel<DH>, Cfg::SMEM, smem_set)) return e;
-  const int grid = sched.total_tiles * s.H;
-  window_attn_kernel<DH><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, kmap, vmap, ckmap, cvmap, m_ctx, sched, s.H, s.T * s.N, scale * 1.4426950408889634f,
-      static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status, ctx.budget_ns);
-  return cudaGetLastError();
-}
-
-// Head dim 128 on the CTA-pair kernel.  kmap_half / ckmap_half read 64-key
-// boxes (each CTA of a pair loads half of a 128-key tile).
-cudaError_t launch_window_pair(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
-                               const CUtensorMap& kmap_half, const CUtensorMap& vmap,
-                               const CUtensorMap& ckmap_half, const CUtensorMap& cvmap,
-                               int m_ctx, const WinSched& sched, float scale, void* o,
-                               int64_t ld_o, float* lse) {
-  using Cfg = WinPairCfg<128>;
-  static std::atomic<uint64_t> smem_set{0};
-  if (cudaError_t e = set_smem_once(window_attn_pair_kernel<128>, Cfg::SMEM, smem_set)) return e;
-  const int grid = 2 * sched.total_pairs * s.H;  // a multiple of the cluster size
-  window_attn_pair_kernel<128><<<grid, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, kmap_half, vmap, ckmap_half, cvmap, m_ctx, sched, s.H, s.T * s.N,
-      scale * 1.4426950408889634f, static_cast<__nv_bfloat16*>(o), ld_o, lse, ctx.status,
-      ctx.budget_ns);
-  return cudaGetLastError();
-}
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-}  // namespace
 }  // namespace vdn
 
 using namespace vdn;

@@ -30,7 +30,8 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_vda_backward_workspace", "vdn_vda_backward", "vdn_vda_backward_debug_buffers",
            "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
            "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8",
-           "vdn_hybrid_fuse_shard_rs", "vdn_window_attn_schedule"]
+           "vdn_hybrid_fuse_shard_rs", "vdn_window_attn_schedule",
+           "vdn_window_attn_mxfp8_workspace", "vdn_window_attn_mxfp8"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -130,6 +131,11 @@ def lib():
     L.vdn_hybrid_fuse_mxfp8.argtypes = [ctypes.c_int] * 3 + [_P] * 6 + [ctypes.c_float, _P, _P,
                                                                          _P, _P, _SZ, _P]
     L.vdn_hybrid_fuse_mxfp8.restype = ctypes.c_int
+    L.vdn_window_attn_mxfp8_workspace.argtypes = [S]
+    L.vdn_window_attn_mxfp8_workspace.restype = _SZ
+    L.vdn_window_attn_mxfp8.argtypes = [S, _P, _P, _P, _I64, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_uint, ctypes.c_float, _P, _I64, _P, _P, _SZ, _P]
+    L.vdn_window_attn_mxfp8.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -435,6 +441,28 @@ def window_attn(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3,
                                          _ptr(out), out.stride(0), _ptr(lse), _ptr(ws),
                                          ws.numel(), _stream(stream))
         _check(code, "vdn_window_attn_ctx")
+    return out, ws
+
+
+def window_attn_mxfp8_workspace(T, N, H, d):
+    return int(lib().vdn_window_attn_mxfp8_workspace(ctypes.byref(_shape(T, N, H, d))))
+
+
+def window_attn_mxfp8(q, k, v, T, N, H, d, chunk_frames=5, window_chunks=1, anchors=3,
+                      scale=0.0, out=None, lse=None, ws=None, stream=None):
+    """Window-and-anchor Softmax with both products on MXFP8 operands (q, k,
+    v quantized into the workspace by the call).  Returns (o, ws)."""
+    _need_cuda(q, k, v, out, lse, ws)
+    shape = _shape(T, N, H, d)
+    if out is None:
+        out = torch.empty((T * N, H * d), dtype=torch.bfloat16, device=q.device)
+    if ws is None:
+        ws = alloc_workspace(window_attn_mxfp8_workspace(T, N, H, d), q.device)
+    code = lib().vdn_window_attn_mxfp8(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v),
+                                       q.stride(0), int(chunk_frames), int(window_chunks),
+                                       int(anchors), float(scale), _ptr(out), out.stride(0),
+                                       _ptr(lse), _ptr(ws), ws.numel(), _stream(stream))
+    _check(code, "vdn_window_attn_mxfp8")
     return out, ws
 
 
