@@ -9,15 +9,18 @@ flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload layer102|layer42|small]
-                    [--part all|layer|vda_backward|fuse_mxfp8|scan_sweep]
+                    [--part all|layer|vda_backward|fuse_mxfp8|window_mxfp8|scan_sweep]
 
-The line also carries two rows timed on their own, not part of the step:
+The line also carries three rows timed on their own, not part of the step:
 ``vda_backward``, the VDA gradient pass (dq, dk, dv, dbeta, dalpha from
-dL/do_vda, forward recomputed inside), and ``fuse_mxfp8``, the fuse with
+dL/do_vda, forward recomputed inside); ``fuse_mxfp8``, the fuse with
 both projection GEMMs in MXFP8 (x quantized inside the timed call, weights
 quantized beforehand), against the FP8 peak and beside the bf16 fuse's
-output.  ``--part vda_backward`` / ``--part fuse_mxfp8`` time only that
-row (for launch lists and captures).  ``--part scan_sweep`` times the VDA
+output; and ``window_mxfp8``, the window Softmax with both products in
+MXFP8 (q, k, v quantized inside the timed call), against its FP8 tensor and
+MUFU bounds and beside the bf16 window Softmax's output.  ``--part
+vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` time only that row (for
+launch lists and captures).  ``--part scan_sweep`` times the VDA
 branch alone at every point of the scan-only sweep (T 42/72/102 x N
 1008/4032 x d 64/128 x H 24/48), each against its roofline.
 
@@ -57,6 +60,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # FP32 (non-tensor) peak from unit counts and clocks: 148 SMs x 128 FMA/clk x
 # 2 FLOP x 1.965 GHz (clocks.max.sm)
 FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+# MUFU exponentials from unit counts and clocks: 148 SMs x 16 per clock x 1.965 GHz
+MUFU_EXP_PER_S = 148 * 16 * 1.965e9
 KERNEL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "window_attn_traffic.json")
 
 
@@ -87,7 +92,7 @@ def work_model(s):
     # two adjoint scans (2 d^3 each) and the combine (two d^3 products, 4 d^3)
     vda_bwd_bytes = 7 * s.L * s.D * 2 + 2 * s.L * s.H * 4
     vda_bwd_alu_flop = vda_alu_flop + s.T * s.H * (4 * s.d ** 3 + 4 * s.d ** 3)
-    return dict(pairs=pairs, softmax_flop=softmax_flop, proj_flop=proj_flop,
+    return dict(pairs=pairs, heads=s.H, softmax_flop=softmax_flop, proj_flop=proj_flop,
                 vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop, vda_bwd_bytes=vda_bwd_bytes,
                 vda_bwd_alu_flop=vda_bwd_alu_flop)
 
@@ -480,6 +485,66 @@ def run_fuse_mxfp8(args, shape, rank, world):
     return ms, dev_rel
 
 
+def run_window_mxfp8(args, shape, rank, world):
+    """Device time of the MXFP8 window Softmax (quantization of q, k, v and
+    the attention; ms, max over ranks) and the max relative deviation of its
+    output from the bf16 window Softmax's on the same inputs."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev)
+    T, N, H, d = shape.T, shape.N, shape.H, shape.d
+    o = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
+    ws = vdn.alloc_workspace(vdn.window_attn_mxfp8_workspace(T, N, H, d), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        vdn.window_attn_mxfp8(inp["q"], inp["k"], inp["v"], T, N, H, d, out=o, ws=ws,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the MXFP8 window warm-up")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    o_bf16, _ = vdn.window_attn(inp["q"], inp["k"], inp["v"], T, N, H, d)
+    dev_rel = float(((o.float() - o_bf16.float()).abs().max() /
+                     o_bf16.float().abs().max()).item())
+    del inp, o, ws, o_bf16
+    torch.cuda.empty_cache()
+    return ms, dev_rel
+
+
+def window_mxfp8_row(work, peaks, ms, dev_rel):
+    """The MXFP8 window Softmax against its two bounds: FP8 tensor work at
+    2 x the measured sustained bf16 rate, and one MUFU exponential per
+    visible (query, key) pair at the MUFU rate from unit counts and the
+    maximum clock (16 per clock per SM, 148 SMs, 1965 MHz)."""
+    peak = 2.0 * peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    tensor_ms = work["softmax_flop"] / (peak * 1e12) * 1e3
+    exps = work["pairs"] * work["heads"]
+    mufu_ms = exps / MUFU_EXP_PER_S * 1e3
+    bound_ms = max(tensor_ms, mufu_ms)
+    tf = work["softmax_flop"] / (ms / 1e3) / 1e12
+    return {"ms": ms, "bound": "mufu" if mufu_ms >= tensor_ms else "tensor",
+            "roofline_ms": bound_ms, "frac": bound_ms / ms, "achieved_tflops": tf,
+            "tensor_ms": tensor_ms, "fp8_peak_tflops": peak, "mufu_ms": mufu_ms,
+            "exponentials": exps, "max_rel_vs_bf16_window": dev_rel,
+            "launches_per_call": 4,
+            "note": "q, k, v quantized inside the timed call (3 launches) + the attention"}
+
+
 def run_scan_sweep(args, rank, world, peaks):
     """The VDA branch alone (prep, solve, both scans, read-out: one
     vdn_vda_scan call) at every point of the scan-only sweep, each timed with
@@ -565,7 +630,8 @@ def main():
                          "scaling), or one video is split over the ranks by token rows with "
                          "head-parallel attention in between (seq, strong scaling)")
     ap.add_argument("--part", default="all",
-                    choices=["all", "layer", "vda_backward", "fuse_mxfp8", "scan_sweep"],
+                    choices=["all", "layer", "vda_backward", "fuse_mxfp8", "window_mxfp8",
+                             "scan_sweep"],
                     help="what to time: the layer step and the two side rows (all), or one "
                          "of them")
     args = ap.parse_args()
@@ -652,6 +718,18 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
+    if args.part == "window_mxfp8":
+        ms, dev_rel = run_window_mxfp8(args, shape, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "MXFP8 window Softmax ms (q, k, v quantized inside)",
+                              "value": ms, "unit": "ms", "higher_is_better": False,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "dtype": "mxfp8 (e4m3, ue8m0 / 32)", "data": "synthetic",
+                              "config": config,
+                              "window_mxfp8": window_mxfp8_row(work, peaks, ms, dev_rel)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.part == "fuse_mxfp8":
         ms, dev_rel = run_fuse_mxfp8(args, shape, rank, world)
         if rank == 0:
@@ -717,6 +795,8 @@ def main():
         line["vda_backward"] = backward_row(work, peaks,
                                             *run_vda_backward(args, shape, rank, world))
         line["fuse_mxfp8"] = mxfp8_row(work, peaks, *run_fuse_mxfp8(args, shape, rank, world))
+        line["window_mxfp8"] = window_mxfp8_row(work, peaks,
+                                                *run_window_mxfp8(args, shape, rank, world))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(shape)
         line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}

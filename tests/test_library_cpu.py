@@ -196,3 +196,25 @@ def test_window_context_entry_rejects_bad_arguments_on_host(L):
     assert ctx(wc=-1) == 1
     assert ctx(anchors=4) == 1
     assert ctx(ws=0) == 3
+
+
+def test_window_mxfp8_rejects_bad_arguments_on_host(L):
+    """Validation before any CUDA call: null pointers, head dims other than
+    128, tokens per frame not a multiple of 32, a missing workspace."""
+    import ctypes
+    lib = L.lib()
+    P = lambda a: ctypes.c_void_p(a)
+    f = lib.vdn_window_attn_mxfp8
+    sh = L.Shape(4, 64, 2, 128)
+    assert f(ctypes.byref(sh), None, P(16), P(16), 256, 5, 1, 3, 0.0, P(16), 256, None, P(256),
+             1 << 30, None) == 1
+    sh_d = L.Shape(4, 64, 2, 64)
+    assert f(ctypes.byref(sh_d), P(16), P(16), P(16), 128, 5, 1, 3, 0.0, P(16), 128, None,
+             P(256), 1 << 30, None) == 2
+    sh_n = L.Shape(4, 40, 2, 128)
+    assert f(ctypes.byref(sh_n), P(16), P(16), P(16), 256, 5, 1, 3, 0.0, P(16), 256, None,
+             P(256), 1 << 30, None) == 2
+    assert f(ctypes.byref(sh), P(16), P(16), P(16), 256, 5, 1, 3, 0.0, P(16), 256, None,
+             None, 0, None) == 3
+    assert lib.vdn_window_attn_mxfp8_workspace(ctypes.byref(sh)) == \
+        256 + 3 * 256 * 256 + 2 * 256 * 8 + 8 * 256

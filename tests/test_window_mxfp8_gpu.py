@@ -133,3 +133,29 @@ def test_window_mxfp8_refuses_unsupported_shapes(vdn):
         with pytest.raises(vdn.VdnError) as e:
             vdn.window_attn_mxfp8(t, t, t, T, N, 1, d, ws=vdn.alloc_workspace(1 << 20))
         assert e.value.code == 2        # VDN_ERR_UNSUPPORTED
+
+
+def test_hybrid_layer_all_mxfp8(vdn):
+    """HybridLayer(softmax="mxfp8", projections="mxfp8"): the Softmax branch
+    against the oracle's MXFP8 window Softmax, y against the oracle's MXFP8
+    fuse on the layer's own branch outputs, and the host-copy path
+    (forward_many) giving the same y."""
+    s = synth.Shape(12, 96, 2, 128)
+    inp = synth.make_inputs(s, seed=8, device="cuda", with_fuse=True)
+    layer = vdn.HybridLayer(s.T, s.N, s.H, s.d, inp["W_gs"], inp["W_gl"], inp["W_os"],
+                            inp["W_ol"], inp["gamma"], projections="mxfp8", softmax="mxfp8")
+    acts = [inp[k] for k in ("q", "k", "v", "beta", "alpha", "x")]
+    y = layer.forward(*acts).clone()
+    assert layer.status() == 0
+    x = {k: host(inp[k]) for k in ("q", "k", "v")}
+    o_ref, _ = omx.window_attn_mxfp8(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d)
+    assert per_head_max_rel(host(layer.o_s), o_ref, s.H, s.d) <= TOL_BF16
+    y_ref = omx.hybrid_fuse_mxfp8(host(inp["x"]), host(layer.o_s), host(layer.o_vda),
+                                  host(inp["W_gs"]), host(inp["W_gl"]), host(inp["gamma"]), 1e-6,
+                                  host(inp["W_os"]), host(inp["W_ol"]), s.H)
+    assert np.abs(host(y) - y_ref).max() / np.abs(y_ref).max() <= TOL_BF16
+    hosts = [[t.cpu().pin_memory() for t in acts]]
+    outs = [torch.empty((s.L, s.D), dtype=torch.bfloat16).pin_memory()]
+    layer.forward_many(hosts, outs)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], y.cpu())

@@ -541,13 +541,15 @@ class HybridLayer:
     copies): host inputs are copied into device buffers owned by the layer
     and, when ``out`` is a host tensor, y is copied back into it.
     ``projections="mxfp8"`` runs both fuse GEMMs on MXFP8 operands (weights
-    quantized once here, x on every call).
+    quantized once here, x on every call); ``softmax="mxfp8"`` runs the
+    window Softmax with both products on MXFP8 operands (q, k, v quantized
+    on every call; head dim 128, tokens per frame a multiple of 32).
     """
 
     KERNELS_PER_FORWARD = 7   # prep, solve, scan, read-out, window Softmax, 2 GEMMs
 
     def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, chunk_frames=5,
-                 window_chunks=1, anchors=3, device=None, projections="bf16"):
+                 window_chunks=1, anchors=3, device=None, projections="bf16", softmax="bf16"):
         self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
         self.L, self.D = self.T * self.N, self.H * self.d
         self.device = torch.device(device or "cuda")
@@ -562,7 +564,12 @@ class HybridLayer:
         self.o_vda = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
         self.y = torch.empty((L, D), dtype=torch.bfloat16, device=dev)
         self.ws_vda = alloc_workspace(vda_scan_workspace(T, N, H, d), dev)
-        self.ws_win = alloc_workspace(window_attn_workspace(T, N, H, d), dev)
+        if softmax not in ("bf16", "mxfp8"):
+            raise ValueError("softmax: 'bf16' or 'mxfp8'")
+        self.softmax = softmax
+        self.ws_win = alloc_workspace(
+            window_attn_mxfp8_workspace(T, N, H, d) if softmax == "mxfp8"
+            else window_attn_workspace(T, N, H, d), dev)
         if projections not in ("bf16", "mxfp8"):
             raise ValueError("projections: 'bf16' or 'mxfp8'")
         self.projections = projections
@@ -574,7 +581,21 @@ class HybridLayer:
         else:
             self.ws_fuse = alloc_workspace(hybrid_fuse_workspace(L, D, H), dev)
             self.kernels_per_forward = self.KERNELS_PER_FORWARD
+        if softmax == "mxfp8":
+            self.kernels_per_forward += 3  # quantization of q, k, v
         self._staging = None
+
+    def _window(self, q, k, v, stream, ctx_k=None, ctx_v=None):
+        T, N, H, d = self.T, self.N, self.H, self.d
+        cf, wc, an = self.mask
+        if self.softmax == "mxfp8":
+            if ctx_k is not None:
+                raise ValueError("the MXFP8 window Softmax takes no context keys")
+            window_attn_mxfp8(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win,
+                              stream=stream)
+        else:
+            window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win,
+                        stream=stream, ctx_k=ctx_k, ctx_v=ctx_v)
 
     def _fuse(self, x, y, stream):
         if self.projections == "mxfp8":
@@ -601,9 +622,7 @@ class HybridLayer:
         stream = stream or torch.cuda.current_stream(self.device)
         q, k, v, beta, alpha, x = self._to_device([q, k, v, beta, alpha, x], stream)
         T, N, H, d = self.T, self.N, self.H, self.d
-        cf, wc, an = self.mask
-        window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win, stream=stream,
-                    ctx_k=ctx_k, ctx_v=ctx_v)
+        self._window(q, k, v, stream, ctx_k, ctx_v)
         vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda, stream=stream)
         self._fuse(x, self.y, stream)
         if out is not None and not out.is_cuda:
@@ -642,7 +661,6 @@ class HybridLayer:
         loaded = [torch.cuda.Event() for _ in batches]
         computed = [torch.cuda.Event() for _ in batches]
         T, N, H, d = self.T, self.N, self.H, self.d
-        cf, wc, an = self.mask
 
         def load(i):
             with torch.cuda.stream(copy_stream):
@@ -664,8 +682,7 @@ class HybridLayer:
                 stream.wait_event(self._read[i - 2])           # y buffer i % 2 is free
             q, k, v, beta, alpha, x = stages[i % 2]
             y = ys[i % 2]
-            window_attn(q, k, v, T, N, H, d, cf, wc, an, out=self.o_s, ws=self.ws_win,
-                        stream=stream)
+            self._window(q, k, v, stream)
             stream.wait_event(loaded[i])                        # beta, alpha, x
             vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
                      stream=stream)
