@@ -28,7 +28,8 @@
 // next S_i product runs during this tile's exponentials.
 //
 // Warps: 0 TMA and scale gathers (all lanes), 1 MMA issue, 4-7 softmax of
-// query tile 0, 8-11 of tile 1 (one thread per query row).
+// query tile 0, 8-11 of tile 1 (one thread per query row).  A quarter of the
+// exponentials run on the FMA pipe (see VDN_MX_EXP2_FMA_PAIRS).
 #include <math.h>
 
 #include "common.cuh"
@@ -62,6 +63,25 @@ static_assert(WinMxCfg::STAGE % 1024 == 0, "stages keep 1024-byte alignment");
 // Instruction descriptor of the block-scaled MMA with B MN-major (bit 16).
 __host__ __device__ constexpr uint32_t idesc_mxf8_bmn(int M, int N) {
   return idesc_mxf8(M, N) | (1u << 16);
+}
+
+// Of every 16 score pairs of a 32-key block, this many take the FMA-pipe
+// exponential (exp2_fma.cuh; relative error 7.5e-5, far below the E4M3 step
+// P is rounded to) and the rest the MUFU.  With the tensor work halved by
+// FP8 the MUFU is this kernel's busiest unit; measured at 102 frames x 4032 x
+// 24 x 128 (CUDA events, one B200): 0 -> 326.0 ms, 4 -> 308.0 ms, 6 -> 319.7
+// ms, 8 -> 332.6 ms.
+#ifndef VDN_MX_EXP2_FMA_PAIRS
+#define VDN_MX_EXP2_FMA_PAIRS 4
+#endif
+static_assert(VDN_MX_EXP2_FMA_PAIRS == 0 || VDN_MX_EXP2_FMA_PAIRS == 4 ||
+                  VDN_MX_EXP2_FMA_PAIRS == 8,
+              "VDN_MX_EXP2_FMA_PAIRS: 0, 4 or 8 of 16 pairs");
+
+__device__ __forceinline__ bool mx_exp2_on_fma(int pair) {
+  if (VDN_MX_EXP2_FMA_PAIRS == 4) return (pair & 3) == 3;
+  if (VDN_MX_EXP2_FMA_PAIRS == 8) return (pair & 1) == 1;
+  return false;
 }
 
 // Scale bytes 0..2 of a row (or column) packed with byte 3 unused (unit scale).
@@ -192,7 +212,15 @@ __device__ __forceinline__ void softmax_mx(int i, uint32_t tmem, uint64_t* s_ful
           const int c0 = 32 * q + 2 * (e2 + u);
           const uint64_t xs =
               f32x2_fma((static_cast<uint64_t>(sr[c0 + 1]) << 32) | sr[c0], cc, nb);
-          const float y0 = exp2_mufu(f32x2_lo(xs)), y1 = exp2_mufu(f32x2_hi(xs));
+          float y0, y1;
+          if (mx_exp2_on_fma(e2 + u)) {
+            const uint64_t yy = exp2_fma_x2(xs);
+            y0 = f32x2_lo(yy);
+            y1 = f32x2_hi(yy);
+          } else {
+            y0 = exp2_mufu(f32x2_lo(xs));
+            y1 = exp2_mufu(f32x2_hi(xs));
+          }
           acc2[u] = f32x2_add(acc2[u], f32x2_pack(y0, y1));
           h2[u] = static_cast<uint32_t>(
               __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3));
