@@ -159,3 +159,46 @@ def test_hybrid_layer_all_mxfp8(vdn):
     layer.forward_many(hosts, outs)
     torch.cuda.synchronize()
     assert torch.equal(outs[0], y.cpu())
+
+
+def test_window_mxfp8_strided_rows_and_output(vdn):
+    """Row strides larger than H*d on the inputs and on the output: the
+    quantizers read through ld, the kernel writes through ld_o and leaves the
+    padding columns untouched."""
+    s = synth.Shape(13, 64, 2, 128)
+    inp = synth.make_inputs(s, seed=77, device="cuda")
+    pad = 64
+    big = {}
+    for n in ("q", "k", "v"):
+        t = torch.full((s.L, s.D + pad), float("nan"), dtype=torch.bfloat16, device="cuda")
+        t[:, :s.D] = inp[n]
+        big[n] = t[:, :s.D]
+    out = torch.full((s.L, s.D + pad), 3.0, dtype=torch.bfloat16, device="cuda")
+    o, ws = vdn.window_attn_mxfp8(big["q"], big["k"], big["v"], s.T, s.N, s.H, s.d,
+                                  out=out[:, :s.D])
+    assert vdn.get_device_status(ws) == 0
+    assert torch.all(out[:, s.D:] == 3.0)
+    x = {k: host(v) for k, v in inp.items() if k in ("q", "k", "v")}
+    o_ref, _ = omx.window_attn_mxfp8(x["q"], x["k"], x["v"], s.T, s.N, s.H, s.d)
+    assert per_head_max_rel(host(out[:, :s.D]), o_ref, s.H, s.d) <= TOL_BF16
+
+
+def test_window_mxfp8_72_frames_sampled_rows(vdn):
+    """The sweep's middle length (72 frames x 1024 tokens, 32-aligned) on
+    sampled rows of two heads."""
+    s = synth.Shape(72, 1024, 4, 128)
+    inp = synth.make_inputs(s, seed=72, device="cuda")
+    o, lse = _run(vdn, s, inp)
+    N, T = s.N, s.T
+    rng = np.random.default_rng(72)
+    rows = sorted(set([0, N - 1, 5 * N, 5 * N - 1, (T - 1) * N, T * N - 1, (T // 2) * N + 3] +
+                      list(rng.integers(0, s.L, 12))))
+    heads = [1, 3]
+    cols = np.concatenate([np.arange(h * 128, (h + 1) * 128) for h in heads])
+    cols_t = torch.as_tensor(cols, device="cuda")
+    rows_t = torch.as_tensor(rows, device="cuda")
+    x = {k: host(inp[k][:, cols_t]) for k in ("q", "k", "v")}
+    o_ref, lse_ref = omx.window_attn_mxfp8_rows(x["q"], x["k"], x["v"], T, N, 2, 128, rows)
+    assert per_head_max_rel(host(o[rows_t][:, cols_t]), o_ref, 2, 128) <= TOL_BF16
+    lse_gpu = host(lse[torch.as_tensor(heads, device="cuda")][:, rows_t])
+    assert np.abs(lse_gpu - lse_ref).max() <= TOL_LSE
