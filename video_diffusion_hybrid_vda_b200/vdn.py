@@ -715,12 +715,21 @@ class HeadShardedLayer:
     no bf16 rounding; each rank receives 1/G of the sum instead of all of
     it).  ``output="rows"`` returns that row block in bf16, ``output="full"``
     also all-gathers the bf16 blocks into the whole y on every rank.
+
+    ``collective="fused"`` replaces the partial and the reduce-scatter with
+    one kernel (vdn_hybrid_fuse_shard_rs): the output GEMM's epilogue adds
+    each row of this rank's partial straight into the row block of the rank
+    that owns it, through peer mappings of the other ranks' fp32 row-block
+    buffers (CUDA IPC handles exchanged once, at construction; plain
+    system-scope atomic adds, no multicast).  Every rank zeroes its own
+    block and the ranks meet on the host before the kernel, and again
+    after it before a block is read.  No kernel waits on another rank.
     ``ops`` replaces the compute calls (tests only).
     """
 
     def __init__(self, T, N, H, d, W_gs, W_gl, W_os, W_ol, gamma, eps=1e-6, group=None,
                  device=None, ops=None, act_dtype=torch.bfloat16, acc_dtype=torch.float32,
-                 output="full"):
+                 output="full", collective="reduce_scatter"):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
@@ -730,7 +739,10 @@ class HeadShardedLayer:
             raise ValueError("heads must divide evenly over the ranks")
         if output not in ("rows", "full"):
             raise ValueError("output: 'rows' or 'full'")
+        if collective not in ("reduce_scatter", "fused"):
+            raise ValueError("collective: 'reduce_scatter' or 'fused'")
         self.output = output
+        self.collective = collective
         self.T, self.N, self.H, self.d = int(T), int(N), int(H), int(d)
         self.L, self.D = self.T * self.N, self.H * self.d
         self.Hl = self.H // self.world
@@ -752,7 +764,8 @@ class HeadShardedLayer:
                 int(lib().vdn_hybrid_fuse_shard_workspace(self.L, self.D, Hl, d)), dev)
             ops = {"window_attn": functools.partial(window_attn, ws=ws_win),
                    "vda_scan": functools.partial(vda_scan, ws=ws_vda),
-                   "fuse_shard": functools.partial(hybrid_fuse_shard, ws=ws_fuse)}
+                   "fuse_shard": functools.partial(hybrid_fuse_shard, ws=ws_fuse),
+                   "fuse_shard_rs": functools.partial(hybrid_fuse_shard_rs, ws=ws_fuse)}
             self.workspaces = (ws_win, ws_vda, ws_fuse)
         self.ops = ops
         self.o_s = torch.empty((self.L, Dl), dtype=act_dtype, device=dev)
@@ -763,6 +776,14 @@ class HeadShardedLayer:
         self.y_rows = torch.empty((self.R, self.D), dtype=act_dtype, device=dev)
         self.y = (torch.empty((self.world * self.R, self.D), dtype=act_dtype, device=dev)
                   if output == "full" else None)
+        if collective == "fused":
+            # this rank's row block, and every rank's block mapped here
+            from torch.multiprocessing.reductions import reduce_tensor
+            self.owner = torch.zeros((self.R, self.D), dtype=acc_dtype, device=dev)
+            handles = [None] * self.world
+            dist.all_gather_object(handles, reduce_tensor(self.owner)[1], group=group)
+            self.owners = [self.owner if g == self.rank else _open_peer_block(handles[g])
+                           for g in range(self.world)]
 
     def forward(self, q, k, v, beta, alpha, x):
         """y (full, [T*N, D]) or this rank's rows of y ([rows, D], rows = self.rows)."""
@@ -773,14 +794,38 @@ class HeadShardedLayer:
         alpha_l = alpha[:, h0:h1].contiguous()
         self.ops["window_attn"](ql, kl, vl, self.T, self.N, Hl, d, out=self.o_s)
         self.ops["vda_scan"](ql, kl, vl, beta_l, alpha_l, self.T, self.N, Hl, d, out=self.o_vda)
-        self.ops["fuse_shard"](x, self.o_s, self.o_vda, *self.W[:2], self.gamma, *self.W[2:], d,
-                               h0, eps=self.eps, out=self.y_partial[:self.L])
-        self.dist.reduce_scatter_tensor(self.y_rows32, self.y_partial, group=self.group)
-        self.y_rows.copy_(self.y_rows32)                    # fp32 sum -> bf16
+        if self.collective == "fused":
+            self.owner.zero_()
+            self._meet()                                    # every block zeroed
+            self.ops["fuse_shard_rs"](x, self.o_s, self.o_vda, *self.W[:2], self.gamma,
+                                      *self.W[2:], d, h0, self.owners, eps=self.eps)
+            self._meet()                                    # every rank's rows added
+            self.y_rows.copy_(self.owner)                   # fp32 sum -> bf16
+        else:
+            self.ops["fuse_shard"](x, self.o_s, self.o_vda, *self.W[:2], self.gamma,
+                                   *self.W[2:], d, h0, eps=self.eps,
+                                   out=self.y_partial[:self.L])
+            self.dist.reduce_scatter_tensor(self.y_rows32, self.y_partial, group=self.group)
+            self.y_rows.copy_(self.y_rows32)                # fp32 sum -> bf16
         if self.output == "rows":
             return self.y_rows[:self.rows.stop - self.rows.start]
         self.dist.all_gather_into_tensor(self.y, self.y_rows, group=self.group)
         return self.y[:self.L]
+
+
+    def _meet(self):
+        """All ranks' work enqueued so far is complete (a host-side meeting)."""
+        if self.device.type == "cuda":
+            torch.cuda.current_stream(self.device).synchronize()
+        self.dist.barrier(group=self.group)
+
+
+def _open_peer_block(args):
+    """A tensor over another process's CUDA allocation, from the arguments
+    torch's CUDA IPC sharing produced for it (the mapping enables peer
+    access lazily; nothing is copied)."""
+    from torch.multiprocessing.reductions import rebuild_cuda_tensor
+    return rebuild_cuda_tensor(*args)
 
 
 class SeqShardedLayer:
