@@ -408,6 +408,19 @@ VDN_API vdn_status vdn_get_device_status(const void* ws, void* stream);
 /* Enqueue a clear of the workspace's device status word on `stream`. */
 VDN_API vdn_status vdn_reset_device_status(void* ws, void* stream);
 
+/* Pitched copy, enqueued on `stream` (cudaMemcpy2DAsync, the direction taken
+ * from the pointers): `rows` rows of `width_bytes` bytes, rows `src_pitch`
+ * bytes apart in the source and `dst_pitch` in the destination.  Data
+ * movement only (the paper has no counterpart): it lets a caller stream a
+ * block of columns of a row-major host activation, for example the heads of
+ * one group, into a device buffer, so that work on those heads can start
+ * before the rest has arrived.  Host memory must be pinned for the copy to
+ * be asynchronous.  VDN_ERR_INVALID_ARG for null pointers or a width above
+ * either pitch; VDN_ERR_CUDA if the copy cannot be enqueued. */
+VDN_API vdn_status vdn_copy2d_async(void* dst, size_t dst_pitch, const void* src,
+                                    size_t src_pitch, size_t width_bytes, size_t rows,
+                                    void* stream);
+
 /* Wall-clock budget (ns) of every bounded wait inside the kernels launched
  * after this call (default 2e9).  0 makes any wait that is not already
  * satisfied fail at once with VDN_ERR_TIMEOUT: a test hook for the timeout

@@ -249,6 +249,17 @@ vdn_status vdn_reset_device_status(void* ws, void* stream) {
   return VDN_OK;
 }
 
+vdn_status vdn_copy2d_async(void* dst, size_t dst_pitch, const void* src, size_t src_pitch,
+                            size_t width_bytes, size_t rows, void* stream) {
+  if (dst == nullptr || src == nullptr || width_bytes > dst_pitch || width_bytes > src_pitch)
+    return VDN_ERR_INVALID_ARG;
+  if (width_bytes == 0 || rows == 0) return VDN_OK;
+  return cudaMemcpy2DAsync(dst, dst_pitch, src, src_pitch, width_bytes, rows, cudaMemcpyDefault,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? VDN_OK
+             : VDN_ERR_CUDA;
+}
+
 vdn_status vdn_get_device_status(const void* ws, void* stream) {
   if (ws == nullptr || !aligned(ws, 256)) return VDN_ERR_WORKSPACE;
   uint32_t word = 0;

@@ -31,7 +31,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
            "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8",
            "vdn_hybrid_fuse_shard_rs", "vdn_window_attn_schedule",
-           "vdn_window_attn_mxfp8_workspace", "vdn_window_attn_mxfp8"]
+           "vdn_window_attn_mxfp8_workspace", "vdn_window_attn_mxfp8", "vdn_copy2d_async"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -136,6 +136,8 @@ def lib():
     L.vdn_window_attn_mxfp8.argtypes = [S, _P, _P, _P, _I64, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_uint, ctypes.c_float, _P, _I64, _P, _P, _SZ, _P]
     L.vdn_window_attn_mxfp8.restype = ctypes.c_int
+    L.vdn_copy2d_async.argtypes = [_P, _SZ, _P, _SZ, _SZ, _SZ, _P]
+    L.vdn_copy2d_async.restype = ctypes.c_int
     L.vdn_version.argtypes = []
     L.vdn_version.restype = ctypes.c_char_p
     _lib = L
@@ -172,6 +174,24 @@ def _need_cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
             raise ValueError("libvdn takes CUDA tensors only")
+
+
+def copy_columns_async(dst, dst_c0, src, src_c0, ncols, stream=None):
+    """ncols columns of the row-major 2-D tensor src, from column src_c0, into
+    dst from column dst_c0 (same row count and dtype; one of them pinned host
+    memory, the other CUDA), as one pitched copy on ``stream``."""
+    if dst.dim() != 2 or src.dim() != 2 or dst.shape[0] != src.shape[0] or \
+            dst.dtype != src.dtype:
+        raise ValueError("copy_columns_async: 2-D tensors with the same rows and dtype")
+    if dst.stride(1) != 1 or src.stride(1) != 1 or dst_c0 + ncols > dst.shape[1] or \
+            src_c0 + ncols > src.shape[1]:
+        raise ValueError("copy_columns_async: contiguous rows holding the columns")
+    e = dst.element_size()
+    _check(lib().vdn_copy2d_async(ctypes.c_void_p(dst.data_ptr() + dst_c0 * e),
+                                  dst.stride(0) * e,
+                                  ctypes.c_void_p(src.data_ptr() + src_c0 * e),
+                                  src.stride(0) * e, ncols * e, dst.shape[0], _stream(stream)),
+           "vdn_copy2d_async")
 
 
 def alloc_workspace(nbytes, device=None):
@@ -585,6 +605,17 @@ class HybridLayer:
             self.kernels_per_forward += 3  # quantization of q, k, v
         self._staging = None
 
+    def _window_heads(self, q, k, v, hg, out, stream):
+        """The window Softmax on hg heads given as column views (row stride D)."""
+        T, N, d = self.T, self.N, self.d
+        cf, wc, an = self.mask
+        if self.softmax == "mxfp8":
+            window_attn_mxfp8(q, k, v, T, N, hg, d, cf, wc, an, out=out, ws=self.ws_win,
+                              stream=stream)
+        else:
+            window_attn(q, k, v, T, N, hg, d, cf, wc, an, out=out, ws=self.ws_win,
+                        stream=stream)
+
     def _window(self, q, k, v, stream, ctx_k=None, ctx_v=None):
         T, N, H, d = self.T, self.N, self.H, self.d
         cf, wc, an = self.mask
@@ -631,17 +662,45 @@ class HybridLayer:
             return out
         return self.y
 
+    def _fuse_rows(self, x, y, r0, r1, stream):
+        """The fuse on token rows [r0, r1) (every step of it is per token)."""
+        if self.projections == "mxfp8":
+            hybrid_fuse_mxfp8(x[r0:r1], self.o_s[r0:r1], self.o_vda[r0:r1], self.wg, self.gamma,
+                              self.wo, self.H, eps=self.eps, out=y[r0:r1], ws=self.ws_fuse,
+                              stream=stream)
+        else:
+            hybrid_fuse(x[r0:r1], self.o_s[r0:r1], self.o_vda[r0:r1], self.W_gs, self.W_gl,
+                        self.gamma, self.W_os, self.W_ol, self.H, eps=self.eps, out=y[r0:r1],
+                        ws=self.ws_fuse, stream=stream)
+
+    def _head_groups(self):
+        """Head groups of the first video of forward_many: up to four."""
+        g = next(n for n in (4, 3, 2, 1) if self.H % n == 0)
+        return [(i * (self.H // g), self.H // g) for i in range(g)]
+
+    def _row_chunks(self):
+        """Row blocks of the last video's fuse and read-back: up to four, of
+        multiples of 128 rows."""
+        step = max(128, (self.L + 4 * 128 - 1) // (4 * 128) * 128)
+        return [(r, min(r + step, self.L)) for r in range(0, self.L, step)]
+
     def forward_many(self, batches, outs, stream=None, copy_stream=None):
         """Run the layer over several videos held in (pinned) host memory.
 
-        ``batches`` is a list of (q, k, v, beta, alpha, x) host tuples and
-        ``outs`` a list of host tensors [T*N, D] bf16 that receive y.  Copies
-        run on ``copy_stream`` into two device staging sets, so the input of
-        video i+1 and the result of video i-1 move while video i computes.
-        q, k, v are copied first: the window Softmax, which needs only them,
-        starts before beta, alpha and x have landed (this shortens the
-        pipeline's fill).  Returns after enqueueing; synchronise the streams
-        to read ``outs``.
+        ``batches`` is a list of (q, k, v, beta, alpha, x) host tensors
+        (q, k, v, x [T*N, D], beta [T*N, H], alpha [T, H], rows contiguous)
+        and ``outs`` a list of host tensors [T*N, D] bf16 that receive y.
+        Copies run on ``copy_stream`` into two device staging sets, so the
+        input of video i+1 and the result of video i-1 move while video i
+        computes.  The pipeline's fill and drain are cut short:
+          * the first video's q, k, v, beta and alpha arrive in head groups
+            (pitched copies of their columns), and both attention branches
+            start on a group as soon as it has landed;
+          * for the other videos q, k, v are copied first: the window
+            Softmax, which needs only them, starts before beta, alpha and x;
+          * the last video's fuse runs in row blocks, each block's y read
+            back while the next one computes.
+        Returns after enqueueing; synchronise the streams to read ``outs``.
         """
         if len(batches) != len(outs):
             raise ValueError("one output per batch")
@@ -650,49 +709,90 @@ class HybridLayer:
         copy_stream = copy_stream or getattr(self, "_copy_stream", None)
         if copy_stream is None:
             copy_stream = self._copy_stream = torch.cuda.Stream(dev)
+        T, N, H, d = self.T, self.N, self.H, self.d
+        groups = self._head_groups()
         if getattr(self, "_stages", None) is None:
             b0 = batches[0]
             self._stages = [[torch.empty(t.shape, dtype=t.dtype, device=dev) for t in b0]
                             for _ in range(2)]
             self._ys = [torch.empty((self.L, self.D), dtype=torch.bfloat16, device=dev)
                         for _ in range(2)]
+            # per head group: its beta and alpha columns, contiguous
+            self._grp_ba = [(torch.empty((self.L, hg), dtype=torch.float32, device=dev),
+                             torch.empty((T, hg), dtype=torch.float32, device=dev))
+                            for _, hg in groups]
         stages, ys = self._stages, self._ys
         loaded_qkv = [torch.cuda.Event() for _ in batches]
         loaded = [torch.cuda.Event() for _ in batches]
         computed = [torch.cuda.Event() for _ in batches]
-        T, N, H, d = self.T, self.N, self.H, self.d
+        grp_loaded = [torch.cuda.Event() for _ in groups]
+        n = len(batches)
 
         def load(i):
             with torch.cuda.stream(copy_stream):
                 if i >= 2:
                     copy_stream.wait_event(computed[i - 2])   # stage i % 2 is free
-                for n, (dst, src) in enumerate(zip(stages[i % 2], batches[i])):
+                for k_, (dst, src) in enumerate(zip(stages[i % 2], batches[i])):
                     dst.copy_(src, non_blocking=True)
-                    if n == 2:
+                    if k_ == 2:
                         loaded_qkv[i].record(copy_stream)
                 loaded[i].record(copy_stream)
 
+        def load_first_by_groups():
+            q, k, v, _, _, x = stages[0]
+            hq, hk, hv, hb, ha, hx = batches[0]
+            with torch.cuda.stream(copy_stream):
+                for (h0, hg), (bg, ag), ev in zip(groups, self._grp_ba, grp_loaded):
+                    copy_columns_async(bg, 0, hb, h0, hg)
+                    copy_columns_async(ag, 0, ha, h0, hg)
+                    for dst, src in ((q, hq), (k, hk), (v, hv)):
+                        copy_columns_async(dst, h0 * d, src, h0 * d, hg * d)
+                    ev.record(copy_stream)
+                x.copy_(hx, non_blocking=True)
+                loaded[0].record(copy_stream)
+
         copy_stream.wait_stream(stream)  # copies start after work already on `stream`
-        load(0)
-        for i in range(len(batches)):
-            if i + 1 < len(batches):
+        load_first_by_groups()
+        self._read = [torch.cuda.Event() for _ in batches]
+        for i in range(n):
+            if i + 1 < n:
                 load(i + 1)
-            stream.wait_event(loaded_qkv[i])
             if i >= 2:
                 stream.wait_event(self._read[i - 2])           # y buffer i % 2 is free
             q, k, v, beta, alpha, x = stages[i % 2]
             y = ys[i % 2]
-            self._window(q, k, v, stream)
-            stream.wait_event(loaded[i])                        # beta, alpha, x
-            vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
-                     stream=stream)
-            self._fuse(x, y, stream)
-            computed[i].record(stream)
             if i == 0:
-                self._read = [torch.cuda.Event() for _ in batches]
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(computed[i])
-                outs[i].copy_(y, non_blocking=True)
+                # both branches per head group, each as soon as it has landed
+                for (h0, hg), (bg, ag), ev in zip(groups, self._grp_ba, grp_loaded):
+                    stream.wait_event(ev)
+                    c = slice(h0 * d, (h0 + hg) * d)
+                    self._window_heads(q[:, c], k[:, c], v[:, c], hg, self.o_s[:, c], stream)
+                    vda_scan(q[:, c], k[:, c], v[:, c], bg, ag, T, N, hg, d,
+                             out=self.o_vda[:, c], ws=self.ws_vda, stream=stream)
+            else:
+                stream.wait_event(loaded_qkv[i])
+                self._window(q, k, v, stream)
+                stream.wait_event(loaded[i])                    # beta, alpha, x
+                vda_scan(q, k, v, beta, alpha, T, N, H, d, out=self.o_vda, ws=self.ws_vda,
+                         stream=stream)
+            stream.wait_event(loaded[i])                        # x
+            if i + 1 < n:
+                self._fuse(x, y, stream)
+                computed[i].record(stream)
+                with torch.cuda.stream(copy_stream):
+                    copy_stream.wait_event(computed[i])
+                    outs[i].copy_(y, non_blocking=True)
+                    self._read[i].record(copy_stream)
+            else:
+                # the last video: fuse and read back in row blocks
+                for r0, r1 in self._row_chunks():
+                    self._fuse_rows(x, y, r0, r1, stream)
+                    done = torch.cuda.Event()
+                    done.record(stream)
+                    with torch.cuda.stream(copy_stream):
+                        copy_stream.wait_event(done)
+                        outs[i][r0:r1].copy_(y[r0:r1], non_blocking=True)
+                computed[i].record(stream)
                 self._read[i].record(copy_stream)
         return outs
 
