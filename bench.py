@@ -9,18 +9,20 @@ flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload layer102|layer42|small]
-                    [--part all|layer|vda_backward|fuse_mxfp8|window_mxfp8|scan_sweep]
+                    [--part all|layer|vda_backward|fuse_mxfp8|window_mxfp8|layer_mxfp8|
+                            scan_sweep]
 
-The line also carries three rows timed on their own, not part of the step:
+The line also carries four rows timed on their own, not part of the step:
 ``vda_backward``, the VDA gradient pass (dq, dk, dv, dbeta, dalpha from
 dL/do_vda, forward recomputed inside); ``fuse_mxfp8``, the fuse with
 both projection GEMMs in MXFP8 (x quantized inside the timed call, weights
 quantized beforehand), against the FP8 peak and beside the bf16 fuse's
 output; and ``window_mxfp8``, the window Softmax with both products in
 MXFP8 (q, k, v quantized inside the timed call), against its FP8 tensor and
-MUFU bounds and beside the bf16 window Softmax's output.  ``--part
-vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` time only that row (for
-launch lists and captures).  ``--part scan_sweep`` times the VDA
+MUFU bounds and beside the bf16 window Softmax's output; and
+``layer_mxfp8``, the whole layer pass with both MXFP8 modes, beside the bf16
+layer's y.  ``--part vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` /
+``layer_mxfp8`` time only that row (for launch lists and captures).  ``--part scan_sweep`` times the VDA
 branch alone at every point of the scan-only sweep (T 42/72/102 x N
 1008/4032 x d 64/128 x H 24/48), each against its roofline.
 
@@ -526,6 +528,55 @@ def run_window_mxfp8(args, shape, rank, world):
     return ms, dev_rel
 
 
+def run_layer_mxfp8(args, shape, rank, world):
+    """Device time of one layer pass with both MXFP8 modes (the window
+    Softmax's products and both fuse GEMMs on MXFP8 operands; ms, max over
+    ranks) and the max relative deviation of its y from the bf16 layer's."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev, with_fuse=True)
+    w = [inp[n] for n in ("W_gs", "W_gl", "W_os", "W_ol")]
+    acts = [inp[n] for n in ("q", "k", "v", "beta", "alpha", "x")]
+    layer = vdn.HybridLayer(shape.T, shape.N, shape.H, shape.d, *w, inp["gamma"], device=dev,
+                            projections="mxfp8", softmax="mxfp8")
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        layer.forward(*acts, stream=stream)
+    torch.cuda.synchronize()
+    if layer.status() != 0:
+        raise RuntimeError("device status after the MXFP8 layer warm-up")
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        y = layer.forward(*acts, stream=stream)
+    e1.record(stream)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    y = y.clone()
+    del layer
+    torch.cuda.empty_cache()
+    ref = vdn.HybridLayer(shape.T, shape.N, shape.H, shape.d, *w, inp["gamma"], device=dev)
+    y_bf16 = ref.forward(*acts, stream=stream)
+    dev_rel = float(((y.float() - y_bf16.float()).abs().max() / y_bf16.float().abs().max()).item())
+    del ref, inp, acts, y, y_bf16
+    torch.cuda.empty_cache()
+    return ms, dev_rel
+
+
+def layer_mxfp8_row(shape, ms, dev_rel):
+    return {"ms": ms, "tokens_per_s": shape.L / (ms / 1e3),
+            "launches_per_pass": 11,
+            "max_rel_vs_bf16_layer": dev_rel,
+            "note": "window Softmax and both projections on MXFP8 operands (q, k, v, x "
+                    "quantized inside the pass, weights beforehand); VDA in bf16 / fp32"}
+
+
 def window_mxfp8_row(work, peaks, ms, dev_rel):
     """The MXFP8 window Softmax against its two bounds: FP8 tensor work at
     2 x the measured sustained bf16 rate, and one MUFU exponential per
@@ -631,7 +682,7 @@ def main():
                          "head-parallel attention in between (seq, strong scaling)")
     ap.add_argument("--part", default="all",
                     choices=["all", "layer", "vda_backward", "fuse_mxfp8", "window_mxfp8",
-                             "scan_sweep"],
+                             "layer_mxfp8", "scan_sweep"],
                     help="what to time: the layer step and the two side rows (all), or one "
                          "of them")
     args = ap.parse_args()
@@ -730,6 +781,18 @@ def main():
         if world > 1:
             torch.distributed.destroy_process_group()
         return
+    if args.part == "layer_mxfp8":
+        ms, dev_rel = run_layer_mxfp8(args, shape, rank, world)
+        if rank == 0:
+            print(json.dumps({"metric": "hybrid layer ms with both MXFP8 modes",
+                              "value": ms, "unit": "ms", "higher_is_better": False,
+                              "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                              "dtype": "mxfp8 (e4m3, ue8m0 / 32) products, fp32 VDA state",
+                              "data": "synthetic", "config": config,
+                              "layer_mxfp8": layer_mxfp8_row(shape, ms, dev_rel)}))
+        if world > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.part == "fuse_mxfp8":
         ms, dev_rel = run_fuse_mxfp8(args, shape, rank, world)
         if rank == 0:
@@ -797,6 +860,7 @@ def main():
         line["fuse_mxfp8"] = mxfp8_row(work, peaks, *run_fuse_mxfp8(args, shape, rank, world))
         line["window_mxfp8"] = window_mxfp8_row(work, peaks,
                                                 *run_window_mxfp8(args, shape, rank, world))
+        line["layer_mxfp8"] = layer_mxfp8_row(shape, *run_layer_mxfp8(args, shape, rank, world))
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(shape)
         line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
