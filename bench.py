@@ -21,7 +21,8 @@ output; and ``window_mxfp8``, the window Softmax with both products in
 MXFP8 (q, k, v quantized inside the timed call), against its FP8 tensor and
 MUFU bounds and beside the bf16 window Softmax's output; and
 ``layer_mxfp8``, the whole layer pass with both MXFP8 modes, beside the bf16
-layer's y.  ``--part vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` /
+layer's y.  ``vda_by_solver`` times the VDA branch with each solve of
+(I + A_t)^-1 (Gauss-Jordan, the default, and Cholesky).  ``--part vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` /
 ``layer_mxfp8`` time only that row (for launch lists and captures).  ``--part scan_sweep`` times the VDA
 branch alone at every point of the scan-only sweep (T 42/72/102 x N
 1008/4032 x d 64/128 x H 24/48), each against its roofline.
@@ -372,6 +373,49 @@ def get_status(ws):
     return vdn.get_device_status(ws)
 
 
+def run_vda_solvers(args, shape, rank, world):
+    """Device time of the VDA branch (prep, solve, scan, read-out; ms, max
+    over ranks) with each solver of (I + A_t)^-1; they differ only in the
+    solve kernel."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=rank, device=dev)
+    T, N, H, d = shape.T, shape.N, shape.H, shape.d
+    o = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
+    ws = vdn.alloc_workspace(vdn.vda_scan_workspace(T, N, H, d), dev)
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, solver in (("gauss_jordan", vdn.SOLVER_GAUSS_JORDAN),
+                         ("cholesky", vdn.SOLVER_CHOLESKY)):
+        vdn.set_vda_solver(solver)
+        for _ in range(args.warmup):
+            vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
+                         out=o, ws=ws, stream=stream)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
+                         out=o, ws=ws, stream=stream)
+        e1.record(stream)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        res[name + "_ms"] = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    if vdn.get_device_status(ws) != 0:
+        raise RuntimeError("device status after the solver comparison")
+    vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN if args.solver == "gauss-jordan"
+                       else vdn.SOLVER_CHOLESKY)
+    del inp, o, ws
+    torch.cuda.empty_cache()
+    res["default"] = "gauss-jordan"
+    res["note"] = "VDA branch (4 launches) timed with each solve; the other three kernels are shared"
+    return res
+
+
 def run_vda_backward(args, shape, rank, world):
     """Device time of one VDA gradient pass (ms, max over ranks)."""
     from video_diffusion_hybrid_vda_b200 import vdn
@@ -674,7 +718,7 @@ def main():
     ap.add_argument("--impl", default="vdn", choices=["vdn", "reference"])
     ap.add_argument("--workload", default="layer102", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--solver", default="cholesky", choices=["cholesky", "gauss-jordan"],
+    ap.add_argument("--solver", default="gauss-jordan", choices=["gauss-jordan", "cholesky"],
                     help="solver of (I + A)^-1 in the VDA branch")
     ap.add_argument("--parallel", default="videos", choices=["videos", "seq"],
                     help="with several GPUs: every rank runs its own video (videos, weak "
@@ -855,6 +899,7 @@ def main():
         "clocks": r["clocks"],
     }
     if args.part == "all":
+        line["vda_by_solver"] = run_vda_solvers(args, shape, rank, world)
         line["vda_backward"] = backward_row(work, peaks,
                                             *run_vda_backward(args, shape, rank, world))
         line["fuse_mxfp8"] = mxfp8_row(work, peaks, *run_fuse_mxfp8(args, shape, rank, world))

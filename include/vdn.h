@@ -436,11 +436,12 @@ VDN_API vdn_status vdn_selftest_exp2(const float* x, float* y_fma, float* y_mufu
                                      void* stream);
 
 /* Solver for (I + A_t)^-1 in the VDA path, process-wide, for calls enqueued
- * after this one: VDN_SOLVER_CHOLESKY (default: blocked Cholesky, W = L^-1,
- * P = W^T W) or VDN_SOLVER_GAUSS_JORDAN (an in-register Gauss-Jordan sweep,
- * the variant the 10100.com article's 消融 section reports for its own
- * kernels).  Returns VDN_ERR_INVALID_ARG for other values.  Not
- * thread-safe against concurrent launches. */
+ * after this one: VDN_SOLVER_GAUSS_JORDAN (default: an in-register
+ * Gauss-Jordan sweep, the variant the 10100.com article's 消融 section
+ * reports for its own kernels) or VDN_SOLVER_CHOLESKY (blocked Cholesky,
+ * W = L^-1, P = W^T W).  Both give P to within a few 1e-5 of the exact
+ * inverse (relative to max |P|).  Returns VDN_ERR_INVALID_ARG for other
+ * values.  Not thread-safe against concurrent launches. */
 #define VDN_SOLVER_CHOLESKY 0
 #define VDN_SOLVER_GAUSS_JORDAN 1
 VDN_API vdn_status vdn_set_vda_solver(int solver);

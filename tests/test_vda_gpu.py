@@ -182,17 +182,19 @@ def test_vda_timeout_path_reports_and_recovers(vdn):
     assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16
 
 
+@pytest.mark.parametrize("solver", ["cholesky", "gauss-jordan"])
 @pytest.mark.parametrize("T,N,H,d", [(7, 200, 2, 128), (17, 33, 2, 64), (3, 4032, 1, 128)])
-def test_vda_gauss_jordan_solver(vdn, T, N, H, d):
-    """The Gauss-Jordan variant of the solve: P against the GPU's own
-    symmetrised A, states and o_vda against the oracle."""
+def test_vda_solvers(vdn, solver, T, N, H, d):
+    """Both solves: P against the GPU's own symmetrised A (inverted in
+    float64 here), states and o_vda against the oracle."""
     shape = synth.Shape(T, N, H, d)
     inp = _inputs(shape, seed=T * 1000 + N + 1)
     try:
-        vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN)
+        vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN if solver == "gauss-jordan"
+                           else vdn.SOLVER_CHOLESKY)
         o, states, ws = _run(vdn, shape, inp)
     finally:
-        vdn.set_vda_solver(vdn.SOLVER_CHOLESKY)
+        vdn.set_vda_solver(vdn.SOLVER_DEFAULT)
     x = {k: host(v) for k, v in inp.items()}
     A, B, P = (host(t) for t in vdn.vda_debug_buffers(ws, T, N, H, d))
     for t in range(T):
@@ -241,7 +243,7 @@ def test_vda_numeric_failure_reports_and_recovers(vdn, solver, fault):
                              *shape_args(shape), ws=ws)
         assert vdn.get_device_status(ws) == 0
     finally:
-        vdn.set_vda_solver(vdn.SOLVER_CHOLESKY)
+        vdn.set_vda_solver(vdn.SOLVER_DEFAULT)
     x = {k: host(v) for k, v in inp.items()}
     o_ref, _, _ = oracle.vda(x["q"], x["k"], x["v"], x["beta"], x["alpha"], *shape_args(shape))
     assert per_head_max_rel(host(o), o_ref, shape.H, shape.d) <= TOL_BF16

@@ -7,13 +7,14 @@
 // (the tensor-core product in the prep rounds beta*k on one operand only, so
 // A is symmetric up to that rounding).  Two solvers:
 //
-//  Cholesky (default): blocked in 16 x 16 blocks; one warp factors and
+//  Cholesky: blocked in 16 x 16 blocks; one warp factors and
 //   inverts each diagonal block with shuffles, every thread takes part in
 //   the panel and trailing block products; then W = L^-1 by blocked forward
 //   substitution and P = W^T W (see the kernel's own comment).
-//  Gauss-Jordan (the inverse the pages' own kernels use):
-//   one in-register sweep over the pivots, publishing the pivot row and
-//   column each step, leaves (I + A_sym)^-1.
+//  Gauss-Jordan (default; the inverse the pages' own kernels use): one
+//   in-register sweep over the pivots, each thread holding a contiguous
+//   block of the matrix, the pivot row and column published each step,
+//   leaves (I + A_sym)^-1.
 // The scan multiplies (alpha S + B_t) by P_t itself, so no B P is formed here.
 //
 // I + A_sym is symmetric positive definite with eigenvalues >= 1 (beta >= 0),
@@ -27,29 +28,6 @@ namespace vdn {
 namespace {
 
 constexpr int kThreads = 256;  // 16 row groups x 16 column groups
-
-// Gauss-Jordan: the matrix in registers (rows ty + 16 a, columns tx + 16 b),
-// the published pivot row and column double-buffered in shared memory.
-template <int DH>
-struct SolveCfg {
-  static constexpr int RA = DH / 16;   // rows per thread (rows ty + 16 a)
-  static constexpr int CB = DH / 16;   // columns per thread (cols tx + 16 b)
-  static constexpr int SMEM = 4 * DH * 4;
-};
-
-// Load (I + A_sym) into the register tile m (rows ty + 16 a, cols tx + 16 b).
-template <int DH>
-__device__ __forceinline__ void load_spd(const float* __restrict__ Am,
-                                         float (&m)[SolveCfg<DH>::RA][SolveCfg<DH>::CB],
-                                         int ty, int tx) {
-#pragma unroll
-  for (int a = 0; a < SolveCfg<DH>::RA; ++a)
-#pragma unroll
-    for (int b = 0; b < SolveCfg<DH>::CB; ++b) {
-      const int i = ty + 16 * a, k = tx + 16 * b;
-      m[a][b] = 0.5f * (__ldg(Am + i * DH + k) + __ldg(Am + k * DH + i)) + (i == k ? 1.f : 0.f);
-    }
-}
 
 // ---------------------------------------------------------------- Cholesky
 //
@@ -332,87 +310,167 @@ __global__ void __launch_bounds__(kThreads, 2)
 //   M[i][k] <- M[i][k] - M[i][p] M[p][k] / piv          (i, k != p)
 // over p = 0..d-1 leaves (I + A_sym)^-1; the pivots are Schur-complement
 // diagonals of an SPD matrix with eigenvalues >= 1.
+//
+// Thread (ty, tx) of the 16 x 16 grid holds the R x R block of rows
+// R ty .. R ty + R-1 and columns R tx .. R tx + R-1 (R = DH / 16) in
+// registers as packed pairs.  The pivots are walked in groups of R, the R
+// pivots of a group unrolled, so the pivot's row or column inside an
+// owner's block is a compile-time index.  Each step: the half-warp holding
+// row p and the lanes holding column p publish them (double-buffered in
+// shared memory, one barrier per step), every thread applies the rank-1
+// update to its block with packed f32x2 FMAs, and the owners overwrite
+// row p, column p and the pivot.
 template <int DH>
 __global__ void __launch_bounds__(kThreads, 2)
     vda_solve_gj_kernel(const float* __restrict__ A, float* __restrict__ P, uint32_t* status) {
-  using Cfg = SolveCfg<DH>;
-  extern __shared__ float sm[];
-  float* rowb = sm;              // 2 x [DH] pivot rows
-  float* colb = rowb + 2 * DH;   // 2 x [DH] pivot columns
+  constexpr int R = DH / 16;  // rows (and columns) per thread
+  constexpr int H2 = R / 2;   // packed pairs per row
+  __shared__ __align__(16) float rowb[2][DH];
+  __shared__ __align__(16) float colb[2][DH];
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
   const int64_t mat = static_cast<int64_t>(blockIdx.x) * DH * DH;
+  const float* Am = A + mat;
   bool bad = false;
 
-  float m[Cfg::RA][Cfg::CB];
-  load_spd<DH>(A + mat, m, ty, tx);
+  // I + (A + A^T) / 2 on this thread's block: its rows, then the rows of
+  // its columns (32 contiguous bytes per lane either way)
+  uint64_t m[R][H2];
+#pragma unroll
+  for (int a = 0; a < R; ++a) {
+    const float* src = Am + (R * ty + a) * DH + R * tx;
+#pragma unroll
+    for (int q = 0; q < R / 4; ++q) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src + 4 * q));
+      m[a][2 * q] = f32x2_pack(v.x, v.y);
+      m[a][2 * q + 1] = f32x2_pack(v.z, v.w);
+    }
+  }
+#pragma unroll
+  for (int b = 0; b < R; ++b) {
+    const float* src = Am + (R * tx + b) * DH + R * ty;
+    float t[R];
+#pragma unroll
+    for (int q = 0; q < R / 4; ++q) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(src + 4 * q));
+      t[4 * q] = v.x;
+      t[4 * q + 1] = v.y;
+      t[4 * q + 2] = v.z;
+      t[4 * q + 3] = v.w;
+    }
+#pragma unroll
+    for (int a = 0; a < R; ++a) {
+      float lo = f32x2_lo(m[a][b / 2]), hi = f32x2_hi(m[a][b / 2]);
+      const float dg = (R * ty + a == R * tx + b) ? 1.f : 0.f;
+      if (b & 1)
+        hi = 0.5f * (hi + t[a]) + dg;
+      else
+        lo = 0.5f * (lo + t[a]) + dg;
+      m[a][b / 2] = f32x2_pack(lo, hi);
+    }
+  }
+
+  // row and column r of the blocks of row / column group g into buffer buf
+  auto publish = [&](int buf, int g, int r) {
+    if (ty == g) {
+#pragma unroll
+      for (int q = 0; q < R / 4; ++q)
+        *reinterpret_cast<float4*>(&rowb[buf][R * tx + 4 * q]) =
+            make_float4(f32x2_lo(m[r][2 * q]), f32x2_hi(m[r][2 * q]),
+                        f32x2_lo(m[r][2 * q + 1]), f32x2_hi(m[r][2 * q + 1]));
+    }
+    if (tx == g) {
+      float c[R];
+#pragma unroll
+      for (int a = 0; a < R; ++a) c[a] = (r & 1) ? f32x2_hi(m[a][r / 2]) : f32x2_lo(m[a][r / 2]);
+#pragma unroll
+      for (int q = 0; q < R / 4; ++q)
+        *reinterpret_cast<float4*>(&colb[buf][R * ty + 4 * q]) =
+            make_float4(c[4 * q], c[4 * q + 1], c[4 * q + 2], c[4 * q + 3]);
+    }
+  };
+  publish(0, 0, 0);
+  __syncthreads();
 #pragma unroll 1
-  for (int p = 0; p < DH; ++p) {
-    float* rb = rowb + (p & 1) * DH;
-    float* cb = colb + (p & 1) * DH;
-    if (ty == (p & 15)) {  // owners of row p
-      const int pa = p >> 4;
+  for (int g = 0; g < 16; ++g) {
 #pragma unroll
-      for (int b = 0; b < Cfg::CB; ++b) {
-        float v = m[0][b];
-#pragma unroll
-        for (int a = 1; a < Cfg::RA; ++a) v = (a == pa) ? m[a][b] : v;
-        rb[tx + 16 * b] = v;
+    for (int r = 0; r < R; ++r) {
+      const int p = R * g + r;
+      const int buf = r & 1;  // R is even: the parity of p
+      float piv = rowb[buf][p];
+      if (!(piv > 0.f)) {  // also catches NaN
+        bad = true;
+        piv = 1.f;
       }
-    }
-    if (tx == (p & 15)) {  // owners of column p
-      const int pb = p >> 4;
+      const float inv = __frcp_rn(piv);
+      const uint64_t ninv2 = f32x2_pack(-inv, -inv);
+      uint64_t nrk[H2];  // -M[p][k] / piv at this thread's columns
 #pragma unroll
-      for (int a = 0; a < Cfg::RA; ++a) {
-        float v = m[a][0];
-#pragma unroll
-        for (int b = 1; b < Cfg::CB; ++b) v = (b == pb) ? m[a][b] : v;
-        cb[ty + 16 * a] = v;
+      for (int q = 0; q < R / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&rowb[buf][R * tx + 4 * q]);
+        nrk[2 * q] = f32x2_mul(f32x2_pack(v.x, v.y), ninv2);
+        nrk[2 * q + 1] = f32x2_mul(f32x2_pack(v.z, v.w), ninv2);
       }
-    }
-    __syncthreads();
-    float piv = rb[p];
-    if (!(piv > 0.f)) {  // also catches NaN
-      bad = true;
-      piv = 1.f;
-    }
-    const float inv = 1.f / piv;
-    float fi[Cfg::RA], rk[Cfg::CB];
+      float col[R];  // M[i][p] at this thread's rows
 #pragma unroll
-    for (int a = 0; a < Cfg::RA; ++a) fi[a] = cb[ty + 16 * a] * inv;
-#pragma unroll
-    for (int b = 0; b < Cfg::CB; ++b) rk[b] = rb[tx + 16 * b];
-#pragma unroll
-    for (int a = 0; a < Cfg::RA; ++a) {
-      const int i = ty + 16 * a;
-#pragma unroll
-      for (int b = 0; b < Cfg::CB; ++b) {
-        const int k = tx + 16 * b;
-        const float upd = fmaf(-fi[a], rk[b], m[a][b]);
-        const float rowp = (k == p) ? inv : rk[b] * inv;
-        m[a][b] = (i == p) ? rowp : ((k == p) ? -fi[a] : upd);
+      for (int q = 0; q < R / 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&colb[buf][R * ty + 4 * q]);
+        col[4 * q] = v.x;
+        col[4 * q + 1] = v.y;
+        col[4 * q + 2] = v.z;
+        col[4 * q + 3] = v.w;
       }
+#pragma unroll
+      for (int a = 0; a < R; ++a) {
+        const uint64_t c2 = f32x2_pack(col[a], col[a]);
+#pragma unroll
+        for (int b = 0; b < H2; ++b) m[a][b] = f32x2_fma(c2, nrk[b], m[a][b]);
+      }
+      if (ty == g) {  // row p: M[p][k] / piv
+#pragma unroll
+        for (int b = 0; b < H2; ++b) m[r][b] = f32x2_mul(nrk[b], f32x2_pack(-1.f, -1.f));
+      }
+      if (tx == g) {  // column p: -M[i][p] / piv, and the pivot 1 / piv
+#pragma unroll
+        for (int a = 0; a < R; ++a) {
+          const float v = (a == r && ty == g) ? inv : -col[a] * inv;
+          float lo = f32x2_lo(m[a][r / 2]), hi = f32x2_hi(m[a][r / 2]);
+          if (r & 1)
+            hi = v;
+          else
+            lo = v;
+          m[a][r / 2] = f32x2_pack(lo, hi);
+        }
+      }
+      // the next step's row and column into the other buffer (its readers
+      // all passed the barrier that ended the step before this one)
+      if (p + 1 < DH) {
+        if (r + 1 < R)
+          publish((r + 1) & 1, g, r + 1);
+        else
+          publish(0, g + 1, 0);
+      }
+      __syncthreads();
     }
-    // one barrier per step: the next step writes the other buffer pair
   }
   float* Pm = P + mat;
 #pragma unroll
-  for (int a = 0; a < Cfg::RA; ++a)
+  for (int a = 0; a < R; ++a)
 #pragma unroll
-    for (int b = 0; b < Cfg::CB; ++b) Pm[(ty + 16 * a) * DH + tx + 16 * b] = m[a][b];
+    for (int q = 0; q < R / 4; ++q)
+      *reinterpret_cast<float4*>(Pm + (R * ty + a) * DH + R * tx + 4 * q) =
+          make_float4(f32x2_lo(m[a][2 * q]), f32x2_hi(m[a][2 * q]), f32x2_lo(m[a][2 * q + 1]),
+                      f32x2_hi(m[a][2 * q + 1]));
   if (bad) record_status(status, kStatusNumeric);
 }
 
 template <int DH>
 cudaError_t launch_solve_dh(const Launch& ctx, const vdn_shape& s, const float* A, float* P,
                             int solver) {
-  using Cfg = SolveCfg<DH>;
   static std::atomic<uint64_t> chol_set{0};
   if (cudaError_t e = set_smem_once(vda_solve_kernel<DH>, CholCfg<DH>::SMEM, chol_set)) return e;
-  static std::atomic<uint64_t> gj_set{0};
-  if (cudaError_t e = set_smem_once(vda_solve_gj_kernel<DH>, Cfg::SMEM, gj_set)) return e;
   if (solver == VDN_SOLVER_GAUSS_JORDAN)
-    vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, Cfg::SMEM, ctx.stream>>>(A, P, ctx.status);
+    vda_solve_gj_kernel<DH><<<s.T * s.H, kThreads, 0, ctx.stream>>>(A, P, ctx.status);
   else
     vda_solve_kernel<DH><<<s.T * s.H, kThreads, CholCfg<DH>::SMEM, ctx.stream>>>(A, P,
                                                                                  ctx.status);

@@ -19,7 +19,7 @@ namespace vdn {
 namespace {
 
 std::atomic<uint64_t> g_budget_ns{2000000000ull};
-std::atomic<int> g_solver{VDN_SOLVER_CHOLESKY};
+std::atomic<int> g_solver{VDN_SOLVER_GAUSS_JORDAN};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -34,9 +34,12 @@ def main(argv=None):
                     metavar=("T", "N", "H", "d"))
     ap.add_argument("--passes", type=int, default=5)
     ap.add_argument("--lib", default=None, help="path of a libvdn.so other than the in-tree one")
+    ap.add_argument("--solver", choices=["gauss-jordan", "cholesky"], default="gauss-jordan")
     args = ap.parse_args(argv)
     if args.lib:
         vdn.LIB_PATH = args.lib
+    vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN if args.solver == "gauss-jordan"
+                       else vdn.SOLVER_CHOLESKY)
     s = synth.Shape(*args.shape)
     inp = synth.make_inputs(s, seed=0, device="cuda")
     if args.part == "vda_forward":
@@ -73,7 +76,8 @@ def main(argv=None):
         if n is not None:
             per[n] = per.get(n, 0.0) + e.device_time_total / 1000.0
     out = {k: round(v / args.passes, 4) for k, v in per.items()}
-    print(json.dumps({"part": args.part, "shape": args.shape, "passes": args.passes,
+    print(json.dumps({"part": args.part, "shape": args.shape, "solver": args.solver,
+                      "passes": args.passes,
                       "ms_per_pass": out, "sum_ms": round(sum(out.values()), 4)}))
 
 

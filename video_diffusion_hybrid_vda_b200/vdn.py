@@ -35,6 +35,7 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
+SOLVER_DEFAULT = SOLVER_GAUSS_JORDAN
 
 
 class VdnError(RuntimeError):
@@ -216,7 +217,7 @@ def set_wait_budget_ns(ns):
 
 
 def set_vda_solver(solver):
-    """SOLVER_CHOLESKY (default) or SOLVER_GAUSS_JORDAN, process-wide."""
+    """SOLVER_GAUSS_JORDAN (default) or SOLVER_CHOLESKY, process-wide."""
     _check(lib().vdn_set_vda_solver(int(solver)), "vdn_set_vda_solver")
 
 
