@@ -86,18 +86,21 @@ def work_model(s):
     proj_flop = 4 * 2 * s.L * s.D * s.D                 # gate GEMMs + output GEMMs
     # VDA HBM bytes: prep reads k, v (bf16) and beta; read-out reads q, writes o
     vda_bytes = 2 * s.L * s.D * 2 + s.L * s.H * 4 + 2 * s.L * s.D * 2
-    # FP32 ALU work in FLOP per (frame, head): the SPD inverse (Cholesky,
-    # W = L^-1 and the triangular product P = W^T W, d^3 / 3 each) and both
-    # scans' (alpha S + B) P, a 2 d^3 product each
-    vda_alu_flop = s.T * s.H * (s.d ** 3 + 4 * s.d ** 3)
+    # FP32 ALU work in FLOP (an FMA is 2, as in the FP32 peak) per (frame,
+    # head): the SPD inverse, d^3 FMA (Gauss-Jordan: d pivots x d^2 updates;
+    # Cholesky: factor, W = L^-1 and P = W^T W, d^3 / 3 each), and both
+    # scans' (alpha S + B) P, a d^3-FMA product each
+    vda_alu_flop = s.T * s.H * (2 * s.d ** 3 + 4 * s.d ** 3)
     # VDA gradient pass: reads q, k, v, dO (bf16) and beta, writes dq, dk, dv
     # (bf16) and dbeta; FP32 ALU: the forward's solve and scans again, the
-    # two adjoint scans (2 d^3 each) and the combine (two d^3 products, 4 d^3)
+    # two adjoint scans (2 d^3 each) and the combine (two d^3 products, 4 d^3);
+    # on a saved forward (P and states kept) only the last two
     vda_bwd_bytes = 7 * s.L * s.D * 2 + 2 * s.L * s.H * 4
-    vda_bwd_alu_flop = vda_alu_flop + s.T * s.H * (4 * s.d ** 3 + 4 * s.d ** 3)
+    vda_bwd_saved_alu_flop = s.T * s.H * (4 * s.d ** 3 + 4 * s.d ** 3)
+    vda_bwd_alu_flop = vda_alu_flop + vda_bwd_saved_alu_flop
     return dict(pairs=pairs, heads=s.H, softmax_flop=softmax_flop, proj_flop=proj_flop,
                 vda_bytes=vda_bytes, vda_alu_flop=vda_alu_flop, vda_bwd_bytes=vda_bwd_bytes,
-                vda_bwd_alu_flop=vda_bwd_alu_flop)
+                vda_bwd_alu_flop=vda_bwd_alu_flop, vda_bwd_saved_alu_flop=vda_bwd_saved_alu_flop)
 
 
 def load_peaks():
@@ -700,14 +703,18 @@ def mxfp8_row(work, peaks, ms, dev_rel):
 
 
 def backward_row(work, peaks, ms, ms_saved):
-    roof_ms = (work["vda_bwd_bytes"] / (peaks["hbm_gbs"] * 1e9) +
-               work["vda_bwd_alu_flop"] / (FP32_TFLOPS * 1e12)) * 1e3
+    hbm_ms = work["vda_bwd_bytes"] / (peaks["hbm_gbs"] * 1e9) * 1e3
+    roof_ms = hbm_ms + work["vda_bwd_alu_flop"] / (FP32_TFLOPS * 1e12) * 1e3
+    roof_saved = hbm_ms + work["vda_bwd_saved_alu_flop"] / (FP32_TFLOPS * 1e12) * 1e3
     return {"ms": ms, "bound": "hbm + fp32 alu", "roofline_ms": roof_ms, "frac": roof_ms / ms,
             "hbm_bytes": work["vda_bwd_bytes"], "fp32_alu_flop": work["vda_bwd_alu_flop"],
             "launches_per_pass": 9,
             "ms_saved_forward": ms_saved, "launches_saved_forward": 6,
+            "roofline_ms_saved_forward": roof_saved, "frac_saved_forward": roof_saved / ms_saved,
+            "fp32_alu_flop_saved_forward": work["vda_bwd_saved_alu_flop"],
             "note": "ms: forward recomputed inside; ms_saved_forward: P and states taken "
-                    "from a forward run on the same workspace"}
+                    "from a forward run on the same workspace (same HBM bytes, without the "
+                    "forward's solve and scans)"}
 
 
 def main():
