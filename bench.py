@@ -79,6 +79,21 @@ def mask_pair_count(T, cf=5, wc=1, anchors=3):
     return n
 
 
+WINDOW_SOURCES = ("window_attn.cu", "window_sched.cuh", "ptx.cuh", "common.cuh", "repack.cuh",
+                  "exp2_fma.cuh")
+
+
+def window_source_hash():
+    """sha256 over the sources the window Softmax kernel is built from (a
+    stored DRAM-traffic figure is used only while these are unchanged)."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in WINDOW_SOURCES:
+        with open(os.path.join(ROOT, "video_diffusion_hybrid_vda_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def work_model(s):
     """Algorithmic work of one layer pass (unmasked pairs only)."""
     pairs = mask_pair_count(s.T) * s.N * s.N          # token pairs per head
@@ -865,7 +880,9 @@ def main():
     if os.path.exists(KERNEL_TRAFFIC_FILE):
         with open(KERNEL_TRAFFIC_FILE) as f:
             tr = json.load(f)
-        if tr.get("workload") == config["workload"]:
+        # only counters taken on this workload and on these kernel sources
+        if (tr.get("workload") == config["workload"] and
+                tr.get("source_sha256") == window_source_hash()):
             traffic = tr.get("bytes_per_launch")
     # layer roofline: sum over steps of the binding resource at the measured peaks
     roof_ms = (work["softmax_flop"] / (peak * 1e12) + work["proj_flop"] / (peak * 1e12) +
