@@ -403,26 +403,30 @@ def run_vda_solvers(args, shape, rank, world):
     o = torch.empty((shape.L, shape.D), dtype=torch.bfloat16, device=dev)
     ws = vdn.alloc_workspace(vdn.vda_scan_workspace(T, N, H, d), dev)
     stream = torch.cuda.current_stream(dev)
-    res = {}
-    for name, solver in (("gauss_jordan", vdn.SOLVER_GAUSS_JORDAN),
-                         ("cholesky", vdn.SOLVER_CHOLESKY)):
-        vdn.set_vda_solver(solver)
-        for _ in range(args.warmup):
-            vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
-                         out=o, ws=ws, stream=stream)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H, d,
-                         out=o, ws=ws, stream=stream)
-        e1.record(stream)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        res[name + "_ms"] = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev, world)[0]
+    solvers = (("gauss_jordan", vdn.SOLVER_GAUSS_JORDAN), ("cholesky", vdn.SOLVER_CHOLESKY))
+    calls = 20  # per round: the branch is ~3.6 ms, so a round is long enough to time
+    best = {name: float("inf") for name, _ in solvers}
+    for rnd in range(3):  # the solvers alternate, so clock drift hits both alike
+        for name, solver in solvers:
+            vdn.set_vda_solver(solver)
+            for _ in range(args.warmup):
+                vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H,
+                             d, out=o, ws=ws, stream=stream)
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(calls):
+                vdn.vda_scan(inp["q"], inp["k"], inp["v"], inp["beta"], inp["alpha"], T, N, H,
+                             d, out=o, ws=ws, stream=stream)
+            e1.record(stream)
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            ms = max_over_ranks([e0.elapsed_time(e1) / calls], dev, world)[0]
+            best[name] = min(best[name], ms)
+    res = {name + "_ms": ms for name, ms in best.items()}
     if vdn.get_device_status(ws) != 0:
         raise RuntimeError("device status after the solver comparison")
     vdn.set_vda_solver(vdn.SOLVER_GAUSS_JORDAN if args.solver == "gauss-jordan"
@@ -430,7 +434,8 @@ def run_vda_solvers(args, shape, rank, world):
     del inp, o, ws
     torch.cuda.empty_cache()
     res["default"] = "gauss-jordan"
-    res["note"] = "VDA branch (4 launches) timed with each solve; the other three kernels are shared"
+    res["note"] = ("VDA branch (4 launches) with each solve, best of 3 alternating rounds of "
+                   "20 calls; the other three kernels are shared")
     return res
 
 
