@@ -124,19 +124,20 @@ cudaError_t launch_vda_gram(const Launch& ctx, const vdn_shape& s, const CUtenso
 cudaError_t launch_vda_adjoint_scan(const Launch& ctx, const vdn_shape& s, const float* P,
                                     const float* G, const float* alpha, float* adj);
 
-// Read-out variants: x (S0 + S1)^T, or x (S0 + S1) when trans_s, rows scaled
-// by row_scale[(t N + i) H + h] when it is non-null.
+// Read-out variants: x (S0 + S1)^T, or x (S0 + S1) when trans_s.
 cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,
-                                  const CUtensorMap& omap, const float* states, bool trans_s,
-                                  const float* row_scale);
+                                  const CUtensorMap& omap, const float* states, bool trans_s);
 
 // E = dA + dA^T with dA = -(S_fwd^T D_fwd + S_bwd^T D_bwd), and dalpha.
 cudaError_t launch_vda_grad_combine(const Launch& ctx, const vdn_shape& s, const float* states,
                                     const float* adj, float* E, float* dalpha);
 
-// dk = beta (K E + V dB) (bf16 through dkmap) and dbeta (fp32 [L, H]).
+// dk = beta (K E + V dB) (bf16 through dkmap), dv = beta K dB^T (bf16 rows
+// of dv, row stride ld_dv elements) and dbeta (fp32 [L, H]), in one pass
+// over k and v.
 cudaError_t launch_vda_grad_k(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, const CUtensorMap& dkmap, const float* E,
-                              const float* adj, const float* beta, float* dbeta);
+                              const float* adj, const float* beta, float* dbeta, void* dv,
+                              int64_t ld_dv);
 
 }  // namespace vdn

@@ -2,8 +2,8 @@
 // 10100.com article, 方法概述 items 2 and 3: the closed-form frame update and
 // the staged alignment that trains the branch).  Two kernels of that pass
 // live here; the others are modes of the forward kernels (gram mode of the
-// prep kernel for G, adjoint mode of the scan for D, transposed and scaled
-// modes of the read-out for dq and dv).
+// prep kernel for G, adjoint mode of the scan for D, the transposed mode of
+// the read-out for dq).
 //
 // With S_t = U_t P_t, U_t = alpha S_prev + B_t, P_t = (I + A_t)^-1 and the
 // adjoint states D_t = dL/dU_t of both scans:
@@ -13,8 +13,10 @@
 //     E_t      = dA_t + dA_t^T                  (A_t is symmetric)
 //     dalpha_t = <D_fwd_t, S_fwd_{t-1}> + <D_bwd_t, S_bwd_{t+1}>
 //   per token i of frame t (dB_t = D_fwd_t + D_bwd_t):
-//     y_i = E_t k_i,  z_i = dB_t^T v_i
-//     dk_i = beta_i (y_i + z_i),  dbeta_i = k_i . (y_i / 2 + z_i)
+//     a_i = E_t k_i + dB_t^T v_i,  w_i = dB_t k_i
+//     dk_i = beta_i a_i,  dv_i = beta_i w_i,
+//     dbeta_i = k_i . (E_t k_i / 2 + dB_t^T v_i) = (k_i . a_i + v_i . w_i) / 2
+//   (v_i . w_i = k_i . dB_t^T v_i), so one pass over k and v gives all three.
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -189,8 +191,8 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
                       const __grid_constant__ CUtensorMap vmap,
                       const __grid_constant__ CUtensorMap dkmap, const float* __restrict__ E,
                       const float* __restrict__ adj, const float* __restrict__ beta,
-                      float* __restrict__ dbeta, int T, int N, int H, uint32_t* status,
-                      uint64_t budget_ns) {
+                      float* __restrict__ dbeta, __nv_bfloat16* __restrict__ dv, int64_t ld_dv,
+                      int T, int N, int H, uint32_t* status, uint64_t budget_ns) {
   using Cfg = GradKCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -269,8 +271,10 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc_y = idesc_bf16(128, DH, false, false);
-      constexpr uint32_t idesc_z = idesc_bf16(128, DH, false, true);
+      // a = K E + V dB (one accumulator), w = K dB^T: dB's tile is the
+      // MN-major B operand of the first and the K-major one of the second
+      constexpr uint32_t idesc_k = idesc_bf16(128, DH, false, false);
+      constexpr uint32_t idesc_mn = idesc_bf16(128, DH, false, true);
       const uint32_t eb = smem_u32(ebuf);
       const uint32_t db = smem_u32(dbbuf);
       for (int j = 0; j < ntiles; ++j) {
@@ -292,10 +296,12 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t eoff = (kk >> 2) * (DH * 128) + (kk & 3) * 32;
-          umma_ss(ty, sdesc_sw128(kb + aoff, 16, 1024), sdesc_sw128(eb + eoff, 16, 1024), idesc_y,
+          umma_ss(ty, sdesc_sw128(kb + aoff, 16, 1024), sdesc_sw128(eb + eoff, 16, 1024), idesc_k,
                   kk > 0);
-          umma_ss(ty + DH, sdesc_sw128(vb + aoff, 16, 1024),
-                  sdesc_sw128(db + kk * 2048, DH * 128, 1024), idesc_z, kk > 0);
+          umma_ss(ty, sdesc_sw128(vb + aoff, 16, 1024),
+                  sdesc_sw128(db + kk * 2048, DH * 128, 1024), idesc_mn, 1);
+          umma_ss(ty + DH, sdesc_sw128(kb + aoff, 16, 1024), sdesc_sw128(db + eoff, 16, 1024),
+                  idesc_k, kk > 0);
         }
         umma_commit(&tfull[b]);
       }
@@ -325,39 +331,50 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
       tc_fence_after();
       uint8_t* ob = obuf + (j % Cfg::OUT_BUFS) * Cfg::TILE;
       const uint8_t* ks = kstage(s);
+      const uint8_t* vs = vstage(s);
       const uint32_t taddr = tmem + b * 2 * DH + ((quarter * 32) << 16);
+      // this token's row of dv, written from registers (16 bytes at a time)
+      __nv_bfloat16* dvrow = dv + (static_cast<int64_t>(t) * N + tok) * ld_dv + h * DH;
       float dbt = 0.f;
 #pragma unroll 1
       for (int c = 0; c < DH; c += 32) {
-        uint32_t ry[32], rz[32];
-        tmem_ld32(taddr + c, ry);
-        tmem_ld32(taddr + DH + c, rz);
+        uint32_t ra[32], rw[32];
+        tmem_ld32(taddr + c, ra);
+        tmem_ld32(taddr + DH + c, rw);
         tmem_ld_wait();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int chunk = ((c & 63) >> 3) + q;  // 16-byte chunk within the 128-byte row
           const uint32_t off = (c >> 6) * 16384 + sw128_offset(row, chunk);
           const uint4 kw = *reinterpret_cast<const uint4*>(ks + off);
+          const uint4 vw = *reinterpret_cast<const uint4*>(vs + off);
           const uint32_t kwa[4] = {kw.x, kw.y, kw.z, kw.w};
-          uint32_t o[4];
+          const uint32_t vwa[4] = {vw.x, vw.y, vw.z, vw.w};
+          uint32_t o[4], ov[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 kf = unpack_bf16x2(kwa[e]);
-            const float y0 = __uint_as_float(ry[8 * q + 2 * e]);
-            const float y1 = __uint_as_float(ry[8 * q + 2 * e + 1]);
-            const float z0 = __uint_as_float(rz[8 * q + 2 * e]);
-            const float z1 = __uint_as_float(rz[8 * q + 2 * e + 1]);
-            dbt = fmaf(kf.x, fmaf(0.5f, y0, z0), dbt);
-            dbt = fmaf(kf.y, fmaf(0.5f, y1, z1), dbt);
-            o[e] = pack_bf16x2(bt * (y0 + z0), bt * (y1 + z1));
+            const float2 vf = unpack_bf16x2(vwa[e]);
+            const float a0 = __uint_as_float(ra[8 * q + 2 * e]);
+            const float a1 = __uint_as_float(ra[8 * q + 2 * e + 1]);
+            const float w0 = __uint_as_float(rw[8 * q + 2 * e]);
+            const float w1 = __uint_as_float(rw[8 * q + 2 * e + 1]);
+            dbt = fmaf(kf.x, a0, dbt);
+            dbt = fmaf(kf.y, a1, dbt);
+            dbt = fmaf(vf.x, w0, dbt);
+            dbt = fmaf(vf.y, w1, dbt);
+            o[e] = pack_bf16x2(bt * a0, bt * a1);
+            ov[e] = pack_bf16x2(bt * w0, bt * w1);
           }
           *reinterpret_cast<uint4*>(ob + off) = make_uint4(o[0], o[1], o[2], o[3]);
+          if (tok < N)
+            *reinterpret_cast<uint4*>(dvrow + c + 8 * q) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[b]);
-      mbar_arrive(&empty[s]);  // k of this stage is no longer needed
-      if (tok < N) dbeta[(static_cast<int64_t>(t) * N + tok) * H + h] = dbt;
+      mbar_arrive(&empty[s]);  // k and v of this stage are no longer needed
+      if (tok < N) dbeta[(static_cast<int64_t>(t) * N + tok) * H + h] = 0.5f * dbt;
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (leader) {
@@ -392,12 +409,14 @@ cudaError_t launch_combine_dh(const Launch& ctx, const vdn_shape& s, const float
 template <int DH>
 cudaError_t launch_grad_k_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                              const CUtensorMap& vmap, const CUtensorMap& dkmap, const float* E,
-                             const float* adj, const float* beta, float* dbeta) {
+                             const float* adj, const float* beta, float* dbeta, void* dv,
+                             int64_t ld_dv) {
   using Cfg = GradKCfg<DH>;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_once(vda_grad_k_kernel<DH>, Cfg::SMEM, smem_set)) return e;
   vda_grad_k_kernel<DH><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      kmap, vmap, dkmap, E, adj, beta, dbeta, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
+      kmap, vmap, dkmap, E, adj, beta, dbeta, static_cast<__nv_bfloat16*>(dv), ld_dv, s.T, s.N,
+      s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
 
@@ -412,9 +431,12 @@ cudaError_t launch_vda_grad_combine(const Launch& ctx, const vdn_shape& s, const
 
 cudaError_t launch_vda_grad_k(const Launch& ctx, const vdn_shape& s, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, const CUtensorMap& dkmap, const float* E,
-                              const float* adj, const float* beta, float* dbeta) {
-  if (s.d == 128) return launch_grad_k_dh<128>(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta);
-  if (s.d == 64) return launch_grad_k_dh<64>(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta);
+                              const float* adj, const float* beta, float* dbeta, void* dv,
+                              int64_t ld_dv) {
+  if (s.d == 128)
+    return launch_grad_k_dh<128>(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta, dv, ld_dv);
+  if (s.d == 64)
+    return launch_grad_k_dh<64>(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta, dv, ld_dv);
   return cudaErrorInvalidValue;
 }
 

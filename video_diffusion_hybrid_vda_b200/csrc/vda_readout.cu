@@ -12,10 +12,9 @@
 // a 3-D frame view, so the ragged last tile of a frame reads zeros and its
 // extra rows are not written.  HBM-bound: q is read once and o written once.
 //
-// The gradient pass reuses the kernel twice: with kTransS the B operand is
-// read MN-major, giving x (S_fwd + S_bwd) instead of x (S_fwd + S_bwd)^T
-// (dq = dO S), and a non-null row_scale multiplies output row i by
-// row_scale[(t N + i) H + h] (dv = beta k (D_fwd + D_bwd)^T).
+// The gradient pass reuses the kernel: with kTransS the B operand is read
+// MN-major, giving x (S_fwd + S_bwd) instead of x (S_fwd + S_bwd)^T
+// (dq = dO S).
 #include "common.cuh"
 #include "ptx.cuh"
 
@@ -40,7 +39,7 @@ template <int DH, bool kTransS>
 __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
     vda_readout_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap omap, const float* __restrict__ states,
-                       const float* __restrict__ row_scale, int T, int N, int H, uint32_t* status,
+                       int T, int N, int H, uint32_t* status,
                        uint64_t budget_ns) {
   using Cfg = ReadoutCfg<DH>;
   extern __shared__ uint8_t smem_raw[];
@@ -165,19 +164,8 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
     const uint32_t quarter = warp & 3;
     const int row = quarter * 32 + lane_id();
     const bool leader = threadIdx.x == 64;
-    // the row's scale for tile j (1 without row_scale), fetched one tile
-    // ahead so its load latency is off the tile's path
-    auto scale_of = [&](int j) {
-      const int tok = j * 128 + row;
-      return row_scale == nullptr ? 1.f
-             : tok < N ? __ldg(row_scale + (static_cast<int64_t>(t) * N + tok) * H + h)
-                       : 0.f;
-    };
-    float rs_next = ntiles > 0 ? scale_of(0) : 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int b = j & 1;
-      const float rs = rs_next;
-      if (j + 1 < ntiles) rs_next = scale_of(j + 1);
       if (leader) bulk_wait_read<Cfg::OUT_BUFS - 1>();  // staging buffer b is free again
       const bool ok = mbar_wait(&tfull[b], (j >> 1) & 1, budget_ns);
       // collective decision (also the barrier that publishes "buffer free"),
@@ -197,10 +185,10 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 u;
-          u.x = pack_bf16x2(rs * __uint_as_float(r[8 * q + 0]), rs * __uint_as_float(r[8 * q + 1]));
-          u.y = pack_bf16x2(rs * __uint_as_float(r[8 * q + 2]), rs * __uint_as_float(r[8 * q + 3]));
-          u.z = pack_bf16x2(rs * __uint_as_float(r[8 * q + 4]), rs * __uint_as_float(r[8 * q + 5]));
-          u.w = pack_bf16x2(rs * __uint_as_float(r[8 * q + 6]), rs * __uint_as_float(r[8 * q + 7]));
+          u.x = pack_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
+          u.y = pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
+          u.z = pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
+          u.w = pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
           const int chunk = ((c & 63) >> 3) + q;  // 16-byte chunk within the 128-byte row
           *reinterpret_cast<uint4*>(ob + (c >> 6) * 16384 + sw128_offset(row, chunk)) = u;
         }
@@ -229,13 +217,12 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
 
 template <int DH, bool kTransS>
 cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
-                              const CUtensorMap& omap, const float* states,
-                              const float* row_scale) {
+                              const CUtensorMap& omap, const float* states) {
   using Cfg = ReadoutCfg<DH>;
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = set_smem_once(vda_readout_kernel<DH, kTransS>, Cfg::SMEM, smem_set)) return e;
   vda_readout_kernel<DH, kTransS><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, omap, states, row_scale, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
+      qmap, omap, states, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
   return cudaGetLastError();
 }
 
@@ -243,20 +230,19 @@ cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUten
 
 cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
                                const CUtensorMap& omap, const float* states) {
-  if (s.d == 128) return launch_readout_dh<128, false>(ctx, s, qmap, omap, states, nullptr);
-  if (s.d == 64) return launch_readout_dh<64, false>(ctx, s, qmap, omap, states, nullptr);
+  if (s.d == 128) return launch_readout_dh<128, false>(ctx, s, qmap, omap, states);
+  if (s.d == 64) return launch_readout_dh<64, false>(ctx, s, qmap, omap, states);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,
-                                  const CUtensorMap& omap, const float* states, bool trans_s,
-                                  const float* row_scale) {
+                                  const CUtensorMap& omap, const float* states, bool trans_s) {
   if (s.d == 128)
-    return trans_s ? launch_readout_dh<128, true>(ctx, s, xmap, omap, states, row_scale)
-                   : launch_readout_dh<128, false>(ctx, s, xmap, omap, states, row_scale);
+    return trans_s ? launch_readout_dh<128, true>(ctx, s, xmap, omap, states)
+                   : launch_readout_dh<128, false>(ctx, s, xmap, omap, states);
   if (s.d == 64)
-    return trans_s ? launch_readout_dh<64, true>(ctx, s, xmap, omap, states, row_scale)
-                   : launch_readout_dh<64, false>(ctx, s, xmap, omap, states, row_scale);
+    return trans_s ? launch_readout_dh<64, true>(ctx, s, xmap, omap, states)
+                   : launch_readout_dh<64, false>(ctx, s, xmap, omap, states);
   return cudaErrorInvalidValue;
 }
 
