@@ -728,8 +728,8 @@ def backward_row(work, peaks, ms, ms_saved):
     roof_saved = hbm_ms + work["vda_bwd_saved_alu_flop"] / (FP32_TFLOPS * 1e12) * 1e3
     return {"ms": ms, "bound": "hbm + fp32 alu", "roofline_ms": roof_ms, "frac": roof_ms / ms,
             "hbm_bytes": work["vda_bwd_bytes"], "fp32_alu_flop": work["vda_bwd_alu_flop"],
-            "launches_per_pass": 8,
-            "ms_saved_forward": ms_saved, "launches_saved_forward": 5,
+            "launches_per_pass": 7,
+            "ms_saved_forward": ms_saved, "launches_saved_forward": 4,
             "roofline_ms_saved_forward": roof_saved, "frac_saved_forward": roof_saved / ms_saved,
             "fp32_alu_flop_saved_forward": work["vda_bwd_saved_alu_flop"],
             "note": "ms: forward recomputed inside; ms_saved_forward: P and states taken "

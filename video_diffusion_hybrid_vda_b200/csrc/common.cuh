@@ -128,6 +128,13 @@ cudaError_t launch_vda_adjoint_scan(const Launch& ctx, const vdn_shape& s, const
 cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,
                                   const CUtensorMap& omap, const float* states, bool trans_s);
 
+// Head dim 128: dq = dO (S0 + S1) (bf16 through dqmap) and, from the same dO
+// tiles, G = sum_i dO_i q_i^T per (t, h) (fp32 [T, H, d, d]); the 128-row
+// frame maps domap and qmap.
+cudaError_t launch_vda_readout_dq_gram(const Launch& ctx, const vdn_shape& s,
+                                       const CUtensorMap& domap, const CUtensorMap& dqmap,
+                                       const CUtensorMap& qmap, const float* states, float* G);
+
 // E = dA + dA^T with dA = -(S_fwd^T D_fwd + S_bwd^T D_bwd), and dalpha.
 cudaError_t launch_vda_grad_combine(const Launch& ctx, const vdn_shape& s, const float* states,
                                     const float* adj, float* E, float* dalpha);

@@ -14,46 +14,53 @@
 //
 // The gradient pass reuses the kernel: with kTransS the B operand is read
 // MN-major, giving x (S_fwd + S_bwd) instead of x (S_fwd + S_bwd)^T
-// (dq = dO S).
+// (dq = dO S).  With kGram (head dim 128) each stage also holds the q tile
+// of the same tokens and the kernel accumulates G = dO^T q (the adjoint
+// scans' input, sum over the frame's tokens of dO_i q_i^T) in a third TMEM
+// region from the dO tile already there, so dO is read once for both.
 #include "common.cuh"
 #include "ptx.cuh"
 
 namespace vdn {
 namespace {
 
-template <int DH>
+template <int DH, bool kGram = false>
 struct ReadoutCfg {
   static constexpr int SLABS = DH / 64;
   static constexpr int QTILE_BYTES = SLABS * 128 * 128;  // 128 tokens x DH bf16
-  static constexpr int STAGES = 3;
+  static constexpr int STAGE_BYTES = (kGram ? 2 : 1) * QTILE_BYTES;  // x tile (then q tile)
+  static constexpr int STAGES = kGram ? 2 : 3;
   static constexpr int S_BYTES = SLABS * DH * 128;       // DH rows x DH bf16
-  static constexpr int OUT_BUFS = 2;
-  static constexpr int TMEM_COLS = 2 * DH;
+  static constexpr int OUT_BUFS = kGram ? 1 : 2;
+  static constexpr int TMEM_COLS = kGram ? 4 * DH : 2 * DH;  // 2 output buffers (+ G)
   static constexpr int THREADS = 192;
   static constexpr int SMEM =
-      1024 + STAGES * QTILE_BYTES + S_BYTES + OUT_BUFS * QTILE_BYTES + 256;
+      1024 + STAGES * STAGE_BYTES + S_BYTES + OUT_BUFS * QTILE_BYTES + 256;
 };
 
 
-template <int DH, bool kTransS>
-__global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
+template <int DH, bool kTransS, bool kGram = false>
+__global__ void __launch_bounds__(ReadoutCfg<DH, kGram>::THREADS, 1)
     vda_readout_kernel(const __grid_constant__ CUtensorMap qmap,
                        const __grid_constant__ CUtensorMap omap, const float* __restrict__ states,
                        int T, int N, int H, uint32_t* status,
-                       uint64_t budget_ns) {
-  using Cfg = ReadoutCfg<DH>;
+                       uint64_t budget_ns, const __grid_constant__ CUtensorMap gmap,
+                       float* __restrict__ G) {
+  static_assert(!kGram || (DH == 128 && kTransS), "G is formed beside dq, head dim 128");
+  using Cfg = ReadoutCfg<DH, kGram>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* qbuf = smem;
-  uint8_t* sbuf = qbuf + Cfg::STAGES * Cfg::QTILE_BYTES;
+  uint8_t* sbuf = qbuf + Cfg::STAGES * Cfg::STAGE_BYTES;
   uint8_t* obuf = sbuf + Cfg::S_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(obuf + Cfg::OUT_BUFS * Cfg::QTILE_BYTES);
   uint64_t* empty = full + Cfg::STAGES;
   uint64_t* tfull = empty + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* g_full = mma_done + 1;  // kGram: every product into G has completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(g_full + 1);
 
   const int t = blockIdx.x / H;
   const int h = blockIdx.x % H;
@@ -70,9 +77,11 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
       mbar_init(&tempty[b], 128);
     }
     mbar_init(mma_done, 1);
+    mbar_init(g_full, 1);
     fence_mbar_init();
     tma_prefetch_desc(&qmap);
     tma_prefetch_desc(&omap);
+    if constexpr (kGram) tma_prefetch_desc(&gmap);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -116,10 +125,14 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
           record_status(status, kStatusTimeout);
           break;
         }
-        mbar_arrive_expect_tx(&full[s], Cfg::QTILE_BYTES);
-        for (int sl = 0; sl < Cfg::SLABS; ++sl)
-          tma_load_3d(qbuf + s * Cfg::QTILE_BYTES + sl * 16384, &qmap, &full[s],
+        mbar_arrive_expect_tx(&full[s], Cfg::STAGE_BYTES);
+        for (int sl = 0; sl < Cfg::SLABS; ++sl) {
+          tma_load_3d(qbuf + s * Cfg::STAGE_BYTES + sl * 16384, &qmap, &full[s],
                       h * DH + 64 * sl, j * 128, t);
+          if constexpr (kGram)
+            tma_load_3d(qbuf + s * Cfg::STAGE_BYTES + Cfg::QTILE_BYTES + sl * 16384, &gmap,
+                        &full[s], h * DH + 64 * sl, j * 128, t);
+        }
         ++issued;
       }
       for (int j = (issued > Cfg::STAGES ? issued - Cfg::STAGES : 0); j < issued; ++j)
@@ -143,7 +156,7 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t qb = smem_u32(qbuf + s * Cfg::QTILE_BYTES);
+        const uint32_t qb = smem_u32(qbuf + s * Cfg::STAGE_BYTES);
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -154,9 +167,20 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
                                                        16, 1024);
           umma_ss(tmem + b * DH, sdesc_sw128(qb + koff, 16, 1024), sdesc, idesc, kk > 0);
         }
+        if constexpr (kGram) {
+          // G += dO^T q over the tile's 128 tokens: both operands MN-major
+          // (16 token rows per step, the two 64-feature slabs 16 KB apart)
+          constexpr uint32_t idesc_g = idesc_bf16(128, DH, true, true);
+          const uint32_t gb = qb + Cfg::QTILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + 2 * DH, sdesc_sw128(qb + kk * 2048, 16384, 1024),
+                    sdesc_sw128(gb + kk * 2048, 16384, 1024), idesc_g, (j | kk) != 0);
+        }
         umma_commit(&empty[s]);
         umma_commit(&tfull[b]);
       }
+      if constexpr (kGram) umma_commit(g_full);
       umma_commit(mma_done);  // every MMA of this CTA, also after an early exit
     }
   } else {
@@ -175,7 +199,7 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
         break;
       }
       tc_fence_after();
-      uint8_t* ob = obuf + b * Cfg::QTILE_BYTES;
+      uint8_t* ob = obuf + (j % Cfg::OUT_BUFS) * Cfg::QTILE_BYTES;
       const uint32_t taddr = tmem + b * DH + ((quarter * 32) << 16);
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
@@ -204,6 +228,27 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
       }
     }
     if (leader) bulk_wait<0>();
+    if constexpr (kGram) {
+      // G: row m of the fp32 matrix from TMEM lane m (warp-uniform wait)
+      if (__all_sync(0xffffffffu, mbar_wait(g_full, 0, budget_ns))) {
+        tc_fence_after();
+        float* dst = G + ((static_cast<int64_t>(t) * H + h) * DH + row) * DH;
+        const uint32_t gaddr = tmem + 2 * DH + ((quarter * 32) << 16);
+#pragma unroll 1
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t r[32];
+          tmem_ld32(gaddr + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + c + e) =
+                make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                            __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+        }
+      } else {
+        record_status(status, kStatusTimeout);
+      }
+    }
   }
 
   tc_fence_before();
@@ -215,14 +260,16 @@ __global__ void __launch_bounds__(ReadoutCfg<DH>::THREADS, 1)
   }
 }
 
-template <int DH, bool kTransS>
+template <int DH, bool kTransS, bool kGram = false>
 cudaError_t launch_readout_dh(const Launch& ctx, const vdn_shape& s, const CUtensorMap& qmap,
-                              const CUtensorMap& omap, const float* states) {
-  using Cfg = ReadoutCfg<DH>;
+                              const CUtensorMap& omap, const float* states,
+                              const CUtensorMap* gmap = nullptr, float* G = nullptr) {
+  using Cfg = ReadoutCfg<DH, kGram>;
   static std::atomic<uint64_t> smem_set{0};
-  if (cudaError_t e = set_smem_once(vda_readout_kernel<DH, kTransS>, Cfg::SMEM, smem_set)) return e;
-  vda_readout_kernel<DH, kTransS><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
-      qmap, omap, states, s.T, s.N, s.H, ctx.status, ctx.budget_ns);
+  if (cudaError_t e = set_smem_once(vda_readout_kernel<DH, kTransS, kGram>, Cfg::SMEM, smem_set))
+    return e;
+  vda_readout_kernel<DH, kTransS, kGram><<<s.T * s.H, Cfg::THREADS, Cfg::SMEM, ctx.stream>>>(
+      qmap, omap, states, s.T, s.N, s.H, ctx.status, ctx.budget_ns, gmap ? *gmap : qmap, G);
   return cudaGetLastError();
 }
 
@@ -233,6 +280,13 @@ cudaError_t launch_vda_readout(const Launch& ctx, const vdn_shape& s, const CUte
   if (s.d == 128) return launch_readout_dh<128, false>(ctx, s, qmap, omap, states);
   if (s.d == 64) return launch_readout_dh<64, false>(ctx, s, qmap, omap, states);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_vda_readout_dq_gram(const Launch& ctx, const vdn_shape& s,
+                                       const CUtensorMap& domap, const CUtensorMap& dqmap,
+                                       const CUtensorMap& qmap, const float* states, float* G) {
+  if (s.d != 128) return cudaErrorInvalidValue;
+  return launch_readout_dh<128, true, true>(ctx, s, domap, dqmap, states, &qmap, G);
 }
 
 cudaError_t launch_vda_readout_ex(const Launch& ctx, const vdn_shape& s, const CUtensorMap& xmap,

@@ -135,7 +135,7 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
                             float* P, float* X, float* states, bool reuse_forward) {
   const int64_t D = static_cast<int64_t>(s.H) * s.d;
   const int prep_rows = s.d == 128 ? 32 : 64;
-  CUtensorMap kmap_p, vmap_p, qmap_p, domap_p, domap, dqmap, kmap, vmap, dkmap;
+  CUtensorMap kmap_p, vmap_p, qmap_p, domap_p, domap, dqmap, kmap, vmap, dkmap, qmap;
   if (!make_frame_map(&kmap_p, k, D, ld, s.N, s.T, prep_rows) ||
       !make_frame_map(&vmap_p, v, D, ld, s.N, s.T, prep_rows) ||
       !make_frame_map(&qmap_p, q, D, ld, s.N, s.T, prep_rows) ||
@@ -143,6 +143,7 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
       !make_frame_map(&domap, d_o, D, ld_do, s.N, s.T, 128) ||
       !make_frame_map(&dqmap, dq, D, ld_g, s.N, s.T, 128) ||
       !make_frame_map(&kmap, k, D, ld, s.N, s.T, 128) ||
+      !make_frame_map(&qmap, q, D, ld, s.N, s.T, 128) ||
       !make_frame_map(&vmap, v, D, ld, s.N, s.T, 128) ||
       !make_frame_map(&dkmap, dk, D, ld_g, s.N, s.T, 128))
     return VDN_ERR_CUDA;
@@ -154,10 +155,17 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
        launch_vda_solve(ctx, s, A, P) != cudaSuccess ||
        launch_vda_scan(ctx, s, P, B, alpha, states) != cudaSuccess))
     return VDN_ERR_CUDA;
-  if (launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
-      launch_vda_adjoint_scan(ctx, s, P, G, alpha, adj) != cudaSuccess ||
+  // dq and G: one pass over dO for head dim 128 (G beside the dq read-out),
+  // the gram mode of the prep kernel and the transposed read-out otherwise
+  if (s.d == 128) {
+    if (launch_vda_readout_dq_gram(ctx, s, domap, dqmap, qmap, states, G) != cudaSuccess)
+      return VDN_ERR_CUDA;
+  } else if (launch_vda_gram(ctx, s, qmap_p, domap_p, G) != cudaSuccess ||
+             launch_vda_readout_ex(ctx, s, domap, dqmap, states, true) != cudaSuccess) {
+    return VDN_ERR_CUDA;
+  }
+  if (launch_vda_adjoint_scan(ctx, s, P, G, alpha, adj) != cudaSuccess ||
       launch_vda_grad_combine(ctx, s, states, adj, E, dalpha) != cudaSuccess ||
-      launch_vda_readout_ex(ctx, s, domap, dqmap, states, true) != cudaSuccess ||
       launch_vda_grad_k(ctx, s, kmap, vmap, dkmap, E, adj, beta, dbeta, dv, ld_g) != cudaSuccess)
     return VDN_ERR_CUDA;
   return VDN_OK;
