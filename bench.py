@@ -11,27 +11,34 @@ flush is needed between steps.
                     [--workload layer102|layer42|small]
                     [--part all|layer|vda_backward|fuse_mxfp8|window_mxfp8|layer_mxfp8|
                             scan_sweep]
+                    [--parallel videos|heads|seq] [--collective reduce_scatter|fused]
+                    [--solver gauss-jordan|cholesky]
 
-The line also carries four rows timed on their own, not part of the step:
+The line also carries rows timed on their own, not part of the step:
 ``vda_backward``, the VDA gradient pass (dq, dk, dv, dbeta, dalpha from
-dL/do_vda, forward recomputed inside); ``fuse_mxfp8``, the fuse with
+dL/do_vda, forward recomputed inside, and on a saved forward);
+``vda_by_solver``, the VDA branch with each solve of (I + A_t)^-1
+(Gauss-Jordan, the default, and Cholesky); ``fuse_mxfp8``, the fuse with
 both projection GEMMs in MXFP8 (x quantized inside the timed call, weights
 quantized beforehand), against the FP8 peak and beside the bf16 fuse's
-output; and ``window_mxfp8``, the window Softmax with both products in
-MXFP8 (q, k, v quantized inside the timed call), against its FP8 tensor and
-MUFU bounds and beside the bf16 window Softmax's output; and
-``layer_mxfp8``, the whole layer pass with both MXFP8 modes, beside the bf16
-layer's y.  ``vda_by_solver`` times the VDA branch with each solve of
-(I + A_t)^-1 (Gauss-Jordan, the default, and Cholesky).  ``--part vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` /
-``layer_mxfp8`` time only that row (for launch lists and captures).  ``--part scan_sweep`` times the VDA
-branch alone at every point of the scan-only sweep (T 42/72/102 x N
-1008/4032 x d 64/128 x H 24/48), each against its roofline.
+output; ``window_mxfp8``, the window Softmax with both products in MXFP8
+(q, k, v quantized inside the timed call), against its FP8 tensor and MUFU
+bounds and beside the bf16 window Softmax's output; and ``layer_mxfp8``,
+the whole layer pass with both MXFP8 modes, beside the bf16 layer's y.
+``--part vda_backward`` / ``fuse_mxfp8`` / ``window_mxfp8`` /
+``layer_mxfp8`` time only that row (for launch lists and captures).
+``--part scan_sweep`` times the VDA branch alone at every point of the
+scan-only sweep (T 42/72/102 x N 1008/4032 x d 64/128 x H 24/48), each
+against its roofline.
 
 With N > 1 (torchrun) every rank runs its own video (independent problems,
 no collective on the data path): weak scaling, time = max over ranks.
-``--parallel seq`` instead splits one video over the ranks by token rows,
-with the attention branches run head-parallel between two all-to-alls
-(strong scaling; on one GPU a one-rank group).
+``--parallel heads`` instead splits one video over the ranks by heads
+(every rank holds the full activations; the row-parallel fuse ends in a
+reduce-scatter of y, NCCL's or the fused GEMM + reduce-scatter kernel's
+with ``--collective fused``), and ``--parallel seq`` by token rows, with
+the attention branches run head-parallel between two all-to-alls (both
+strong scaling; on one GPU a one-rank group).
 ``--impl reference`` times the float64 CPU oracle instead, on a bounded
 sample of the same workload, extrapolated by work.
 """
@@ -376,6 +383,41 @@ def run_seq_sharded(args, shape, rank, world):
     start.record(stream)
     for _ in range(args.steps):
         layer.forward(*mine)
+    end.record(stream)
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = clocks_stop(clk)
+    if max(get_status(w) for w in layer.workspaces) != 0:
+        raise RuntimeError("device status after the sharded steps")
+    ms = max_over_ranks([start.elapsed_time(end)], dev, world)[0]
+    return ms / args.steps, clocks
+
+
+def run_head_sharded(args, shape, rank, world):
+    """One video split over the ranks by heads (HeadShardedLayer): every rank
+    holds the full activations, runs both branches on its H/G heads and the
+    row-parallel fuse on its columns, and one reduce-scatter (NCCL, or the
+    fused GEMM + reduce-scatter over peer mappings) leaves it a row block of
+    y; time of `steps` layer passes, max over ranks."""
+    from video_diffusion_hybrid_vda_b200 import vdn
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(shape, seed=0, device=dev, with_fuse=True)
+    layer = vdn.HeadShardedLayer(shape.T, shape.N, shape.H, shape.d, inp["W_gs"], inp["W_gl"],
+                                 inp["W_os"], inp["W_ol"], inp["gamma"], device=dev,
+                                 output="rows", collective=args.collective)
+    acts = [inp[n] for n in ("q", "k", "v", "beta", "alpha", "x")]
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        layer.forward(*acts)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = clocks_start()
+    torch.distributed.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        layer.forward(*acts)
     end.record(stream)
     torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -747,10 +789,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--solver", default="gauss-jordan", choices=["gauss-jordan", "cholesky"],
                     help="solver of (I + A)^-1 in the VDA branch")
-    ap.add_argument("--parallel", default="videos", choices=["videos", "seq"],
+    ap.add_argument("--parallel", default="videos", choices=["videos", "heads", "seq"],
                     help="with several GPUs: every rank runs its own video (videos, weak "
-                         "scaling), or one video is split over the ranks by token rows with "
-                         "head-parallel attention in between (seq, strong scaling)")
+                         "scaling); or one video is split over the ranks (strong scaling) by "
+                         "heads, every rank holding the full activations and keeping a row "
+                         "block of y (heads), or by token rows with head-parallel attention "
+                         "in between (seq)")
+    ap.add_argument("--collective", default="reduce_scatter",
+                    choices=["reduce_scatter", "fused"],
+                    help="--parallel heads: NCCL reduce-scatter of the fp32 partials, or the "
+                         "output GEMM adding its rows into the owners' blocks over peer "
+                         "mappings")
     ap.add_argument("--part", default="all",
                     choices=["all", "layer", "vda_backward", "fuse_mxfp8", "window_mxfp8",
                              "layer_mxfp8", "scan_sweep"],
@@ -796,15 +845,21 @@ def main():
             "nccl", device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0))),
             timeout=__import__("datetime").timedelta(seconds=300))
     peaks, peak_kind = load_peaks()
-    if args.parallel == "seq":
+    if args.parallel in ("seq", "heads"):
         if world == 1:
             torch.distributed.init_process_group(
                 "nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:%d" % free_port(),
                 device_id=torch.device("cuda", 0))
-        ms, clocks = run_seq_sharded(args, shape, rank, world)
+        if args.parallel == "seq":
+            ms, clocks = run_seq_sharded(args, shape, rank, world)
+            par = f"sequence x{world}, head-parallel attention (all-to-all)"
+        else:
+            ms, clocks = run_head_sharded(args, shape, rank, world)
+            par = (f"heads x{world}, row-parallel fuse + "
+                   + ("NCCL reduce-scatter" if args.collective == "reduce_scatter"
+                      else "fused GEMM + reduce-scatter over peer mappings"))
         if rank == 0:
-            config.update({"global_batch": 1, "parallelism": f"sequence x{world}, "
-                           "head-parallel attention (all-to-all)"})
+            config.update({"global_batch": 1, "parallelism": par})
             print(json.dumps({
                 "metric": METRIC, "value": shape.L / (ms / 1e3), "unit": "tokens/s",
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
