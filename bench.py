@@ -425,6 +425,7 @@ def run_head_sharded(args, shape, rank, world):
     if max(get_status(w) for w in layer.workspaces) != 0:
         raise RuntimeError("device status after the sharded steps")
     ms = max_over_ranks([start.elapsed_time(end)], dev, world)[0]
+    layer.close()
     return ms / args.steps, clocks
 
 

@@ -98,6 +98,7 @@ def _fused_rs_worker(rank, world, port, out):
             y = layer.forward(*[inp[n] for n in names])
             torch.cuda.synchronize()
             errs.append(max_rel(host(y), host(ref[layer.rows])))
+        layer.close()                                   # peer mappings released on both ranks
         out[rank] = (layer.rows.start, layer.rows.stop, errs)
     finally:
         dist_.destroy_process_group()

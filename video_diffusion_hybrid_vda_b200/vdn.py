@@ -879,12 +879,15 @@ class HeadShardedLayer:
                   if output == "full" else None)
         if collective == "fused":
             # this rank's row block, and every rank's block mapped here
-            from torch.multiprocessing.reductions import reduce_tensor
             self.owner = torch.zeros((self.R, self.D), dtype=acc_dtype, device=dev)
-            handles = [None] * self.world
-            dist.all_gather_object(handles, reduce_tensor(self.owner)[1], group=group)
-            self.owners = [self.owner if g == self.rank else _open_peer_block(handles[g])
-                           for g in range(self.world)]
+            if self.world == 1:
+                self.owners = [self.owner]
+            else:
+                from torch.multiprocessing.reductions import reduce_tensor
+                handles = [None] * self.world
+                dist.all_gather_object(handles, reduce_tensor(self.owner)[1], group=group)
+                self.owners = [self.owner if g == self.rank else _open_peer_block(handles[g])
+                               for g in range(self.world)]
 
     def forward(self, q, k, v, beta, alpha, x):
         """y (full, [T*N, D]) or this rank's rows of y ([rows, D], rows = self.rows)."""
@@ -913,6 +916,15 @@ class HeadShardedLayer:
         self.dist.all_gather_into_tensor(self.y, self.y_rows, group=self.group)
         return self.y[:self.L]
 
+
+    def close(self):
+        """Release the peer mappings of the fused collective; every rank calls
+        it before the process group goes away, so no rank's block is freed
+        while another still maps it."""
+        if self.collective == "fused" and self.world > 1:
+            self._meet()
+            self.owners = [self.owner]
+            self._meet()
 
     def _meet(self):
         """All ranks' work enqueued so far is complete (a host-side meeting)."""
