@@ -38,8 +38,9 @@
  *  - Host-side argument errors return VDN_ERR_INVALID_ARG or
  *    VDN_ERR_UNSUPPORTED before anything is enqueued.  A failed launch
  *    returns VDN_ERR_CUDA.  Errors detected on the device (a non-positive
- *    Cholesky pivot or NaN, a wait that ran out of time) are OR-ed into the
- *    workspace status word; no kernel traps.
+ *    Cholesky pivot or NaN, a wait that ran out of time, and in debug builds
+ *    an index outside its tensor) are OR-ed into the workspace status word;
+ *    no kernel traps.
  *  - Head dims: 64 and 128 run directly; 16 and 32 run on zero-padded
  *    64-wide copies of every head in the workspace (exact).  N, T, H >= 1.
  */
@@ -66,7 +67,8 @@ typedef enum {
   VDN_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required      */
   VDN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed               */
   VDN_ERR_NUMERIC = 5,     /* device: non-positive pivot or NaN in a solve    */
-  VDN_ERR_TIMEOUT = 6      /* device: a bounded wait ran out                   */
+  VDN_ERR_TIMEOUT = 6,     /* device: a bounded wait ran out                   */
+  VDN_ERR_BOUNDS = 7       /* device, debug builds: an index outside its tensor */
 } vdn_status;
 
 /* Problem shape: T latent frames, N tokens per frame, H heads, head dim d
@@ -407,6 +409,22 @@ VDN_API vdn_status vdn_get_device_status(const void* ws, void* stream);
 
 /* Enqueue a clear of the workspace's device status word on `stream`. */
 VDN_API vdn_status vdn_reset_device_status(void* ws, void* stream);
+
+/* 1 if this library was built with VDN_DEBUG_BOUNDS=1: every hand-computed
+ * global store (and tile start) is checked against its tensor's extents,
+ * and a miss is recorded as VDN_ERR_BOUNDS in the status word and the
+ * access skipped, instead of faulting; 0 for release builds, where the
+ * checks are compiled out.  Debug scaffolding (the paper has no
+ * counterpart). */
+VDN_API int vdn_debug_bounds_enabled(void);
+
+/* Self-test of the bounds check: one device thread checks row `r` and
+ * columns [c, c + width) against a rows x cols tensor, touching no memory
+ * but the status word of `ws`.  In a debug build an out-of-range index sets
+ * VDN_ERR_BOUNDS (read it with vdn_get_device_status); a release build
+ * records nothing.  Enqueued on `stream`. */
+VDN_API vdn_status vdn_selftest_bounds(void* ws, int64_t r, int64_t rows, int64_t c,
+                                       int64_t width, int64_t cols, void* stream);
 
 /* Pitched copy, enqueued on `stream` (cudaMemcpy2DAsync, the direction taken
  * from the pointers): `rows` rows of `width_bytes` bytes, rows `src_pitch`

@@ -63,7 +63,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings(L):
-    for code in range(7):
+    for code in range(8):
         assert L.status_string(code)
     assert "unknown" in L.status_string(99)
     assert "sm_100a" in L.version()
@@ -218,3 +218,17 @@ def test_window_mxfp8_rejects_bad_arguments_on_host(L):
              None, 0, None) == 3
     assert lib.vdn_window_attn_mxfp8_workspace(ctypes.byref(sh)) == \
         256 + 3 * 256 * 256 + 2 * 256 * 8 + 8 * 256
+
+
+def test_release_library_has_no_bounds_checks(L):
+    assert L.debug_bounds_enabled() is False
+
+
+def test_debug_bounds_variant_builds_and_reports_itself():
+    """The VDN_DEBUG_BOUNDS=1 variant (libvdn_debug.so) cross-compiles for
+    sm_100a and says so; its checks run on the GPU (test_debug_bounds_gpu)."""
+    from video_diffusion_hybrid_vda_b200 import build
+    path = build.build(debug_bounds=True)
+    dbg = ctypes.CDLL(path)
+    dbg.vdn_debug_bounds_enabled.restype = ctypes.c_int
+    assert dbg.vdn_debug_bounds_enabled() == 1

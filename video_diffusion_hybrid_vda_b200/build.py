@@ -1,6 +1,7 @@
 """Build libvdn.so in-tree from csrc/*.cu for sm_100a (nvcc cross-compiles
 without a GPU).  Usage: ``python -m video_diffusion_hybrid_vda_b200.build``
-(``--force`` rebuilds, ``-v`` prints ptxas register and spill counts).
+(``--force`` rebuilds, ``-v`` prints ptxas register and spill counts,
+``--debug-bounds`` builds the bounds-checking libvdn_debug.so instead).
 
 Build-time switches of the kernels are passed as preprocessor definitions
 in ``VDN_NVCC_DEFINES`` (comma-separated ``NAME=VALUE``), e.g.
@@ -37,10 +38,13 @@ def headers():
                   glob.glob(os.path.join(os.path.dirname(HERE), "include", "*.h")))
 
 
-def up_to_date():
-    if not os.path.exists(LIB):
+DEBUG_LIB = os.path.join(HERE, "libvdn_debug.so")  # VDN_DEBUG_BOUNDS=1 variant
+
+
+def up_to_date(lib=LIB):
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in sources() + headers() + [__file__])
 
 
@@ -56,13 +60,19 @@ def defines():
     return out
 
 
-def build(force=False, verbose=False, jobs=None):
-    """Compile every csrc/*.cu to an object and link libvdn.so."""
-    if not force and up_to_date():
-        return LIB
-    objdir = os.path.join(HERE, "_build")
+def build(force=False, verbose=False, jobs=None, debug_bounds=False):
+    """Compile every csrc/*.cu to an object and link libvdn.so, or with
+    ``debug_bounds`` the libvdn_debug.so variant built with
+    VDN_DEBUG_BOUNDS=1 (every hand-computed global store checked against
+    its tensor's extents on the device)."""
+    lib = DEBUG_LIB if debug_bounds else LIB
+    if not force and up_to_date(lib):
+        return lib
+    objdir = os.path.join(HERE, "_build_debug" if debug_bounds else "_build")
     os.makedirs(objdir, exist_ok=True)
     inc = ["-I", os.path.join(os.path.dirname(HERE), "include"), *defines()]
+    if debug_bounds:
+        inc.append("-DVDN_DEBUG_BOUNDS=1")
     procs, objs = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
@@ -80,12 +90,12 @@ def build(force=False, verbose=False, jobs=None):
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed on: " + ", ".join(failed))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-ldl"])
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+                debug_bounds="--debug-bounds" in sys.argv))

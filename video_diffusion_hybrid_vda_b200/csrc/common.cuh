@@ -16,12 +16,34 @@ namespace vdn {
 // Bits of the device status word (first 4 bytes of every workspace).
 constexpr uint32_t kStatusNumeric = 1u << 0;
 constexpr uint32_t kStatusTimeout = 1u << 1;
+constexpr uint32_t kStatusBounds = 1u << 2;  // debug builds: an index outside its tensor
+
+// Debug builds (VDN_DEBUG_BOUNDS=1) check the row and column range of every
+// hand-computed global store, and the start of hand-computed tile
+// coordinates, against the tensor's extents; a violation is recorded in the
+// status word and the access skipped.  Release builds compile the checks out.
+#ifndef VDN_DEBUG_BOUNDS
+#define VDN_DEBUG_BOUNDS 0
+#endif
 
 // Workspace bytes reserved in front of every workspace for the status word.
 constexpr size_t kStatusBytes = 256;
 
 __device__ __forceinline__ void record_status(uint32_t* status, uint32_t bits) {
   if (status != nullptr) atomicOr(status, bits);
+}
+
+// Rows [r, r + 1) and columns [c, c + width) inside a rows x cols tensor?
+// Always true in release builds; in debug builds a miss is recorded.
+__device__ __forceinline__ bool in_bounds(uint32_t* status, int64_t r, int64_t rows, int64_t c,
+                                          int64_t width, int64_t cols) {
+  if constexpr (VDN_DEBUG_BOUNDS) {
+    if (r < 0 || r >= rows || c < 0 || width < 0 || c + width > cols) {
+      record_status(status, kStatusBounds);
+      return false;
+    }
+  }
+  return true;
 }
 
 // NVTX range around a C-ABI call (a no-op unless a profiler is attached).

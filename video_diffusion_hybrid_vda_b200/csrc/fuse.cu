@@ -63,7 +63,8 @@ struct StoreF32Args {
 // arrive summed in their owners' buffers without a separate collective.
 struct RedScatterArgs {
   float* owner[8];
-  int rows;
+  int rows;   // rows of each owner's block
+  int count;  // owners
 };
 
 __device__ __forceinline__ float sigmoidf_fast(float x) {
@@ -289,14 +290,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             gate_chunk(args, r, n, acc, rinv, c == c0);
           } else if constexpr (std::is_same<Args, RedScatterArgs>::value) {
             const int o = static_cast<int>(r / args.rows);
-            float4* dst = reinterpret_cast<float4*>(
-                args.owner[o] + (r - static_cast<int64_t>(o) * args.rows) * N + n);
+            // the owning rank's block, and the row within it (checked in
+            // debug builds)
+            if (in_bounds(status, o, args.count, n, 32, N) &&
+                in_bounds(status, r - static_cast<int64_t>(o) * args.rows, args.rows, n, 32, N)) {
+              float4* dst = reinterpret_cast<float4*>(
+                  args.owner[o] + (r - static_cast<int64_t>(o) * args.rows) * N + n);
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              atomicAdd_system(dst + e, make_float4(__uint_as_float(acc[4 * e]),
-                                                    __uint_as_float(acc[4 * e + 1]),
-                                                    __uint_as_float(acc[4 * e + 2]),
-                                                    __uint_as_float(acc[4 * e + 3])));
+              for (int e = 0; e < 8; ++e)
+                atomicAdd_system(dst + e, make_float4(__uint_as_float(acc[4 * e]),
+                                                      __uint_as_float(acc[4 * e + 1]),
+                                                      __uint_as_float(acc[4 * e + 2]),
+                                                      __uint_as_float(acc[4 * e + 3])));
+            }
           } else if constexpr (sizeof(args.y[0]) == 4) {
             float4* dst = reinterpret_cast<float4*>(args.y + r * N + n);
 #pragma unroll
@@ -765,6 +771,7 @@ vdn_status vdn_hybrid_fuse_shard_rs(int L, int D, int H_local, int d, int head0,
     out.owner[o] = y_owners[o];
   }
   out.rows = (L + G - 1) / G;
+  out.count = G;
   return fuse_shard_impl(L, D, H_local, d, head0, x, o_s, o_vda, ld_o, W_gs, W_gl, gamma, eps,
                          W_os, W_ol, out, y_owners[0], ws, ws_bytes, stream);
 }

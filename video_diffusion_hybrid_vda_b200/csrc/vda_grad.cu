@@ -316,6 +316,12 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
       const int s = j % Cfg::STAGES;
       const int b = j & 1;
       const int tok = j * 128 + row;
+      // this token's rows of dk, dv and dbeta are stored only inside the
+      // frame (and inside the tensors: checked in debug builds)
+      const bool store = tok < N && in_bounds(status, static_cast<int64_t>(t) * N + tok,
+                                              static_cast<int64_t>(T) * N,
+                                              static_cast<int64_t>(h) * DH, DH,
+                                              static_cast<int64_t>(H) * DH);
       const float bt =
           tok < N ? __ldg(beta + (static_cast<int64_t>(t) * N + tok) * H + h) : 0.f;
       if (leader) bulk_wait_read<Cfg::OUT_BUFS - 1>();  // staging buffer free again
@@ -367,14 +373,14 @@ __global__ void __launch_bounds__(GradKCfg<DH>::THREADS, 1)
             ov[e] = pack_bf16x2(bt * w0, bt * w1);
           }
           *reinterpret_cast<uint4*>(ob + off) = make_uint4(o[0], o[1], o[2], o[3]);
-          if (tok < N)
+          if (store)
             *reinterpret_cast<uint4*>(dvrow + c + 8 * q) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[b]);
       mbar_arrive(&empty[s]);  // k and v of this stage are no longer needed
-      if (tok < N) dbeta[(static_cast<int64_t>(t) * N + tok) * H + h] = 0.5f * dbt;
+      if (store) dbeta[(static_cast<int64_t>(t) * N + tok) * H + h] = 0.5f * dbt;
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
       if (leader) {

@@ -175,6 +175,11 @@ vdn_status run_vda_backward(const Launch& ctx, const vdn_shape& s, const void* q
 
 uint64_t current_wait_budget_ns() { return g_budget_ns.load(); }
 
+__global__ void bounds_selftest_kernel(uint32_t* status, int64_t r, int64_t rows, int64_t c,
+                                       int64_t width, int64_t cols) {
+  in_bounds(status, r, rows, c, width, cols);
+}
+
 int current_vda_solver() { return g_solver.load(); }
 
 bool make_frame_map(CUtensorMap* map, const void* base, int64_t cols, int64_t ld, int N, int T,
@@ -235,6 +240,7 @@ const char* vdn_status_string(vdn_status s) {
     case VDN_ERR_CUDA: return "CUDA runtime or driver call failed";
     case VDN_ERR_NUMERIC: return "numeric failure on the device (non-positive pivot or NaN)";
     case VDN_ERR_TIMEOUT: return "a bounded wait on the device ran out of time";
+    case VDN_ERR_BOUNDS: return "an index outside its tensor (debug bounds check)";
   }
   return "unknown status";
 }
@@ -275,7 +281,18 @@ vdn_status vdn_get_device_status(const void* ws, void* stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return VDN_ERR_CUDA;
   if (word & kStatusTimeout) return VDN_ERR_TIMEOUT;
   if (word & kStatusNumeric) return VDN_ERR_NUMERIC;
+  if (word & kStatusBounds) return VDN_ERR_BOUNDS;
   return VDN_OK;
+}
+
+int vdn_debug_bounds_enabled(void) { return VDN_DEBUG_BOUNDS ? 1 : 0; }
+
+vdn_status vdn_selftest_bounds(void* ws, int64_t r, int64_t rows, int64_t c, int64_t width,
+                               int64_t cols, void* stream) {
+  if (ws == nullptr || !aligned(ws, 256)) return VDN_ERR_WORKSPACE;
+  bounds_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint32_t*>(ws), r, rows, c, width, cols);
+  return cudaGetLastError() == cudaSuccess ? VDN_OK : VDN_ERR_CUDA;
 }
 
 // ----------------------------------------------------------------- VDA

@@ -88,7 +88,7 @@ template <int DH, bool P_SMEM, class ArriveHalf, class ArriveReady, class SFree>
 __device__ __forceinline__ void softmax_warpgroup(
     int i, uint32_t tmem, uint64_t* s_full, uint64_t* o_done, ArriveHalf arrive_half,
     ArriveReady arrive_ready, SFree s_free, uint8_t* pbuf, const KvRange& kr, int nkv,
-    float scale_log2, int q0, int q_end, int h, int L, __nv_bfloat16* __restrict__ out,
+    float scale_log2, int q0, int q_end, int h, int H, int L, __nv_bfloat16* __restrict__ out,
     int64_t ld_o, float* __restrict__ lse, uint32_t* status, uint64_t budget_ns) {
   const uint32_t quarter = warp_id() & 3;
   const int row = quarter * 32 + lane_id();
@@ -258,7 +258,10 @@ __device__ __forceinline__ void softmax_warpgroup(
   if (__all_sync(0xffffffffu, ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns))) {
     tc_fence_after();
     const int r = q0 + 128 * i + row;
-    const bool live = r < q_end;
+    // rows past the segment are not stored; a stored row lies in [0, L) and
+    // its head's columns in [0, H d) (checked in debug builds)
+    const bool live = r < q_end && in_bounds(status, r, L, static_cast<int64_t>(h) * DH, DH,
+                                             static_cast<int64_t>(H) * DH);
     const float inv = 1.f / l;
     __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * DH;
 #pragma unroll 1
@@ -489,8 +492,8 @@ __global__ void __launch_bounds__(WinCfg<DH>::THREADS, 1)
     const int i = (warp - 4) >> 2;  // query tile of this warpgroup
     softmax_warpgroup<DH, false>(
         i, tmem, s_full, o_done, [&] { mbar_arrive(&p_half[i]); },
-        [&] { mbar_arrive(&p_ready[i]); }, [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, L,
-        out, ld_o, lse, status, budget_ns);
+        [&] { mbar_arrive(&p_ready[i]); }, [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, H,
+        L, out, ld_o, lse, status, budget_ns);
   }
 
   tc_fence_before();
@@ -751,7 +754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WinPairCfg<DH>::THRE
           __syncwarp();
           if (lane_id() == 0) mbar_arrive_cluster(lp_ready);
         },
-        [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse, status,
+        [] {}, nullptr, kr, nkv, scale_log2, q0, q_end, h, H, L, out, ld_o, lse, status,
         budget_ns);
   }
 

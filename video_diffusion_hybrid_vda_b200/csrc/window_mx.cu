@@ -99,8 +99,8 @@ __device__ __forceinline__ uint32_t pack_sf3(uint32_t b0, uint32_t b1, uint32_t 
 __device__ __forceinline__ void softmax_mx(int i, uint32_t tmem, uint64_t* s_full,
                                            uint64_t* s_free, uint64_t* p_ready, uint64_t* o_done,
                                            uint8_t* pbuf, uint8_t* psf, const KvRange& kr, int nkv,
-                                           float scale_log2, int q0, int q_end, int h, int L,
-                                           __nv_bfloat16* __restrict__ out, int64_t ld_o,
+                                           float scale_log2, int q0, int q_end, int h, int H,
+                                           int L, __nv_bfloat16* __restrict__ out, int64_t ld_o,
                                            float* __restrict__ lse, uint32_t* status,
                                            uint64_t budget_ns) {
   using Cfg = WinMxCfg;
@@ -255,7 +255,9 @@ __device__ __forceinline__ void softmax_mx(int i, uint32_t tmem, uint64_t* s_ful
   if (__all_sync(0xffffffffu, ok && mbar_wait(&o_done[i], (nkv - 1) & 1, budget_ns))) {
     tc_fence_after();
     const int r = q0 + 128 * i + row;
-    const bool live = r < q_end;
+    // rows past the segment are not stored (bounds checked in debug builds)
+    const bool live = r < q_end && in_bounds(status, r, L, static_cast<int64_t>(h) * 128, 128,
+                                             static_cast<int64_t>(H) * 128);
     const float inv = 1.f / l;
     __nv_bfloat16* dst = out + static_cast<int64_t>(r) * ld_o + h * 128;
 #pragma unroll 1
@@ -539,8 +541,8 @@ __global__ void __launch_bounds__(WinMxCfg::THREADS, 1)
     asm volatile("setmaxnreg.inc.sync.aligned.u32 200;\n" ::: "memory");
     const int i = (warp - 4) >> 2;
     softmax_mx(i, tmem, s_full, s_free, p_ready, o_done, pbuf + i * Cfg::P_TILE,
-               psf + i * Cfg::SF, kr, nkv, scale_log2, q0, q_end, h, L, out, ld_o, lse, status,
-               budget_ns);
+               psf + i * Cfg::SF, kr, nkv, scale_log2, q0, q_end, h, H, L, out, ld_o, lse,
+               status, budget_ns);
   }
 
   tc_fence_before();

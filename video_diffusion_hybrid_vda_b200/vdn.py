@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libvdn.so")
 VDN_OK = 0
 STATUS_NAMES = {0: "VDN_OK", 1: "VDN_ERR_INVALID_ARG", 2: "VDN_ERR_UNSUPPORTED",
                 3: "VDN_ERR_WORKSPACE", 4: "VDN_ERR_CUDA", 5: "VDN_ERR_NUMERIC",
-                6: "VDN_ERR_TIMEOUT"}
+                6: "VDN_ERR_TIMEOUT", 7: "VDN_ERR_BOUNDS"}
 
 # every symbol include/vdn.h declares
 EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
@@ -31,7 +31,8 @@ EXPORTS = ["vdn_vda_scan_workspace", "vdn_vda_scan", "vdn_vda_debug_buffers",
            "vdn_mxfp8_scale_bytes", "vdn_mxfp8_quantize", "vdn_gemm_mxfp8",
            "vdn_hybrid_fuse_mxfp8_workspace", "vdn_hybrid_fuse_mxfp8",
            "vdn_hybrid_fuse_shard_rs", "vdn_window_attn_schedule",
-           "vdn_window_attn_mxfp8_workspace", "vdn_window_attn_mxfp8", "vdn_copy2d_async"]
+           "vdn_window_attn_mxfp8_workspace", "vdn_window_attn_mxfp8", "vdn_copy2d_async",
+           "vdn_debug_bounds_enabled", "vdn_selftest_bounds"]
 
 SOLVER_CHOLESKY = 0
 SOLVER_GAUSS_JORDAN = 1
@@ -68,6 +69,10 @@ def lib():
     S = ctypes.POINTER(Shape)
     L.vdn_vda_scan_workspace.argtypes = [S]
     L.vdn_vda_scan_workspace.restype = _SZ
+    L.vdn_debug_bounds_enabled.argtypes = []
+    L.vdn_debug_bounds_enabled.restype = ctypes.c_int
+    L.vdn_selftest_bounds.argtypes = [_P, _I64, _I64, _I64, _I64, _I64, _P]
+    L.vdn_selftest_bounds.restype = ctypes.c_int
     L.vdn_vda_scan.argtypes = [S, _P, _P, _P, _I64, _P, _P, _P, _I64, _P, _P, _SZ, _P]
     L.vdn_vda_scan.restype = ctypes.c_int
     L.vdn_vda_debug_buffers.argtypes = [S, _P] + [ctypes.POINTER(_P)] * 3
@@ -219,6 +224,20 @@ def set_wait_budget_ns(ns):
 def set_vda_solver(solver):
     """SOLVER_GAUSS_JORDAN (default) or SOLVER_CHOLESKY, process-wide."""
     _check(lib().vdn_set_vda_solver(int(solver)), "vdn_set_vda_solver")
+
+
+def debug_bounds_enabled():
+    """True if the loaded library checks store indices against their
+    tensors on the device (built with VDN_DEBUG_BOUNDS=1)."""
+    return bool(lib().vdn_debug_bounds_enabled())
+
+
+def selftest_bounds(ws, r, rows, c, width, cols, stream=None):
+    """One device-side bounds check of row r and columns [c, c + width)
+    against a rows x cols tensor (no memory touched but ws's status word)."""
+    _need_cuda(ws)
+    _check(lib().vdn_selftest_bounds(_ptr(ws), int(r), int(rows), int(c), int(width), int(cols),
+                                     _stream(stream)), "vdn_selftest_bounds")
 
 
 def selftest_exp2(x, stream=None):
