@@ -1,9 +1,10 @@
 // Gradient pass of Video DeltaNet's linear branch ("Video DeltaNet",
 // 10100.com article, 方法概述 items 2 and 3: the closed-form frame update and
 // the staged alignment that trains the branch).  Two kernels of that pass
-// live here; the others are modes of the forward kernels (gram mode of the
-// prep kernel for G, adjoint mode of the scan for D, the transposed mode of
-// the read-out for dq).
+// live here; the others are modes of the forward kernels (the transposed
+// mode of the read-out for dq, which at head dim 128 also forms G, and the
+// gram mode of the prep kernel for G at head dims 64 and below; the
+// adjoint mode of the scan for D).
 //
 // With S_t = U_t P_t, U_t = alpha S_prev + B_t, P_t = (I + A_t)^-1 and the
 // adjoint states D_t = dL/dU_t of both scans:
