@@ -80,11 +80,21 @@ def test_tiny_layer(vdn, T, N, H, d):
     assert max_rel(host(y2), y2_ref) <= TOL_BF16
 
 
-def test_forward_many_pipelined_host_path(vdn):
+@pytest.mark.parametrize("T,N,H,d,nvid", [
+    (12, 96, 2, 128, 3),   # two head groups, three videos
+    (7, 100, 3, 128, 1),   # one video: head-group fill and row-block drain on it; ragged rows
+    (5, 64, 5, 128, 2),    # H = 5: a single head group
+    (9, 128, 4, 128, 2),   # four head groups
+    (7, 100, 4, 64, 2),    # head dim 64
+])
+def test_forward_many_pipelined_host_path(vdn, T, N, H, d, nvid):
     """HybridLayer.forward_many (pinned host in/out, copies overlapping the
-    compute) gives the same y as forward() on device tensors."""
-    s = synth.Shape(12, 96, 2, 128)
-    vids = [synth.make_inputs(s, seed=20 + i, device="cuda", with_fuse=True) for i in range(3)]
+    compute; the first video's inputs arriving by head groups, the last
+    video's fuse and read-back in row blocks) gives y bit-identical to
+    forward() on device tensors."""
+    s = synth.Shape(T, N, H, d)
+    vids = [synth.make_inputs(s, seed=20 + i, device="cuda", with_fuse=True)
+            for i in range(nvid)]
     w = vids[0]
     layer = vdn.HybridLayer(s.T, s.N, s.H, s.d, w["W_gs"], w["W_gl"], w["W_os"], w["W_ol"],
                             w["gamma"])
