@@ -109,3 +109,23 @@ def test_forward_many_pipelined_host_path(vdn, T, N, H, d, nvid):
     assert layer.status() == 0
     for o, r in zip(outs, refs):
         assert torch.equal(o, r.cpu())
+
+
+def test_forward_many_after_the_grouping_changes(vdn):
+    """Changing the fill and drain granularity between forward_many calls
+    (the per-group beta/alpha buffers are rebuilt for the new grouping)
+    keeps y bit-identical to forward()."""
+    s = synth.Shape(7, 100, 4, 128)
+    v = synth.make_inputs(s, seed=31, device="cuda", with_fuse=True)
+    layer = vdn.HybridLayer(s.T, s.N, s.H, s.d, v["W_gs"], v["W_gl"], v["W_os"], v["W_ol"],
+                            v["gamma"])
+    names = ("q", "k", "v", "beta", "alpha", "x")
+    ref = layer.forward(*[v[n] for n in names]).clone().cpu()
+    batch = [[v[n].to("cpu").pin_memory() for n in names]]
+    for fg, db in ((4, 4), (2, 3), (1, 1), (4, 8)):
+        layer.FILL_GROUPS, layer.DRAIN_BLOCKS = fg, db
+        out = [torch.empty((s.L, s.D), dtype=torch.bfloat16).pin_memory()]
+        layer.forward_many(batch, out)
+        torch.cuda.synchronize()
+        assert layer.status() == 0
+        assert torch.equal(out[0], ref), (fg, db)

@@ -693,15 +693,22 @@ class HybridLayer:
                         self.gamma, self.W_os, self.W_ol, self.H, eps=self.eps, out=y[r0:r1],
                         ws=self.ws_fuse, stream=stream)
 
+    # forward_many's fill and drain granularity: the first video's inputs
+    # arrive in up to FILL_GROUPS head groups (the largest count that divides
+    # H), the last video's fuse and read-back run in up to DRAIN_BLOCKS row
+    # blocks (multiples of 128 rows)
+    FILL_GROUPS = 4
+    DRAIN_BLOCKS = 4
+
     def _head_groups(self):
-        """Head groups of the first video of forward_many: up to four."""
-        g = next(n for n in (4, 3, 2, 1) if self.H % n == 0)
+        """Head groups of the first video of forward_many."""
+        g = next(n for n in range(min(self.FILL_GROUPS, self.H), 0, -1) if self.H % n == 0)
         return [(i * (self.H // g), self.H // g) for i in range(g)]
 
     def _row_chunks(self):
-        """Row blocks of the last video's fuse and read-back: up to four, of
-        multiples of 128 rows."""
-        step = max(128, (self.L + 4 * 128 - 1) // (4 * 128) * 128)
+        """Row blocks of the last video's fuse and read-back."""
+        nb = max(1, int(self.DRAIN_BLOCKS))
+        step = max(128, (self.L + nb * 128 - 1) // (nb * 128) * 128)
         return [(r, min(r + step, self.L)) for r in range(0, self.L, step)]
 
     def forward_many(self, batches, outs, stream=None, copy_stream=None):
@@ -737,10 +744,15 @@ class HybridLayer:
                             for _ in range(2)]
             self._ys = [torch.empty((self.L, self.D), dtype=torch.bfloat16, device=dev)
                         for _ in range(2)]
-            # per head group: its beta and alpha columns, contiguous
+        if getattr(self, "_grp_key", None) != tuple(groups):
+            # per head group: its beta and alpha columns, contiguous (rebuilt
+            # whenever the grouping changes)
             self._grp_ba = [(torch.empty((self.L, hg), dtype=torch.float32, device=dev),
                              torch.empty((T, hg), dtype=torch.float32, device=dev))
                             for _, hg in groups]
+            self._grp_key = tuple(groups)
+        if len(self._grp_ba) != len(groups):
+            raise RuntimeError("forward_many: head-group buffers out of step with the grouping")
         stages, ys = self._stages, self._ys
         loaded_qkv = [torch.cuda.Event() for _ in batches]
         loaded = [torch.cuda.Event() for _ in batches]
