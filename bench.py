@@ -804,8 +804,9 @@ def main():
     ap.add_argument("--part", default="all",
                     choices=["all", "layer", "vda_backward", "fuse_mxfp8", "window_mxfp8",
                              "layer_mxfp8", "scan_sweep"],
-                    help="what to time: the layer step and the two side rows (all), or one "
-                         "of them")
+                    help="what to time: the layer step and its side rows (all), one side "
+                         "row, the layer step alone (layer), or the VDA branch over the "
+                         "scan-only sweep (scan_sweep)")
     args = ap.parse_args()
     shape = WORKLOADS[args.workload]
     world = int(os.environ.get("WORLD_SIZE", "1"))
