@@ -818,7 +818,8 @@ def main():
               "mask": "chunk 5, +-1 chunk, first/last-frame anchors",
               "global_batch": world, "parallelism": f"independent videos x{world}",
               "vda_solver": args.solver,
-              "l2": "inputs larger than L2 (2.5 GB per activation), no flush"}
+              "l2": "inputs larger than L2 (%.2f GB per activation), no flush"
+                    % (shape.L * shape.D * 2 / 1e9)}
 
     if args.impl == "reference":
         if rank != 0:
